@@ -1,0 +1,427 @@
+#!/usr/bin/env python
+"""Benchmark of the MoE token-routing path (gate + align + permute-gather + combine) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = moe_topk_softmax -> moe_align_permute -> moe_gather -> moe_combine over one batch
+(the stand-in expert outputs replace the expert MLPs between gather and combine), replayed as
+one CUDA graph.  Inputs are resident in HBM; L2 is flushed (a 256 MiB write) between timed
+steps; every step is timed with CUDA events on the launching stream and the K step times are
+summed; the result is the max over ranks.  N > 1 runs one independent batch per GPU (weak
+scaling: the path has no cross-token exchange).  Rank 0 prints one JSON line.
+
+Also reported: per-stage device times and achieved HBM bandwidth from the algorithmic bytes,
+the roofline of the dominant kernel against the measured copy peak, an end-to-end figure
+through MoeRouter.step_from_host (pinned host inputs copied in and the output copied back
+inside the timed region), SM clocks sampled during the timed region, and the CPU oracle
+timed on this host as a baseline.  ``--impl reference`` times the CPU oracle alone.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "routed tokens/s (gate+align+permute+combine) and achieved HBM GB/s vs ~8 TB/s"
+UNIT = "tokens/s"
+L2_FLUSH_BYTES = 256 << 20
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = {
+    "topk_softmax_kernel": "token_dispatch_topk_b200/csrc/topk_softmax.cu",
+    "align_count_kernel+align_place_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
+    "gather_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
+    "combine_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
+}
+STAGE_KERNEL = {"topk": "topk_softmax_kernel", "align": "align_count_kernel+align_place_kernel",
+                "gather": "gather_kernel", "combine": "combine_kernel"}
+
+
+def parse_args():
+    p = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    p.add_argument("--workload", default=None, help="workload name (default: the Qwen3-MoE-like prefill)")
+    p.add_argument("--seed", type=int, default=0)
+    p.add_argument("--no-graph", action="store_true", help="launch the four calls directly instead of a graph")
+    p.add_argument("--stage-steps", type=int, default=None, help="timed iterations per stage (default: steps)")
+    p.add_argument("--e2e-steps", type=int, default=None, help="timed end-to-end steps (default: min(steps, 200))")
+    p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle baseline budget (rank 0, N=1)")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--reference-seconds", type=float, default=150.0, help="--impl reference: total time budget")
+    return p.parse_args()
+
+
+# ------------------------------------------------------------------------- helpers --
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, burst copy)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback 6.65 TB/s (no MEASURED_PEAKS.json)"
+
+
+def source_sha(rel: str) -> str:
+    with open(os.path.join(ROOT, rel), "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged since."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            table = json.load(f)
+        ent = table[f"{kernel}|{workload}"]
+        if ent.get("source_sha256") != source_sha(KERNEL_SOURCES[kernel]):
+            return None
+        return float(ent["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def algorithmic_bytes(wl, R: int, C: int, NB: int) -> dict:
+    """Bytes each stage must move (each input read once, each output written once)."""
+    lb = 2 if wl.logits_dtype == "bf16" else 4
+    T, E, k, H, El = wl.T, wl.E, wl.k, wl.H, wl.experts_local
+    mp = E * 4 if wl.E_local is not None else 0
+    return {
+        "topk": T * E * lb + T * k * 8,
+        "align": 2 * T * k * 4 + mp + C * 4 + NB * 4 + (2 * El + 2) * 4,
+        "gather": T * H * 2 + R * H * 2 + T * k * 4,
+        "combine": R * H * 2 + T * k * 8 + T * H * 2,
+    }
+
+
+class ClockSampler:
+    """nvidia-smi SM clock / throttle-reason sampling in the background (200 ms period)."""
+    FIELDS = ("uuid,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, uuid: str | None):
+        self.uuid = uuid
+        self.proc = None
+        self.file = None
+
+    def start(self):
+        try:
+            self.file = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=self.file, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0, "note": "nvidia-smi unavailable"}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.file.flush()
+        self.file.seek(0)
+        rows = [ln.split(",") for ln in self.file.read().splitlines() if ln.strip()]
+        os.unlink(self.file.name)
+        rows = [[c.strip() for c in r] for r in rows if len(r) >= 10]
+        if self.uuid:
+            mine = [r for r in rows if self.uuid in r[0]]
+            rows = mine or rows
+        sm = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        mx = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower().startswith("active")})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ CPU oracle leg --
+def oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, t0: int, n: int):
+    """The oracle pipeline on tokens [t0, t0+n) of the workload (gate, align, gather, combine)."""
+    w, ids = oracle_mod.topk_softmax(logits_np[t0:t0 + n], wl.k, wl.renormalize)
+    al = oracle_mod.align_permute(ids, wl.E, wl.block_size, emap_np, wl.experts_local)
+    npad = int(al["num_tokens_post_pad"][0])
+    oracle_mod.gather(hidden_bits[t0:t0 + n], wl.k, al["sorted_token_ids"], npad, al["capacity"])
+    oracle_mod.combine(y_bits[:al["capacity"]], w, al["inv_perm"])
+    return n
+
+
+def host_inputs_numpy(wl, seed: int, T_max: int):
+    import numpy as np
+    import torch
+    from token_dispatch_topk_b200 import inputs as I
+    T = min(wl.T, T_max)
+    logits = I.make_logits(wl, seed=seed, T=T)
+    logits_np = logits.view(torch.int16).numpy().view(np.uint16) if logits.dtype == torch.bfloat16 else logits.numpy()
+    hidden = I.make_hidden(wl, seed=seed, T=T)
+    hidden_bits = hidden.view(torch.int16).numpy().view(np.uint16)
+    cap = T * wl.k + wl.experts_local * (wl.block_size - 1)
+    y = I.make_expert_out(cap, wl.H, seed=seed)
+    y_bits = y.view(torch.int16).numpy().view(np.uint16)
+    emap = I.expert_map(wl)
+    return logits_np, hidden_bits, y_bits, None if emap is None else emap.numpy()
+
+
+def cpu_oracle_rate(wl, seed: int, budget_s: float, T_max: int = 4096):
+    """Tokens/s of the oracle on this host over a bounded sample (single-threaded)."""
+    import oracle as oracle_mod
+    oracle_mod.default()
+    logits_np, hidden_bits, y_bits, emap_np = host_inputs_numpy(wl, seed, T_max)
+    T = logits_np.shape[0]
+    done, reps = 0, 0
+    t_start = time.perf_counter()
+    while True:
+        done += oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, T)
+        reps += 1
+        el = time.perf_counter() - t_start
+        if el >= budget_s or reps >= 1000:
+            break
+    return {"value": done / el, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{reps} oracle passes over the first {T} tokens of the workload ({el:.1f} s, single thread)"}
+
+
+def run_reference(args, wl):
+    """--impl reference: the CPU oracle on this host as the reference arm."""
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import oracle as oracle_mod
+    oracle_mod.default()
+    steps, warm = args.steps, args.warmup
+    # calibrate the per-step sample so that warmup + steps fit the time budget
+    T_cal = min(wl.T, 64)
+    logits_np, hidden_bits, y_bits, emap_np = host_inputs_numpy(wl, args.seed, min(wl.T, 4096))
+    t = time.perf_counter()
+    oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, T_cal)
+    per_token = max((time.perf_counter() - t) / T_cal, 1e-7)
+    per_step_budget = args.reference_seconds / max(1, steps + warm)
+    n = int(max(1, min(logits_np.shape[0], per_step_budget / per_token)))
+    for i in range(warm):
+        oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, n)
+    t = time.perf_counter()
+    for i in range(steps):
+        t0 = (i * n) % max(1, logits_np.shape[0] - n + 1)
+        oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, t0, n)
+    el = time.perf_counter() - t
+    value = steps * n / el
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps,
+            "warmup": warm, "ms_per_step": 1e3 * el / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64 softmax, fp32 combine", "data": "synthetic",
+            "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"}},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                             "sample": f"{n} tokens of the workload per step, single-threaded C++ oracle"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------ GPU leg --
+def main():
+    args = parse_args()
+    from token_dispatch_topk_b200 import inputs as I
+    wl = I.WORKLOADS[args.workload or I.DEFAULT_WORKLOAD]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+    import token_dispatch_topk_b200 as tdt
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    seed = args.seed + rank  # an independent batch per rank
+    tdt.load_library()
+
+    # ---- inputs resident in HBM
+    logits_h = I.make_logits(wl, seed=seed)
+    hidden_h = I.make_hidden(wl, seed=seed)
+    logits = logits_h.to(dev)
+    hidden = hidden_h.to(dev)
+    y = I.make_expert_out(wl.capacity, wl.H, seed=seed, device=dev)
+    r = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, E_local=wl.E_local,
+                      expert_map=I.expert_map(wl), logits_dtype=logits.dtype, device=dev)
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def flush(i=0):
+        flush_buf.fill_(i & 0xFF)
+
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            r.step(logits, hidden, y)
+    stream.synchronize()
+    if r.device_status() != tdt.MOE_OK:
+        raise RuntimeError("device status after warm-up steps is not MOE_OK")
+    R = int(r.align.counts.sum().item())
+    npad = int(r.align.num_tokens_post_pad.item())
+    NB = r.align.expert_ids.numel()
+    align_launches = 1 if tdt.moe_align_workspace_bytes(wl.T, wl.k, wl.experts_local) <= 256 else 2
+    launches_per_step = 1 + align_launches + 1 + 1
+
+    use_graph = not args.no_graph
+    graphs = {}
+    if use_graph:
+        def capture(fn):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                fn()
+            return g
+        graphs["step"] = capture(lambda: r.step(logits, hidden, y))
+        graphs["topk"] = capture(lambda: r.gate(logits))
+        graphs["align"] = capture(lambda: r.align_permute())
+        graphs["gather"] = capture(lambda: r.gather(hidden))
+        graphs["combine"] = capture(lambda: r.combine(y))
+    stage_fns = {"step": lambda: r.step(logits, hidden, y), "topk": lambda: r.gate(logits),
+                 "align": lambda: r.align_permute(), "gather": lambda: r.gather(hidden),
+                 "combine": lambda: r.combine(y)}
+
+    def run(name):
+        if use_graph:
+            graphs[name].replay()
+        else:
+            stage_fns[name]()
+
+    def timed(name, iters, warm):
+        """Sum of per-iteration event times (ms), L2 flushed before each iteration."""
+        with torch.cuda.stream(stream):
+            for i in range(warm):
+                flush(i)
+                run(name)
+            evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+            for i, (a, b) in enumerate(evs):
+                flush(i)
+                a.record(stream)
+                run(name)
+                b.record(stream)
+        stream.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs)
+
+    # ---- the timed region: K steps
+    uuid = None
+    try:
+        uuid = str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    sampler = ClockSampler(uuid) if rank == 0 else None
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if sampler:
+        sampler.start()
+        time.sleep(0.4)
+    total_ms = timed("step", args.steps, args.warmup)
+    torch.cuda.synchronize()
+    clocks = sampler.stop() if sampler else None
+    if ws > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+        dist.barrier()
+    ms_per_step = total_ms / args.steps
+    value = ws * wl.T * args.steps / (total_ms / 1e3)
+
+    # ---- per-stage times (same flush protocol) and roofline
+    peak, peak_src = measured_peaks()
+    abytes = algorithmic_bytes(wl, R, r.capacity, NB)
+    st_iters = args.stage_steps or args.steps
+    stages = {}
+    for name in ("topk", "align", "gather", "combine"):
+        ms = timed(name, st_iters, min(args.warmup, 10)) / st_iters
+        stages[name] = {"us": 1e3 * ms, "algorithmic_bytes": abytes[name],
+                        "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": STAGE_KERNEL[name]}
+    dom = max(("gather", "combine"), key=lambda s: stages[s]["us"])
+    ach = stages[dom]["achieved_gbs"]
+    total_bytes = sum(abytes.values())
+    roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                "traffic": ncu_traffic(STAGE_KERNEL[dom], wl.name), "kernel": STAGE_KERNEL[dom],
+                "peak_source": peak_src,
+                "algorithmic_bytes_per_launch": abytes[dom]}
+
+    # ---- end to end through the public API, from pinned host buffers
+    e2e_steps = args.e2e_steps or min(args.steps, 200)
+    lp, hp = logits_h.pin_memory(), hidden_h.pin_memory()
+    out_h = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            r.step_from_host(lp, hp, y, out_h, stream)
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
+        for a, b in evs:
+            a.record(stream)
+            r.step_from_host(lp, hp, y, out_h, stream)
+            b.record(stream)
+    stream.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in evs)
+    if ws > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    h2d = lp.numel() * lp.element_size() + hp.numel() * hp.element_size()
+    d2h = out_h.numel() * out_h.element_size()
+    e2e = {"value": ws * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+           "api": "MoeRouter.step_from_host (pinned H2D of logits+hidden, 4 C-ABI calls, D2H of out)"}
+
+    if r.device_status() != tdt.MOE_OK:
+        raise RuntimeError("device status after the timed steps is not MOE_OK")
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_rate(wl, seed, args.cpu_seconds)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "dtype_detail": "bf16 activations, fp32 gating math and combine accumulation, int32 indices",
+            "data": "synthetic (seeded; see token_dispatch_topk_b200/inputs.py)",
+            "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                       "cuda_graph": use_graph,
+                       "parallelism": "one independent batch per GPU" if ws > 1 else "single GPU"},
+            "achieved_hbm_gbs": total_bytes / (ms_per_step * 1e-3) / 1e9,
+            "algorithmic_bytes_per_step": total_bytes,
+            "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
+            "routed_slots_local": R, "num_tokens_post_pad": npad,
+            "roofline": roofline, "stages": stages, "e2e": e2e, "cpu_baseline": cpu,
+            "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    del graphs
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,117 @@
+"""The C-ABI library on the CPU: it loads, exports every symbol include/moe_route.h declares,
+and its host-side logic (sizes, validation, status strings) behaves as documented.
+No call here reaches a CUDA launch: each one is rejected (or is a no-op) before that."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+import token_dispatch_topk_b200 as tdt
+from token_dispatch_topk_b200 import binding as B
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_route.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_four_stages():
+    names = declared_symbols()
+    for stage in ("moe_topk_softmax", "moe_align_permute", "moe_gather", "moe_combine"):
+        assert stage in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = B.load_library()
+    names = declared_symbols()
+    assert names, "no MOE_API declarations found"
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in moe_route.h but not exported"
+    assert set(names) == set(B.SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(RuntimeError, match="no CPU fallback"):
+        B.load_library(str(tmp_path / "absent.so"))
+
+
+def test_sizes_match_the_oracle():
+    for T, k, El, bs in [(64, 2, 8, 16), (4096, 8, 128, 64), (2, 6, 40, 8), (16384, 4, 60, 64),
+                         (65536, 8, 256, 128), (0, 3, 5, 7), (1, 1, 1, 1)]:
+        assert tdt.moe_align_capacity(T, k, El, bs) == oracle.align_capacity(T, k, El, bs)
+        C = tdt.moe_align_capacity(T, k, El, bs)
+        assert tdt.moe_align_num_blocks(T, k, El, bs) == -(-C // bs)
+        assert tdt.moe_align_workspace_bytes(T, k, El) >= 256
+    assert tdt.moe_align_capacity(-1, 2, 3, 4) == -1
+    assert tdt.moe_align_capacity(4, 0, 3, 4) == -1
+
+
+def test_status_strings():
+    for code in range(8):
+        assert B.status_string(code).startswith("MOE_")
+    assert "UNKNOWN" in B.status_string(99)
+    assert tdt.moe_version() >= 100
+
+
+N = None
+
+
+def test_topk_validation_before_launch():
+    lib = B.load_library()
+    f = lib.moe_topk_softmax
+    assert f(N, B.MOE_DTYPE_BF16, 4, 8, 9, 0, N, N, N) == B.MOE_ERR_INVALID_ARG       # k > E
+    assert f(N, B.MOE_DTYPE_BF16, 4, 8, 0, 0, N, N, N) == B.MOE_ERR_INVALID_ARG       # k < 1
+    assert f(N, B.MOE_DTYPE_BF16, -1, 8, 2, 0, N, N, N) == B.MOE_ERR_INVALID_ARG      # T < 0
+    assert f(N, 7, 4, 8, 2, 0, N, N, N) == B.MOE_ERR_INVALID_ARG                      # dtype
+    assert f(N, B.MOE_DTYPE_F32, 4, 8, 2, 0x10, N, N, N) == B.MOE_ERR_INVALID_ARG     # flags
+    assert f(N, B.MOE_DTYPE_F32, 4, 2048, 2, 0, N, N, N) == B.MOE_ERR_UNSUPPORTED     # E > 1024
+    assert f(N, B.MOE_DTYPE_F32, 4, 64, 33, 0, N, N, N) == B.MOE_ERR_UNSUPPORTED      # k > 32
+    assert f(N, B.MOE_DTYPE_F32, 4, 64, 8, 0, N, N, N) == B.MOE_ERR_INVALID_ARG       # null pointers
+    assert f(N, B.MOE_DTYPE_F32, 0, 64, 8, 1, N, N, N) == B.MOE_OK                    # T == 0: no-op
+
+
+def test_align_validation_before_launch():
+    lib = B.load_library()
+    f = lib.moe_align_permute
+    buf = ctypes.c_void_p(16)  # never dereferenced: every call below is rejected on the host
+    args = lambda T=4, k=2, Eg=8, emap=N, El=8, bs=4, ws=buf, wsb=1 << 20: (
+        buf, T, k, Eg, emap, El, bs, buf, buf, buf, buf, buf, buf, ws, wsb, N)
+    assert f(*args(El=9)) == B.MOE_ERR_INVALID_ARG            # E_local > E_global
+    assert f(*args(El=4)) == B.MOE_ERR_INVALID_ARG            # identity map needs E_local == E_global
+    assert f(*args(bs=0)) == B.MOE_ERR_INVALID_ARG
+    assert f(*args(T=-1)) == B.MOE_ERR_INVALID_ARG
+    assert f(*args(Eg=2048, El=2048)) == B.MOE_ERR_UNSUPPORTED
+    assert f(*args(ws=N)) == B.MOE_ERR_WORKSPACE
+    assert f(*args(wsb=8)) == B.MOE_ERR_WORKSPACE
+    assert f(*args(T=1 << 28, k=8)) == B.MOE_ERR_INVALID_ARG  # T*k >= 2^30
+    assert f(*args(ws=ctypes.c_void_p(20))) == B.MOE_ERR_INVALID_ARG  # misaligned workspace
+
+
+def test_gather_combine_validation_before_launch():
+    lib = B.load_library()
+    buf = ctypes.c_void_p(16)
+    odd = ctypes.c_void_p(24)
+    g = lib.moe_gather
+    assert g(buf, 4, 12, 2, buf, N, N, 100, 0, buf, N, N) == B.MOE_ERR_INVALID_ARG    # H % 8
+    assert g(odd, 4, 16, 2, buf, N, N, 100, 0, buf, N, N) == B.MOE_ERR_INVALID_ARG    # misaligned hidden
+    assert g(buf, 4, 16, 2, buf, N, N, 100, 0x8, buf, N, N) == B.MOE_ERR_INVALID_ARG  # flags
+    assert g(buf, 4, 16, 2, buf, N, N, 100, B.MOE_GATHER_ZERO_PAD, buf, N, N) == B.MOE_ERR_INVALID_ARG
+    assert g(buf, 4, 16, 33, buf, N, N, 100, 0, buf, N, N) == B.MOE_ERR_UNSUPPORTED
+    assert g(N, 0, 16, 2, N, N, N, 0, 0, N, N, N) == B.MOE_OK                         # nothing to do
+    c = lib.moe_combine
+    assert c(buf, buf, buf, 4, 2, 12, 100, buf, N, N) == B.MOE_ERR_INVALID_ARG        # H % 8
+    assert c(buf, buf, buf, 4, 2, 16, 100, odd, N, N) == B.MOE_ERR_INVALID_ARG        # misaligned out
+    assert c(buf, N, buf, 4, 2, 16, 100, buf, N, N) == B.MOE_ERR_INVALID_ARG          # null weights
+    assert c(N, N, N, 0, 2, 16, 0, N, N, N) == B.MOE_OK                               # T == 0
+    assert lib.moe_read_status(N, N, N) == B.MOE_ERR_INVALID_ARG
+
+
+def test_binding_rejects_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError, match="CUDA tensor"):
+        tdt.moe_topk_softmax(torch.zeros(4, 8, dtype=torch.bfloat16), 2, True)

@@ -1,0 +1,185 @@
+"""End-to-end GPU parity on the five routing workloads, at their full sizes, through
+MoeRouter.step (the four C-ABI calls the bench times) against the CPU oracle pipeline.
+
+The tiny, prefill, decode and non-power-of-2 workloads are compared in full.  The
+skewed 65 536-token workload (about 17 GB on the device) is compared in full for gating
+and align, and on sampled rows for gather and combine: the oracle computes those rows one
+by one from the same inputs, the expert outputs being read back for the sampled rows only.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_dispatch_topk_b200 as tdt
+from token_dispatch_topk_b200 import inputs as I
+
+from gpu_helpers import (COMBINE_MAX_ULP, TOPK_WEIGHT_ATOL, assert_align_equal, bf16_bits, logits_for_oracle,
+                         np_i32, require_gpu, ulp_distance_bf16)
+
+pytestmark = pytest.mark.gpu
+
+FULL = ["tiny_T64_E8_k2", "qwen3moe_prefill_T4096_E128_k8", "nonpow2_T16384_E60_k4"]
+
+
+def _router(wl, dev):
+    emap = I.expert_map(wl)
+    return tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, E_local=wl.E_local,
+                         expert_map=emap, logits_dtype=torch.bfloat16 if wl.logits_dtype == "bf16" else torch.float32,
+                         device=dev)
+
+
+def _oracle_pipeline(wl, logits, hidden_bits, y_bits, ids_override=None, w_override=None):
+    w, ids = oracle.topk_softmax(logits_for_oracle(logits), wl.k, wl.renormalize)
+    if ids_override is not None:
+        ids = ids_override
+    if w_override is not None:
+        w = w_override
+    emap = I.expert_map(wl)
+    al = oracle.align_permute(ids, wl.E, wl.block_size, None if emap is None else emap.numpy(), wl.experts_local)
+    npad = int(al["num_tokens_post_pad"][0])
+    perm = oracle.gather(hidden_bits, wl.k, al["sorted_token_ids"], npad, al["capacity"])
+    out = oracle.combine(y_bits, w, al["inv_perm"])
+    return w, ids, al, perm, out
+
+
+def _check_all(r, wl, ref, what):
+    w_ref, ids_ref, al_ref, perm_ref, out_ref = ref
+    assert np.array_equal(np_i32(r.topk_ids), ids_ref), what
+    assert np.abs(r.topk_weights.cpu().numpy() - w_ref).max() <= TOPK_WEIGHT_ATOL, what
+    assert_align_equal(r.align, al_ref, what)
+    npad = int(al_ref["num_tokens_post_pad"][0])
+    real = al_ref["sorted_token_ids"][:npad] != wl.T * wl.k
+    got = bf16_bits(r.permuted[:npad])
+    assert np.array_equal(got[real], perm_ref[:npad][real]), what
+    d = ulp_distance_bf16(bf16_bits(r.out), out_ref)
+    assert d.max() <= COMBINE_MAX_ULP, (what, d.max())
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_workload_full_size(name):
+    dev = require_gpu()
+    wl = I.WORKLOADS[name]
+    logits = I.make_logits(wl)
+    hidden = I.make_hidden(wl)
+    y = I.make_expert_out(wl.capacity, wl.H)
+    r = _router(wl, dev)
+    r.step(logits.to(dev), hidden.to(dev), y.to(dev))
+    torch.cuda.synchronize()
+    ref = _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y))
+    _check_all(r, wl, ref, name)
+    assert r.device_status() == tdt.MOE_OK
+
+
+def test_ep_decode_every_route_pattern():
+    """M=2, top-k 6, rank 1 of 4 (40 local experts): the logits-derived routing and every
+    injected route pattern, including the valid all-remote rank."""
+    dev = require_gpu()
+    wl = I.WORKLOADS["ep_decode_T2_E160_local40_k6"]
+    logits = I.make_logits(wl)
+    hidden = I.make_hidden(wl)
+    y = I.make_expert_out(wl.capacity, wl.H)
+    r = _router(wl, dev)
+    r.step(logits.to(dev), hidden.to(dev), y.to(dev))
+    torch.cuda.synchronize()
+    _check_all(r, wl, _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y)), "logits-derived")
+    w_inj = I.decode_pattern_weights()
+    for name in I.DECODE_PATTERNS:
+        ids = I.decode_pattern_ids(name)
+        r.gate(logits.to(dev))
+        r.topk_ids.copy_(ids.to(dev))
+        r.topk_weights.copy_(w_inj.to(dev))
+        r.align_permute()
+        r.gather(hidden.to(dev))
+        r.combine(y.to(dev))
+        torch.cuda.synchronize()
+        w_ref, _, al, perm, out = _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y),
+                                                   ids_override=ids.numpy(), w_override=w_inj.numpy())
+        assert_align_equal(r.align, al, name)
+        npad = int(al["num_tokens_post_pad"][0])
+        real = al["sorted_token_ids"][:npad] != wl.T * wl.k
+        assert np.array_equal(bf16_bits(r.permuted[:npad])[real], perm[:npad][real]), name
+        assert np.array_equal(bf16_bits(r.out), out), name
+        if name == "all_remote":
+            assert npad == 0 and (bf16_bits(r.out) == 0).all()
+
+
+def test_skewed_prefill_full_size_sampled():
+    dev = require_gpu()
+    wl = I.WORKLOADS["zipf_prefill_T65536_E256_k8_H7168"]
+    logits = I.make_logits(wl)
+    hidden = I.make_hidden(wl)
+    y_dev = I.make_expert_out(wl.capacity, wl.H, device=dev)
+    r = _router(wl, dev)
+    r.step(logits.to(dev), hidden.to(dev), y_dev)
+    torch.cuda.synchronize()
+    # gating and align in full
+    w_ref, ids_ref = oracle.topk_softmax(logits_for_oracle(logits), wl.k, wl.renormalize)
+    assert np.array_equal(np_i32(r.topk_ids), ids_ref)
+    assert np.abs(r.topk_weights.cpu().numpy() - w_ref).max() <= TOPK_WEIGHT_ATOL
+    al = oracle.align_permute(ids_ref, wl.E, wl.block_size)
+    assert_align_equal(r.align, al, "skewed")
+    counts = al["counts"]
+    assert counts.max() > 0.5 * wl.T and (counts == 0).any() or counts.max() > 8 * counts.mean()
+    # gather: sampled rows, each recomputed by the oracle from its slot id
+    rng = np.random.default_rng(0)
+    npad = int(al["num_tokens_post_pad"][0])
+    rows = np.unique(np.concatenate([rng.integers(0, npad, 512), [0, npad - 1]]))
+    sti = al["sorted_token_ids"][rows]
+    want = oracle.gather(bf16_bits(hidden), wl.k, sti, len(rows), len(rows))
+    got = bf16_bits(r.permuted[torch.from_numpy(rows).to(dev)])
+    real = sti != wl.T * wl.k
+    assert np.array_equal(got[real], want[real])
+    # combine: sampled tokens; the expert-output rows they read are copied back
+    toks = np.unique(np.concatenate([rng.integers(0, wl.T, 256), [0, wl.T - 1]]))
+    inv = al["inv_perm"].reshape(wl.T, wl.k)[toks]
+    used = np.unique(inv[inv >= 0])
+    y_rows = bf16_bits(y_dev[torch.from_numpy(used).long().to(dev)])
+    remap = np.full(wl.capacity, -1, np.int64)
+    remap[used] = np.arange(len(used))
+    inv_c = np.where(inv >= 0, remap[np.maximum(inv, 0)], -1).astype(np.int32).reshape(-1)
+    want = oracle.combine(y_rows, w_ref[toks], inv_c)
+    got = bf16_bits(r.out[torch.from_numpy(toks).long().to(dev)])
+    assert ulp_distance_bf16(got, want).max() <= COMBINE_MAX_ULP
+
+
+def test_repeat_steps_are_bit_identical():
+    dev = require_gpu()
+    wl = I.WORKLOADS["qwen3moe_prefill_T4096_E128_k8"]
+    logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)
+    y = I.make_expert_out(wl.capacity, wl.H, device=dev)
+    r = _router(wl, dev)
+    first = None
+    for _ in range(5):
+        r.step(logits, hidden, y)
+        snap = [t.clone() for t in (r.topk_ids, r.topk_weights, r.align.sorted_token_ids, r.align.inv_perm,
+                                    r.align.expert_ids, r.out)]
+        if first is None:
+            first = snap
+        else:
+            for a, b in zip(first, snap):
+                assert torch.equal(a, b)
+
+
+def test_end_to_end_from_host_buffers():
+    dev = require_gpu()
+    wl = I.WORKLOADS["tiny_T64_E8_k2"]
+    logits, hidden = I.make_logits(wl).pin_memory(), I.make_hidden(wl).pin_memory()
+    y = I.make_expert_out(wl.capacity, wl.H)
+    out_host = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
+    r = _router(wl, dev)
+    r.step_from_host(logits, hidden, y.to(dev), out_host)
+    torch.cuda.synchronize()
+    ref = _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y))
+    assert np.array_equal(bf16_bits(out_host), ref[4])
+
+
+def test_zero_tokens():
+    dev = require_gpu()
+    r = tdt.MoeRouter(0, 16, 4, 64, 8, True, device=dev)
+    r.step(torch.empty((0, 16), dtype=torch.bfloat16, device=dev), torch.empty((0, 64), dtype=torch.bfloat16,
+                                                                                 device=dev),
+           torch.empty((r.capacity, 64), dtype=torch.bfloat16, device=dev))
+    torch.cuda.synchronize()
+    ref = oracle.align_permute(np.zeros((0, 4), np.int32), 16, 8)
+    assert_align_equal(r.align, ref, "T=0")

@@ -1,0 +1,418 @@
+// align_permute.cu -- per-expert histogram, block-padded prefix and stable placement.
+//
+// Operation: "Upstream Reference: Deep-Spark xllm + vllm", "File Index"
+// (moe_align_sum_kernels.cu: block alignment for scatter), with the expert-parallel
+// remap of the 2026-07-16 MTP1 M=2 compact scheduler closure note (scheduler
+// paragraph: each local expert's row count and remapped-row prefix come from topk_ids
+// plus expert_map; coverage paragraph: an all-remote rank is valid).
+//
+// Slots s = t*k + j are cut into tiles of `tile_slots` consecutive slots.
+//   count kernel (one CTA per tile): local expert of every slot, warp-aggregated
+//     shared-memory histogram (match.any groups equal experts so one lane adds for
+//     the whole group), tile counts to the workspace.  The CTA that finishes last
+//     (completion ticket, no spinning) scans the tile counts per expert into
+//     exclusive per-tile prefixes, writes counts, the block-padded offsets and
+//     N_pad, and resets the ticket for the next call.
+//   place kernel (one CTA per tile): every warp owns a contiguous run of the
+//     tile's slots; per-warp histograms are scanned across warps, then each warp
+//     walks its run in order and gives every slot the row
+//        offsets[e] + tile prefix[e] + warp prefix[e] + rank among equal experts
+//     in its 32-slot chunk (ballot-free: match.any + popc of the lower lanes).
+//     Rows therefore follow (expert, slot) order exactly, with no dependence on
+//     atomic ordering.  The same kernel writes the pad value into the pad rows,
+//     the tail rows past N_pad, and expert_ids.
+// When all slots fit one tile (decode, small batches), the count kernel does
+// everything in one CTA and the place kernel is not launched.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kAlignThreads = 512;
+constexpr int kAlignWarps = kAlignThreads / 32;
+constexpr int kWsHeaderBytes = 256;  // status word, ticket, padding
+
+struct AlignArgs {
+  const int32_t* topk_ids;
+  const int32_t* expert_map;
+  int64_t P;  // slots = T*k
+  int E_global;
+  int E_local;
+  int bs;
+  int64_t C;  // capacity rows
+  int NB;     // blocks
+  int tile_slots;
+  int num_tiles;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_ids;
+  int32_t* expert_ids;
+  int32_t* n_pad;
+  int32_t* inv_perm;
+  int32_t* status;
+  unsigned int* ticket;
+  int32_t* tile_counts;  // [num_tiles][E_local]
+};
+
+// Local expert of slot s, or -1 (remote).  Bad ids are remote and flagged.
+__device__ __forceinline__ int local_expert(const AlignArgs& a, int64_t s) {
+  const int g = a.topk_ids[s];
+  if (static_cast<unsigned>(g) >= static_cast<unsigned>(a.E_global)) {
+    moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+    return -1;
+  }
+  const int le = a.expert_map != nullptr ? a.expert_map[g] : g;
+  if (le < -1 || le >= a.E_local) {
+    moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+    return -1;
+  }
+  return le;
+}
+
+// Block-wide exclusive scan of n <= 2*kAlignThreads ints in shared memory (in place).
+// Returns the total.  Every thread of the block must call it.
+__device__ int block_exclusive_scan(int* data, int n, int* warp_sums) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = 2 * tid, i1 = 2 * tid + 1;
+  const int a = i0 < n ? data[i0] : 0;
+  const int b = i1 < n ? data[i1] : 0;
+  int incl = a + b;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kAlignWarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += v;
+    }
+    if (lane < kAlignWarps) warp_sums[lane] = w;  // inclusive warp prefix
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - (a + b);
+  const int total = warp_sums[kAlignWarps - 1];
+  __syncthreads();
+  if (i0 < n) data[i0] = before;
+  if (i1 < n) data[i1] = before + a;
+  __syncthreads();
+  return total;
+}
+
+// counts (s_cnt) -> block-padded exclusive offsets (s_off, E_local+1 entries); writes the
+// counts/offsets/N_pad outputs.  Block-wide.
+__device__ void padded_offsets(const AlignArgs& a, const int* s_cnt, int* s_off, int* warp_sums) {
+  for (int e = threadIdx.x; e < a.E_local; e += blockDim.x) {
+    const int c = s_cnt[e];
+    s_off[e] = ((c + a.bs - 1) / a.bs) * a.bs;
+  }
+  __syncthreads();
+  const int total = block_exclusive_scan(s_off, a.E_local, warp_sums);
+  if (threadIdx.x == 0) {
+    s_off[a.E_local] = total;
+    a.offsets[a.E_local] = total;
+    a.n_pad[0] = total;
+  }
+  for (int e = threadIdx.x; e < a.E_local; e += blockDim.x) {
+    a.offsets[e] = s_off[e];
+    a.counts[e] = s_cnt[e];
+  }
+  __syncthreads();
+}
+
+// Pad value into every non-slot row, expert_ids for every block.  Work is split over
+// `nworkers` CTAs; this CTA is `worker`.
+__device__ void fill_pads_and_blocks(const AlignArgs& a, const int* s_cnt, const int* s_off, int worker,
+                                     int nworkers) {
+  const int npad = s_off[a.E_local];
+  const int64_t pad_items = static_cast<int64_t>(a.E_local) * a.bs;
+  const int64_t tail = a.C - npad;
+  const int32_t pad_value = static_cast<int32_t>(a.P);
+  const int64_t stride = static_cast<int64_t>(nworkers) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(worker) * blockDim.x + threadIdx.x; i < pad_items + tail; i += stride) {
+    if (i < pad_items) {
+      const int e = static_cast<int>(i / a.bs);
+      const int r = static_cast<int>(i - static_cast<int64_t>(e) * a.bs);
+      const int p = s_off[e] + s_cnt[e] + r;
+      if (p < s_off[e + 1]) a.sorted_ids[p] = pad_value;
+    } else {
+      a.sorted_ids[npad + (i - pad_items)] = pad_value;
+    }
+  }
+  // expert of each block: the largest e with offsets[e] <= b*bs (empty experts share offsets
+  // with their successor, so the largest such e is the non-empty one), -1 past N_pad.
+  for (int64_t b = static_cast<int64_t>(worker) * blockDim.x + threadIdx.x; b < a.NB; b += stride) {
+    const int64_t row = b * a.bs;
+    int e = -1;
+    if (row < npad) {
+      int lo = 0, hi = a.E_local - 1;  // invariant: s_off[lo] <= row
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    a.expert_ids[b] = e;
+  }
+}
+
+// Stable placement of one tile.  s_base[e] = first row of this tile's slots of expert e.
+// s_whist: [kAlignWarps][E_local] scratch, s_le: [tile_slots] scratch.
+__device__ void place_tile(const AlignArgs& a, int tile, const int* s_base, int* s_whist, int* s_le) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t s0 = static_cast<int64_t>(tile) * a.tile_slots;
+  const int64_t s1 = (s0 + a.tile_slots < a.P) ? s0 + a.tile_slots : a.P;
+  const int per_warp = ((a.tile_slots / kAlignWarps) + 31) & ~31;
+  const int64_t w0 = s0 + static_cast<int64_t>(warp) * per_warp;
+  const int64_t w1 = (w0 + per_warp < s1) ? w0 + per_warp : s1;
+  int* my_hist = s_whist + warp * a.E_local;
+
+  for (int i = tid; i < kAlignWarps * a.E_local; i += blockDim.x) s_whist[i] = 0;
+  __syncthreads();
+  // pass 1: per-warp histogram of its own run (one adding lane per group of equal experts)
+  for (int64_t base = w0; base < w1; base += 32) {
+    const int64_t s = base + lane;
+    const int le = s < w1 ? local_expert(a, s) : -1;
+    if (s < w1) s_le[s - s0] = le;
+    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // pass 2: exclusive scan over warps, seeded with the tile's base row
+  for (int e = tid; e < a.E_local; e += blockDim.x) {
+    int run = s_base[e];
+    for (int w = 0; w < kAlignWarps; ++w) {
+      const int c = s_whist[w * a.E_local + e];
+      s_whist[w * a.E_local + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  // pass 3: rows in slot order
+  for (int64_t base = w0; base < w1; base += 32) {
+    const int64_t s = base + lane;
+    const int le = s < w1 ? s_le[s - s0] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    if (le >= 0) {
+      const int row = my_hist[le] + __popc(peers & moe::lanemask_lt());
+      a.sorted_ids[row] = static_cast<int32_t>(s);
+      a.inv_perm[s] = row;
+    } else if (s < w1) {
+      a.inv_perm[s] = -1;
+    }
+    __syncwarp();
+    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
+    __syncwarp();
+  }
+}
+
+// Shared-memory layout of both kernels (ints):
+//   s_cnt[E_local] | s_off[E_local+1] | warp_sums[32] | s_whist[kAlignWarps*E_local] | s_le[tile_slots]
+//   | s_tile_base[E_local] (place kernel)
+__host__ __device__ inline size_t align_smem_ints(int E_local, int tile_slots) {
+  return static_cast<size_t>(E_local) + (E_local + 1) + 32 + static_cast<size_t>(kAlignWarps) * E_local +
+         tile_slots + E_local;
+}
+
+__global__ void __launch_bounds__(kAlignThreads) align_count_kernel(AlignArgs a) {
+  extern __shared__ int smem[];
+  int* s_cnt = smem;
+  int* s_off = s_cnt + a.E_local;
+  int* warp_sums = s_off + a.E_local + 1;
+  int* s_whist = warp_sums + 32;
+  int* s_le = s_whist + kAlignWarps * a.E_local;
+  __shared__ int s_is_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x;
+  const int64_t s0 = static_cast<int64_t>(tile) * a.tile_slots;
+  const int64_t s1 = (s0 + a.tile_slots < a.P) ? s0 + a.tile_slots : a.P;
+
+  for (int e = tid; e < a.E_local; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  for (int64_t base = s0 + static_cast<int64_t>(warp) * 32; base < s1; base += kAlignThreads) {
+    const int64_t s = base + lane;
+    const int le = s < s1 ? local_expert(a, s) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    if (le >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_cnt[le], __popc(peers));
+  }
+  __syncthreads();
+
+  if (a.num_tiles == 1) {
+    // everything in this CTA
+    padded_offsets(a, s_cnt, s_off, warp_sums);
+    place_tile(a, 0, s_off, s_whist, s_le);
+    fill_pads_and_blocks(a, s_cnt, s_off, 0, 1);
+    return;
+  }
+
+  int32_t* mine = a.tile_counts + static_cast<int64_t>(tile) * a.E_local;
+  for (int e = tid; e < a.E_local; e += blockDim.x) mine[e] = s_cnt[e];
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_is_last = (atomicAdd(a.ticket, 1u) == static_cast<unsigned>(a.num_tiles - 1)) ? 1 : 0;
+  __syncthreads();
+  if (!s_is_last) return;
+  __threadfence();
+
+  // Last CTA: per-expert exclusive scan over tiles.  `parts` threads share one expert, each
+  // scanning a contiguous range of tiles, so all threads work when E_local is small.
+  int parts = 1;
+  while (parts * 2 * a.E_local <= kAlignThreads && parts * 2 <= 32) parts *= 2;
+  const int experts_per_pass = kAlignThreads / parts;
+  const int part = tid % parts;
+  const int per = (a.num_tiles + parts - 1) / parts;
+  const int t0 = part * per;
+  const int t1 = (t0 + per < a.num_tiles) ? t0 + per : a.num_tiles;
+  for (int e0 = 0; e0 < a.E_local; e0 += experts_per_pass) {  // uniform trip count
+    const int e = e0 + tid / parts;
+    int sum = 0;
+    if (e < a.E_local) {
+      for (int t = t0; t < t1; ++t) sum += __ldcg(a.tile_counts + static_cast<int64_t>(t) * a.E_local + e);
+    }
+    // exclusive prefix of the part sums inside each group of `parts` lanes (groups never straddle a warp)
+    int incl = sum;
+    for (int off = 1; off < parts; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off, parts);
+      if (part >= off) incl += v;
+    }
+    if (e < a.E_local) {
+      int run = incl - sum;
+      for (int t = t0; t < t1; ++t) {
+        int32_t* p = a.tile_counts + static_cast<int64_t>(t) * a.E_local + e;
+        const int c = __ldcg(p);
+        *p = run;
+        run += c;
+      }
+      if (part == parts - 1) s_cnt[e] = run;
+    }
+  }
+  __syncthreads();
+  padded_offsets(a, s_cnt, s_off, warp_sums);
+  if (tid == 0) *a.ticket = 0u;  // ready for the next call
+}
+
+__global__ void __launch_bounds__(kAlignThreads) align_place_kernel(AlignArgs a) {
+  extern __shared__ int smem[];
+  int* s_cnt = smem;
+  int* s_off = s_cnt + a.E_local;
+  int* warp_sums = s_off + a.E_local + 1;
+  int* s_whist = warp_sums + 32;
+  int* s_le = s_whist + kAlignWarps * a.E_local;
+  int* s_tile_base = s_le + a.tile_slots;  // [E_local]: first row of this tile's slots per expert
+  const int tile = blockIdx.x;
+  for (int e = threadIdx.x; e <= a.E_local; e += blockDim.x) {
+    s_off[e] = a.offsets[e];
+    if (e < a.E_local) {
+      s_cnt[e] = a.counts[e];
+      s_tile_base[e] = a.offsets[e] + a.tile_counts[static_cast<int64_t>(tile) * a.E_local + e];
+    }
+  }
+  __syncthreads();
+  place_tile(a, tile, s_tile_base, s_whist, s_le);
+  __syncthreads();
+  fill_pads_and_blocks(a, s_cnt, s_off, tile, a.num_tiles);
+}
+
+// Tiling: one tile for up to 4096 slots (single-CTA path); otherwise tiles of 2048 slots,
+// grown up to 8192 so that the last CTA's per-expert scan over tiles stays short.
+int tile_slots_for(int64_t P) {
+  if (P <= 4096) return 4096;
+  int ts = 2048;
+  while ((P + ts - 1) / ts > 256 && ts < 8192) ts *= 2;
+  return ts;
+}
+
+int num_tiles_for(int64_t P, int ts) {
+  const int64_t nt = (P + ts - 1) / ts;
+  return nt < 1 ? 1 : static_cast<int>(nt);
+}
+
+}  // namespace
+
+extern "C" int64_t moe_align_capacity(int64_t T, int32_t k, int32_t E_local, int32_t block_size) {
+  if (T < 0 || k < 1 || E_local < 1 || block_size < 1) return -1;
+  if (T > (int64_t{1} << 40)) return -1;
+  return T * k + static_cast<int64_t>(E_local) * (block_size - 1);
+}
+
+extern "C" int64_t moe_align_num_blocks(int64_t T, int32_t k, int32_t E_local, int32_t block_size) {
+  const int64_t C = moe_align_capacity(T, k, E_local, block_size);
+  if (C < 0) return -1;
+  return (C + block_size - 1) / block_size;
+}
+
+extern "C" size_t moe_align_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
+  if (T < 0 || k < 1 || E_local < 1) return 0;
+  const int64_t P = T * k;
+  const int ts = tile_slots_for(P);
+  const int nt = num_tiles_for(P, ts);
+  const size_t tiles = nt > 1 ? static_cast<size_t>(nt) : 0;
+  return kWsHeaderBytes + tiles * static_cast<size_t>(E_local) * sizeof(int32_t);
+}
+
+extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
+                                          const int32_t* expert_map, int32_t E_local, int32_t block_size,
+                                          int32_t* counts, int32_t* offsets, int32_t* sorted_token_ids,
+                                          int32_t* expert_ids, int32_t* num_tokens_post_pad, int32_t* inv_perm,
+                                          void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || k < 1 || E_global < 1 || E_local < 1 || block_size < 1) return MOE_ERR_INVALID_ARG;
+  if (E_local > E_global) return MOE_ERR_INVALID_ARG;
+  if (expert_map == nullptr && E_local != E_global) return MOE_ERR_INVALID_ARG;
+  if (E_local > 1024) return MOE_ERR_UNSUPPORTED;
+  const int64_t P = T * k;
+  if (T > (int64_t{1} << 40) || P >= (int64_t{1} << 30)) return MOE_ERR_INVALID_ARG;
+  const int64_t C = moe_align_capacity(T, k, E_local, block_size);
+  if (C < 0 || C >= (int64_t{1} << 31)) return MOE_ERR_INVALID_ARG;
+  if (counts == nullptr || offsets == nullptr || sorted_token_ids == nullptr || expert_ids == nullptr ||
+      num_tokens_post_pad == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (P > 0 && (topk_ids == nullptr || inv_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < moe_align_workspace_bytes(T, k, E_local)) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return MOE_ERR_INVALID_ARG;
+
+  AlignArgs a{};
+  a.topk_ids = topk_ids;
+  a.expert_map = expert_map;
+  a.P = P;
+  a.E_global = E_global;
+  a.E_local = E_local;
+  a.bs = block_size;
+  a.C = C;
+  a.NB = static_cast<int>((C + block_size - 1) / block_size);
+  a.tile_slots = tile_slots_for(P);
+  a.num_tiles = num_tiles_for(P, a.tile_slots);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.sorted_ids = sorted_token_ids;
+  a.expert_ids = expert_ids;
+  a.n_pad = num_tokens_post_pad;
+  a.inv_perm = inv_perm;
+  a.status = static_cast<int32_t*>(workspace);
+  a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 4);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kWsHeaderBytes);
+
+  const size_t smem = align_smem_ints(E_local, a.tile_slots) * sizeof(int);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(align_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(align_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  align_count_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (a.num_tiles > 1) {
+    align_place_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}

@@ -1,0 +1,279 @@
+// topk_softmax.cu -- fused softmax + top-k gating over router logits.
+//
+// Operation: "Upstream Reference: Deep-Spark xllm + vllm", "File Index"
+// (moe_topk_softmax_kernels.cuh: fused softmax+topk; vLLM topk_softmax_kernels.cu),
+// placed by "Call Chain: MoE topk_softmax on BI-V100" between the router and the experts.
+//
+// Design (sm_100a): a sub-warp of G lanes (G a power of two, 1..32) owns one row.
+// Each lane loads its share of the row with 16-byte vector loads (8-, 4- or
+// 2-byte, or scalar, when the row length or base pointer does not allow 16),
+// keeps it in registers as 64-bit ordered keys (value bits above, inverted
+// index below), and the k experts are chosen by k rounds of a shuffle-xor max
+// over the G lanes.  Because the key orders by value first and by lower index
+// second, the round's maximum is the largest logit with the lowest index among
+// equals, and the winner is retired by zeroing its key (0 is below every real
+// key, so retired and padding slots can never win while k <= E).  Round 0 also
+// yields the row maximum m, from which the full-row sum Z of exp(x - m) is
+// reduced the same way.  Selected probabilities exp(x_j - m) are staged per
+// warp in shared memory and written out with contiguous stores after the
+// division by Z (or by their own sum when renormalising).
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "common.cuh"
+
+namespace {
+
+constexpr int kMaxWarps = 8;
+
+__device__ __forceinline__ uint32_t ordered_bits(float x) {
+  uint32_t u = __float_as_uint(x);
+  if ((u & 0x7fffffffu) == 0u) u = 0u;  // -0 and +0 compare equal
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float ordered_to_float(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+__device__ __forceinline__ uint64_t make_key(float x, int e) {
+  return (static_cast<uint64_t>(ordered_bits(x)) << 32) | static_cast<uint32_t>(0xffffffffu - static_cast<uint32_t>(e));
+}
+
+// Load VEC consecutive logits of a row as fp32.
+template <typename TIn, int VEC>
+struct VecLoad;
+
+template <>
+struct VecLoad<__nv_bfloat16, 8> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[8]) {
+    uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    v[0] = moe::bf16_lo(u.x); v[1] = moe::bf16_hi(u.x); v[2] = moe::bf16_lo(u.y); v[3] = moe::bf16_hi(u.y);
+    v[4] = moe::bf16_lo(u.z); v[5] = moe::bf16_hi(u.z); v[6] = moe::bf16_lo(u.w); v[7] = moe::bf16_hi(u.w);
+  }
+};
+template <>
+struct VecLoad<__nv_bfloat16, 4> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[4]) {
+    uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
+    v[0] = moe::bf16_lo(u.x); v[1] = moe::bf16_hi(u.x); v[2] = moe::bf16_lo(u.y); v[3] = moe::bf16_hi(u.y);
+  }
+};
+template <>
+struct VecLoad<__nv_bfloat16, 2> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[2]) {
+    uint32_t u = __ldcs(reinterpret_cast<const unsigned int*>(p));
+    v[0] = moe::bf16_lo(u); v[1] = moe::bf16_hi(u);
+  }
+};
+template <>
+struct VecLoad<__nv_bfloat16, 1> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[1]) {
+    uint32_t u = __ldcs(reinterpret_cast<const unsigned short*>(p));
+    v[0] = moe::bf16_lo(u);
+  }
+};
+template <>
+struct VecLoad<float, 4> {
+  static __device__ __forceinline__ void run(const float* p, float (&v)[4]) {
+    float4 u = __ldcs(reinterpret_cast<const float4*>(p));
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+  }
+};
+template <>
+struct VecLoad<float, 2> {
+  static __device__ __forceinline__ void run(const float* p, float (&v)[2]) {
+    float2 u = __ldcs(reinterpret_cast<const float2*>(p));
+    v[0] = u.x; v[1] = u.y;
+  }
+};
+template <>
+struct VecLoad<float, 1> {
+  static __device__ __forceinline__ void run(const float* p, float (&v)[1]) { v[0] = __ldcs(p); }
+};
+
+// One sub-warp of G = 2^g_log2 lanes per row; CPL vector chunks of VEC logits per lane.
+template <typename TIn, int VEC, int CPL>
+__global__ void __launch_bounds__(kMaxWarps * 32)
+topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int g_log2, int renormalize,
+                    float* __restrict__ topk_weights, int32_t* __restrict__ topk_ids) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  constexpr int NV = CPL * VEC;
+  const int G = 1 << g_log2;
+  const int rows_per_warp = 32 >> g_log2;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const int g = lane & (G - 1);
+  const int sub = lane >> g_log2;
+
+  const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp) * rows_per_warp;
+  if (row0 >= T) return;  // uniform per warp
+
+  // per-warp staging: ids, probabilities (rows_per_warp * k each), then one denominator per row
+  const int stage = rows_per_warp * k;
+  int32_t* s_id = reinterpret_cast<int32_t*>(smem_raw) + warp * (2 * stage + rows_per_warp);
+  float* s_p = reinterpret_cast<float*>(s_id + stage);
+  float* s_den = s_p + stage;
+
+  const int64_t row = row0 + sub;
+  const bool row_ok = row < T;
+  const int n_chunks = E / VEC;
+  const TIn* rp = logits + (row_ok ? row : row0) * static_cast<int64_t>(E);
+
+  uint64_t key[NV];
+#pragma unroll
+  for (int c = 0; c < CPL; ++c) {
+    const int chunk = g + c * G;
+    if (row_ok && chunk < n_chunks) {
+      float v[VEC];
+      VecLoad<TIn, VEC>::run(rp + chunk * VEC, v);
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) key[c * VEC + i] = make_key(v[i], chunk * VEC + i);
+    } else {
+#pragma unroll
+      for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0ull;
+    }
+  }
+
+  float m = 0.f, Z = 0.f, S = 0.f;
+  for (int j = 0; j < k; ++j) {
+    uint64_t best = 0ull;
+#pragma unroll
+    for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
+    for (int off = G >> 1; off >= 1; off >>= 1) {
+      const uint64_t o = __shfl_xor_sync(0xffffffffu, best, off);
+      best = o > best ? o : best;
+    }
+    const float xj = ordered_to_float(static_cast<uint32_t>(best >> 32));
+    if (j == 0) {
+      // the first winner is the row maximum; reduce Z = sum over the row of exp(x - m)
+      m = xj;
+      float z = 0.f;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) {
+        if (key[i] != 0ull) z += expf(ordered_to_float(static_cast<uint32_t>(key[i] >> 32)) - m);
+      }
+      for (int off = G >> 1; off >= 1; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+      Z = z;
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
+    const float p = expf(xj - m);
+    S += p;
+    if (g == 0) {
+      s_id[sub * k + j] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(best));
+      s_p[sub * k + j] = p;
+    }
+  }
+  if (g == 0) s_den[sub] = renormalize ? S : Z;
+  __syncwarp();
+
+  const int64_t rows_here = (T - row0) < rows_per_warp ? (T - row0) : rows_per_warp;
+  const int n_out = static_cast<int>(rows_here) * k;
+  float* wdst = topk_weights + row0 * k;
+  int32_t* idst = topk_ids + row0 * k;
+  for (int idx = lane; idx < n_out; idx += 32) {
+    const int r = idx / k;
+    wdst[idx] = s_p[idx] / s_den[r];
+    idst[idx] = s_id[idx];
+  }
+}
+
+using TopkKernel = void (*)(const void*, int64_t, int, int, int, int, float*, int32_t*);
+
+template <typename TIn, int VEC, int CPL>
+TopkKernel instance() {
+  if constexpr (VEC * CPL <= 32) {
+    return reinterpret_cast<TopkKernel>(&topk_softmax_kernel<TIn, VEC, CPL>);
+  } else {
+    return nullptr;
+  }
+}
+
+template <typename TIn, int VEC>
+TopkKernel pick_cpl(int cpl) {
+  switch (cpl) {
+    case 1: return instance<TIn, VEC, 1>();
+    case 2: return instance<TIn, VEC, 2>();
+    case 4: return instance<TIn, VEC, 4>();
+    case 8: return instance<TIn, VEC, 8>();
+    case 16: return instance<TIn, VEC, 16>();
+    case 32: return instance<TIn, VEC, 32>();
+    default: return nullptr;
+  }
+}
+
+template <typename TIn>
+TopkKernel pick_kernel(int vec, int cpl) {
+  if constexpr (sizeof(TIn) == 2) {
+    switch (vec) {
+      case 8: return pick_cpl<TIn, 8>(cpl);
+      case 4: return pick_cpl<TIn, 4>(cpl);
+      case 2: return pick_cpl<TIn, 2>(cpl);
+      default: return pick_cpl<TIn, 1>(cpl);
+    }
+  } else {
+    switch (vec) {
+      case 4: return pick_cpl<TIn, 4>(cpl);
+      case 2: return pick_cpl<TIn, 2>(cpl);
+      default: return pick_cpl<TIn, 1>(cpl);
+    }
+  }
+}
+
+// Launch geometry for one logits layout: vector width, lanes per row, chunks per lane.
+struct TopkGeometry {
+  int vec, g_log2, cpl, warps, smem;
+};
+
+TopkGeometry topk_geometry(int elem_bytes, const void* logits, int E, int k) {
+  TopkGeometry geo{};
+  int vec = 16 / elem_bytes;
+  while (vec > 1 && ((E % vec) != 0 || (reinterpret_cast<uintptr_t>(logits) % (vec * elem_bytes)) != 0)) vec >>= 1;
+  const int n_chunks = E / vec;
+  int G = 1, g_log2 = 0;
+  while (G < n_chunks && G < 32) { G <<= 1; ++g_log2; }
+  int cpl = 1;
+  while (cpl * G < n_chunks) cpl <<= 1;
+  geo.vec = vec;
+  geo.g_log2 = g_log2;
+  geo.cpl = cpl;
+  const int rows_per_warp = 32 >> g_log2;
+  const int per_warp = (2 * rows_per_warp * k + rows_per_warp) * 4;
+  int warps = kMaxWarps;
+  while (warps > 1 && warps * per_warp > 48 * 1024) warps >>= 1;
+  geo.warps = warps;
+  geo.smem = warps * per_warp;
+  return geo;
+}
+
+}  // namespace
+
+extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, int64_t T, int32_t E, int32_t k,
+                                         uint32_t flags, float* topk_weights, int32_t* topk_ids, void* stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~MOE_RENORMALIZE) != 0u) return MOE_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32) return MOE_ERR_UNSUPPORTED;
+  if (T == 0) return MOE_OK;
+  if (logits == nullptr || topk_weights == nullptr || topk_ids == nullptr) return MOE_ERR_INVALID_ARG;
+  if (T > (int64_t{1} << 40)) return MOE_ERR_INVALID_ARG;
+
+  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  const TopkGeometry geo = topk_geometry(elem, logits, E, k);
+  TopkKernel kern = dtype == MOE_DTYPE_BF16 ? pick_kernel<__nv_bfloat16>(geo.vec, geo.cpl)
+                                            : pick_kernel<float>(geo.vec, geo.cpl);
+  if (kern == nullptr) return MOE_ERR_UNSUPPORTED;
+  const int64_t rows_per_cta = static_cast<int64_t>(geo.warps) * (32 >> geo.g_log2);
+  const int64_t grid = (T + rows_per_cta - 1) / rows_per_cta;
+  if (grid > 0x7fffffff) return MOE_ERR_INVALID_ARG;
+  int renorm = (flags & MOE_RENORMALIZE) ? 1 : 0;
+  int g_log2 = geo.g_log2;
+  const void* logits_arg = logits;
+  void* args[] = {&logits_arg, &T, &E, &k, &g_log2, &renorm, &topk_weights, &topk_ids};
+  cudaError_t err = cudaLaunchKernel(reinterpret_cast<const void*>(kern), dim3(static_cast<unsigned>(grid)),
+                                     dim3(geo.warps * 32), args, static_cast<size_t>(geo.smem),
+                                     static_cast<cudaStream_t>(stream));
+  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}

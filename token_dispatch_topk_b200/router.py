@@ -1,0 +1,81 @@
+"""MoeRouter: the routing path for fixed sizes with every buffer preallocated on the device.
+
+One ``step`` runs the four library stages back to back on one stream:
+moe_topk_softmax -> moe_align_permute -> moe_gather -> (caller's experts) -> moe_combine.
+No allocation, host synchronisation or Python-side arithmetic happens inside a step, so
+it can be captured in a CUDA graph.  ``step_from_host`` is the end-to-end form: it copies
+the step's inputs from (pinned) host memory, runs the step and copies the result back.
+"""
+from __future__ import annotations
+
+from typing import Optional
+
+import torch
+
+from . import binding as B
+
+
+class MoeRouter:
+    def __init__(self, T: int, E: int, k: int, H: int, block_size: int, renormalize: bool,
+                 E_local: Optional[int] = None, expert_map: Optional[torch.Tensor] = None,
+                 logits_dtype: torch.dtype = torch.bfloat16, device="cuda"):
+        B.load_library()
+        self.T, self.E, self.k, self.H, self.block_size = T, E, k, H, block_size
+        self.renormalize = renormalize
+        self.E_local = E if E_local is None else E_local
+        self.device = torch.device(device)
+        self.expert_map = None if expert_map is None else expert_map.to(self.device, torch.int32).contiguous()
+        self.logits_dtype = logits_dtype
+        self.topk_weights = torch.empty((T, k), dtype=torch.float32, device=self.device)
+        self.topk_ids = torch.empty((T, k), dtype=torch.int32, device=self.device)
+        self.align = B.alloc_align_outputs(T, k, self.E_local, block_size, self.device)
+        self.capacity = self.align.capacity
+        self.workspace = B.alloc_workspace(T, k, self.E_local, self.device)
+        self.permuted = torch.empty((self.capacity, H), dtype=torch.bfloat16, device=self.device)
+        self.out = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+        # device-side inputs for the end-to-end path
+        self.logits_dev = torch.empty((T, E), dtype=logits_dtype, device=self.device)
+        self.hidden_dev = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
+
+    # ------------------------------------------------------------------ stages --
+    def gate(self, logits: torch.Tensor, stream=None):
+        return B.moe_topk_softmax(logits, self.k, self.renormalize, self.topk_weights, self.topk_ids, stream)
+
+    def align_permute(self, topk_ids: Optional[torch.Tensor] = None, stream=None) -> B.AlignResult:
+        ids = self.topk_ids if topk_ids is None else topk_ids
+        return B.moe_align_permute(ids, self.E, self.block_size, self.expert_map, self.E_local, self.align,
+                                   self.workspace, stream)
+
+    def gather(self, hidden: torch.Tensor, stream=None) -> torch.Tensor:
+        return B.moe_gather(hidden, self.k, self.align.inv_perm, self.capacity, permuted=self.permuted,
+                            device_status=self.workspace, stream=stream)
+
+    def combine(self, expert_out: torch.Tensor, topk_weights: Optional[torch.Tensor] = None,
+                stream=None) -> torch.Tensor:
+        w = self.topk_weights if topk_weights is None else topk_weights
+        return B.moe_combine(expert_out, w, self.align.inv_perm, self.out, device_status=self.workspace,
+                             stream=stream)
+
+    def step(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
+        """gate + align + permute-gather + combine (expert_out stands in for the expert MLPs' output)."""
+        self.gate(logits, stream)
+        self.align_permute(stream=stream)
+        self.gather(hidden, stream)
+        return self.combine(expert_out, stream=stream)
+
+    def step_from_host(self, logits_host: torch.Tensor, hidden_host: torch.Tensor, expert_out: torch.Tensor,
+                       out_host: torch.Tensor, stream=None) -> torch.Tensor:
+        """End to end: H2D copies of the step's inputs, the step, D2H copy of the combined output.
+
+        Host tensors should be pinned for asynchronous copies; the caller synchronises."""
+        s = torch.cuda.current_stream() if stream is None else stream
+        with torch.cuda.stream(s):
+            self.logits_dev.copy_(logits_host, non_blocking=True)
+            self.hidden_dev.copy_(hidden_host, non_blocking=True)
+            out = self.step(self.logits_dev, self.hidden_dev, expert_out, s)
+            out_host.copy_(out, non_blocking=True)
+        return out_host
+
+    def device_status(self, stream=None) -> int:
+        """Read and reset the device status word (synchronises)."""
+        return B.moe_read_status(self.workspace, stream)
