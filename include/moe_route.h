@@ -163,6 +163,33 @@ MOE_API moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32
                                void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * moe_align_permute_noalloc -- moe_align_permute without a workspace argument.  The pages
+ * have no counterpart of this entry point; it exists for callers that cannot allocate device
+ * memory: a host framework whose custom-op interface passes only the op's own inputs and
+ * outputs and does not let the op call cudaMalloc (for example because the call may run while
+ * the stream is being captured, or because another component owns the device memory budget).
+ *   Same arguments, outputs, ordering and errors as moe_align_permute, except:
+ *   - no workspace: the completion ticket and the per-tile expert counters live in a fixed
+ *     1 MiB array inside the library, one per GPU that loads it, held until the process exits;
+ *   - sizes whose scratch would exceed that array (moe_align_workspace_bytes(T, k, E_local)
+ *     > 1 MiB, e.g. E_local = 1024 with more than about 1M slots) return MOE_ERR_UNSUPPORTED
+ *     before anything is enqueued;
+ *   - device_status: a caller device int32 that collects device-side errors, or NULL.
+ *   It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on each
+ *   device looks up the array's device address (cudaGetSymbolAddress) with that device
+ *   current; make that first call before any stream capture.  Each call clears the ticket
+ *   with an asynchronous 4-byte memset on `stream`; the counters are rewritten before they
+ *   are read.  All calls on a device share the one array and it keeps the last call's
+ *   contents, so calls that overlap on the GPU (different streams, concurrent graphs) race
+ *   and give wrong results: serialise them.
+ */
+MOE_API moe_status_t moe_align_permute_noalloc(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
+                                               const int32_t* expert_map, int32_t E_local, int32_t block_size,
+                                               int32_t* counts, int32_t* offsets, int32_t* sorted_token_ids,
+                                               int32_t* expert_ids, int32_t* num_tokens_post_pad,
+                                               int32_t* inv_perm, int32_t* device_status, void* stream);
+
+/*
  * moe_gather -- permute-gather of the activations into the expert-grouped
  * layout ("expand" of the FusedMoE pipeline, "Upstream Reference", "File Index";
  * "final permuted gather" of the compact scheduler note).

@@ -41,6 +41,8 @@ SIGNATURES = {
     "moe_align_workspace_bytes": (_SZ, [_I64, _I32, _I32]),
     "moe_workspace_init": (ctypes.c_int, [_P, _SZ, _P]),
     "moe_align_permute": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_align_permute_noalloc": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P, _P, _P, _P, _P, _P,
+                                                  _P]),
     "moe_gather": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _I64, _U32, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _I64, _P, _P, _P]),
     "moe_read_status": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
@@ -195,6 +197,27 @@ def moe_align_permute(topk_ids: torch.Tensor, E_global: int, block_size: int,
         _dev(out.inv_perm, "inv_perm"), _dev(workspace, "workspace"),
         workspace.numel() * workspace.element_size(), _stream(stream))
     _check(st, "moe_align_permute")
+    return out
+
+
+def moe_align_permute_noalloc(topk_ids: torch.Tensor, E_global: int, block_size: int,
+                              expert_map: Optional[torch.Tensor] = None, E_local: Optional[int] = None,
+                              out: Optional[AlignResult] = None, device_status: Optional[torch.Tensor] = None,
+                              stream=None) -> AlignResult:
+    """moe_align_permute without a workspace: the library's fixed per-device scratch is used instead
+    (for callers that cannot allocate; calls must not overlap on the GPU).  ``out`` may be preallocated."""
+    T, k = topk_ids.shape
+    if E_local is None:
+        E_local = E_global
+    if out is None:
+        out = alloc_align_outputs(T, k, E_local, block_size, topk_ids.device)
+    assert topk_ids.dtype == torch.int32 and (expert_map is None or expert_map.dtype == torch.int32)
+    st = load_library().moe_align_permute_noalloc(
+        _dev(topk_ids, "topk_ids"), T, k, E_global, _dev(expert_map, "expert_map"), E_local, block_size,
+        _dev(out.counts, "counts"), _dev(out.offsets, "offsets"), _dev(out.sorted_token_ids, "sorted_token_ids"),
+        _dev(out.expert_ids, "expert_ids"), _dev(out.num_tokens_post_pad, "num_tokens_post_pad"),
+        _dev(out.inv_perm, "inv_perm"), _dev(device_status, "device_status"), _stream(stream))
+    _check(st, "moe_align_permute_noalloc")
     return out
 
 

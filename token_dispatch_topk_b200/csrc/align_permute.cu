@@ -416,3 +416,104 @@ extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, in
   }
   return MOE_OK;
 }
+
+// ---------------------------------------------------------------------------------------------
+// moe_align_permute_noalloc: the same two align kernels, with their scratch (completion ticket
+// and per-tile expert counters) in a file-scope device array instead of a caller workspace.
+// For callers that cannot allocate device memory at all (see the header).
+// ---------------------------------------------------------------------------------------------
+#include <mutex>
+
+namespace {
+constexpr size_t kNoAllocScratchBytes = size_t{1} << 20;  // 1 MiB per device, held until process exit
+constexpr int kNoAllocMaxDevices = 64;
+}  // namespace
+
+// Host code may not use this name as an address: it is a host-side stand-in.  The device address
+// comes from cudaGetSymbolAddress, fetched once per device below.
+static __device__ __align__(256) unsigned char g_align_noalloc_scratch[kNoAllocScratchBytes];
+
+namespace {
+std::mutex g_noalloc_mutex;
+void* g_noalloc_scratch_addr[kNoAllocMaxDevices] = {};
+
+// Device address of the scratch array on the current device (looked up on first use).
+moe_status_t noalloc_scratch(void** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_align_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_noalloc_scratch_addr[dev] = p;
+  }
+  *out = g_noalloc_scratch_addr[dev];
+  return MOE_OK;
+}
+}  // namespace
+
+extern "C" moe_status_t moe_align_permute_noalloc(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
+                                                  const int32_t* expert_map, int32_t E_local, int32_t block_size,
+                                                  int32_t* counts, int32_t* offsets, int32_t* sorted_token_ids,
+                                                  int32_t* expert_ids, int32_t* num_tokens_post_pad,
+                                                  int32_t* inv_perm, int32_t* device_status, void* stream) {
+  if (T < 0 || k < 1 || E_global < 1 || E_local < 1 || block_size < 1) return MOE_ERR_INVALID_ARG;
+  if (E_local > E_global) return MOE_ERR_INVALID_ARG;
+  if (expert_map == nullptr && E_local != E_global) return MOE_ERR_INVALID_ARG;
+  if (E_local > 1024) return MOE_ERR_UNSUPPORTED;
+  const int64_t P = T * k;
+  if (T > (int64_t{1} << 40) || P >= (int64_t{1} << 30)) return MOE_ERR_INVALID_ARG;
+  const int64_t C = moe_align_capacity(T, k, E_local, block_size);
+  if (C < 0 || C >= (int64_t{1} << 31)) return MOE_ERR_INVALID_ARG;
+  if (counts == nullptr || offsets == nullptr || sorted_token_ids == nullptr || expert_ids == nullptr ||
+      num_tokens_post_pad == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (P > 0 && (topk_ids == nullptr || inv_perm == nullptr)) return MOE_ERR_INVALID_ARG;
+  // the scratch these sizes need must fit the fixed array
+  if (moe_align_workspace_bytes(T, k, E_local) > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
+
+  void* scratch = nullptr;
+  const moe_status_t st_scratch = noalloc_scratch(&scratch);
+  if (st_scratch != MOE_OK) return st_scratch;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // the completion ticket must start at zero whatever an earlier call left behind
+  if (cudaMemsetAsync(static_cast<char*>(scratch) + 4, 0, 4, st) != cudaSuccess) return MOE_ERR_CUDA;
+
+  AlignArgs a{};
+  a.topk_ids = topk_ids;
+  a.expert_map = expert_map;
+  a.P = P;
+  a.E_global = E_global;
+  a.E_local = E_local;
+  a.bs = block_size;
+  a.C = C;
+  a.NB = static_cast<int>((C + block_size - 1) / block_size);
+  a.tile_slots = tile_slots_for(P);
+  a.num_tiles = num_tiles_for(P, a.tile_slots);
+  a.counts = counts;
+  a.offsets = offsets;
+  a.sorted_ids = sorted_token_ids;
+  a.expert_ids = expert_ids;
+  a.n_pad = num_tokens_post_pad;
+  a.inv_perm = inv_perm;
+  a.status = device_status;
+  a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(scratch) + 4);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(scratch) + kWsHeaderBytes);
+
+  const size_t smem = align_smem_ints(E_local, a.tile_slots) * sizeof(int);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(align_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(align_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  align_count_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (a.num_tiles > 1) {
+    align_place_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
