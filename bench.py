@@ -6,7 +6,8 @@
 One step = moe_topk_softmax -> moe_align_permute -> moe_gather -> moe_combine over one batch
 (the stand-in expert outputs replace the expert MLPs between gather and combine), replayed as
 one CUDA graph.  Inputs are resident in HBM; L2 is flushed (a 256 MiB write) between timed
-steps; every step is timed with CUDA events on the launching stream and the K step times are
+steps (then a 256 MiB read, so no dirty flush lines are written back inside a timed step);
+every step is timed with CUDA events on the launching stream and the K step times are
 summed; the result is the max over ranks.  N > 1 runs one independent batch per GPU (weak
 scaling: the path has no cross-token exchange).  Rank 0 prints one JSON line.
 
@@ -268,9 +269,13 @@ def main():
     r = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, E_local=wl.E_local,
                       expert_map=I.expert_map(wl), logits_dtype=logits.dtype, device=dev)
     flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+    flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
 
     def flush(i=0):
+        # write a buffer larger than L2, then read another one: L2 is left holding only clean
+        # lines of a buffer the step never touches, so no flush write-back lands in a timed step
         flush_buf.fill_(i & 0xFF)
+        flush_read.max()
 
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
@@ -404,7 +409,8 @@ def main():
             "dtype_detail": "bf16 activations, fp32 gating math and combine accumulation, int32 indices",
             "data": "synthetic (seeded; see token_dispatch_topk_b200/inputs.py)",
             "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
-                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write)",
+                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write + "
+                             f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)",
                        "cuda_graph": use_graph,
                        "parallelism": "one independent batch per GPU" if ws > 1 else "single GPU"},
             "achieved_hbm_gbs": total_bytes / (ms_per_step * 1e-3) / 1e9,

@@ -23,6 +23,7 @@
 //     the tail rows past N_pad, and expert_ids.
 // When all slots fit one tile (decode, small batches), the count kernel does
 // everything in one CTA and the place kernel is not launched.
+#include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -321,6 +322,145 @@ __global__ void __launch_bounds__(kAlignThreads) align_place_kernel(AlignArgs a)
   fill_pads_and_blocks(a, s_cnt, s_off, tile, a.num_tiles);
 }
 
+// ------------------------------------------------------------------------------------------
+// Single-launch align on one thread-block cluster (up to 16 CTAs on distinct SMs).
+// Global warp g = rank*32 + w owns the contiguous slot run [g*run, (g+1)*run).
+//   1. every warp counts its run into its own shared-memory row (match.any aggregation);
+//   2. per expert, the CTA turns its warp rows into exclusive prefixes and publishes its total;
+//   3. cluster barrier; every CTA reads the totals of all CTAs of the cluster through
+//      distributed shared memory: the sum over lower ranks is its base, the sum over all ranks
+//      is the expert's count; cluster barrier (no CTA leaves while others read its totals);
+//   4. block-padded offsets (each CTA computes them; rank 0 writes counts/offsets/N_pad);
+//   5. every warp walks its run again and places its slots in order;
+//   6. pad rows, tail rows and expert_ids, split over the cluster.
+// No global scratch, no atomics on global memory, no spinning: the cluster barrier is the only
+// inter-CTA synchronisation.
+// ------------------------------------------------------------------------------------------
+constexpr int kClusterThreads = 1024;
+constexpr int kClusterWarps = kClusterThreads / 32;
+constexpr int kMaxClusterCtas = 16;
+
+// Exclusive scan of n <= 1024 ints in shared memory, one per thread of a 1024-thread block.
+__device__ int block_exclusive_scan_1024(int* data, int n, int* warp_sums) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int v = tid < n ? data[tid] : 0;
+  int incl = v;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int x = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += x;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += x;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - v;
+  const int total = warp_sums[31];
+  __syncthreads();
+  if (tid < n) data[tid] = before;
+  __syncthreads();
+  return total;
+}
+
+__global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArgs a, int64_t run) {
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int nc = static_cast<int>(cluster.num_blocks());
+  const int rank = static_cast<int>(cluster.block_rank());
+  const int El = a.E_local;
+  extern __shared__ int smem[];
+  int* whist = smem;                         // [kClusterWarps][El]: per-warp counts, then prefixes
+  int* cta_cnt = whist + kClusterWarps * El;  // [El] this CTA's totals (read by the cluster)
+  int* s_cnt = cta_cnt + El;                 // [El] counts over the whole cluster
+  int* s_off = s_cnt + El;                   // [El+1] block-padded offsets
+  int* s_base = s_off + El + 1;              // [El] first row of this CTA's slots per expert
+  int* warp_sums = s_base + El;              // [32]
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t g = static_cast<int64_t>(rank) * kClusterWarps + warp;
+  const int64_t w0 = g * run;
+  const int64_t w1 = (w0 + run < a.P) ? w0 + run : a.P;
+  int* my_hist = whist + warp * El;
+
+  for (int i = tid; i < kClusterWarps * El; i += kClusterThreads) whist[i] = 0;
+  __syncthreads();
+  // 1. per-warp counts of the warp's own run
+  for (int64_t base = w0; base < w1; base += 32) {
+    const int64_t s = base + lane;
+    const int le = s < w1 ? local_expert(a, s) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  // 2. exclusive prefixes over this CTA's warps; CTA totals
+  for (int e = tid; e < El; e += kClusterThreads) {
+    int run_sum = 0;
+    for (int w = 0; w < kClusterWarps; ++w) {
+      const int c = whist[w * El + e];
+      whist[w * El + e] = run_sum;
+      run_sum += c;
+    }
+    cta_cnt[e] = run_sum;
+  }
+  // 3. exchange totals across the cluster
+  cluster.sync();
+  for (int e = tid; e < El; e += kClusterThreads) {
+    int below = 0, all = 0;
+    for (int r = 0; r < nc; ++r) {
+      const int c = *cluster.map_shared_rank(cta_cnt + e, r);
+      if (r < rank) below += c;
+      all += c;
+    }
+    s_base[e] = below;
+    s_cnt[e] = all;
+  }
+  cluster.sync();
+  // 4. block-padded offsets
+  for (int e = tid; e < El; e += kClusterThreads) s_off[e] = ((s_cnt[e] + a.bs - 1) / a.bs) * a.bs;
+  __syncthreads();
+  const int total = block_exclusive_scan_1024(s_off, El, warp_sums);
+  if (tid == 0) s_off[El] = total;
+  __syncthreads();
+  if (rank == 0) {
+    for (int e = tid; e <= El; e += kClusterThreads) a.offsets[e] = s_off[e];
+    for (int e = tid; e < El; e += kClusterThreads) a.counts[e] = s_cnt[e];
+    if (tid == 0) a.n_pad[0] = total;
+  }
+  for (int e = tid; e < El; e += kClusterThreads) s_base[e] += s_off[e];
+  __syncthreads();
+  // 5. placement in slot order
+  for (int64_t base = w0; base < w1; base += 32) {
+    const int64_t s = base + lane;
+    const int le = s < w1 ? local_expert(a, s) : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    if (le >= 0) {
+      const int row = s_base[le] + my_hist[le] + __popc(peers & moe::lanemask_lt());
+      a.sorted_ids[row] = static_cast<int32_t>(s);
+      a.inv_perm[s] = row;
+    } else if (s < w1) {
+      a.inv_perm[s] = -1;
+    }
+    __syncwarp();
+    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
+    __syncwarp();
+  }
+  // 6. pads, tail, expert_ids
+  fill_pads_and_blocks(a, s_cnt, s_off, rank, nc);
+}
+
+__host__ inline size_t align_cluster_smem_bytes(int E_local) {
+  return (static_cast<size_t>(kClusterWarps) * E_local + 4 * static_cast<size_t>(E_local) + 1 + 32) * sizeof(int);
+}
+
 // Tiling: one tile for up to 4096 slots (single-CTA path); otherwise tiles of 2048 slots,
 // grown up to 8192 so that the last CTA's per-expert scan over tiles stays short.
 int tile_slots_for(int64_t P) {
@@ -333,6 +473,64 @@ int tile_slots_for(int64_t P) {
 int num_tiles_for(int64_t P, int ts) {
   const int64_t nt = (P + ts - 1) / ts;
   return nt < 1 ? 1 : static_cast<int>(nt);
+}
+
+}  // namespace
+
+namespace {
+
+// CTAs in the align cluster: one for small batches, else 8 (portable) or 16 when the device
+// can co-schedule a 16-CTA cluster of this kernel.
+int align_cluster_ctas(int64_t P, size_t smem) {
+  if (P <= 4096) return 1;
+  if (P <= 16384) return 8;
+  if (cudaFuncSetAttribute(align_cluster_kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return 8;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kMaxClusterCtas);
+  cfg.blockDim = dim3(kClusterThreads);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kMaxClusterCtas;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int clusters = 0;
+  if (cudaOccupancyMaxActiveClusters(&clusters, align_cluster_kernel, &cfg) != cudaSuccess || clusters < 1) {
+    (void)cudaGetLastError();
+    return 8;
+  }
+  return kMaxClusterCtas;
+}
+
+moe_status_t launch_align_cluster(const AlignArgs& a, cudaStream_t st) {
+  const size_t smem = align_cluster_smem_bytes(a.E_local);
+  if (cudaFuncSetAttribute(align_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int nc = align_cluster_ctas(a.P, smem);
+  const int64_t warps = static_cast<int64_t>(nc) * kClusterWarps;
+  int64_t run = (a.P + warps - 1) / warps;
+  run = (run + 31) & ~int64_t{31};
+  if (run < 32) run = 32;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(nc);
+  cfg.blockDim = dim3(kClusterThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = nc;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  AlignArgs args = a;
+  return cudaLaunchKernelEx(&cfg, align_cluster_kernel, args, run) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
@@ -399,22 +597,7 @@ extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, in
   a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 4);
   a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kWsHeaderBytes);
 
-  const size_t smem = align_smem_ints(E_local, a.tile_slots) * sizeof(int);
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (smem > 48 * 1024) {
-    if (cudaFuncSetAttribute(align_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess ||
-        cudaFuncSetAttribute(align_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-  }
-  align_count_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
-  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-  if (a.num_tiles > 1) {
-    align_place_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
-  }
-  return MOE_OK;
+  return launch_align_cluster(a, static_cast<cudaStream_t>(stream));
 }
 
 // ---------------------------------------------------------------------------------------------

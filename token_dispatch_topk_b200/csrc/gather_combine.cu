@@ -6,15 +6,16 @@
 // weighted sum back to token order; moe_align_sum_kernels.cu names the "sum"), and
 // the "final permuted gather" of the 2026-07-16 MTP1 M=2 compact scheduler closure note.
 //
-// Both kernels are token-major and bandwidth-bound: one warp owns one token (or one
-// segment of a long row when there are too few tokens to fill the GPU).  Lane j < k
-// holds the row inv_perm[t*k+j] of the token's j-th slot (and its weight) and hands
-// it to the warp by shuffle, so the per-slot indices are read once per warp.
-//   gather:  each hidden row is read once (16-byte loads, U vectors in flight per
-//            lane) and stored to every local destination row.
-//   combine: for each 16-byte column chunk, up to 8 slot rows are loaded before the
-//            fp32 fused multiply-adds run in ascending j from +0, then one bf16
-//            round-to-nearest-even store.
+// Both stages are token-major and bandwidth-bound.  The main kernels move rows with TMA
+// bulk copies (cp.async.bulk, no multicast) through shared memory:
+//   gather_tma_kernel:  each hidden row is bulk-loaded once and bulk-stored to every
+//                       local destination row of its token.
+//   combine_tma_kernel: a producer warp bulk-loads the local slot rows of each (token,
+//                       column chunk) into a 3-stage ring; consumer warps run the fp32
+//                       fused multiply-adds in ascending slot order from +0 and store one
+//                       bf16 round-to-nearest-even result.
+// The register-staged gather_kernel (one warp per token or row segment, lane j < k holding
+// the row of slot j) covers rows too long to stage; zero_pad_kernel fills pad rows on request.
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -85,59 +86,232 @@ zero_pad_kernel(const int32_t* __restrict__ sorted_ids, const int32_t* __restric
   for (int v = lane; v < NV; v += 32) moe::st_plain(dst + v, z);
 }
 
-__global__ void __launch_bounds__(kWarpsPerCta * 32)
-combine_kernel(const uint4* __restrict__ expert_out, const float* __restrict__ topk_weights,
-               const int32_t* __restrict__ inv_perm, int64_t T, int NV, int k, int seg, int seg_len, int64_t capacity,
-               uint4* __restrict__ out, int32_t* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
-  const int64_t t = gw / seg;
-  if (t >= T) return;  // uniform per warp
-  const int sg = static_cast<int>(gw - t * seg);
-  const int v0 = sg * seg_len;
-  const int v1 = (v0 + seg_len < NV) ? v0 + seg_len : NV;
-  const int myrow = lane_row(inv_perm, t, k, capacity, lane, status);
-  const float myw = lane < k ? topk_weights[t * k + lane] : 0.f;
-  uint4* dst = out + t * NV;
+// ------------------------------------------------------------------------------------------
+// TMA kernels.  Rows move as whole bulk copies through shared memory: the copy engine keeps
+// many kilobytes in flight per SM without holding registers, which register-staged copies
+// cannot (occupancy-limited, one dependent load/store phase per iteration).
+// ------------------------------------------------------------------------------------------
+constexpr int kGatherMaxTokensPerCta = 8;
+constexpr uint32_t kGatherCtaBytes = 32u * 1024u;  // hidden rows staged per CTA
 
-  for (int vb = v0; vb < v1; vb += 32) {
-    const int v = vb + lane;
-    const bool ok = v < v1;
-    float acc[8];
+// One warp per CTA: lane 0 bulk-loads the CTA's `tokens_per_cta` hidden rows into shared memory
+// while the lanes read the rows' destinations; then every lane bulk-stores the staged rows of its
+// slots to their expert-grouped rows.
+__global__ void __launch_bounds__(32)
+gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_bytes, int k, int tokens_per_cta,
+                  const int32_t* __restrict__ inv_perm, int64_t capacity, uint8_t* __restrict__ permuted,
+                  int32_t* status) {
+  extern __shared__ __align__(128) uint8_t rows[];
+  __shared__ __align__(8) uint64_t bar;
+  const int lane = threadIdx.x;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * tokens_per_cta;
+  const int n = static_cast<int>((T - t0) < tokens_per_cta ? (T - t0) : tokens_per_cta);
+  if (lane == 0) {
+    moe::mbar_init(&bar, 1);
+    moe::fence_barrier_init();
+  }
+  __syncwarp();
+  if (lane == 0) {
+    moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
+    for (int i = 0; i < n; ++i) {
+      moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes, hidden + (t0 + i) * static_cast<int64_t>(row_bytes),
+                     row_bytes, &bar);
+    }
+  }
+  const int nslots = n * k;  // <= 8 * 32
+  int32_t dst[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    for (int j0 = 0; j0 < k; j0 += 8) {
-      uint4 yv[8];
-      int rr[8];
-#pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        rr[jj] = __shfl_sync(0xffffffffu, myrow, (j0 + jj) & 31);  // lanes >= k hold -1
-        yv[jj] = make_uint4(0u, 0u, 0u, 0u);
-        if (j0 + jj < k && rr[jj] >= 0 && ok) yv[jj] = moe::ld_stream(expert_out + static_cast<int64_t>(rr[jj]) * NV + v);
+  for (int m = 0; m < 8; ++m) {
+    const int e = lane + 32 * m;
+    int r = -1;
+    if (e < nslots) {
+      r = inv_perm[t0 * k + e];
+      if (r < -1 || static_cast<int64_t>(r) >= capacity) {
+        moe::record_status(status, MOE_ERR_BAD_ROW);
+        r = -1;
       }
+    }
+    dst[m] = r;
+  }
+  if (!moe::mbar_wait(&bar, 0)) {
+    moe::record_status(status, MOE_ERR_TIMEOUT);
+    moe::mbar_wait(&bar, 0);  // give the loads in flight one more bounded wait before leaving
+    return;
+  }
 #pragma unroll
-      for (int jj = 0; jj < 8; ++jj) {
-        const float w = __shfl_sync(0xffffffffu, myw, (j0 + jj) & 31);
-        if (j0 + jj < k && rr[jj] >= 0) {
-          acc[0] = fmaf(w, moe::bf16_lo(yv[jj].x), acc[0]);
-          acc[1] = fmaf(w, moe::bf16_hi(yv[jj].x), acc[1]);
-          acc[2] = fmaf(w, moe::bf16_lo(yv[jj].y), acc[2]);
-          acc[3] = fmaf(w, moe::bf16_hi(yv[jj].y), acc[3]);
-          acc[4] = fmaf(w, moe::bf16_lo(yv[jj].z), acc[4]);
-          acc[5] = fmaf(w, moe::bf16_hi(yv[jj].z), acc[5]);
-          acc[6] = fmaf(w, moe::bf16_lo(yv[jj].w), acc[6]);
-          acc[7] = fmaf(w, moe::bf16_hi(yv[jj].w), acc[7]);
+  for (int m = 0; m < 8; ++m) {
+    const int e = lane + 32 * m;
+    if (e < nslots && dst[m] >= 0) {
+      moe::bulk_store(permuted + static_cast<int64_t>(dst[m]) * row_bytes, rows + static_cast<size_t>(e / k) * row_bytes,
+                      row_bytes);
+    }
+  }
+  moe::bulk_commit();
+  moe::bulk_wait_read_all();  // the staged rows must outlive the stores that read them
+}
+
+constexpr int kCombineConsumerWarps = 8;
+constexpr int kCombineStages = 3;
+
+struct CombineArgs {
+  const uint8_t* y;        // expert_out [capacity, H] bf16
+  const float* w;          // [T, k]
+  const int32_t* inv_perm; // [T*k]
+  int64_t T;
+  int k;
+  uint32_t row_bytes;      // H * 2
+  uint32_t chunk_bytes;    // bytes of one row chunk (a unit covers one chunk of one token)
+  int nchunks;
+  int64_t units;           // T * nchunks
+  int64_t capacity;
+  uint8_t* out;            // [T, H] bf16
+  int32_t* status;
+};
+
+// Persistent, warp-specialised: warp 0 produces, warps 1..8 consume.  A unit is one column chunk
+// of one token.  The producer bulk-loads the chunk of each local slot row into a stage of a
+// 3-deep shared-memory ring (mbarrier `full`), with the slot weights and a validity mask beside
+// it; the consumers accumulate in fp32 (packed f32x2 fused multiply-adds: two independent
+// correctly rounded fmas, ascending slot order, from +0), store the bf16 result and release the
+// stage (mbarrier `empty`, one arrival per consumer warp).
+__global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_kernel(CombineArgs a) {
+  constexpr int S = kCombineStages;
+  extern __shared__ __align__(128) uint8_t smem[];
+  const int k = a.k;
+  const uint32_t stage_bytes = static_cast<uint32_t>(k) * a.chunk_bytes;
+  uint8_t* buf = smem;
+  uint64_t* s_w2 = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);  // [S][k] packed {w, w}
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_w2 + S * k);         // [S]
+  uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_mask + S) + 7) & ~uintptr_t(7));
+  uint64_t* empty = full + S;
+  __shared__ int s_abort;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int64_t per = (a.units + gridDim.x - 1) / gridDim.x;
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * per;
+  const int64_t u1 = (u0 + per < a.units) ? u0 + per : a.units;
+  if (tid == 0) {
+    for (int s = 0; s < S; ++s) {
+      moe::mbar_init(&full[s], 1);
+      moe::mbar_init(&empty[s], kCombineConsumerWarps);
+    }
+    s_abort = 0;
+    moe::fence_barrier_init();
+  }
+  __syncthreads();
+  if (u0 >= u1) return;
+
+  if (warp == 0) {
+    // ---- producer
+    int64_t cur_t = u0 / a.nchunks;
+    auto load_meta = [&](int64_t t, int& r, float& w) {
+      r = -1;
+      w = 0.f;
+      if (t < a.T && lane < k) {
+        r = a.inv_perm[t * k + lane];
+        w = a.w[t * k + lane];
+        if (r < -1 || static_cast<int64_t>(r) >= a.capacity) {
+          moe::record_status(a.status, MOE_ERR_BAD_ROW);
+          r = -1;
         }
       }
+    };
+    int r_cur, r_next;
+    float w_cur, w_next;
+    load_meta(cur_t, r_cur, w_cur);
+    load_meta(cur_t + 1, r_next, w_next);
+    int64_t issued = 0;
+    for (int64_t u = u0; u < u1; ++u, ++issued) {
+      const int64_t t = u / a.nchunks;
+      const int c = static_cast<int>(u - t * a.nchunks);
+      if (t != cur_t) {  // advance one token (units are in token order) and prefetch the next
+        cur_t = t;
+        r_cur = r_next;
+        w_cur = w_next;
+        load_meta(t + 1, r_next, w_next);
+      }
+      const int s = static_cast<int>(issued % S);
+      const uint32_t n = static_cast<uint32_t>(issued / S);
+      if (n > 0 && !moe::mbar_wait(&empty[s], (n - 1) & 1u)) {
+        moe::record_status(a.status, MOE_ERR_TIMEOUT);
+        s_abort = 1;
+        break;
+      }
+      const uint32_t mask = __ballot_sync(0xffffffffu, lane < k && r_cur >= 0);
+      const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
+      if (lane < k) s_w2[s * k + lane] = moe::f32x2(w_cur, w_cur);
+      if (lane == 0) s_mask[s] = mask;
+      __threadfence_block();
+      __syncwarp();
+      if (lane == 0) moe::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(mask)) * cb);
+      __syncwarp();
+      if (lane < k && r_cur >= 0) {
+        moe::bulk_load(buf + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * a.chunk_bytes,
+                       a.y + static_cast<int64_t>(r_cur) * a.row_bytes + static_cast<int64_t>(c) * a.chunk_bytes, cb,
+                       &full[s]);
+      }
     }
-    if (ok) {
+    if (s_abort && lane == 0) {
+      // never leave with loads in flight into this CTA's shared memory: fills older than the
+      // last S were consumed before their stage was refilled, so wait (bounded) for those S
+      for (int64_t q = issued > S ? issued - S : 0; q < issued; ++q) {
+        moe::mbar_wait(&full[q % S], static_cast<uint32_t>(q / S) & 1u);
+      }
+    }
+    return;
+  }
+
+  // ---- consumers
+  const int ct = tid - 32;
+  constexpr int NCT = kCombineConsumerWarps * 32;
+  int64_t done = 0;
+  for (int64_t u = u0; u < u1; ++u, ++done) {
+    const int s = static_cast<int>(done % S);
+    const uint32_t n = static_cast<uint32_t>(done / S);
+    if (!moe::mbar_wait(&full[s], n & 1u)) {
+      moe::record_status(a.status, MOE_ERR_TIMEOUT);
+      s_abort = 1;
+      break;
+    }
+    const int64_t t = u / a.nchunks;
+    const int c = static_cast<int>(u - t * a.nchunks);
+    const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
+    const uint32_t mask = s_mask[s];
+    const uint8_t* stage = buf + static_cast<size_t>(s) * stage_bytes;
+    uint8_t* dst = a.out + t * static_cast<int64_t>(a.row_bytes) + static_cast<int64_t>(c) * a.chunk_bytes;
+    const int nvec = static_cast<int>(cb >> 4);
+    const uint64_t* w2 = s_w2 + s * k;
+    for (int v = ct; v < nvec; v += NCT) {
+      uint64_t acc01 = 0ull, acc23 = 0ull, acc45 = 0ull, acc67 = 0ull;  // +0.0f pairs
+      const uint8_t* col = stage + static_cast<size_t>(v) * 16;
+      for (int j0 = 0; j0 < k; j0 += 8) {
+#pragma unroll
+        for (int jj = 0; jj < 8; ++jj) {
+          const int j = j0 + jj;
+          if (j < k && ((mask >> j) & 1u)) {  // ascending j, as the reference order requires
+            const uint4 yv = moe::lds128(col + static_cast<size_t>(j) * a.chunk_bytes);
+            const uint64_t ww = moe::lds64(w2 + j);
+            acc01 = moe::fma_bf16x2(ww, yv.x, acc01);
+            acc23 = moe::fma_bf16x2(ww, yv.y, acc23);
+            acc45 = moe::fma_bf16x2(ww, yv.z, acc45);
+            acc67 = moe::fma_bf16x2(ww, yv.w, acc67);
+          }
+        }
+      }
+      float r[8];
+      moe::f32x2_split(acc01, r[0], r[1]);
+      moe::f32x2_split(acc23, r[2], r[3]);
+      moe::f32x2_split(acc45, r[4], r[5]);
+      moe::f32x2_split(acc67, r[6], r[7]);
       uint4 o;
-      o.x = moe::pack_bf16x2(acc[0], acc[1]);
-      o.y = moe::pack_bf16x2(acc[2], acc[3]);
-      o.z = moe::pack_bf16x2(acc[4], acc[5]);
-      o.w = moe::pack_bf16x2(acc[6], acc[7]);
-      moe::st_plain(dst + v, o);
+      o.x = moe::pack_bf16x2(r[0], r[1]);
+      o.y = moe::pack_bf16x2(r[2], r[3]);
+      o.z = moe::pack_bf16x2(r[4], r[5]);
+      o.w = moe::pack_bf16x2(r[6], r[7]);
+      moe::st_plain(reinterpret_cast<uint4*>(dst + static_cast<size_t>(v) * 16), o);
     }
+    __syncwarp();
+    if (lane == 0) moe::mbar_arrive(&empty[s]);
   }
 }
 
@@ -175,7 +349,23 @@ extern "C" moe_status_t moe_gather(const void* hidden, int64_t T, int32_t H, int
     return MOE_ERR_INVALID_ARG;
   const int NV = H / 8;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (T > 0) {
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+  if (T > 0 && row_bytes <= kGatherCtaBytes * 4u) {
+    int tpc = static_cast<int>(kGatherCtaBytes / row_bytes);
+    if (tpc < 1) tpc = 1;
+    if (tpc > kGatherMaxTokensPerCta) tpc = kGatherMaxTokensPerCta;
+    const int64_t blocks = (T + tpc - 1) / tpc;
+    const size_t smem = static_cast<size_t>(tpc) * row_bytes;
+    if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(gather_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+            cudaSuccess)
+      return MOE_ERR_CUDA;
+    gather_tma_kernel<<<static_cast<unsigned>(blocks), 32, smem, st>>>(
+        static_cast<const uint8_t*>(hidden), T, row_bytes, k, tpc, inv_perm, capacity, static_cast<uint8_t*>(permuted),
+        device_status);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  } else if (T > 0) {  // rows beyond 128 KB: register-staged copy
     int seg, seg_len;
     segment_rows(T, NV, &seg, &seg_len);
     const int64_t warps = T * seg;
@@ -208,14 +398,35 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   if (topk_weights == nullptr || inv_perm == nullptr || out == nullptr) return MOE_ERR_INVALID_ARG;
   if (capacity > 0 && expert_out == nullptr) return MOE_ERR_INVALID_ARG;
   if ((expert_out && !moe_host::aligned16(expert_out)) || !moe_host::aligned16(out)) return MOE_ERR_INVALID_ARG;
-  const int NV = H / 8;
-  int seg, seg_len;
-  segment_rows(T, NV, &seg, &seg_len);
-  const int64_t warps = T * seg;
-  const int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
-  if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
-  combine_kernel<<<static_cast<unsigned>(blocks), kWarpsPerCta * 32, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<const uint4*>(expert_out), topk_weights, inv_perm, T, NV, k, seg, seg_len, capacity,
-      static_cast<uint4*>(out), device_status);
+  CombineArgs a{};
+  a.y = static_cast<const uint8_t*>(expert_out);
+  a.w = topk_weights;
+  a.inv_perm = inv_perm;
+  a.T = T;
+  a.k = k;
+  a.row_bytes = static_cast<uint32_t>(H) * 2u;
+  // one stage holds k row chunks: at most 32 KB
+  const uint32_t chunk_cap = k <= 8 ? 4096u : (k <= 16 ? 2048u : 1024u);
+  a.chunk_bytes = a.row_bytes < chunk_cap ? a.row_bytes : chunk_cap;
+  a.nchunks = static_cast<int>((a.row_bytes + a.chunk_bytes - 1) / a.chunk_bytes);
+  a.units = T * a.nchunks;
+  a.capacity = capacity;
+  a.out = static_cast<uint8_t*>(out);
+  a.status = device_status;
+  const size_t smem = static_cast<size_t>(kCombineStages) * k * a.chunk_bytes +
+                      static_cast<size_t>(kCombineStages) * k * sizeof(uint64_t) + kCombineStages * sizeof(uint32_t) +
+                      8 + 2 * kCombineStages * sizeof(uint64_t);
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  const int per_sm = smem <= 48 * 1024 ? 4 : 2;
+  const int64_t grid = a.units < static_cast<int64_t>(sms) * per_sm ? a.units : static_cast<int64_t>(sms) * per_sm;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(combine_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  combine_tma_kernel<<<static_cast<unsigned>(grid), (1 + kCombineConsumerWarps) * 32, smem,
+                       static_cast<cudaStream_t>(stream)>>>(a);
   return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }

@@ -4,7 +4,10 @@
 // (moe_topk_softmax_kernels.cuh: fused softmax+topk; vLLM topk_softmax_kernels.cu),
 // placed by "Call Chain: MoE topk_softmax on BI-V100" between the router and the experts.
 //
-// Design (sm_100a): a sub-warp of G lanes (G a power of two, 1..32) owns one row.
+// Design (sm_100a).  Rows of E >= 16 experts: one warp per row (topk_row_warp_kernel below),
+// one warp-wide redux.sync max per selection round.  Short rows (E < 16): the sub-warp kernel
+// described here.
+// Sub-warp kernel: a sub-warp of G lanes (G a power of two, 1..32) owns one row.
 // Each lane loads its share of the row with 16-byte vector loads (8-, 4- or
 // 2-byte, or scalar, when the row length or base pointer does not allow 16),
 // keeps it in registers as 64-bit ordered keys (value bits above, inverted
@@ -180,6 +183,166 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// One warp per row (E >= 16).  Lane l holds chunks l, l+32, ... of VEC logits.  bf16 logits fit
+// a 32-bit key (ordered 16-bit value above, 0xFFFF - index below), so each round is a single
+// warp-wide redux max; fp32 logits use the 64-bit key, reduced as its high word, then the low
+// word among the lanes holding that high word.  Lane j keeps round j's expert and probability.
+// ------------------------------------------------------------------------------------------
+constexpr int kRowWarps = 4;
+
+__device__ __forceinline__ uint32_t ordered16(uint32_t b) {
+  b &= 0xffffu;
+  if ((b & 0x7fffu) == 0u) b = 0u;  // -0 == +0
+  return (b & 0x8000u) ? (~b & 0xffffu) : (b | 0x8000u);
+}
+
+__device__ __forceinline__ float ordered16_to_float(uint32_t o) {
+  const uint32_t b = (o & 0x8000u) ? (o & 0x7fffu) : (~o & 0xffffu);
+  return __uint_as_float(b << 16);
+}
+
+// Raw 16-bit patterns of VEC consecutive bf16 logits.
+template <int VEC>
+struct Bf16Bits;
+template <>
+struct Bf16Bits<8> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[8]) {
+    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
+    b[0] = u.x & 0xffffu; b[1] = u.x >> 16; b[2] = u.y & 0xffffu; b[3] = u.y >> 16;
+    b[4] = u.z & 0xffffu; b[5] = u.z >> 16; b[6] = u.w & 0xffffu; b[7] = u.w >> 16;
+  }
+};
+template <>
+struct Bf16Bits<4> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[4]) {
+    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
+    b[0] = u.x & 0xffffu; b[1] = u.x >> 16; b[2] = u.y & 0xffffu; b[3] = u.y >> 16;
+  }
+};
+template <>
+struct Bf16Bits<2> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[2]) {
+    const uint32_t u = __ldcs(reinterpret_cast<const unsigned int*>(p));
+    b[0] = u & 0xffffu; b[1] = u >> 16;
+  }
+};
+template <>
+struct Bf16Bits<1> {
+  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[1]) {
+    b[0] = __ldcs(reinterpret_cast<const unsigned short*>(p));
+  }
+};
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+template <typename TIn, int VEC, int CPL>
+__global__ void __launch_bounds__(kRowWarps * 32)
+topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int g_log2_unused, int renormalize,
+                     float* __restrict__ topk_weights, int32_t* __restrict__ topk_ids) {
+  (void)g_log2_unused;
+  constexpr int NV = CPL * VEC;
+  const int lane = threadIdx.x & 31;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
+  if (row >= T) return;  // uniform per warp
+  const int n_chunks = E / VEC;
+  const TIn* rp = logits + row * static_cast<int64_t>(E);
+  float m = 0.f, Z = 0.f, S = 0.f, my_p = 0.f;
+  int my_e = 0;
+
+  if constexpr (sizeof(TIn) == 2) {
+    uint32_t key[NV];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int chunk = lane + 32 * c;
+      if (chunk < n_chunks) {
+        uint32_t b[VEC];
+        Bf16Bits<VEC>::run(rp + chunk * VEC, b);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = (ordered16(b[i]) << 16) | (0xffffu - static_cast<uint32_t>(chunk * VEC + i));
+      } else {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0u;
+      }
+    }
+    for (int j = 0; j < k; ++j) {
+      uint32_t best = 0u;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
+      best = __reduce_max_sync(0xffffffffu, best);
+      const float xj = ordered16_to_float(best >> 16);
+      if (j == 0) {
+        m = xj;
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          if (key[i] != 0u) z += expf(ordered16_to_float(key[i] >> 16) - m);
+        }
+        Z = warp_sum(z);
+      }
+#pragma unroll
+      for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0u : key[i];
+      const float p = expf(xj - m);
+      S += p;
+      if (lane == j) {
+        my_e = static_cast<int>(0xffffu - (best & 0xffffu));
+        my_p = p;
+      }
+    }
+  } else {
+    uint64_t key[NV];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) {
+      const int chunk = lane + 32 * c;
+      if (chunk < n_chunks) {
+        float v[VEC];
+        VecLoad<TIn, VEC>::run(rp + chunk * VEC, v);
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = make_key(v[i], chunk * VEC + i);
+      } else {
+#pragma unroll
+        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0ull;
+      }
+    }
+    for (int j = 0; j < k; ++j) {
+      uint64_t mine = 0ull;
+#pragma unroll
+      for (int i = 0; i < NV; ++i) mine = key[i] > mine ? key[i] : mine;
+      const uint32_t hi = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32));
+      const uint32_t lo = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32) == hi
+                                                             ? static_cast<uint32_t>(mine) : 0u);
+      const uint64_t best = (static_cast<uint64_t>(hi) << 32) | lo;
+      const float xj = ordered_to_float(hi);
+      if (j == 0) {
+        m = xj;
+        float z = 0.f;
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+          if (key[i] != 0ull) z += expf(ordered_to_float(static_cast<uint32_t>(key[i] >> 32)) - m);
+        }
+        Z = warp_sum(z);
+      }
+#pragma unroll
+      for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
+      const float p = expf(xj - m);
+      S += p;
+      if (lane == j) {
+        my_e = static_cast<int>(0xffffffffu - lo);
+        my_p = p;
+      }
+    }
+  }
+  if (lane < k) {
+    const float den = renormalize ? S : Z;
+    topk_weights[row * k + lane] = my_p / den;
+    topk_ids[row * k + lane] = my_e;
+  }
+}
+
 using TopkKernel = void (*)(const void*, int64_t, int, int, int, int, float*, int32_t*);
 
 template <typename TIn, int VEC, int CPL>
@@ -201,6 +364,46 @@ TopkKernel pick_cpl(int cpl) {
     case 16: return instance<TIn, VEC, 16>();
     case 32: return instance<TIn, VEC, 32>();
     default: return nullptr;
+  }
+}
+
+template <typename TIn, int VEC, int CPL>
+TopkKernel row_instance() {
+  if constexpr (VEC * CPL <= 32) {
+    return reinterpret_cast<TopkKernel>(&topk_row_warp_kernel<TIn, VEC, CPL>);
+  } else {
+    return nullptr;
+  }
+}
+
+template <typename TIn, int VEC>
+TopkKernel pick_row_cpl(int cpl) {
+  switch (cpl) {
+    case 1: return row_instance<TIn, VEC, 1>();
+    case 2: return row_instance<TIn, VEC, 2>();
+    case 4: return row_instance<TIn, VEC, 4>();
+    case 8: return row_instance<TIn, VEC, 8>();
+    case 16: return row_instance<TIn, VEC, 16>();
+    case 32: return row_instance<TIn, VEC, 32>();
+    default: return nullptr;
+  }
+}
+
+template <typename TIn>
+TopkKernel pick_row_kernel(int vec, int cpl) {
+  if constexpr (sizeof(TIn) == 2) {
+    switch (vec) {
+      case 8: return pick_row_cpl<TIn, 8>(cpl);
+      case 4: return pick_row_cpl<TIn, 4>(cpl);
+      case 2: return pick_row_cpl<TIn, 2>(cpl);
+      default: return pick_row_cpl<TIn, 1>(cpl);
+    }
+  } else {
+    switch (vec) {
+      case 4: return pick_row_cpl<TIn, 4>(cpl);
+      case 2: return pick_row_cpl<TIn, 2>(cpl);
+      default: return pick_row_cpl<TIn, 1>(cpl);
+    }
   }
 }
 
@@ -261,6 +464,30 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
   if (T > (int64_t{1} << 40)) return MOE_ERR_INVALID_ARG;
 
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  int renorm_flag = (flags & MOE_RENORMALIZE) ? 1 : 0;
+  if (E >= 16) {
+    // one warp per row: the widest aligned vector that still spreads the row over all 32 lanes
+    int vec_max = 16 / elem;
+    while (vec_max > 1 && ((E % vec_max) != 0 || (reinterpret_cast<uintptr_t>(logits) % (vec_max * elem)) != 0))
+      vec_max >>= 1;
+    int vec = 1;
+    for (int v = vec_max; v >= 1; v >>= 1) {
+      if ((E % v) == 0 && E / v >= 32) { vec = v; break; }
+    }
+    const int n_chunks = E / vec;
+    int cpl = 1;
+    while (cpl * 32 < n_chunks) cpl <<= 1;
+    TopkKernel rk = dtype == MOE_DTYPE_BF16 ? pick_row_kernel<__nv_bfloat16>(vec, cpl) : pick_row_kernel<float>(vec, cpl);
+    if (rk == nullptr) return MOE_ERR_UNSUPPORTED;
+    const int64_t grid = (T + kRowWarps - 1) / kRowWarps;
+    if (grid > 0x7fffffff) return MOE_ERR_INVALID_ARG;
+    int unused = 0;
+    const void* logits_arg = logits;
+    void* args[] = {&logits_arg, &T, &E, &k, &unused, &renorm_flag, &topk_weights, &topk_ids};
+    cudaError_t err = cudaLaunchKernel(reinterpret_cast<const void*>(rk), dim3(static_cast<unsigned>(grid)),
+                                       dim3(kRowWarps * 32), args, 0, static_cast<cudaStream_t>(stream));
+    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  }
   const TopkGeometry geo = topk_geometry(elem, logits, E, k);
   TopkKernel kern = dtype == MOE_DTYPE_BF16 ? pick_kernel<__nv_bfloat16>(geo.vec, geo.cpl)
                                             : pick_kernel<float>(geo.vec, geo.cpl);
@@ -268,10 +495,9 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
   const int64_t rows_per_cta = static_cast<int64_t>(geo.warps) * (32 >> geo.g_log2);
   const int64_t grid = (T + rows_per_cta - 1) / rows_per_cta;
   if (grid > 0x7fffffff) return MOE_ERR_INVALID_ARG;
-  int renorm = (flags & MOE_RENORMALIZE) ? 1 : 0;
   int g_log2 = geo.g_log2;
   const void* logits_arg = logits;
-  void* args[] = {&logits_arg, &T, &E, &k, &g_log2, &renorm, &topk_weights, &topk_ids};
+  void* args[] = {&logits_arg, &T, &E, &k, &g_log2, &renorm_flag, &topk_weights, &topk_ids};
   cudaError_t err = cudaLaunchKernel(reinterpret_cast<const void*>(kern), dim3(static_cast<unsigned>(grid)),
                                      dim3(geo.warps * 32), args, static_cast<size_t>(geo.smem),
                                      static_cast<cudaStream_t>(stream));
