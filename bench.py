@@ -57,7 +57,8 @@ def parse_args():
     p.add_argument("--workload", default=None, help="workload name (default: the Qwen3-MoE-like prefill)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-graph", action="store_true", help="launch the four calls directly instead of a graph")
-    p.add_argument("--stage-steps", type=int, default=None, help="timed iterations per stage (default: steps)")
+    p.add_argument("--stage-steps", type=int, default=None,
+                   help="instrumented steps for the per-stage breakdown (default: min(steps, 500))")
     p.add_argument("--e2e-steps", type=int, default=None, help="timed end-to-end steps (default: min(steps, 200))")
     p.add_argument("--cpu-seconds", type=float, default=10.0, help="CPU-oracle baseline budget (rank 0, N=1)")
     p.add_argument("--no-cpu-baseline", action="store_true")
@@ -300,13 +301,7 @@ def main():
                 fn()
             return g
         graphs["step"] = capture(lambda: r.step(logits, hidden, y))
-        graphs["topk"] = capture(lambda: r.gate(logits))
-        graphs["align"] = capture(lambda: r.align_permute())
-        graphs["gather"] = capture(lambda: r.gather(hidden))
-        graphs["combine"] = capture(lambda: r.combine(y))
-    stage_fns = {"step": lambda: r.step(logits, hidden, y), "topk": lambda: r.gate(logits),
-                 "align": lambda: r.align_permute(), "gather": lambda: r.gather(hidden),
-                 "combine": lambda: r.combine(y)}
+    stage_fns = {"step": lambda: r.step(logits, hidden, y)}
 
     def run(name):
         if use_graph:
@@ -353,15 +348,44 @@ def main():
     ms_per_step = total_ms / args.steps
     value = ws * wl.T * args.steps / (total_ms / 1e3)
 
-    # ---- per-stage times (same flush protocol) and roofline
+    # ---- per-stage times inside the step, and roofline
+    # The step is captured once more with external event records between its stages, so each
+    # stage is timed on the launching stream exactly as it runs inside a step (same flush protocol).
     peak, peak_src = measured_peaks()
     abytes = algorithmic_bytes(wl, R, r.capacity, NB)
-    st_iters = args.stage_steps or args.steps
+    st_iters = args.stage_steps or min(args.steps, 500)
+    names = ("topk", "align", "gather", "combine")
+    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
+    stage_calls = [lambda: r.gate(logits), lambda: r.align_permute(), lambda: r.gather(hidden), lambda: r.combine(y)]
+
+    def instrumented_step():
+        marks[0].record()
+        for i, fn in enumerate(stage_calls):
+            fn()
+            marks[i + 1].record()
+
+    if use_graph:
+        g_inst = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_inst, stream=stream):
+            instrumented_step()
+    sums = [0.0] * len(names)
+    with torch.cuda.stream(stream):
+        for i in range(min(args.warmup, 10) + st_iters):
+            flush(i)
+            if use_graph:
+                g_inst.replay()
+            else:
+                instrumented_step()
+            stream.synchronize()
+            if i >= min(args.warmup, 10):
+                for j in range(len(names)):
+                    sums[j] += marks[j].elapsed_time(marks[j + 1])
     stages = {}
-    for name in ("topk", "align", "gather", "combine"):
-        ms = timed(name, st_iters, min(args.warmup, 10)) / st_iters
+    for j, name in enumerate(names):
+        ms = sums[j] / st_iters
         stages[name] = {"us": 1e3 * ms, "algorithmic_bytes": abytes[name],
-                        "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": STAGE_KERNEL[name]}
+                        "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": STAGE_KERNEL[name],
+                        "timing": "CUDA events between the stages of the step graph"}
     dom = max(("gather", "combine"), key=lambda s: stages[s]["us"])
     ach = stages[dom]["achieved_gbs"]
     total_bytes = sum(abytes.values())
@@ -423,6 +447,8 @@ def main():
         }
         print(json.dumps(line), flush=True)
     del graphs
+    if use_graph:
+        del g_inst
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -23,6 +23,11 @@
  *     0 and 8 in the all-duplicate case) and coverage paragraph (a valid
  *     all-remote expert-parallel rank; bitwise-exact checks).
  *
+ * Kernel launches use programmatic dependent launch: each kernel lets the next kernel in the
+ * stream be scheduled early and waits (griddepcontrol.wait) for the previous one before reading
+ * its outputs.  A caller kernel launched right after one of these with programmatic stream
+ * serialisation must likewise wait before reading their outputs; ordinary launches need nothing.
+ *
  * Conventions shared by every entry point
  *   Notation: T tokens, E (= E_global) experts, E_local experts on this rank,
  *   k experts per token, H hidden size, bs block size.  Slot s = t*k + j is the
@@ -77,6 +82,9 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 /* flags */
 #define MOE_RENORMALIZE 1u     /* moe_topk_softmax: renormalise the k weights to sum to 1 */
 #define MOE_GATHER_ZERO_PAD 2u /* moe_gather: write +0 into the pad rows below N_pad */
+#define MOE_GATHER_HIDDEN_READY 4u /* moe_gather: `hidden` was complete before the previous kernel in
+                                      the stream was launched, so it may be read before waiting for
+                                      that kernel (true when hidden is an input of the routing step) */
 
 /* Human-readable name of a status code (static string, never NULL). */
 MOE_API const char* moe_status_string(moe_status_t status);

@@ -29,6 +29,7 @@ MOE_DTYPE_F32 = 0
 MOE_DTYPE_BF16 = 1
 MOE_RENORMALIZE = 1
 MOE_GATHER_ZERO_PAD = 2
+MOE_GATHER_HIDDEN_READY = 4
 
 # Every symbol include/moe_route.h declares, with (restype, argtypes).
 _P, _I32, _I64, _U32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t
@@ -224,8 +225,11 @@ def moe_align_permute_noalloc(topk_ids: torch.Tensor, E_global: int, block_size:
 def moe_gather(hidden: torch.Tensor, k: int, inv_perm: torch.Tensor, capacity: int,
                sorted_token_ids: Optional[torch.Tensor] = None, num_tokens_post_pad: Optional[torch.Tensor] = None,
                zero_pad: bool = False, permuted: Optional[torch.Tensor] = None,
-               device_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
-    """hidden [T, H] bf16 -> permuted [capacity, H] bf16 (expert-grouped rows)."""
+               device_status: Optional[torch.Tensor] = None, stream=None, hidden_ready: bool = False) -> torch.Tensor:
+    """hidden [T, H] bf16 -> permuted [capacity, H] bf16 (expert-grouped rows).
+
+    hidden_ready: hidden was complete before the previous kernel in the stream was launched
+    (MOE_GATHER_HIDDEN_READY), so the kernel may start loading it before that kernel finishes."""
     T, H = hidden.shape
     assert hidden.dtype == torch.bfloat16
     if permuted is None:
@@ -233,7 +237,8 @@ def moe_gather(hidden: torch.Tensor, k: int, inv_perm: torch.Tensor, capacity: i
     st = load_library().moe_gather(_dev(hidden, "hidden"), T, H, k, _dev(inv_perm, "inv_perm"),
                                    _dev(sorted_token_ids, "sorted_token_ids"),
                                    _dev(num_tokens_post_pad, "num_tokens_post_pad"), capacity,
-                                   MOE_GATHER_ZERO_PAD if zero_pad else 0, _dev(permuted, "permuted"),
+                                   (MOE_GATHER_ZERO_PAD if zero_pad else 0) |
+                                   (MOE_GATHER_HIDDEN_READY if hidden_ready else 0), _dev(permuted, "permuted"),
                                    _dev(device_status, "device_status"), _stream(stream))
     _check(st, "moe_gather")
     return permuted

@@ -72,6 +72,20 @@ __device__ __forceinline__ int local_expert(const AlignArgs& a, int64_t s) {
   return le;
 }
 
+// Lanes of this warp that hold the same value v >= 0, as a bit mask (0 for v < 0).  Uses a
+// per-warp array of masks in shared memory, indexed by value, that is all zero on entry and is
+// left all zero: one atomic OR, one read and one reset per lane, whatever the number of distinct
+// values (match.any costs grow with it).
+__device__ __forceinline__ unsigned peers_smem(unsigned* masks, int v, int lane) {
+  if (v >= 0) atomicOr(&masks[v], 1u << lane);
+  __syncwarp();
+  const unsigned p = v >= 0 ? masks[v] : 0u;
+  __syncwarp();
+  if (v >= 0) masks[v] = 0u;
+  __syncwarp();
+  return p;
+}
+
 // Block-wide exclusive scan of n <= 2*kAlignThreads ints in shared memory (in place).
 // Returns the total.  Every thread of the block must call it.
 __device__ int block_exclusive_scan(int* data, int n, int* warp_sums) {
@@ -164,8 +178,10 @@ __device__ void fill_pads_and_blocks(const AlignArgs& a, const int* s_cnt, const
 }
 
 // Stable placement of one tile.  s_base[e] = first row of this tile's slots of expert e.
-// s_whist: [kAlignWarps][E_local] scratch, s_le: [tile_slots] scratch.
-__device__ void place_tile(const AlignArgs& a, int tile, const int* s_base, int* s_whist, int* s_le) {
+// s_whist: [kAlignWarps][E_local] scratch, s_le: [tile_slots] scratch, s_masks:
+// [kAlignWarps][E_local] all-zero masks (left all zero).
+__device__ void place_tile(const AlignArgs& a, int tile, const int* s_base, int* s_whist, int* s_le,
+                           unsigned* s_masks) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t s0 = static_cast<int64_t>(tile) * a.tile_slots;
   const int64_t s1 = (s0 + a.tile_slots < a.P) ? s0 + a.tile_slots : a.P;
@@ -173,17 +189,15 @@ __device__ void place_tile(const AlignArgs& a, int tile, const int* s_base, int*
   const int64_t w0 = s0 + static_cast<int64_t>(warp) * per_warp;
   const int64_t w1 = (w0 + per_warp < s1) ? w0 + per_warp : s1;
   int* my_hist = s_whist + warp * a.E_local;
+  unsigned* my_masks = s_masks + warp * a.E_local;
 
   for (int i = tid; i < kAlignWarps * a.E_local; i += blockDim.x) s_whist[i] = 0;
   __syncthreads();
-  // pass 1: per-warp histogram of its own run (one adding lane per group of equal experts)
-  for (int64_t base = w0; base < w1; base += 32) {
-    const int64_t s = base + lane;
-    const int le = s < w1 ? local_expert(a, s) : -1;
-    if (s < w1) s_le[s - s0] = le;
-    const unsigned peers = __match_any_sync(0xffffffffu, le);
-    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
-    __syncwarp();
+  // pass 1: per-warp histogram of its own run
+  for (int64_t s = w0 + lane; s < w1; s += 32) {
+    const int le = local_expert(a, s);
+    s_le[s - s0] = le;
+    if (le >= 0) atomicAdd(&my_hist[le], 1);
   }
   __syncthreads();
   // pass 2: exclusive scan over warps, seeded with the tile's base row
@@ -200,7 +214,7 @@ __device__ void place_tile(const AlignArgs& a, int tile, const int* s_base, int*
   for (int64_t base = w0; base < w1; base += 32) {
     const int64_t s = base + lane;
     const int le = s < w1 ? s_le[s - s0] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    const unsigned peers = peers_smem(my_masks, le, lane);
     if (le >= 0) {
       const int row = my_hist[le] + __popc(peers & moe::lanemask_lt());
       a.sorted_ids[row] = static_cast<int32_t>(s);
@@ -216,10 +230,10 @@ __device__ void place_tile(const AlignArgs& a, int tile, const int* s_base, int*
 
 // Shared-memory layout of both kernels (ints):
 //   s_cnt[E_local] | s_off[E_local+1] | warp_sums[32] | s_whist[kAlignWarps*E_local] | s_le[tile_slots]
-//   | s_tile_base[E_local] (place kernel)
+//   | s_tile_base[E_local] (place kernel) | s_masks[kAlignWarps*E_local]
 __host__ __device__ inline size_t align_smem_ints(int E_local, int tile_slots) {
   return static_cast<size_t>(E_local) + (E_local + 1) + 32 + static_cast<size_t>(kAlignWarps) * E_local +
-         tile_slots + E_local;
+         tile_slots + E_local + static_cast<size_t>(kAlignWarps) * E_local;
 }
 
 __global__ void __launch_bounds__(kAlignThreads) align_count_kernel(AlignArgs a) {
@@ -229,27 +243,27 @@ __global__ void __launch_bounds__(kAlignThreads) align_count_kernel(AlignArgs a)
   int* warp_sums = s_off + a.E_local + 1;
   int* s_whist = warp_sums + 32;
   int* s_le = s_whist + kAlignWarps * a.E_local;
+  unsigned* s_masks = reinterpret_cast<unsigned*>(s_le + a.tile_slots + a.E_local);
   __shared__ int s_is_last;
 
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int64_t s0 = static_cast<int64_t>(tile) * a.tile_slots;
   const int64_t s1 = (s0 + a.tile_slots < a.P) ? s0 + a.tile_slots : a.P;
 
   for (int e = tid; e < a.E_local; e += blockDim.x) s_cnt[e] = 0;
+  for (int i = tid; i < kAlignWarps * a.E_local; i += blockDim.x) s_masks[i] = 0u;
   __syncthreads();
-  for (int64_t base = s0 + static_cast<int64_t>(warp) * 32; base < s1; base += kAlignThreads) {
-    const int64_t s = base + lane;
-    const int le = s < s1 ? local_expert(a, s) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, le);
-    if (le >= 0 && lane == __ffs(peers) - 1) atomicAdd(&s_cnt[le], __popc(peers));
+  for (int64_t s = s0 + tid; s < s1; s += kAlignThreads) {
+    const int le = local_expert(a, s);
+    if (le >= 0) atomicAdd(&s_cnt[le], 1);
   }
   __syncthreads();
 
   if (a.num_tiles == 1) {
     // everything in this CTA
     padded_offsets(a, s_cnt, s_off, warp_sums);
-    place_tile(a, 0, s_off, s_whist, s_le);
+    place_tile(a, 0, s_off, s_whist, s_le, s_masks);
     fill_pads_and_blocks(a, s_cnt, s_off, 0, 1);
     return;
   }
@@ -308,7 +322,9 @@ __global__ void __launch_bounds__(kAlignThreads) align_place_kernel(AlignArgs a)
   int* s_whist = warp_sums + 32;
   int* s_le = s_whist + kAlignWarps * a.E_local;
   int* s_tile_base = s_le + a.tile_slots;  // [E_local]: first row of this tile's slots per expert
+  unsigned* s_masks = reinterpret_cast<unsigned*>(s_tile_base + a.E_local);
   const int tile = blockIdx.x;
+  for (int i = threadIdx.x; i < kAlignWarps * a.E_local; i += blockDim.x) s_masks[i] = 0u;
   for (int e = threadIdx.x; e <= a.E_local; e += blockDim.x) {
     s_off[e] = a.offsets[e];
     if (e < a.E_local) {
@@ -317,28 +333,34 @@ __global__ void __launch_bounds__(kAlignThreads) align_place_kernel(AlignArgs a)
     }
   }
   __syncthreads();
-  place_tile(a, tile, s_tile_base, s_whist, s_le);
+  place_tile(a, tile, s_tile_base, s_whist, s_le, s_masks);
   __syncthreads();
   fill_pads_and_blocks(a, s_cnt, s_off, tile, a.num_tiles);
 }
 
 // ------------------------------------------------------------------------------------------
-// Single-launch align on one thread-block cluster (up to 16 CTAs on distinct SMs).
-// Global warp g = rank*32 + w owns the contiguous slot run [g*run, (g+1)*run).
-//   1. every warp counts its run into its own shared-memory row (match.any aggregation);
-//   2. per expert, the CTA turns its warp rows into exclusive prefixes and publishes its total;
-//   3. cluster barrier; every CTA reads the totals of all CTAs of the cluster through
-//      distributed shared memory: the sum over lower ranks is its base, the sum over all ranks
-//      is the expert's count; cluster barrier (no CTA leaves while others read its totals);
+// Single-launch align on one thread-block cluster (up to 16 CTAs on distinct SMs), used up to
+// 65536 slots with at most 512 local experts (larger batches take the two tile kernels above,
+// which spread over every SM).  Global warp g = rank*32 + w owns the slot run [g*run, (g+1)*run).
+//   1. every warp counts its run into its own shared-memory row (shared atomics; the ids of up
+//      to 8 chunks are loaded at once and their experts kept for step 5);
+//   2. per expert, the CTA turns its warp rows into exclusive prefixes and writes its total to
+//      row `rank` of a table in the workspace;
+//   3. cluster barrier (release/acquire at cluster scope); each CTA scans the table: the sum
+//      over lower ranks is its base, the sum over all ranks is the expert's count;
 //   4. block-padded offsets (each CTA computes them; rank 0 writes counts/offsets/N_pad);
-//   5. every warp walks its run again and places its slots in order;
+//   5. every warp walks its run again and places its slots in order (peer masks from shared
+//      memory, rank = earlier peers in the chunk);
 //   6. pad rows, tail rows and expert_ids, split over the cluster.
-// No global scratch, no atomics on global memory, no spinning: the cluster barrier is the only
+// Steps 2 and 3 are warp shuffle scans: lane = warp index (32 warps) or lane = CTA rank; four
+// experts are scanned at once to overlap the shuffle latencies.  The cluster barrier is the only
 // inter-CTA synchronisation.
 // ------------------------------------------------------------------------------------------
 constexpr int kClusterThreads = 1024;
 constexpr int kClusterWarps = kClusterThreads / 32;
 constexpr int kMaxClusterCtas = 16;
+constexpr int64_t kClusterMaxSlots = 65536;
+constexpr int kClusterMaxExperts = 512;
 
 // Exclusive scan of n <= 1024 ints in shared memory, one per thread of a 1024-thread block.
 __device__ int block_exclusive_scan_1024(int* data, int n, int* warp_sums) {
@@ -370,60 +392,143 @@ __device__ int block_exclusive_scan_1024(int* data, int n, int* warp_sums) {
   return total;
 }
 
+// Row stride of the per-warp counters and of the cluster table: odd, so that 32 lanes reading one
+// expert column of 32 rows hit 32 different banks.
+__host__ __device__ inline int warp_row_stride(int E_local) { return E_local | 1; }
+
+constexpr int kAlignBatch = 8;  // 32-slot chunks whose ids a warp loads at once
+
+// Local experts of one batch of a warp's run: slot base + 32*b + lane for b < kAlignBatch.  All
+// id loads (then all map loads) are issued before any is used.
+__device__ __forceinline__ void load_batch(const AlignArgs& a, int64_t base, int64_t end, int lane,
+                                           int (&le)[kAlignBatch]) {
+  int g[kAlignBatch];
+#pragma unroll
+  for (int b = 0; b < kAlignBatch; ++b) {
+    const int64_t s = base + 32 * b + lane;
+    g[b] = s < end ? a.topk_ids[s] : -2;
+  }
+#pragma unroll
+  for (int b = 0; b < kAlignBatch; ++b) {
+    int v = -1;
+    if (g[b] != -2) {
+      if (static_cast<unsigned>(g[b]) >= static_cast<unsigned>(a.E_global)) {
+        moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+      } else {
+        v = a.expert_map != nullptr ? a.expert_map[g[b]] : g[b];
+        if (v < -1 || v >= a.E_local) {
+          moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+          v = -1;
+        }
+      }
+    }
+    le[b] = v;
+  }
+}
+
 __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArgs a, int64_t run) {
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int nc = static_cast<int>(cluster.num_blocks());
   const int rank = static_cast<int>(cluster.block_rank());
   const int El = a.E_local;
+  const int ES = warp_row_stride(El);
   extern __shared__ int smem[];
-  int* whist = smem;                         // [kClusterWarps][El]: per-warp counts, then prefixes
-  int* cta_cnt = whist + kClusterWarps * El;  // [El] this CTA's totals (read by the cluster)
-  int* s_cnt = cta_cnt + El;                 // [El] counts over the whole cluster
-  int* s_off = s_cnt + El;                   // [El+1] block-padded offsets
-  int* s_base = s_off + El + 1;              // [El] first row of this CTA's slots per expert
-  int* warp_sums = s_base + El;              // [32]
+  int* whist = smem;                                                          // [32][ES] counts, then prefixes
+  unsigned* masks = reinterpret_cast<unsigned*>(whist + kClusterWarps * ES);  // [32][El] peer masks
+  int* s_cnt = reinterpret_cast<int*>(masks + kClusterWarps * El);            // [El] cluster counts
+  int* s_off = s_cnt + El;                                                    // [El+1] padded offsets
+  int* s_base = s_off + El + 1;                                               // [El] this CTA's first rows
+  int* warp_sums = s_base + El;                                               // [32]
+  int32_t* gtable = a.tile_counts;  // [nc][El] in the workspace: every CTA's totals
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t g = static_cast<int64_t>(rank) * kClusterWarps + warp;
   const int64_t w0 = g * run;
   const int64_t w1 = (w0 + run < a.P) ? w0 + run : a.P;
-  int* my_hist = whist + warp * El;
+  int* my_hist = whist + warp * ES;
+  unsigned* my_masks = masks + warp * El;
+  const bool one_batch = run <= 32 * kAlignBatch;  // the whole run's experts stay in registers
 
-  for (int i = tid; i < kClusterWarps * El; i += kClusterThreads) whist[i] = 0;
+  for (int i = tid; i < kClusterWarps * ES; i += kClusterThreads) whist[i] = 0;
+  for (int i = tid; i < kClusterWarps * El; i += kClusterThreads) masks[i] = 0u;
   __syncthreads();
+  moe::pdl_wait();  // topk_ids come from the previous kernel
+  moe::pdl_launch_dependents();
   // 1. per-warp counts of the warp's own run
-  for (int64_t base = w0; base < w1; base += 32) {
-    const int64_t s = base + lane;
-    const int le = s < w1 ? local_expert(a, s) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, le);
-    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
-    __syncwarp();
+  int le[kAlignBatch];
+  for (int64_t base = w0; base < w1; base += 32 * kAlignBatch) {
+    load_batch(a, base, w1, lane, le);
+#pragma unroll
+    for (int b = 0; b < kAlignBatch; ++b) {
+      if (le[b] >= 0) atomicAdd(&my_hist[le[b]], 1);
+    }
   }
   __syncthreads();
-  // 2. exclusive prefixes over this CTA's warps; CTA totals
-  for (int e = tid; e < El; e += kClusterThreads) {
-    int run_sum = 0;
-    for (int w = 0; w < kClusterWarps; ++w) {
-      const int c = whist[w * El + e];
-      whist[w * El + e] = run_sum;
-      run_sum += c;
+  // 2. per expert, exclusive prefix over this CTA's 32 warps (lane = warp index); the CTA total
+  //    goes to row `rank` of the cluster table
+  for (int e0 = warp; e0 < El; e0 += 4 * kClusterWarps) {
+    int c[4], incl[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = e0 + q * kClusterWarps;
+      c[q] = e < El ? whist[lane * ES + e] : 0;
+      incl[q] = c[q];
     }
-    cta_cnt[e] = run_sum;
-  }
-  // 3. exchange totals across the cluster
-  cluster.sync();
-  for (int e = tid; e < El; e += kClusterThreads) {
-    int below = 0, all = 0;
-    for (int r = 0; r < nc; ++r) {
-      const int c = *cluster.map_shared_rank(cta_cnt + e, r);
-      if (r < rank) below += c;
-      all += c;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int x = __shfl_up_sync(0xffffffffu, incl[q], off);
+        if (lane >= off) incl[q] += x;
+      }
     }
-    s_base[e] = below;
-    s_cnt[e] = all;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = e0 + q * kClusterWarps;
+      if (e < El) {
+        whist[lane * ES + e] = incl[q] - c[q];
+        if (lane == 31 && nc > 1) gtable[static_cast<int64_t>(rank) * El + e] = incl[q];
+        if (nc == 1 && lane == 31) {
+          s_base[e] = 0;
+          s_cnt[e] = incl[q];
+        }
+      }
+    }
   }
-  cluster.sync();
+  // 3. after the cluster barrier (release/acquire at cluster scope), each CTA scans the table:
+  //    lane = rank; the sum over lower ranks is its base, the sum over all ranks the count
+  if (nc > 1) {
+    cluster.sync();
+    for (int e0 = warp; e0 < El; e0 += 4 * kClusterWarps) {
+      int c[4], incl[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = e0 + q * kClusterWarps;
+        c[q] = (e < El && lane < nc) ? __ldcg(gtable + static_cast<int64_t>(lane) * El + e) : 0;
+        incl[q] = c[q];
+      }
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int x = __shfl_up_sync(0xffffffffu, incl[q], off);
+          if (lane >= off) incl[q] += x;
+        }
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int e = e0 + q * kClusterWarps;
+        const int all = __shfl_sync(0xffffffffu, incl[q], 31);
+        const int below = __shfl_sync(0xffffffffu, incl[q] - c[q], rank);
+        if (lane == 0 && e < El) {
+          s_base[e] = below;
+          s_cnt[e] = all;
+        }
+      }
+    }
+  }
+  __syncthreads();
   // 4. block-padded offsets
   for (int e = tid; e < El; e += kClusterThreads) s_off[e] = ((s_cnt[e] + a.bs - 1) / a.bs) * a.bs;
   __syncthreads();
@@ -438,27 +543,53 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
   for (int e = tid; e < El; e += kClusterThreads) s_base[e] += s_off[e];
   __syncthreads();
   // 5. placement in slot order
-  for (int64_t base = w0; base < w1; base += 32) {
-    const int64_t s = base + lane;
-    const int le = s < w1 ? local_expert(a, s) : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, le);
-    if (le >= 0) {
-      const int row = s_base[le] + my_hist[le] + __popc(peers & moe::lanemask_lt());
-      a.sorted_ids[row] = static_cast<int32_t>(s);
-      a.inv_perm[s] = row;
-    } else if (s < w1) {
-      a.inv_perm[s] = -1;
+  for (int64_t base = w0; base < w1; base += 32 * kAlignBatch) {
+    if (!one_batch) load_batch(a, base, w1, lane, le);
+#pragma unroll
+    for (int b = 0; b < kAlignBatch; ++b) {
+      const int64_t s = base + 32 * b + lane;
+      const unsigned peers = peers_smem(my_masks, le[b], lane);
+      if (le[b] >= 0) {
+        const int row = s_base[le[b]] + my_hist[le[b]] + __popc(peers & moe::lanemask_lt());
+        a.sorted_ids[row] = static_cast<int32_t>(s);
+        a.inv_perm[s] = row;
+      } else if (s < w1) {
+        a.inv_perm[s] = -1;
+      }
+      __syncwarp();
+      if (le[b] >= 0 && lane == __ffs(peers) - 1) my_hist[le[b]] += __popc(peers);
+      __syncwarp();
     }
-    __syncwarp();
-    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
-    __syncwarp();
   }
-  // 6. pads, tail, expert_ids
-  fill_pads_and_blocks(a, s_cnt, s_off, rank, nc);
+  // 6. pad rows (one warp per expert: fewer than bs rows each), tail rows, expert_ids
+  const int32_t pad_value = static_cast<int32_t>(a.P);
+  for (int e = rank * kClusterWarps + warp; e < El; e += nc * kClusterWarps) {
+    const int p1 = s_off[e + 1];
+    for (int p = s_off[e] + s_cnt[e] + lane; p < p1; p += 32) a.sorted_ids[p] = pad_value;
+  }
+  const uint32_t tail = static_cast<uint32_t>(a.C - total);
+  for (uint32_t i = static_cast<uint32_t>(rank) * kClusterThreads + tid; i < tail;
+       i += static_cast<uint32_t>(nc) * kClusterThreads)
+    a.sorted_ids[total + i] = pad_value;
+  for (int b = rank * kClusterThreads + tid; b < a.NB; b += nc * kClusterThreads) {
+    const int64_t row = static_cast<int64_t>(b) * a.bs;
+    int e = -1;
+    if (row < total) {
+      int lo = 0, hi = El - 1;  // largest e with s_off[e] <= row (empty experts share offsets)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    a.expert_ids[b] = e;
+  }
 }
 
 __host__ inline size_t align_cluster_smem_bytes(int E_local) {
-  return (static_cast<size_t>(kClusterWarps) * E_local + 4 * static_cast<size_t>(E_local) + 1 + 32) * sizeof(int);
+  return (static_cast<size_t>(kClusterWarps) * warp_row_stride(E_local) + static_cast<size_t>(kClusterWarps) * E_local +
+          3 * static_cast<size_t>(E_local) + 1 + 32) *
+         sizeof(int);
 }
 
 // Tiling: one tile for up to 4096 slots (single-CTA path); otherwise tiles of 2048 slots,
@@ -522,13 +653,15 @@ moe_status_t launch_align_cluster(const AlignArgs& a, cudaStream_t st) {
   cfg.blockDim = dim3(kClusterThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = nc;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   AlignArgs args = a;
   return cudaLaunchKernelEx(&cfg, align_cluster_kernel, args, run) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
@@ -552,8 +685,9 @@ extern "C" size_t moe_align_workspace_bytes(int64_t T, int32_t k, int32_t E_loca
   const int64_t P = T * k;
   const int ts = tile_slots_for(P);
   const int nt = num_tiles_for(P, ts);
-  const size_t tiles = nt > 1 ? static_cast<size_t>(nt) : 0;
-  return kWsHeaderBytes + tiles * static_cast<size_t>(E_local) * sizeof(int32_t);
+  size_t rows = nt > 1 ? static_cast<size_t>(nt) : 0;  // per-tile counters of the tile kernels
+  if (P > 4096 && rows < static_cast<size_t>(kMaxClusterCtas)) rows = kMaxClusterCtas;  // cluster table
+  return kWsHeaderBytes + rows * static_cast<size_t>(E_local) * sizeof(int32_t);
 }
 
 extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
@@ -597,7 +731,24 @@ extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, in
   a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 4);
   a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kWsHeaderBytes);
 
-  return launch_align_cluster(a, static_cast<cudaStream_t>(stream));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (P <= kClusterMaxSlots && E_local <= kClusterMaxExperts) return launch_align_cluster(a, st);
+  // large batches or many local experts: count + place tile kernels over every SM
+  const size_t smem = align_smem_ints(E_local, a.tile_slots) * sizeof(int);
+  if (smem > 48 * 1024) {
+    if (cudaFuncSetAttribute(align_count_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaFuncSetAttribute(align_place_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  align_count_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
+  if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  if (a.num_tiles > 1) {
+    align_place_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
 }
 
 // ---------------------------------------------------------------------------------------------

@@ -43,6 +43,7 @@ __device__ __forceinline__ int lane_row(const int32_t* inv_perm, int64_t t, int 
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 gather_kernel(const uint4* __restrict__ hidden, int64_t T, int NV, int k, int seg, int seg_len,
               const int32_t* __restrict__ inv_perm, int64_t capacity, uint4* __restrict__ permuted, int32_t* status) {
+  moe::pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t gw = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
   const int64_t t = gw / seg;
@@ -77,6 +78,7 @@ gather_kernel(const uint4* __restrict__ hidden, int64_t T, int NV, int k, int se
 __global__ void __launch_bounds__(kWarpsPerCta * 32)
 zero_pad_kernel(const int32_t* __restrict__ sorted_ids, const int32_t* __restrict__ n_pad, int64_t capacity, int NV,
                 int32_t pad_value, uint4* __restrict__ permuted) {
+  moe::pdl_wait();
   const int lane = threadIdx.x & 31;
   const int64_t p = static_cast<int64_t>(blockIdx.x) * kWarpsPerCta + (threadIdx.x >> 5);
   if (p >= capacity || p >= static_cast<int64_t>(n_pad[0])) return;
@@ -100,7 +102,7 @@ constexpr uint32_t kGatherCtaBytes = 32u * 1024u;  // hidden rows staged per CTA
 __global__ void __launch_bounds__(32)
 gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_bytes, int k, int tokens_per_cta,
                   const int32_t* __restrict__ inv_perm, int64_t capacity, uint8_t* __restrict__ permuted,
-                  int32_t* status) {
+                  int32_t* status, int hidden_ready) {
   extern __shared__ __align__(128) uint8_t rows[];
   __shared__ __align__(8) uint64_t bar;
   const int lane = threadIdx.x;
@@ -111,13 +113,19 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
     moe::fence_barrier_init();
   }
   __syncwarp();
-  if (lane == 0) {
-    moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
-    for (int i = 0; i < n; ++i) {
-      moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes, hidden + (t0 + i) * static_cast<int64_t>(row_bytes),
-                     row_bytes, &bar);
+  auto load_rows = [&]() {
+    if (lane == 0) {
+      moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
+      for (int i = 0; i < n; ++i) {
+        moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes,
+                       hidden + (t0 + i) * static_cast<int64_t>(row_bytes), row_bytes, &bar);
+      }
     }
-  }
+  };
+  if (hidden_ready) load_rows();  // hidden predates the previous kernel: load it while that kernel finishes
+  moe::pdl_launch_dependents();
+  moe::pdl_wait();                 // inv_perm comes from the previous kernel
+  if (!hidden_ready) load_rows();
   const int nslots = n * k;  // <= 8 * 32
   int32_t dst[8];
 #pragma unroll
@@ -199,6 +207,8 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
     moe::fence_barrier_init();
   }
   __syncthreads();
+  moe::pdl_launch_dependents();
+  moe::pdl_wait();  // slot rows, weights and expert outputs come from earlier kernels
   if (u0 >= u1) return;
 
   if (warp == 0) {
@@ -338,7 +348,7 @@ extern "C" moe_status_t moe_gather(const void* hidden, int64_t T, int32_t H, int
   if (T < 0 || H < 1 || k < 1 || capacity < 0) return MOE_ERR_INVALID_ARG;
   if (k > 32) return MOE_ERR_UNSUPPORTED;
   if ((H % 8) != 0) return MOE_ERR_INVALID_ARG;
-  if ((flags & ~MOE_GATHER_ZERO_PAD) != 0u) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~(MOE_GATHER_ZERO_PAD | MOE_GATHER_HIDDEN_READY)) != 0u) return MOE_ERR_INVALID_ARG;
   const bool zero_pad = (flags & MOE_GATHER_ZERO_PAD) != 0u;
   if (T > (int64_t{1} << 40) || T * k >= (int64_t{1} << 30) || capacity >= (int64_t{1} << 31))
     return MOE_ERR_INVALID_ARG;
@@ -361,27 +371,28 @@ extern "C" moe_status_t moe_gather(const void* hidden, int64_t T, int32_t H, int
         cudaFuncSetAttribute(gather_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
             cudaSuccess)
       return MOE_ERR_CUDA;
-    gather_tma_kernel<<<static_cast<unsigned>(blocks), 32, smem, st>>>(
-        static_cast<const uint8_t*>(hidden), T, row_bytes, k, tpc, inv_perm, capacity, static_cast<uint8_t*>(permuted),
-        device_status);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    const int ready = (flags & MOE_GATHER_HIDDEN_READY) ? 1 : 0;
+    if (moe_host::launch_pdl(gather_tma_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32), smem, st,
+                             static_cast<const uint8_t*>(hidden), T, row_bytes, k, tpc, inv_perm, capacity,
+                             static_cast<uint8_t*>(permuted), device_status, ready) != MOE_OK)
+      return MOE_ERR_CUDA;
   } else if (T > 0) {  // rows beyond 128 KB: register-staged copy
     int seg, seg_len;
     segment_rows(T, NV, &seg, &seg_len);
     const int64_t warps = T * seg;
     const int64_t blocks = (warps + kWarpsPerCta - 1) / kWarpsPerCta;
     if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
-    gather_kernel<<<static_cast<unsigned>(blocks), kWarpsPerCta * 32, 0, st>>>(
-        static_cast<const uint4*>(hidden), T, NV, k, seg, seg_len, inv_perm, capacity, static_cast<uint4*>(permuted),
-        device_status);
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe_host::launch_pdl(gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kWarpsPerCta * 32), 0, st,
+                             static_cast<const uint4*>(hidden), T, NV, k, seg, seg_len, inv_perm, capacity,
+                             static_cast<uint4*>(permuted), device_status) != MOE_OK)
+      return MOE_ERR_CUDA;
   }
   if (zero_pad && capacity > 0) {
     const int64_t blocks = (capacity + kWarpsPerCta - 1) / kWarpsPerCta;
-    zero_pad_kernel<<<static_cast<unsigned>(blocks), kWarpsPerCta * 32, 0, st>>>(
-        sorted_token_ids, num_tokens_post_pad, capacity, NV, static_cast<int32_t>(T * k),
-        static_cast<uint4*>(permuted));
-    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    if (moe_host::launch_pdl(zero_pad_kernel, dim3(static_cast<unsigned>(blocks)), dim3(kWarpsPerCta * 32), 0, st,
+                             sorted_token_ids, num_tokens_post_pad, capacity, NV, static_cast<int32_t>(T * k),
+                             static_cast<uint4*>(permuted)) != MOE_OK)
+      return MOE_ERR_CUDA;
   }
   return MOE_OK;
 }
@@ -426,7 +437,6 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
       cudaFuncSetAttribute(combine_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
-  combine_tma_kernel<<<static_cast<unsigned>(grid), (1 + kCombineConsumerWarps) * 32, smem,
-                       static_cast<cudaStream_t>(stream)>>>(a);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return moe_host::launch_pdl(combine_tma_kernel, dim3(static_cast<unsigned>(grid)),
+                              dim3((1 + kCombineConsumerWarps) * 32), smem, static_cast<cudaStream_t>(stream), a);
 }

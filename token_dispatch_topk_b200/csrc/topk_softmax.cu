@@ -110,6 +110,8 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
   const int g = lane & (G - 1);
   const int sub = lane >> g_log2;
 
+  moe::pdl_wait();
+  moe::pdl_launch_dependents();
   const int64_t row0 = (static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + warp) * rows_per_warp;
   if (row0 >= T) return;  // uniform per warp
 
@@ -187,7 +189,9 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
 // One warp per row (E >= 16).  Lane l holds chunks l, l+32, ... of VEC logits.  bf16 logits fit
 // a 32-bit key (ordered 16-bit value above, 0xFFFF - index below), so each round is a single
 // warp-wide redux max; fp32 logits use the 64-bit key, reduced as its high word, then the low
-// word among the lanes holding that high word.  Lane j keeps round j's expert and probability.
+// word among the lanes holding that high word.  Lane j keeps round j's key; after the rounds each
+// of lanes 0..k-1 takes one exp, and a warp sum gives the renormalising denominator (the
+// full-row denominator Z is reduced in round 0 only when not renormalising).
 // ------------------------------------------------------------------------------------------
 constexpr int kRowWarps = 4;
 
@@ -247,6 +251,8 @@ topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, in
   (void)g_log2_unused;
   constexpr int NV = CPL * VEC;
   const int lane = threadIdx.x & 31;
+  moe::pdl_wait();  // the logits may come from the previous kernel (the router projection)
+  moe::pdl_launch_dependents();
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
   if (row >= T) return;  // uniform per warp
   const int n_chunks = E / VEC;
@@ -269,30 +275,34 @@ topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, in
         for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0u;
       }
     }
+    uint32_t my_key = 0u, best0 = 0u;
     for (int j = 0; j < k; ++j) {
       uint32_t best = 0u;
 #pragma unroll
       for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
       best = __reduce_max_sync(0xffffffffu, best);
-      const float xj = ordered16_to_float(best >> 16);
       if (j == 0) {
-        m = xj;
-        float z = 0.f;
+        best0 = best;
+        if (!renormalize) {  // full-row denominator, from the keys before any is retired
+          m = ordered16_to_float(best >> 16);
+          float z = 0.f;
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
-          if (key[i] != 0u) z += expf(ordered16_to_float(key[i] >> 16) - m);
+          for (int i = 0; i < NV; ++i) {
+            if (key[i] != 0u) z += expf(ordered16_to_float(key[i] >> 16) - m);
+          }
+          Z = warp_sum(z);
         }
-        Z = warp_sum(z);
       }
 #pragma unroll
       for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0u : key[i];
-      const float p = expf(xj - m);
-      S += p;
-      if (lane == j) {
-        my_e = static_cast<int>(0xffffu - (best & 0xffffu));
-        my_p = p;
-      }
+      if (lane == j) my_key = best;
     }
+    m = ordered16_to_float(best0 >> 16);
+    if (lane < k) {
+      my_p = expf(ordered16_to_float(my_key >> 16) - m);
+      my_e = static_cast<int>(0xffffu - (my_key & 0xffffu));
+    }
+    if (renormalize) S = warp_sum(my_p);
   } else {
     uint64_t key[NV];
 #pragma unroll
@@ -308,6 +318,8 @@ topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, in
         for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0ull;
       }
     }
+    uint64_t my_key = 0ull;
+    uint32_t hi0 = 0u;
     for (int j = 0; j < k; ++j) {
       uint64_t mine = 0ull;
 #pragma unroll
@@ -316,25 +328,28 @@ topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, in
       const uint32_t lo = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32) == hi
                                                              ? static_cast<uint32_t>(mine) : 0u);
       const uint64_t best = (static_cast<uint64_t>(hi) << 32) | lo;
-      const float xj = ordered_to_float(hi);
       if (j == 0) {
-        m = xj;
-        float z = 0.f;
+        hi0 = hi;
+        if (!renormalize) {
+          m = ordered_to_float(hi);
+          float z = 0.f;
 #pragma unroll
-        for (int i = 0; i < NV; ++i) {
-          if (key[i] != 0ull) z += expf(ordered_to_float(static_cast<uint32_t>(key[i] >> 32)) - m);
+          for (int i = 0; i < NV; ++i) {
+            if (key[i] != 0ull) z += expf(ordered_to_float(static_cast<uint32_t>(key[i] >> 32)) - m);
+          }
+          Z = warp_sum(z);
         }
-        Z = warp_sum(z);
       }
 #pragma unroll
       for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
-      const float p = expf(xj - m);
-      S += p;
-      if (lane == j) {
-        my_e = static_cast<int>(0xffffffffu - lo);
-        my_p = p;
-      }
+      if (lane == j) my_key = best;
     }
+    m = ordered_to_float(hi0);
+    if (lane < k) {
+      my_p = expf(ordered_to_float(static_cast<uint32_t>(my_key >> 32)) - m);
+      my_e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(my_key));
+    }
+    if (renormalize) S = warp_sum(my_p);
   }
   if (lane < k) {
     const float den = renormalize ? S : Z;
@@ -344,6 +359,22 @@ topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, in
 }
 
 using TopkKernel = void (*)(const void*, int64_t, int, int, int, int, float*, int32_t*);
+
+// Launch a gating kernel (any instance, arguments as a void* array) with programmatic stream
+// serialisation.
+cudaError_t launch_topk(TopkKernel kern, int64_t grid, int block, size_t smem, cudaStream_t st, void** args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(block);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelExC(&cfg, reinterpret_cast<const void*>(kern), args);
+}
 
 template <typename TIn, int VEC, int CPL>
 TopkKernel instance() {
@@ -484,9 +515,9 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
     int unused = 0;
     const void* logits_arg = logits;
     void* args[] = {&logits_arg, &T, &E, &k, &unused, &renorm_flag, &topk_weights, &topk_ids};
-    cudaError_t err = cudaLaunchKernel(reinterpret_cast<const void*>(rk), dim3(static_cast<unsigned>(grid)),
-                                       dim3(kRowWarps * 32), args, 0, static_cast<cudaStream_t>(stream));
-    return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+    return launch_topk(rk, grid, kRowWarps * 32, 0, static_cast<cudaStream_t>(stream), args) == cudaSuccess
+               ? MOE_OK
+               : MOE_ERR_CUDA;
   }
   const TopkGeometry geo = topk_geometry(elem, logits, E, k);
   TopkKernel kern = dtype == MOE_DTYPE_BF16 ? pick_kernel<__nv_bfloat16>(geo.vec, geo.cpl)
@@ -498,8 +529,8 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
   int g_log2 = geo.g_log2;
   const void* logits_arg = logits;
   void* args[] = {&logits_arg, &T, &E, &k, &g_log2, &renorm_flag, &topk_weights, &topk_ids};
-  cudaError_t err = cudaLaunchKernel(reinterpret_cast<const void*>(kern), dim3(static_cast<unsigned>(grid)),
-                                     dim3(geo.warps * 32), args, static_cast<size_t>(geo.smem),
-                                     static_cast<cudaStream_t>(stream));
-  return err == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_topk(kern, grid, geo.warps * 32, static_cast<size_t>(geo.smem), static_cast<cudaStream_t>(stream),
+                     args) == cudaSuccess
+             ? MOE_OK
+             : MOE_ERR_CUDA;
 }

@@ -46,9 +46,9 @@ class MoeRouter:
         return B.moe_align_permute(ids, self.E, self.block_size, self.expert_map, self.E_local, self.align,
                                    self.workspace, stream)
 
-    def gather(self, hidden: torch.Tensor, stream=None) -> torch.Tensor:
+    def gather(self, hidden: torch.Tensor, stream=None, hidden_ready: bool = False) -> torch.Tensor:
         return B.moe_gather(hidden, self.k, self.align.inv_perm, self.capacity, permuted=self.permuted,
-                            device_status=self.workspace, stream=stream)
+                            device_status=self.workspace, stream=stream, hidden_ready=hidden_ready)
 
     def combine(self, expert_out: torch.Tensor, topk_weights: Optional[torch.Tensor] = None,
                 stream=None) -> torch.Tensor:
@@ -60,7 +60,7 @@ class MoeRouter:
         """gate + align + permute-gather + combine (expert_out stands in for the expert MLPs' output)."""
         self.gate(logits, stream)
         self.align_permute(stream=stream)
-        self.gather(hidden, stream)
+        self.gather(hidden, stream, hidden_ready=True)  # hidden is an input of the step: ready before gating
         return self.combine(expert_out, stream=stream)
 
     def step_from_host(self, logits_host: torch.Tensor, hidden_host: torch.Tensor, expert_out: torch.Tensor,
