@@ -235,6 +235,32 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
                          int32_t k, int32_t H, int64_t capacity, void* out, int32_t* device_status, void* stream);
 
 /*
+ * moe_route_dispatch -- gating, align and permute-gather in one call, as two kernels instead of
+ * four ("Upstream Reference", "File Index": the gate -> topk -> expand part of the FusedMoE
+ * pipeline).  Every output is the same as from moe_topk_softmax (flags: MOE_RENORMALIZE) then
+ * moe_align_permute then moe_gather (without MOE_GATHER_ZERO_PAD), bit for bit:
+ *   topk_weights [T,k], topk_ids [T,k], counts [E_local], offsets [E_local+1],
+ *   sorted_token_ids [C], expert_ids [NB], num_tokens_post_pad [1], inv_perm [T*k],
+ *   permuted [C, H] (rows of local slots; pad rows untouched).
+ * The first kernel gates tiles of tokens and counts each tile's slots per local expert with
+ * their ranks inside the tile; the last of its CTAs to finish turns the tile counts into the
+ * padded layout.  The second kernel gives every slot its row and copies the hidden rows there.
+ *   logits [T, E] bf16/fp32 (dtype); hidden [T, H] bf16, 16-byte aligned, H % 8 == 0 and
+ *   H <= 65536; expert_map and E_local as for moe_align_permute.
+ *   workspace: >= moe_route_dispatch_workspace_bytes(T, k, E_local) bytes, zeroed before its
+ *   first use and left ready by every call; its first 4 bytes are the device status word.
+ *   Errors: as the three calls it replaces; UNSUPPORTED also for H > 65536.
+ */
+MOE_API size_t moe_route_dispatch_workspace_bytes(int64_t T, int32_t k, int32_t E_local);
+
+MOE_API moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, const void* hidden, int64_t T,
+                                        int32_t E, int32_t k, int32_t H, uint32_t flags, const int32_t* expert_map,
+                                        int32_t E_local, int32_t block_size, float* topk_weights, int32_t* topk_ids,
+                                        int32_t* counts, int32_t* offsets, int32_t* sorted_token_ids,
+                                        int32_t* expert_ids, int32_t* num_tokens_post_pad, int32_t* inv_perm,
+                                        void* permuted, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Read the device status word (first 4 bytes of an align workspace, or any
  * device int32 used as device_status), reset it to MOE_OK, and return the
  * value in *device_status.  Synchronises `stream`.  Not capturable.

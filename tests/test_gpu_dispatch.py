@@ -1,0 +1,103 @@
+"""GPU parity of the fused dispatch (moe_route_dispatch: gating + align + permute-gather in two
+kernels) against the CPU oracle pipeline, through the C ABI.
+
+Shapes cover one and many gating tiles with a ragged last tile, maps with remote and out-of-range
+values, every gating vector width, k up to 32, 1024 experts, T = 0 and the decode size.  Bars as
+for the stage entry points: ids, align outputs and gathered rows bit-exact, weights within 2e-6.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import token_dispatch_topk_b200 as tdt
+from token_dispatch_topk_b200 import inputs as I
+
+from gpu_helpers import TOPK_WEIGHT_ATOL, assert_align_equal, bf16_bits, logits_for_oracle, np_i32, require_gpu
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    # name, T, E, k, dtype, renorm, map kind, E_local, bs, H
+    ("tiny", 64, 8, 2, torch.bfloat16, True, None, 8, 16, 256),
+    ("prefill_ragged", 4100, 128, 8, torch.bfloat16, True, None, 128, 64, 2048),
+    ("decode_rank1", 2, 160, 6, torch.bfloat16, True, "rank1", 40, 8, 4096),
+    ("nonpow2_fp32", 3000, 60, 4, torch.float32, False, None, 60, 64, 264),
+    ("strided_map", 777, 160, 6, torch.bfloat16, True, "strided", 40, 8, 512),
+    ("bad_map_values", 500, 64, 4, torch.bfloat16, True, "bad", 16, 16, 64),
+    ("k32_fp32", 300, 64, 32, torch.float32, True, None, 64, 8, 128),
+    ("wide_1024", 257, 1024, 8, torch.bfloat16, False, None, 1024, 4, 128),
+    ("odd_e_bf16", 333, 61, 5, torch.bfloat16, True, None, 61, 3, 16),
+    ("many_tiles_small_bs", 9000, 32, 2, torch.bfloat16, True, None, 32, 1, 8),
+    ("zero_tokens", 0, 16, 4, torch.bfloat16, True, None, 16, 8, 64),
+]
+
+
+def _map(kind, E, E_local):
+    if kind is None:
+        return None
+    if kind == "rank1":
+        m = np.full(E, -1, np.int32)
+        m[E_local:2 * E_local] = np.arange(E_local)
+        return m
+    if kind == "strided":
+        return I.strided_expert_map(E, 4, 1).numpy()
+    if kind == "bad":  # some globals map past E_local or below -1: those slots are dropped and flagged
+        m = np.full(E, -1, np.int32)
+        m[:E_local] = np.arange(E_local)
+        m[E_local] = E_local + 3
+        m[E_local + 1] = -5
+        return m
+    raise ValueError(kind)
+
+
+@pytest.mark.parametrize("name,T,E,k,dtype,renorm,kind,E_local,bs,H", CASES, ids=[c[0] for c in CASES])
+def test_dispatch_parity(name, T, E, k, dtype, renorm, kind, E_local, bs, H):
+    dev = require_gpu()
+    g = torch.Generator().manual_seed(T + 7 * E + k)
+    x = torch.randn((T, E), generator=g).to(dtype)
+    if kind == "bad":  # make the flagged globals win often
+        x[:, E_local] += 3.0
+        x[:, E_local + 1] += 3.0
+    hidden = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    emap = _map(kind, E, E_local)
+    emap_d = None if emap is None else torch.from_numpy(emap).to(dev)
+    ws = tdt.alloc_dispatch_workspace(T, k, E_local, dev)
+    w_ref, ids_ref = oracle.topk_softmax(logits_for_oracle(x), k, renorm)
+    al = oracle.align_permute(ids_ref, E, bs, emap, E_local)
+    npad = int(al["num_tokens_post_pad"][0])
+    perm_ref = oracle.gather(bf16_bits(hidden), k, al["sorted_token_ids"], npad, al["capacity"])
+    real = al["sorted_token_ids"][:npad] != T * k
+    for call in range(2):  # the second call checks that the workspace was left ready
+        w, ids, align, perm = tdt.moe_route_dispatch(x.to(dev), hidden.to(dev), k, renorm, bs, emap_d, E_local,
+                                                     workspace=ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(np_i32(ids), ids_ref), (name, call)
+        if T:
+            assert np.abs(w.cpu().numpy() - w_ref).max() <= TOPK_WEIGHT_ATOL, (name, call)
+        assert_align_equal(align, al, f"{name} call {call}")
+        assert np.array_equal(bf16_bits(perm[:npad])[real], perm_ref[:npad][real]), (name, call)
+        status = tdt.moe_read_status(ws)
+        assert status == (tdt.MOE_ERR_BAD_EXPERT_ID if kind == "bad" else tdt.MOE_OK), (name, status)
+
+
+def test_dispatch_matches_stage_entry_points():
+    """The fused dispatch and the three stage calls it replaces give identical outputs."""
+    dev = require_gpu()
+    wl = I.WORKLOADS["qwen3moe_prefill_T4096_E128_k8"]
+    logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)
+    a = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, device=dev)
+    b = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, device=dev)
+    a.dispatch(logits, hidden)
+    b.gate(logits)
+    b.align_permute()
+    b.gather(hidden)
+    torch.cuda.synchronize()
+    for name in ("counts", "offsets", "sorted_token_ids", "expert_ids", "num_tokens_post_pad", "inv_perm"):
+        assert torch.equal(getattr(a.align, name), getattr(b.align, name)), name
+    assert torch.equal(a.topk_ids, b.topk_ids) and torch.equal(a.topk_weights, b.topk_weights)
+    npad = int(a.align.num_tokens_post_pad.item())
+    real = (a.align.sorted_token_ids[:npad] != wl.T * wl.k)
+    assert torch.equal(a.permuted[:npad][real], b.permuted[:npad][real])

@@ -63,8 +63,13 @@ def _check_all(r, wl, ref, what, y, y_bits):
     assert d.max() <= COMBINE_MAX_ULP, (what, d.max())
 
 
+def _run(r, path, logits, hidden, y):
+    return r.step(logits, hidden, y) if path == "fused" else r.step_staged(logits, hidden, y)
+
+
+@pytest.mark.parametrize("path", ["fused", "staged"])
 @pytest.mark.parametrize("name", FULL)
-def test_workload_full_size(name):
+def test_workload_full_size(name, path):
     dev = require_gpu()
     wl = I.WORKLOADS[name]
     logits = I.make_logits(wl)
@@ -72,14 +77,15 @@ def test_workload_full_size(name):
     y = I.make_expert_out(wl.capacity, wl.H)
     r = _router(wl, dev)
     yd = y.to(dev)
-    r.step(logits.to(dev), hidden.to(dev), yd)
+    _run(r, path, logits.to(dev), hidden.to(dev), yd)
     torch.cuda.synchronize()
     ref = _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y))
     _check_all(r, wl, ref, name, yd, bf16_bits(y))
     assert r.device_status() == tdt.MOE_OK
 
 
-def test_ep_decode_every_route_pattern():
+@pytest.mark.parametrize("path", ["fused", "staged"])
+def test_ep_decode_every_route_pattern(path):
     """M=2, top-k 6, rank 1 of 4 (40 local experts): the logits-derived routing and every
     injected route pattern, including the valid all-remote rank."""
     dev = require_gpu()
@@ -89,7 +95,7 @@ def test_ep_decode_every_route_pattern():
     y = I.make_expert_out(wl.capacity, wl.H)
     r = _router(wl, dev)
     yd = y.to(dev)
-    r.step(logits.to(dev), hidden.to(dev), yd)
+    _run(r, path, logits.to(dev), hidden.to(dev), yd)
     torch.cuda.synchronize()
     _check_all(r, wl, _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y)), "logits-derived", yd,
                bf16_bits(y))
@@ -114,14 +120,15 @@ def test_ep_decode_every_route_pattern():
             assert npad == 0 and (bf16_bits(r.out) == 0).all()
 
 
-def test_skewed_prefill_full_size_sampled():
+@pytest.mark.parametrize("path", ["fused", "staged"])
+def test_skewed_prefill_full_size_sampled(path):
     dev = require_gpu()
     wl = I.WORKLOADS["zipf_prefill_T65536_E256_k8_H7168"]
     logits = I.make_logits(wl)
     hidden = I.make_hidden(wl)
     y_dev = I.make_expert_out(wl.capacity, wl.H, device=dev)
     r = _router(wl, dev)
-    r.step(logits.to(dev), hidden.to(dev), y_dev)
+    _run(r, path, logits.to(dev), hidden.to(dev), y_dev)
     torch.cuda.synchronize()
     # gating and align in full
     w_ref, ids_ref = oracle.topk_softmax(logits_for_oracle(logits), wl.k, wl.renormalize)
@@ -165,8 +172,8 @@ def test_repeat_steps_are_bit_identical():
     y = I.make_expert_out(wl.capacity, wl.H, device=dev)
     r = _router(wl, dev)
     first = None
-    for _ in range(5):
-        r.step(logits, hidden, y)
+    for i in range(6):
+        (r.step if i % 2 == 0 else r.step_staged)(logits, hidden, y)
         snap = [t.clone() for t in (r.topk_ids, r.topk_weights, r.align.sorted_token_ids, r.align.inv_perm,
                                     r.align.expert_ids, r.out)]
         if first is None:

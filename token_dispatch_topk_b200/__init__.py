@@ -11,7 +11,8 @@ from .binding import (  # noqa: F401
     MOE_RENORMALIZE,
     AlignResult, MoeError, alloc_align_outputs, alloc_workspace, load_library, moe_align_capacity,
     moe_align_num_blocks, moe_align_permute, moe_align_permute_noalloc, moe_align_workspace_bytes, moe_combine, moe_gather, moe_read_status,
-    moe_topk_softmax, moe_version, moe_workspace_init, status_string,
+    moe_route_dispatch, moe_route_dispatch_workspace_bytes, moe_topk_softmax, moe_version, moe_workspace_init,
+    status_string, alloc_dispatch_workspace,
 )
 from .router import MoeRouter  # noqa: F401
 

@@ -47,6 +47,9 @@ SIGNATURES = {
     "moe_gather": (ctypes.c_int, [_P, _I64, _I32, _I32, _P, _P, _P, _I64, _U32, _P, _P, _P]),
     "moe_combine": (ctypes.c_int, [_P, _P, _P, _I64, _I32, _I32, _I64, _P, _P, _P]),
     "moe_read_status": (ctypes.c_int, [_P, _P, ctypes.POINTER(ctypes.c_int)]),
+    "moe_route_dispatch_workspace_bytes": (_SZ, [_I64, _I32, _I32]),
+    "moe_route_dispatch": (ctypes.c_int, [_P, ctypes.c_int, _P, _I64, _I32, _I32, _I32, _U32, _P, _I32, _I32, _P, _P,
+                                          _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -258,6 +261,57 @@ def moe_combine(expert_out: torch.Tensor, topk_weights: torch.Tensor, inv_perm: 
                                     _dev(device_status, "device_status"), _stream(stream))
     _check(st, "moe_combine")
     return out
+
+
+def moe_route_dispatch_workspace_bytes(T: int, k: int, E_local: int) -> int:
+    return int(load_library().moe_route_dispatch_workspace_bytes(T, k, E_local))
+
+
+def alloc_dispatch_workspace(T: int, k: int, E_local: int, device) -> torch.Tensor:
+    """A zeroed workspace for moe_route_dispatch (int32 words; word 0 is the device status word)."""
+    nbytes = moe_route_dispatch_workspace_bytes(T, k, E_local)
+    return torch.zeros((nbytes + 3) // 4, dtype=torch.int32, device=device)
+
+
+def moe_route_dispatch(logits: torch.Tensor, hidden: torch.Tensor, k: int, renormalize: bool, block_size: int,
+                       expert_map: Optional[torch.Tensor] = None, E_local: Optional[int] = None,
+                       topk_weights: Optional[torch.Tensor] = None, topk_ids: Optional[torch.Tensor] = None,
+                       align: Optional[AlignResult] = None, permuted: Optional[torch.Tensor] = None,
+                       workspace: Optional[torch.Tensor] = None, stream=None):
+    """Gating + align + permute-gather in one call.  Returns (topk_weights, topk_ids, AlignResult, permuted)."""
+    T, E = logits.shape
+    H = hidden.shape[1]
+    if logits.dtype == torch.bfloat16:
+        dt = MOE_DTYPE_BF16
+    elif logits.dtype == torch.float32:
+        dt = MOE_DTYPE_F32
+    else:
+        raise ValueError(f"logits dtype {logits.dtype} unsupported (bf16 or fp32)")
+    assert hidden.dtype == torch.bfloat16
+    if E_local is None:
+        E_local = E
+    dev = logits.device
+    if topk_weights is None:
+        topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
+    if topk_ids is None:
+        topk_ids = torch.empty((T, k), dtype=torch.int32, device=dev)
+    if align is None:
+        align = alloc_align_outputs(T, k, E_local, block_size, dev)
+    if permuted is None:
+        permuted = torch.empty((align.capacity, H), dtype=torch.bfloat16, device=dev)
+    if workspace is None:
+        workspace = alloc_dispatch_workspace(T, k, E_local, dev)
+    assert expert_map is None or expert_map.dtype == torch.int32
+    st = load_library().moe_route_dispatch(
+        _dev(logits, "logits"), dt, _dev(hidden, "hidden"), T, E, k, H, MOE_RENORMALIZE if renormalize else 0,
+        _dev(expert_map, "expert_map"), E_local, block_size, _dev(topk_weights, "topk_weights"),
+        _dev(topk_ids, "topk_ids"), _dev(align.counts, "counts"), _dev(align.offsets, "offsets"),
+        _dev(align.sorted_token_ids, "sorted_token_ids"), _dev(align.expert_ids, "expert_ids"),
+        _dev(align.num_tokens_post_pad, "num_tokens_post_pad"), _dev(align.inv_perm, "inv_perm"),
+        _dev(permuted, "permuted"), _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+        _stream(stream))
+    _check(st, "moe_route_dispatch")
+    return topk_weights, topk_ids, align, permuted
 
 
 def moe_read_status(device_status_word: torch.Tensor, stream=None) -> int:

@@ -159,37 +159,44 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
 }
 
 constexpr int kCombineConsumerWarps = 8;
-constexpr int kCombineStages = 3;
+constexpr int kCombineMaxStages = 8;
+constexpr uint32_t kCombineStageTarget = 32u * 1024u;  // bytes of slot rows per stage (about)
+constexpr uint32_t kCombineRingTarget = 96u * 1024u;   // bytes of stages per CTA (about)
 
 struct CombineArgs {
-  const uint8_t* y;        // expert_out [capacity, H] bf16
-  const float* w;          // [T, k]
-  const int32_t* inv_perm; // [T*k]
+  const uint8_t* y;         // expert_out [capacity, H] bf16
+  const float* w;           // [T, k]
+  const int32_t* inv_perm;  // [T*k]
   int64_t T;
   int k;
-  uint32_t row_bytes;      // H * 2
-  uint32_t chunk_bytes;    // bytes of one row chunk (a unit covers one chunk of one token)
+  int tpu;                  // tokens per unit (tpu * k <= 32)
+  int stages;               // depth of the shared-memory ring
+  uint32_t row_bytes;       // H * 2
+  uint32_t chunk_bytes;     // bytes of one row chunk (a unit covers one chunk of tpu tokens)
   int nchunks;
-  int64_t units;           // T * nchunks
+  int64_t units;            // ceil(T / tpu) * nchunks
   int64_t capacity;
-  uint8_t* out;            // [T, H] bf16
+  uint8_t* out;             // [T, H] bf16
   int32_t* status;
 };
 
 // Persistent, warp-specialised: warp 0 produces, warps 1..8 consume.  A unit is one column chunk
-// of one token.  The producer bulk-loads the chunk of each local slot row into a stage of a
-// 3-deep shared-memory ring (mbarrier `full`), with the slot weights and a validity mask beside
-// it; the consumers accumulate in fp32 (packed f32x2 fused multiply-adds: two independent
-// correctly rounded fmas, ascending slot order, from +0), store the bf16 result and release the
-// stage (mbarrier `empty`, one arrival per consumer warp).
+// of `tpu` consecutive tokens (tpu * k slot rows, about 32 KB).  The producer bulk-loads the chunk
+// of every local slot row of the unit into a stage of a shared-memory ring (mbarrier `full`), with
+// the slot weights and a validity mask beside it; one consumer thread waits for the stage and the
+// consumer warps are released together by a named barrier (waiting warps take no issue slots).
+// Consumers accumulate in fp32 (packed f32x2 fused multiply-adds: two independent correctly
+// rounded fmas, ascending slot order, from +0), store the bf16 result and release the stage
+// (mbarrier `empty`, one arrival per consumer warp).
 __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_kernel(CombineArgs a) {
-  constexpr int S = kCombineStages;
   extern __shared__ __align__(128) uint8_t smem[];
   const int k = a.k;
-  const uint32_t stage_bytes = static_cast<uint32_t>(k) * a.chunk_bytes;
+  const int S = a.stages;
+  const int spu = a.tpu * k;  // slot rows per unit (<= 32)
+  const uint32_t stage_bytes = static_cast<uint32_t>(spu) * a.chunk_bytes;
   uint8_t* buf = smem;
-  uint64_t* s_w2 = reinterpret_cast<uint64_t*>(smem + S * stage_bytes);  // [S][k] packed {w, w}
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_w2 + S * k);         // [S]
+  uint64_t* s_w2 = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);  // [S][32] {w, w}
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_w2 + S * 32);                              // [S]
   uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_mask + S) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + S;
   __shared__ int s_abort;
@@ -212,53 +219,59 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
   if (u0 >= u1) return;
 
   if (warp == 0) {
-    // ---- producer
-    int64_t cur_t = u0 / a.nchunks;
-    auto load_meta = [&](int64_t t, int& r, float& w) {
+    // ---- producer: lane l < spu handles slot l of the unit (token t0 + l / k, rank l % k)
+    auto load_meta = [&](int64_t grp, int& r, float& w) {
       r = -1;
       w = 0.f;
-      if (t < a.T && lane < k) {
-        r = a.inv_perm[t * k + lane];
-        w = a.w[t * k + lane];
+      const int64_t t = grp * a.tpu + lane / k;
+      if (lane < spu && t < a.T) {
+        const int64_t s = t * k + lane % k;
+        r = a.inv_perm[s];
+        w = a.w[s];
         if (r < -1 || static_cast<int64_t>(r) >= a.capacity) {
           moe::record_status(a.status, MOE_ERR_BAD_ROW);
           r = -1;
         }
       }
     };
+    int64_t cur = u0 / a.nchunks;  // token group
     int r_cur, r_next;
     float w_cur, w_next;
-    load_meta(cur_t, r_cur, w_cur);
-    load_meta(cur_t + 1, r_next, w_next);
+    load_meta(cur, r_cur, w_cur);
+    load_meta(cur + 1, r_next, w_next);
+    int s = 0;
+    uint32_t round = 0;  // completed passes over the ring
     int64_t issued = 0;
     for (int64_t u = u0; u < u1; ++u, ++issued) {
-      const int64_t t = u / a.nchunks;
-      const int c = static_cast<int>(u - t * a.nchunks);
-      if (t != cur_t) {  // advance one token (units are in token order) and prefetch the next
-        cur_t = t;
+      const int64_t grp = u / a.nchunks;
+      const int c = static_cast<int>(u - grp * a.nchunks);
+      if (grp != cur) {  // units are in group order: advance one group and prefetch the next
+        cur = grp;
         r_cur = r_next;
         w_cur = w_next;
-        load_meta(t + 1, r_next, w_next);
+        load_meta(grp + 1, r_next, w_next);
       }
-      const int s = static_cast<int>(issued % S);
-      const uint32_t n = static_cast<uint32_t>(issued / S);
-      if (n > 0 && !moe::mbar_wait(&empty[s], (n - 1) & 1u)) {
+      if (issued >= S && !moe::mbar_wait(&empty[s], (round - 1) & 1u)) {
         moe::record_status(a.status, MOE_ERR_TIMEOUT);
         s_abort = 1;
         break;
       }
-      const uint32_t mask = __ballot_sync(0xffffffffu, lane < k && r_cur >= 0);
+      const uint32_t mask = __ballot_sync(0xffffffffu, r_cur >= 0);
       const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
-      if (lane < k) s_w2[s * k + lane] = moe::f32x2(w_cur, w_cur);
+      s_w2[s * 32 + lane] = moe::f32x2(w_cur, w_cur);
       if (lane == 0) s_mask[s] = mask;
       __threadfence_block();
       __syncwarp();
       if (lane == 0) moe::mbar_arrive_expect_tx(&full[s], static_cast<uint32_t>(__popc(mask)) * cb);
       __syncwarp();
-      if (lane < k && r_cur >= 0) {
+      if (r_cur >= 0) {
         moe::bulk_load(buf + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * a.chunk_bytes,
                        a.y + static_cast<int64_t>(r_cur) * a.row_bytes + static_cast<int64_t>(c) * a.chunk_bytes, cb,
                        &full[s]);
+      }
+      if (++s == S) {
+        s = 0;
+        ++round;
       }
     }
     if (s_abort && lane == 0) {
@@ -274,33 +287,39 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
   // ---- consumers
   const int ct = tid - 32;
   constexpr int NCT = kCombineConsumerWarps * 32;
-  int64_t done = 0;
-  for (int64_t u = u0; u < u1; ++u, ++done) {
-    const int s = static_cast<int>(done % S);
-    const uint32_t n = static_cast<uint32_t>(done / S);
-    if (!moe::mbar_wait(&full[s], n & 1u)) {
+  int s = 0;
+  uint32_t round = 0;
+  for (int64_t u = u0; u < u1; ++u) {
+    if (ct == 0 && !moe::mbar_wait(&full[s], round & 1u)) {
       moe::record_status(a.status, MOE_ERR_TIMEOUT);
       s_abort = 1;
-      break;
     }
-    const int64_t t = u / a.nchunks;
-    const int c = static_cast<int>(u - t * a.nchunks);
+    moe::named_barrier(1, NCT);
+    if (s_abort) break;
+    while (!moe::mbar_try_wait(&full[s], round & 1u)) {
+    }  // completed already: gives this thread its own acquire of the stage
+    const int64_t grp = u / a.nchunks;
+    const int c = static_cast<int>(u - grp * a.nchunks);
     const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
     const uint32_t mask = s_mask[s];
     const uint8_t* stage = buf + static_cast<size_t>(s) * stage_bytes;
-    uint8_t* dst = a.out + t * static_cast<int64_t>(a.row_bytes) + static_cast<int64_t>(c) * a.chunk_bytes;
+    const uint64_t* w2 = s_w2 + s * 32;
     const int nvec = static_cast<int>(cb >> 4);
-    const uint64_t* w2 = s_w2 + s * k;
-    for (int v = ct; v < nvec; v += NCT) {
+    for (int item = ct; item < a.tpu * nvec; item += NCT) {
+      const int ti = item / nvec;
+      const int v = item - ti * nvec;
+      const int64_t t = grp * a.tpu + ti;
+      if (t >= a.T) break;  // items are in token order
       uint64_t acc01 = 0ull, acc23 = 0ull, acc45 = 0ull, acc67 = 0ull;  // +0.0f pairs
-      const uint8_t* col = stage + static_cast<size_t>(v) * 16;
+      const uint8_t* col = stage + static_cast<size_t>(ti) * k * a.chunk_bytes + static_cast<size_t>(v) * 16;
+      const uint32_t tmask = mask >> (ti * k);
       for (int j0 = 0; j0 < k; j0 += 8) {
 #pragma unroll
         for (int jj = 0; jj < 8; ++jj) {
           const int j = j0 + jj;
-          if (j < k && ((mask >> j) & 1u)) {  // ascending j, as the reference order requires
+          if (j < k && ((tmask >> j) & 1u)) {  // ascending j
             const uint4 yv = moe::lds128(col + static_cast<size_t>(j) * a.chunk_bytes);
-            const uint64_t ww = moe::lds64(w2 + j);
+            const uint64_t ww = moe::lds64(w2 + ti * k + j);
             acc01 = moe::fma_bf16x2(ww, yv.x, acc01);
             acc23 = moe::fma_bf16x2(ww, yv.y, acc23);
             acc45 = moe::fma_bf16x2(ww, yv.z, acc45);
@@ -318,10 +337,15 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
       o.y = moe::pack_bf16x2(r[2], r[3]);
       o.z = moe::pack_bf16x2(r[4], r[5]);
       o.w = moe::pack_bf16x2(r[6], r[7]);
+      uint8_t* dst = a.out + t * static_cast<int64_t>(a.row_bytes) + static_cast<int64_t>(c) * a.chunk_bytes;
       moe::st_plain(reinterpret_cast<uint4*>(dst + static_cast<size_t>(v) * 16), o);
     }
     __syncwarp();
     if (lane == 0) moe::mbar_arrive(&empty[s]);
+    if (++s == S) {
+      s = 0;
+      ++round;
+    }
   }
 }
 
@@ -416,22 +440,30 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   a.T = T;
   a.k = k;
   a.row_bytes = static_cast<uint32_t>(H) * 2u;
-  // one stage holds k row chunks: at most 32 KB
+  // a unit: `tpu` tokens x k slot rows x one chunk of each row, about 32 KB
   const uint32_t chunk_cap = k <= 8 ? 4096u : (k <= 16 ? 2048u : 1024u);
   a.chunk_bytes = a.row_bytes < chunk_cap ? a.row_bytes : chunk_cap;
   a.nchunks = static_cast<int>((a.row_bytes + a.chunk_bytes - 1) / a.chunk_bytes);
-  a.units = T * a.nchunks;
+  int tpu = static_cast<int>(kCombineStageTarget / (static_cast<uint32_t>(k) * a.chunk_bytes));
+  if (tpu < 1) tpu = 1;
+  if (tpu * k > 32) tpu = 32 / k;
+  a.tpu = tpu;
+  const uint32_t stage_bytes = static_cast<uint32_t>(tpu * k) * a.chunk_bytes;
+  int stages = static_cast<int>(kCombineRingTarget / stage_bytes);
+  stages = stages < 2 ? 2 : (stages > kCombineMaxStages ? kCombineMaxStages : stages);
+  a.stages = stages;
+  a.units = ((T + tpu - 1) / tpu) * a.nchunks;
   a.capacity = capacity;
   a.out = static_cast<uint8_t*>(out);
   a.status = device_status;
-  const size_t smem = static_cast<size_t>(kCombineStages) * k * a.chunk_bytes +
-                      static_cast<size_t>(kCombineStages) * k * sizeof(uint64_t) + kCombineStages * sizeof(uint32_t) +
-                      8 + 2 * kCombineStages * sizeof(uint64_t);
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes + static_cast<size_t>(stages) * 32 * sizeof(uint64_t) +
+                      stages * sizeof(uint32_t) + 8 + 2 * stages * sizeof(uint64_t);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MOE_ERR_CUDA;
-  const int per_sm = smem <= 48 * 1024 ? 4 : 2;
+  int per_sm = static_cast<int>((200u * 1024u) / (smem + 1024));
+  per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
   const int64_t grid = a.units < static_cast<int64_t>(sms) * per_sm ? a.units : static_cast<int64_t>(sms) * per_sm;
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(combine_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=

@@ -1,0 +1,514 @@
+// route_fused.cu -- fused dispatch: gating and expert counting in one kernel, placement and the
+// activation gather in the next.
+//
+// Operations: the FusedMoE pipeline of "Upstream Reference: Deep-Spark xllm + vllm", "File
+// Index" (gate -> topk -> expand -> ...): topk_softmax (moe_topk_softmax_kernels.cuh), the
+// block alignment for scatter (moe_align_sum_kernels.cu) and the permute-gather ("expand"),
+// with the expert_map remap and the all-remote rank of the 2026-07-16 MTP1 M=2 compact
+// scheduler closure note.  The outputs are exactly those of moe_topk_softmax +
+// moe_align_permute + moe_gather; only the kernel boundaries move.
+//
+// gate_count_kernel (one CTA per tile of `rows_per_tile` tokens):
+//   A. each warp gates rows of the tile (gate_row: one warp per row) and writes topk_weights and
+//      topk_ids; the local expert of every slot of the tile goes to shared memory;
+//   B. stable ranks inside the tile: each warp owns a contiguous run of the tile's slots, counts
+//      it into its own shared-memory row, the rows are scanned across warps, and each slot's rank
+//      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm and the
+//      tile's per-expert counts go to the workspace;
+//   C. the CTA that finishes last (completion ticket, no spinning) scans the tile counts per
+//      expert into per-tile bases, writes counts, the block-padded offsets, N_pad and expert_ids,
+//      and resets the ticket.
+// place_gather_kernel (one warp per CTA, up to 8 tokens, TMA staging as in gather_tma_kernel):
+//   each slot's row = offsets[e] + tile base[e] + rank; the CTA writes sorted_token_ids and
+//   inv_perm for its slots, bulk-loads its hidden rows (before waiting for the previous kernel:
+//   hidden is an input of the call) and bulk-stores them to their rows; the pad rows, the tail
+//   rows past N_pad are spread over the CTAs.
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "gate_row.cuh"
+
+namespace {
+
+constexpr int kGcWarps = 16;
+constexpr int kGcThreads = kGcWarps * 32;
+constexpr int kWsHeaderBytes = 256;  // status word, ticket, padding
+constexpr int64_t kMaxTileCounters = 65536;
+constexpr int kPgMaxTokens = 8;
+constexpr uint32_t kPgCtaBytes = 32u * 1024u;
+
+struct DispatchArgs {
+  const void* logits;
+  int64_t T;
+  int E;
+  int k;
+  int renormalize;
+  const int32_t* expert_map;
+  int E_local;
+  int bs;
+  int64_t P;  // T * k
+  int64_t C;  // capacity rows
+  int NB;     // blocks
+  int rows_per_tile;
+  int num_tiles;
+  float* topk_weights;
+  int32_t* topk_ids;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* sorted_ids;
+  int32_t* expert_ids;
+  int32_t* n_pad;
+  int32_t* inv_perm;
+  int32_t* status;
+  unsigned int* ticket;
+  int32_t* tile_counts;  // [num_tiles][E_local]: tile counts, then per-tile bases
+};
+
+// Local expert of global expert g (or -1: remote); out-of-range values are flagged.
+__device__ __forceinline__ int to_local(const DispatchArgs& a, int g) {
+  if (static_cast<unsigned>(g) >= static_cast<unsigned>(a.E)) {
+    moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+    return -1;
+  }
+  const int le = a.expert_map != nullptr ? a.expert_map[g] : g;
+  if (le < -1 || le >= a.E_local) {
+    moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+    return -1;
+  }
+  return le;
+}
+
+// Lanes of this warp holding the same value v >= 0 (0 for v < 0), through a per-warp array of
+// masks in shared memory that is zero on entry and left zero.
+__device__ __forceinline__ unsigned peers_of(unsigned* masks, int v, int lane) {
+  if (v >= 0) atomicOr(&masks[v], 1u << lane);
+  __syncwarp();
+  const unsigned p = v >= 0 ? masks[v] : 0u;
+  __syncwarp();
+  if (v >= 0) masks[v] = 0u;
+  __syncwarp();
+  return p;
+}
+
+// Exclusive scan of n <= 2 * kGcThreads ints in shared memory (block-wide, in place); returns the total.
+__device__ int scan_block(int* data, int n, int* warp_sums) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int i0 = 2 * tid, i1 = 2 * tid + 1;
+  const int x0 = i0 < n ? data[i0] : 0;
+  const int x1 = i1 < n ? data[i1] : 0;
+  int incl = x0 + x1;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < kGcWarps ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += v;
+    }
+    if (lane < kGcWarps) warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - (x0 + x1);
+  const int total = warp_sums[kGcWarps - 1];
+  __syncthreads();
+  if (i0 < n) data[i0] = before;
+  if (i1 < n) data[i1] = before + x0;
+  __syncthreads();
+  return total;
+}
+
+// Shared memory of gate_count_kernel (ints):
+//   s_le[rows_per_tile * k] | whist[kGcWarps][E_local] | masks[kGcWarps][E_local]
+//   | s_cnt[E_local] | s_off[E_local + 1] | warp_sums[32]
+__host__ __device__ inline size_t gc_smem_ints(int rows_per_tile, int k, int E_local) {
+  return static_cast<size_t>(rows_per_tile) * k + 2 * static_cast<size_t>(kGcWarps) * E_local + 2 * E_local + 1 + 32;
+}
+
+template <typename TIn, int VEC, int CPL>
+__global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) {
+  extern __shared__ int smem[];
+  const int k = a.k, El = a.E_local, RT = a.rows_per_tile;
+  int* s_le = smem;
+  int* whist = s_le + RT * k;
+  unsigned* masks = reinterpret_cast<unsigned*>(whist + kGcWarps * El);
+  int* s_cnt = reinterpret_cast<int*>(masks + kGcWarps * El);
+  int* s_off = s_cnt + El;
+  int* warp_sums = s_off + El + 1;
+  __shared__ int s_is_last;
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x;
+  const int64_t row0 = static_cast<int64_t>(tile) * RT;
+  const int rows = static_cast<int>((a.T - row0) < RT ? (a.T - row0) : RT);
+  for (int i = tid; i < kGcWarps * El; i += kGcThreads) {
+    whist[i] = 0;
+    masks[i] = 0u;
+  }
+  __syncthreads();
+  moe::pdl_wait();  // the logits may come from the previous kernel
+  moe::pdl_launch_dependents();
+
+  // A. gating, one warp per row
+  const TIn* logits = static_cast<const TIn*>(a.logits);
+  for (int r = warp; r < rows; r += kGcWarps) {
+    const int64_t row = row0 + r;
+    int my_e;
+    float my_w;
+    moe_gate::gate_row<TIn, VEC, CPL>(logits + row * static_cast<int64_t>(a.E), a.E, k, a.renormalize, lane, my_e,
+                                      my_w);
+    if (lane < k) {
+      a.topk_weights[row * k + lane] = my_w;
+      a.topk_ids[row * k + lane] = my_e;
+      s_le[r * k + lane] = to_local(a, my_e);
+    }
+  }
+  __syncthreads();
+
+  // B. stable ranks inside the tile
+  const int nslots = rows * k;
+  const int nch = (nslots + 31) / 32;
+  const int cpw = (nch + kGcWarps - 1) / kGcWarps;
+  const int c0 = warp * cpw;
+  const int c1 = (c0 + cpw < nch) ? c0 + cpw : nch;
+  int* my_hist = whist + warp * El;
+  unsigned* my_masks = masks + warp * El;
+  for (int c = c0; c < c1; ++c) {
+    const int i = c * 32 + lane;
+    const int le = i < nslots ? s_le[i] : -1;
+    if (le >= 0) atomicAdd(&my_hist[le], 1);
+  }
+  __syncthreads();
+  for (int e = tid; e < El; e += kGcThreads) {
+    int run = 0;
+    for (int w = 0; w < kGcWarps; ++w) {
+      const int c = whist[w * El + e];
+      whist[w * El + e] = run;
+      run += c;
+    }
+    a.tile_counts[static_cast<int64_t>(tile) * El + e] = run;
+  }
+  __syncthreads();
+  for (int c = c0; c < c1; ++c) {
+    const int i = c * 32 + lane;
+    const int le = i < nslots ? s_le[i] : -1;
+    const unsigned peers = peers_of(my_masks, le, lane);
+    if (le >= 0) {
+      a.inv_perm[row0 * k + i] = my_hist[le] + __popc(peers & moe::lanemask_lt());  // rank in the tile
+    } else if (i < nslots) {
+      a.inv_perm[row0 * k + i] = -1;
+    }
+    __syncwarp();
+    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
+    __syncwarp();
+  }
+
+  // C. the last CTA turns the tile counts into per-tile bases and writes the expert layout
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_is_last = (atomicAdd(a.ticket, 1u) == static_cast<unsigned>(a.num_tiles - 1)) ? 1 : 0;
+  __syncthreads();
+  if (!s_is_last) return;
+  __threadfence();
+  int parts = 1;  // threads sharing one expert column, each scanning a contiguous range of tiles
+  while (parts * 2 * El <= kGcThreads && parts * 2 <= 32) parts *= 2;
+  const int per = (a.num_tiles + parts - 1) / parts;
+  const int part = tid % parts;
+  const int t0 = part * per;
+  const int t1 = (t0 + per < a.num_tiles) ? t0 + per : a.num_tiles;
+  for (int e0 = 0; e0 < El; e0 += kGcThreads / parts) {  // uniform trip count
+    const int e = e0 + tid / parts;
+    int sum = 0;
+    if (e < El) {
+      for (int t = t0; t < t1; ++t) sum += __ldcg(a.tile_counts + static_cast<int64_t>(t) * El + e);
+    }
+    int incl = sum;
+    for (int off = 1; off < parts; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off, parts);
+      if (part >= off) incl += v;
+    }
+    if (e < El) {
+      int run = incl - sum;
+      for (int t = t0; t < t1; ++t) {
+        int32_t* p = a.tile_counts + static_cast<int64_t>(t) * El + e;
+        const int c = __ldcg(p);
+        *p = run;
+        run += c;
+      }
+      if (part == parts - 1) s_cnt[e] = run;
+    }
+  }
+  __syncthreads();
+  for (int e = tid; e < El; e += kGcThreads) s_off[e] = ((s_cnt[e] + a.bs - 1) / a.bs) * a.bs;
+  __syncthreads();
+  const int total = scan_block(s_off, El, warp_sums);
+  if (tid == 0) {
+    s_off[El] = total;
+    a.offsets[El] = total;
+    a.n_pad[0] = total;
+    *a.ticket = 0u;  // ready for the next call
+  }
+  for (int e = tid; e < El; e += kGcThreads) {
+    a.offsets[e] = s_off[e];
+    a.counts[e] = s_cnt[e];
+  }
+  __syncthreads();
+  for (int b = tid; b < a.NB; b += kGcThreads) {
+    const int64_t row = static_cast<int64_t>(b) * a.bs;
+    int e = -1;
+    if (row < total) {
+      int lo = 0, hi = El - 1;  // largest e with s_off[e] <= row (empty experts share offsets)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    a.expert_ids[b] = e;
+  }
+}
+
+// One warp per CTA: slots of tokens [t0, t0 + n) get their rows, the hidden rows are staged with
+// a bulk load and bulk-stored to every local row; then a share of the pad and tail rows.
+__global__ void __launch_bounds__(32)
+place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t row_bytes, int tpc,
+                    uint8_t* __restrict__ permuted) {
+  extern __shared__ __align__(128) uint8_t rows[];
+  __shared__ __align__(8) uint64_t bar;
+  const int lane = threadIdx.x;
+  const int k = a.k, El = a.E_local;
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * tpc;
+  const int64_t left = a.T - t0;
+  const int n = left <= 0 ? 0 : static_cast<int>(left < tpc ? left : tpc);
+  if (lane == 0) {
+    moe::mbar_init(&bar, 1);
+    moe::fence_barrier_init();
+  }
+  __syncwarp();
+  if (lane == 0 && n > 0) {  // hidden is an input of the call: complete before the previous kernel ran
+    moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
+    for (int i = 0; i < n; ++i) {
+      moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes, hidden + (t0 + i) * static_cast<int64_t>(row_bytes),
+                     row_bytes, &bar);
+    }
+  }
+  moe::pdl_launch_dependents();
+  moe::pdl_wait();  // ids, ranks, offsets and tile bases come from gate_count_kernel
+
+  const int nslots = n * k;  // <= kPgMaxTokens * 32
+  int32_t dst[kPgMaxTokens];
+#pragma unroll
+  for (int m = 0; m < kPgMaxTokens; ++m) {
+    const int e = lane + 32 * m;
+    int r = -1;
+    if (e < nslots) {
+      const int64_t s = t0 * k + e;
+      const int le = to_local(a, a.topk_ids[s]);
+      if (le >= 0) {
+        const int64_t tile = (t0 + e / k) / a.rows_per_tile;
+        r = a.offsets[le] + a.tile_counts[tile * El + le] + a.inv_perm[s];
+        if (r < 0 || static_cast<int64_t>(r) >= a.C) {  // cannot happen for consistent inputs
+          moe::record_status(a.status, MOE_ERR_BAD_ROW);
+          r = -1;
+        } else {
+          a.sorted_ids[r] = static_cast<int32_t>(s);
+          a.inv_perm[s] = r;
+        }
+      }
+    }
+    dst[m] = r;
+  }
+  if (n > 0) {
+    if (!moe::mbar_wait(&bar, 0)) {
+      moe::record_status(a.status, MOE_ERR_TIMEOUT);
+      moe::mbar_wait(&bar, 0);  // one more bounded wait for the loads in flight before leaving
+      return;
+    }
+#pragma unroll
+    for (int m = 0; m < kPgMaxTokens; ++m) {
+      const int e = lane + 32 * m;
+      if (e < nslots && dst[m] >= 0) {
+        moe::bulk_store(permuted + static_cast<int64_t>(dst[m]) * row_bytes,
+                        rows + static_cast<size_t>(e / k) * row_bytes, row_bytes);
+      }
+    }
+    moe::bulk_commit();
+  }
+  // pad rows of every expert and the tail past N_pad hold the pad value
+  const int32_t pad_value = static_cast<int32_t>(a.P);
+  const int npad = a.offsets[El];
+  for (int e = blockIdx.x; e < El; e += gridDim.x) {
+    const int p1 = a.offsets[e + 1];
+    for (int p = a.offsets[e] + a.counts[e] + lane; p < p1; p += 32) a.sorted_ids[p] = pad_value;
+  }
+  const int64_t tail = a.C - npad;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 32 + lane; i < tail; i += static_cast<int64_t>(gridDim.x) * 32)
+    a.sorted_ids[npad + i] = pad_value;
+  if (n > 0) moe::bulk_wait_read_all();  // the staged rows must outlive the stores that read them
+}
+
+using GcKernel = void (*)(DispatchArgs);
+
+template <typename TIn, int VEC, int CPL>
+GcKernel gc_instance() {
+  if constexpr (VEC * CPL <= 32) {
+    return &gate_count_kernel<TIn, VEC, CPL>;
+  } else {
+    return nullptr;
+  }
+}
+
+template <typename TIn, int VEC>
+GcKernel gc_pick_cpl(int cpl) {
+  switch (cpl) {
+    case 1: return gc_instance<TIn, VEC, 1>();
+    case 2: return gc_instance<TIn, VEC, 2>();
+    case 4: return gc_instance<TIn, VEC, 4>();
+    case 8: return gc_instance<TIn, VEC, 8>();
+    case 16: return gc_instance<TIn, VEC, 16>();
+    case 32: return gc_instance<TIn, VEC, 32>();
+    default: return nullptr;
+  }
+}
+
+template <typename TIn>
+GcKernel gc_pick(int vec, int cpl) {
+  if constexpr (sizeof(TIn) == 2) {
+    switch (vec) {
+      case 8: return gc_pick_cpl<TIn, 8>(cpl);
+      case 4: return gc_pick_cpl<TIn, 4>(cpl);
+      case 2: return gc_pick_cpl<TIn, 2>(cpl);
+      default: return gc_pick_cpl<TIn, 1>(cpl);
+    }
+  } else {
+    switch (vec) {
+      case 4: return gc_pick_cpl<TIn, 4>(cpl);
+      case 2: return gc_pick_cpl<TIn, 2>(cpl);
+      default: return gc_pick_cpl<TIn, 1>(cpl);
+    }
+  }
+}
+
+// Tokens per gating tile: 32, doubled (up to 512) while the tile counters would exceed 64K.
+int rows_per_tile_for(int64_t T, int E_local) {
+  int rt = 32;
+  while (rt < 512 && ((T + rt - 1) / rt) * E_local > kMaxTileCounters) rt *= 2;
+  return rt;
+}
+
+}  // namespace
+
+extern "C" size_t moe_route_dispatch_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
+  if (T < 0 || k < 1 || E_local < 1) return 0;
+  const int rt = rows_per_tile_for(T, E_local);
+  int64_t nt = (T + rt - 1) / rt;
+  if (nt < 1) nt = 1;
+  return kWsHeaderBytes + static_cast<size_t>(nt) * static_cast<size_t>(E_local) * sizeof(int32_t);
+}
+
+extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, const void* hidden, int64_t T,
+                                           int32_t E, int32_t k, int32_t H, uint32_t flags, const int32_t* expert_map,
+                                           int32_t E_local, int32_t block_size, float* topk_weights,
+                                           int32_t* topk_ids, int32_t* counts, int32_t* offsets,
+                                           int32_t* sorted_token_ids, int32_t* expert_ids,
+                                           int32_t* num_tokens_post_pad, int32_t* inv_perm, void* permuted,
+                                           void* workspace, size_t workspace_bytes, void* stream) {
+  if (T < 0 || E < 1 || k < 1 || k > E || H < 1 || E_local < 1 || block_size < 1) return MOE_ERR_INVALID_ARG;
+  if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~MOE_RENORMALIZE) != 0u) return MOE_ERR_INVALID_ARG;
+  if (E_local > E || (expert_map == nullptr && E_local != E)) return MOE_ERR_INVALID_ARG;
+  if (E > 1024 || k > 32 || E_local > 1024) return MOE_ERR_UNSUPPORTED;
+  if ((H % 8) != 0) return MOE_ERR_INVALID_ARG;
+  const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
+  if (row_bytes > 4u * kPgCtaBytes) return MOE_ERR_UNSUPPORTED;
+  const int64_t P = T * k;
+  if (T > (int64_t{1} << 40) || P >= (int64_t{1} << 30)) return MOE_ERR_INVALID_ARG;
+  const int64_t C = moe_align_capacity(T, k, E_local, block_size);
+  if (C < 0 || C >= (int64_t{1} << 31)) return MOE_ERR_INVALID_ARG;
+  if (counts == nullptr || offsets == nullptr || sorted_token_ids == nullptr || expert_ids == nullptr ||
+      num_tokens_post_pad == nullptr)
+    return MOE_ERR_INVALID_ARG;
+  if (T > 0 && (logits == nullptr || hidden == nullptr || topk_weights == nullptr || topk_ids == nullptr ||
+                inv_perm == nullptr || permuted == nullptr))
+    return MOE_ERR_INVALID_ARG;
+  if ((hidden && !moe_host::aligned16(hidden)) || (permuted && !moe_host::aligned16(permuted)))
+    return MOE_ERR_INVALID_ARG;
+  if (workspace == nullptr || workspace_bytes < moe_route_dispatch_workspace_bytes(T, k, E_local))
+    return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 15u) != 0) return MOE_ERR_INVALID_ARG;
+
+  DispatchArgs a{};
+  a.logits = logits;
+  a.T = T;
+  a.E = E;
+  a.k = k;
+  a.renormalize = (flags & MOE_RENORMALIZE) ? 1 : 0;
+  a.expert_map = expert_map;
+  a.E_local = E_local;
+  a.bs = block_size;
+  a.P = P;
+  a.C = C;
+  a.NB = static_cast<int>((C + block_size - 1) / block_size);
+  a.rows_per_tile = rows_per_tile_for(T, E_local);
+  const int64_t nt = (T + a.rows_per_tile - 1) / a.rows_per_tile;
+  a.num_tiles = nt < 1 ? 1 : static_cast<int>(nt);
+  a.topk_weights = topk_weights;
+  a.topk_ids = topk_ids;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.sorted_ids = sorted_token_ids;
+  a.expert_ids = expert_ids;
+  a.n_pad = num_tokens_post_pad;
+  a.inv_perm = inv_perm;
+  a.status = static_cast<int32_t*>(workspace);
+  a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 4);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kWsHeaderBytes);
+
+  // gating geometry: one warp per row, widest aligned vector that spreads the row over the warp
+  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  int vec_max = 16 / elem;
+  while (vec_max > 1 && ((E % vec_max) != 0 || (reinterpret_cast<uintptr_t>(logits) % (vec_max * elem)) != 0))
+    vec_max >>= 1;
+  int vec = 1;
+  for (int v = vec_max; v >= 1; v >>= 1) {
+    if ((E % v) == 0 && E / v >= 32) {
+      vec = v;
+      break;
+    }
+  }
+  if (E < 32) vec = 1;
+  const int n_chunks = E / vec;
+  int cpl = 1;
+  while (cpl * 32 < n_chunks) cpl <<= 1;
+  GcKernel gk = dtype == MOE_DTYPE_BF16 ? gc_pick<__nv_bfloat16>(vec, cpl) : gc_pick<float>(vec, cpl);
+  if (gk == nullptr) return MOE_ERR_UNSUPPORTED;
+
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
+  if (smem1 > 48 * 1024 &&
+      cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem1)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
+    return MOE_ERR_CUDA;
+
+  int tpc = static_cast<int>(kPgCtaBytes / row_bytes);
+  tpc = tpc < 1 ? 1 : (tpc > kPgMaxTokens ? kPgMaxTokens : tpc);
+  int64_t blocks = (T + tpc - 1) / tpc;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
+  const size_t smem2 = static_cast<size_t>(tpc) * row_bytes;
+  if (smem2 > 48 * 1024 &&
+      cudaFuncSetAttribute(place_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2)) !=
+          cudaSuccess)
+    return MOE_ERR_CUDA;
+  return moe_host::launch_pdl(place_gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st, a,
+                              static_cast<const uint8_t*>(hidden), row_bytes, tpc, static_cast<uint8_t*>(permuted));
+}

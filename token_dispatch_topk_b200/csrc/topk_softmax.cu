@@ -25,76 +25,14 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "gate_row.cuh"
 
 namespace {
 
+using namespace moe_gate;
+
 constexpr int kMaxWarps = 8;
 
-__device__ __forceinline__ uint32_t ordered_bits(float x) {
-  uint32_t u = __float_as_uint(x);
-  if ((u & 0x7fffffffu) == 0u) u = 0u;  // -0 and +0 compare equal
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ float ordered_to_float(uint32_t o) {
-  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
-}
-
-__device__ __forceinline__ uint64_t make_key(float x, int e) {
-  return (static_cast<uint64_t>(ordered_bits(x)) << 32) | static_cast<uint32_t>(0xffffffffu - static_cast<uint32_t>(e));
-}
-
-// Load VEC consecutive logits of a row as fp32.
-template <typename TIn, int VEC>
-struct VecLoad;
-
-template <>
-struct VecLoad<__nv_bfloat16, 8> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[8]) {
-    uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-    v[0] = moe::bf16_lo(u.x); v[1] = moe::bf16_hi(u.x); v[2] = moe::bf16_lo(u.y); v[3] = moe::bf16_hi(u.y);
-    v[4] = moe::bf16_lo(u.z); v[5] = moe::bf16_hi(u.z); v[6] = moe::bf16_lo(u.w); v[7] = moe::bf16_hi(u.w);
-  }
-};
-template <>
-struct VecLoad<__nv_bfloat16, 4> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[4]) {
-    uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
-    v[0] = moe::bf16_lo(u.x); v[1] = moe::bf16_hi(u.x); v[2] = moe::bf16_lo(u.y); v[3] = moe::bf16_hi(u.y);
-  }
-};
-template <>
-struct VecLoad<__nv_bfloat16, 2> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[2]) {
-    uint32_t u = __ldcs(reinterpret_cast<const unsigned int*>(p));
-    v[0] = moe::bf16_lo(u); v[1] = moe::bf16_hi(u);
-  }
-};
-template <>
-struct VecLoad<__nv_bfloat16, 1> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, float (&v)[1]) {
-    uint32_t u = __ldcs(reinterpret_cast<const unsigned short*>(p));
-    v[0] = moe::bf16_lo(u);
-  }
-};
-template <>
-struct VecLoad<float, 4> {
-  static __device__ __forceinline__ void run(const float* p, float (&v)[4]) {
-    float4 u = __ldcs(reinterpret_cast<const float4*>(p));
-    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
-  }
-};
-template <>
-struct VecLoad<float, 2> {
-  static __device__ __forceinline__ void run(const float* p, float (&v)[2]) {
-    float2 u = __ldcs(reinterpret_cast<const float2*>(p));
-    v[0] = u.x; v[1] = u.y;
-  }
-};
-template <>
-struct VecLoad<float, 1> {
-  static __device__ __forceinline__ void run(const float* p, float (&v)[1]) { v[0] = __ldcs(p); }
-};
 
 // One sub-warp of G = 2^g_log2 lanes per row; CPL vector chunks of VEC logits per lane.
 template <typename TIn, int VEC, int CPL>
@@ -195,165 +133,22 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
 // ------------------------------------------------------------------------------------------
 constexpr int kRowWarps = 4;
 
-__device__ __forceinline__ uint32_t ordered16(uint32_t b) {
-  b &= 0xffffu;
-  if ((b & 0x7fffu) == 0u) b = 0u;  // -0 == +0
-  return (b & 0x8000u) ? (~b & 0xffffu) : (b | 0x8000u);
-}
-
-__device__ __forceinline__ float ordered16_to_float(uint32_t o) {
-  const uint32_t b = (o & 0x8000u) ? (o & 0x7fffu) : (~o & 0xffffu);
-  return __uint_as_float(b << 16);
-}
-
-// Raw 16-bit patterns of VEC consecutive bf16 logits.
-template <int VEC>
-struct Bf16Bits;
-template <>
-struct Bf16Bits<8> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[8]) {
-    const uint4 u = __ldcs(reinterpret_cast<const uint4*>(p));
-    b[0] = u.x & 0xffffu; b[1] = u.x >> 16; b[2] = u.y & 0xffffu; b[3] = u.y >> 16;
-    b[4] = u.z & 0xffffu; b[5] = u.z >> 16; b[6] = u.w & 0xffffu; b[7] = u.w >> 16;
-  }
-};
-template <>
-struct Bf16Bits<4> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[4]) {
-    const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
-    b[0] = u.x & 0xffffu; b[1] = u.x >> 16; b[2] = u.y & 0xffffu; b[3] = u.y >> 16;
-  }
-};
-template <>
-struct Bf16Bits<2> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[2]) {
-    const uint32_t u = __ldcs(reinterpret_cast<const unsigned int*>(p));
-    b[0] = u & 0xffffu; b[1] = u >> 16;
-  }
-};
-template <>
-struct Bf16Bits<1> {
-  static __device__ __forceinline__ void run(const __nv_bfloat16* p, uint32_t (&b)[1]) {
-    b[0] = __ldcs(reinterpret_cast<const unsigned short*>(p));
-  }
-};
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
 
 template <typename TIn, int VEC, int CPL>
 __global__ void __launch_bounds__(kRowWarps * 32)
 topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int g_log2_unused, int renormalize,
                      float* __restrict__ topk_weights, int32_t* __restrict__ topk_ids) {
   (void)g_log2_unused;
-  constexpr int NV = CPL * VEC;
   const int lane = threadIdx.x & 31;
   moe::pdl_wait();  // the logits may come from the previous kernel (the router projection)
   moe::pdl_launch_dependents();
   const int64_t row = static_cast<int64_t>(blockIdx.x) * kRowWarps + (threadIdx.x >> 5);
   if (row >= T) return;  // uniform per warp
-  const int n_chunks = E / VEC;
-  const TIn* rp = logits + row * static_cast<int64_t>(E);
-  float m = 0.f, Z = 0.f, S = 0.f, my_p = 0.f;
-  int my_e = 0;
-
-  if constexpr (sizeof(TIn) == 2) {
-    uint32_t key[NV];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const int chunk = lane + 32 * c;
-      if (chunk < n_chunks) {
-        uint32_t b[VEC];
-        Bf16Bits<VEC>::run(rp + chunk * VEC, b);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = (ordered16(b[i]) << 16) | (0xffffu - static_cast<uint32_t>(chunk * VEC + i));
-      } else {
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0u;
-      }
-    }
-    uint32_t my_key = 0u, best0 = 0u;
-    for (int j = 0; j < k; ++j) {
-      uint32_t best = 0u;
-#pragma unroll
-      for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
-      best = __reduce_max_sync(0xffffffffu, best);
-      if (j == 0) {
-        best0 = best;
-        if (!renormalize) {  // full-row denominator, from the keys before any is retired
-          m = ordered16_to_float(best >> 16);
-          float z = 0.f;
-#pragma unroll
-          for (int i = 0; i < NV; ++i) {
-            if (key[i] != 0u) z += expf(ordered16_to_float(key[i] >> 16) - m);
-          }
-          Z = warp_sum(z);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0u : key[i];
-      if (lane == j) my_key = best;
-    }
-    m = ordered16_to_float(best0 >> 16);
-    if (lane < k) {
-      my_p = expf(ordered16_to_float(my_key >> 16) - m);
-      my_e = static_cast<int>(0xffffu - (my_key & 0xffffu));
-    }
-    if (renormalize) S = warp_sum(my_p);
-  } else {
-    uint64_t key[NV];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      const int chunk = lane + 32 * c;
-      if (chunk < n_chunks) {
-        float v[VEC];
-        VecLoad<TIn, VEC>::run(rp + chunk * VEC, v);
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = make_key(v[i], chunk * VEC + i);
-      } else {
-#pragma unroll
-        for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0ull;
-      }
-    }
-    uint64_t my_key = 0ull;
-    uint32_t hi0 = 0u;
-    for (int j = 0; j < k; ++j) {
-      uint64_t mine = 0ull;
-#pragma unroll
-      for (int i = 0; i < NV; ++i) mine = key[i] > mine ? key[i] : mine;
-      const uint32_t hi = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32));
-      const uint32_t lo = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32) == hi
-                                                             ? static_cast<uint32_t>(mine) : 0u);
-      const uint64_t best = (static_cast<uint64_t>(hi) << 32) | lo;
-      if (j == 0) {
-        hi0 = hi;
-        if (!renormalize) {
-          m = ordered_to_float(hi);
-          float z = 0.f;
-#pragma unroll
-          for (int i = 0; i < NV; ++i) {
-            if (key[i] != 0ull) z += expf(ordered_to_float(static_cast<uint32_t>(key[i] >> 32)) - m);
-          }
-          Z = warp_sum(z);
-        }
-      }
-#pragma unroll
-      for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
-      if (lane == j) my_key = best;
-    }
-    m = ordered_to_float(hi0);
-    if (lane < k) {
-      my_p = expf(ordered_to_float(static_cast<uint32_t>(my_key >> 32)) - m);
-      my_e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(my_key));
-    }
-    if (renormalize) S = warp_sum(my_p);
-  }
+  int my_e;
+  float my_w;
+  moe_gate::gate_row<TIn, VEC, CPL>(logits + row * static_cast<int64_t>(E), E, k, renormalize, lane, my_e, my_w);
   if (lane < k) {
-    const float den = renormalize ? S : Z;
-    topk_weights[row * k + lane] = my_p / den;
+    topk_weights[row * k + lane] = my_w;
     topk_ids[row * k + lane] = my_e;
   }
 }

@@ -31,6 +31,7 @@ class MoeRouter:
         self.align = B.alloc_align_outputs(T, k, self.E_local, block_size, self.device)
         self.capacity = self.align.capacity
         self.workspace = B.alloc_workspace(T, k, self.E_local, self.device)
+        self.dispatch_workspace = B.alloc_dispatch_workspace(T, k, self.E_local, self.device)
         self.permuted = torch.empty((self.capacity, H), dtype=torch.bfloat16, device=self.device)
         self.out = torch.empty((T, H), dtype=torch.bfloat16, device=self.device)
         # device-side inputs for the end-to-end path
@@ -56,8 +57,20 @@ class MoeRouter:
         return B.moe_combine(expert_out, w, self.align.inv_perm, self.out, device_status=self.workspace,
                              stream=stream)
 
+    def dispatch(self, logits: torch.Tensor, hidden: torch.Tensor, stream=None):
+        """gate + align + permute-gather through the fused entry point (two kernels)."""
+        return B.moe_route_dispatch(logits, hidden, self.k, self.renormalize, self.block_size, self.expert_map,
+                                    self.E_local, self.topk_weights, self.topk_ids, self.align, self.permuted,
+                                    self.dispatch_workspace, stream)
+
     def step(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
-        """gate + align + permute-gather + combine (expert_out stands in for the expert MLPs' output)."""
+        """gate + align + permute-gather (fused dispatch) + combine; expert_out stands in for the expert MLPs."""
+        self.dispatch(logits, hidden, stream)
+        return self.combine(expert_out, stream=stream)
+
+    def step_staged(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor,
+                    stream=None) -> torch.Tensor:
+        """The same step through the four stage entry points (four or five kernels)."""
         self.gate(logits, stream)
         self.align_permute(stream=stream)
         self.gather(hidden, stream, hidden_ready=True)  # hidden is an input of the step: ready before gating
@@ -77,5 +90,7 @@ class MoeRouter:
         return out_host
 
     def device_status(self, stream=None) -> int:
-        """Read and reset the device status word (synchronises)."""
-        return B.moe_read_status(self.workspace, stream)
+        """Read and reset the device status words of both paths (synchronises); the first error seen."""
+        a = B.moe_read_status(self.workspace, stream)
+        b = B.moe_read_status(self.dispatch_workspace, stream)
+        return a if a != B.MOE_OK else b
