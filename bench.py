@@ -39,13 +39,14 @@ UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = {
-    "topk_softmax_kernel": "token_dispatch_topk_b200/csrc/topk_softmax.cu",
-    "align_count_kernel+align_place_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
-    "gather_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
-    "combine_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
+    "topk_row_warp_kernel": "token_dispatch_topk_b200/csrc/topk_softmax.cu",
+    "align_cluster_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
+    "gather_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
+    "combine_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
+    "gate_count_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
 }
-STAGE_KERNEL = {"topk": "topk_softmax_kernel", "align": "align_count_kernel+align_place_kernel",
-                "gather": "gather_kernel", "combine": "combine_kernel"}
+STAGE_KERNEL = {"topk": "topk_row_warp_kernel", "align": "align_cluster_kernel", "gather": "gather_tma_kernel",
+                "combine": "combine_tma_kernel", "dispatch": "gate_count_kernel+place_gather_kernel"}
 
 
 def parse_args():
@@ -289,8 +290,9 @@ def main():
     R = int(r.align.counts.sum().item())
     npad = int(r.align.num_tokens_post_pad.item())
     NB = r.align.expert_ids.numel()
-    align_launches = 1 if tdt.moe_align_workspace_bytes(wl.T, wl.k, wl.experts_local) <= 256 else 2
-    launches_per_step = 1 + align_launches + 1 + 1
+    launches_per_step = 4  # topk_row_warp_kernel, align_cluster_kernel (or 2 tile kernels), gather, combine
+    if wl.T * wl.k > 65536 or wl.experts_local > 512:
+        launches_per_step = 5
 
     use_graph = not args.no_graph
     graphs = {}
@@ -350,45 +352,57 @@ def main():
 
     # ---- per-stage times inside the step, and roofline
     # The step is captured once more with external event records between its stages, so each
-    # stage is timed on the launching stream exactly as it runs inside a step (same flush protocol).
+    # stage is timed on the launching stream as it runs inside a step (same flush protocol).  The
+    # fused step has two stages (dispatch = gate_count + place_gather kernels, then combine); the
+    # four stage entry points are timed the same way for comparison.
     peak, peak_src = measured_peaks()
     abytes = algorithmic_bytes(wl, R, r.capacity, NB)
+    abytes["dispatch"] = abytes["topk"] + abytes["align"] + abytes["gather"]
     st_iters = args.stage_steps or min(args.steps, 500)
-    names = ("topk", "align", "gather", "combine")
-    marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
-    stage_calls = [lambda: r.gate(logits), lambda: r.align_permute(), lambda: r.gather(hidden), lambda: r.combine(y)]
 
-    def instrumented_step():
-        marks[0].record()
-        for i, fn in enumerate(stage_calls):
-            fn()
-            marks[i + 1].record()
+    def stage_times(names, calls):
+        marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
 
-    if use_graph:
-        g_inst = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_inst, stream=stream):
-            instrumented_step()
-    sums = [0.0] * len(names)
-    with torch.cuda.stream(stream):
-        for i in range(min(args.warmup, 10) + st_iters):
-            flush(i)
-            if use_graph:
-                g_inst.replay()
-            else:
-                instrumented_step()
-            stream.synchronize()
-            if i >= min(args.warmup, 10):
-                for j in range(len(names)):
-                    sums[j] += marks[j].elapsed_time(marks[j + 1])
-    stages = {}
-    for j, name in enumerate(names):
-        ms = sums[j] / st_iters
-        stages[name] = {"us": 1e3 * ms, "algorithmic_bytes": abytes[name],
-                        "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": STAGE_KERNEL[name],
-                        "timing": "CUDA events between the stages of the step graph"}
-    dom = max(("gather", "combine"), key=lambda s: stages[s]["us"])
+        def instrumented():
+            marks[0].record()
+            for i, fn in enumerate(calls):
+                fn()
+                marks[i + 1].record()
+
+        if use_graph:
+            g_inst = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_inst, stream=stream):
+                instrumented()
+        sums = [0.0] * len(names)
+        warm = min(args.warmup, 10)
+        with torch.cuda.stream(stream):
+            for i in range(warm + st_iters):
+                flush(i)
+                if use_graph:
+                    g_inst.replay()
+                else:
+                    instrumented()
+                stream.synchronize()
+                if i >= warm:
+                    for j in range(len(names)):
+                        sums[j] += marks[j].elapsed_time(marks[j + 1])
+        if use_graph:
+            del g_inst
+        out = {}
+        for j, name in enumerate(names):
+            ms = sums[j] / st_iters
+            out[name] = {"us": 1e3 * ms, "algorithmic_bytes": abytes[name],
+                         "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": STAGE_KERNEL[name],
+                         "timing": "CUDA events between the stages of the step graph"}
+        return out
+
+    stages = stage_times(("topk", "align", "gather", "combine"),
+                         [lambda: r.gate(logits), lambda: r.align_permute(),
+                          lambda: r.gather(hidden, hidden_ready=True), lambda: r.combine(y)])
+    stages_fused = stage_times(("dispatch", "combine"), [lambda: r.dispatch(logits, hidden), lambda: r.combine(y)])
+    dom = "combine"  # the dominant single kernel of the step (about half of its bytes)
     ach = stages[dom]["achieved_gbs"]
-    total_bytes = sum(abytes.values())
+    total_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
     roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": ncu_traffic(STAGE_KERNEL[dom], wl.name), "kernel": STAGE_KERNEL[dom],
                 "peak_source": peak_src,
@@ -441,14 +455,13 @@ def main():
             "algorithmic_bytes_per_step": total_bytes,
             "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
             "routed_slots_local": R, "num_tokens_post_pad": npad,
-            "roofline": roofline, "stages": stages, "e2e": e2e, "cpu_baseline": cpu,
+            "roofline": roofline, "stages": stages, "stages_fused_dispatch_path": stages_fused, "e2e": e2e,
+            "cpu_baseline": cpu,
             "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
     del graphs
-    if use_graph:
-        del g_inst
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -64,7 +64,7 @@ def _check_all(r, wl, ref, what, y, y_bits):
 
 
 def _run(r, path, logits, hidden, y):
-    return r.step(logits, hidden, y) if path == "fused" else r.step_staged(logits, hidden, y)
+    return r.step_fused(logits, hidden, y) if path == "fused" else r.step(logits, hidden, y)
 
 
 @pytest.mark.parametrize("path", ["fused", "staged"])
@@ -173,7 +173,7 @@ def test_repeat_steps_are_bit_identical():
     r = _router(wl, dev)
     first = None
     for i in range(6):
-        (r.step if i % 2 == 0 else r.step_staged)(logits, hidden, y)
+        (r.step if i % 2 == 0 else r.step_fused)(logits, hidden, y)
         snap = [t.clone() for t in (r.topk_ids, r.topk_weights, r.align.sorted_token_ids, r.align.inv_perm,
                                     r.align.expert_ids, r.out)]
         if first is None:

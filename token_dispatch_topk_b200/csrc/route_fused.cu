@@ -15,11 +15,14 @@
 //      it into its own shared-memory row, the rows are scanned across warps, and each slot's rank
 //      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm and the
 //      tile's per-expert counts go to the workspace;
-//   C. the CTA that finishes last (completion ticket, no spinning) scans the tile counts per
-//      expert into per-tile bases, writes counts, the block-padded offsets, N_pad and expert_ids,
-//      and resets the ticket.
+//   C. two-level scan with completion tickets (no spinning): the CTA that finishes last in its
+//      group of tiles scans the group's tile counters (staged through shared memory) into bases
+//      inside the group and publishes the group totals; the group that finishes last scans the
+//      group totals into group bases and writes counts, the block-padded offsets, N_pad and
+//      expert_ids.  Every ticket is reset by the CTA that used it last.
 // place_gather_kernel (one warp per CTA, up to 8 tokens, TMA staging as in gather_tma_kernel):
-//   each slot's row = offsets[e] + tile base[e] + rank; the CTA writes sorted_token_ids and
+//   each slot's row = offsets[e] + group base[e] + tile base[e] + rank (the rank and the expert
+//   were parked in inv_perm by the first kernel); the CTA writes sorted_token_ids and
 //   inv_perm for its slots, bulk-loads its hidden rows (before waiting for the previous kernel:
 //   hidden is an input of the call) and bulk-stores them to their rows; the pad rows, the tail
 //   rows past N_pad are spread over the CTAs.
@@ -35,7 +38,8 @@ namespace {
 constexpr int kGcWarps = 16;
 constexpr int kGcThreads = kGcWarps * 32;
 constexpr int kWsHeaderBytes = 256;  // status word, ticket, padding
-constexpr int64_t kMaxTileCounters = 65536;
+constexpr int kRowsPerTile = 32;
+constexpr int kScanCap = 16384;  // ints of shared memory for staging a block of tile counters
 constexpr int kPgMaxTokens = 8;
 constexpr uint32_t kPgCtaBytes = 32u * 1024u;
 
@@ -63,7 +67,11 @@ struct DispatchArgs {
   int32_t* inv_perm;
   int32_t* status;
   unsigned int* ticket;
-  int32_t* tile_counts;  // [num_tiles][E_local]: tile counts, then per-tile bases
+  int32_t* tile_counts;         // [num_tiles][E_local]: tile counts, then bases inside the group
+  int tiles_per_group;
+  int num_groups;
+  unsigned int* group_tickets;  // [num_groups]
+  int32_t* group_counts;        // [num_groups][E_local]: group totals, then group bases
 };
 
 // Local expert of global expert g (or -1: remote); out-of-range values are flagged.
@@ -126,10 +134,61 @@ __device__ int scan_block(int* data, int n, int* warp_sums) {
 }
 
 // Shared memory of gate_count_kernel (ints):
-//   s_le[rows_per_tile * k] | whist[kGcWarps][E_local] | masks[kGcWarps][E_local]
-//   | s_cnt[E_local] | s_off[E_local + 1] | warp_sums[32]
+//   s_le[rows_per_tile * k] | work region: whist[kGcWarps][E_local] + masks[kGcWarps][E_local],
+//   later the staging buffer of the tile-counter scans | s_cnt[E_local] | s_off[E_local + 1] | warp_sums[32]
+__host__ __device__ inline size_t gc_work_ints(int E_local) {
+  const size_t w = 2 * static_cast<size_t>(kGcWarps) * E_local;
+  return w > static_cast<size_t>(kScanCap) ? w : static_cast<size_t>(kScanCap);
+}
 __host__ __device__ inline size_t gc_smem_ints(int rows_per_tile, int k, int E_local) {
-  return static_cast<size_t>(rows_per_tile) * k + 2 * static_cast<size_t>(kGcWarps) * E_local + 2 * E_local + 1 + 32;
+  return static_cast<size_t>(rows_per_tile) * k + gc_work_ints(E_local) + 2 * E_local + 1 + 32;
+}
+
+// In-place exclusive scan down the rows of a rows x cols int32 block in global memory (row
+// stride `cols`), column by column; column totals to `totals`.  The block is staged through
+// `buf` (cap ints of shared memory) in slices of columns, with coalesced, batched loads.
+// Block-wide (kGcThreads threads).
+__device__ void scan_columns(int32_t* g, int rows, int cols, int* buf, int cap, int* totals) {
+  const int tid = threadIdx.x;
+  int ec = cap / (rows > 0 ? rows : 1);
+  if (ec > cols) ec = cols;
+  if (ec < 1) ec = 1;
+  for (int c0 = 0; c0 < cols; c0 += ec) {
+    const int w = (cols - c0) < ec ? (cols - c0) : ec;
+    const int n = rows * w;
+    for (int i0 = tid; i0 < n; i0 += kGcThreads * 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kGcThreads;
+        if (i < n) {
+          const int r = i / w;
+          v[u] = __ldcg(g + static_cast<int64_t>(r) * cols + c0 + (i - r * w));
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = i0 + u * kGcThreads;
+        if (i < n) buf[i] = v[u];
+      }
+    }
+    __syncthreads();
+    for (int j = tid; j < w; j += kGcThreads) {
+      int run = 0;
+      for (int r = 0; r < rows; ++r) {
+        const int x = buf[r * w + j];
+        buf[r * w + j] = run;
+        run += x;
+      }
+      totals[c0 + j] = run;
+    }
+    __syncthreads();
+    for (int i = tid; i < n; i += kGcThreads) {
+      const int r = i / w;
+      g[static_cast<int64_t>(r) * cols + c0 + (i - r * w)] = buf[i];
+    }
+    __syncthreads();
+  }
 }
 
 template <typename TIn, int VEC, int CPL>
@@ -139,7 +198,9 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   int* s_le = smem;
   int* whist = s_le + RT * k;
   unsigned* masks = reinterpret_cast<unsigned*>(whist + kGcWarps * El);
-  int* s_cnt = reinterpret_cast<int*>(masks + kGcWarps * El);
+  int* work = whist;  // whist + masks, reused as the scan staging buffer
+  const int work_cap = static_cast<int>(gc_work_ints(El));
+  int* s_cnt = work + work_cap;
   int* s_off = s_cnt + El;
   int* warp_sums = s_off + El + 1;
   __shared__ int s_is_last;
@@ -201,7 +262,8 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
     const int le = i < nslots ? s_le[i] : -1;
     const unsigned peers = peers_of(my_masks, le, lane);
     if (le >= 0) {
-      a.inv_perm[row0 * k + i] = my_hist[le] + __popc(peers & moe::lanemask_lt());  // rank in the tile
+      // parked until place_gather_kernel: (rank in the tile) << 10 | local expert
+      a.inv_perm[row0 * k + i] = ((my_hist[le] + __popc(peers & moe::lanemask_lt())) << 10) | le;
     } else if (i < nslots) {
       a.inv_perm[row0 * k + i] = -1;
     }
@@ -210,41 +272,28 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
     __syncwarp();
   }
 
-  // C. the last CTA turns the tile counts into per-tile bases and writes the expert layout
+  // C. two-level scan of the tile counters.  The last CTA of each group of tiles turns the group's
+  //    tile counts into bases inside the group and publishes the group totals; the last group
+  //    to finish turns the group totals into group bases and writes the expert layout.
   __threadfence();
   __syncthreads();
-  if (tid == 0) s_is_last = (atomicAdd(a.ticket, 1u) == static_cast<unsigned>(a.num_tiles - 1)) ? 1 : 0;
+  const int grp = tile / a.tiles_per_group;
+  const int g0 = grp * a.tiles_per_group;
+  const int gt = (a.num_tiles - g0) < a.tiles_per_group ? (a.num_tiles - g0) : a.tiles_per_group;
+  if (tid == 0) s_is_last = (atomicAdd(&a.group_tickets[grp], 1u) == static_cast<unsigned>(gt - 1)) ? 1 : 0;
   __syncthreads();
   if (!s_is_last) return;
   __threadfence();
-  int parts = 1;  // threads sharing one expert column, each scanning a contiguous range of tiles
-  while (parts * 2 * El <= kGcThreads && parts * 2 <= 32) parts *= 2;
-  const int per = (a.num_tiles + parts - 1) / parts;
-  const int part = tid % parts;
-  const int t0 = part * per;
-  const int t1 = (t0 + per < a.num_tiles) ? t0 + per : a.num_tiles;
-  for (int e0 = 0; e0 < El; e0 += kGcThreads / parts) {  // uniform trip count
-    const int e = e0 + tid / parts;
-    int sum = 0;
-    if (e < El) {
-      for (int t = t0; t < t1; ++t) sum += __ldcg(a.tile_counts + static_cast<int64_t>(t) * El + e);
-    }
-    int incl = sum;
-    for (int off = 1; off < parts; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off, parts);
-      if (part >= off) incl += v;
-    }
-    if (e < El) {
-      int run = incl - sum;
-      for (int t = t0; t < t1; ++t) {
-        int32_t* p = a.tile_counts + static_cast<int64_t>(t) * El + e;
-        const int c = __ldcg(p);
-        *p = run;
-        run += c;
-      }
-      if (part == parts - 1) s_cnt[e] = run;
-    }
-  }
+  scan_columns(a.tile_counts + static_cast<int64_t>(g0) * El, gt, El, work, work_cap, s_cnt);
+  for (int e = tid; e < El; e += kGcThreads) a.group_counts[static_cast<int64_t>(grp) * El + e] = s_cnt[e];
+  if (tid == 0) a.group_tickets[grp] = 0u;  // ready for the next call
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) s_is_last = (atomicAdd(a.ticket, 1u) == static_cast<unsigned>(a.num_groups - 1)) ? 1 : 0;
+  __syncthreads();
+  if (!s_is_last) return;
+  __threadfence();
+  scan_columns(a.group_counts, a.num_groups, El, work, work_cap, s_cnt);
   __syncthreads();
   for (int e = tid; e < El; e += kGcThreads) s_off[e] = ((s_cnt[e] + a.bs - 1) / a.bs) * a.bs;
   __syncthreads();
@@ -310,10 +359,12 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     int r = -1;
     if (e < nslots) {
       const int64_t s = t0 * k + e;
-      const int le = to_local(a, a.topk_ids[s]);
-      if (le >= 0) {
+      const int v = a.inv_perm[s];  // (rank in the tile) << 10 | local expert, or -1
+      if (v >= 0) {
+        const int le = v & 1023;
         const int64_t tile = (t0 + e / k) / a.rows_per_tile;
-        r = a.offsets[le] + a.tile_counts[tile * El + le] + a.inv_perm[s];
+        const int64_t grp = tile / a.tiles_per_group;
+        r = a.offsets[le] + a.group_counts[grp * El + le] + a.tile_counts[tile * El + le] + (v >> 10);
         if (r < 0 || static_cast<int64_t>(r) >= a.C) {  // cannot happen for consistent inputs
           moe::record_status(a.status, MOE_ERR_BAD_ROW);
           r = -1;
@@ -396,21 +447,35 @@ GcKernel gc_pick(int vec, int cpl) {
   }
 }
 
-// Tokens per gating tile: 32, doubled (up to 512) while the tile counters would exceed 64K.
-int rows_per_tile_for(int64_t T, int E_local) {
-  int rt = 32;
-  while (rt < 512 && ((T + rt - 1) / rt) * E_local > kMaxTileCounters) rt *= 2;
-  return rt;
+// Tiles per group: a group's block of tile counters fits the shared-memory scan buffer.
+int tiles_per_group_for(int E_local) {
+  int g = kScanCap / E_local;
+  return g < 2 ? 2 : (g > 64 ? 64 : g);
+}
+
+struct FusedLayout {
+  int num_tiles, tiles_per_group, num_groups;
+  size_t group_tickets_off, tile_counts_off, group_counts_off, bytes;
+};
+
+FusedLayout fused_layout(int64_t T, int E_local) {
+  FusedLayout l{};
+  const int64_t nt = (T + kRowsPerTile - 1) / kRowsPerTile;
+  l.num_tiles = nt < 1 ? 1 : static_cast<int>(nt);
+  l.tiles_per_group = tiles_per_group_for(E_local);
+  l.num_groups = (l.num_tiles + l.tiles_per_group - 1) / l.tiles_per_group;
+  l.group_tickets_off = kWsHeaderBytes;
+  l.tile_counts_off = l.group_tickets_off + ((static_cast<size_t>(l.num_groups) * 4 + 255) & ~size_t{255});
+  l.group_counts_off = l.tile_counts_off + static_cast<size_t>(l.num_tiles) * E_local * 4;
+  l.bytes = l.group_counts_off + static_cast<size_t>(l.num_groups) * E_local * 4;
+  return l;
 }
 
 }  // namespace
 
 extern "C" size_t moe_route_dispatch_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
   if (T < 0 || k < 1 || E_local < 1) return 0;
-  const int rt = rows_per_tile_for(T, E_local);
-  int64_t nt = (T + rt - 1) / rt;
-  if (nt < 1) nt = 1;
-  return kWsHeaderBytes + static_cast<size_t>(nt) * static_cast<size_t>(E_local) * sizeof(int32_t);
+  return fused_layout(T, E_local).bytes;
 }
 
 extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, const void* hidden, int64_t T,
@@ -456,9 +521,11 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.P = P;
   a.C = C;
   a.NB = static_cast<int>((C + block_size - 1) / block_size);
-  a.rows_per_tile = rows_per_tile_for(T, E_local);
-  const int64_t nt = (T + a.rows_per_tile - 1) / a.rows_per_tile;
-  a.num_tiles = nt < 1 ? 1 : static_cast<int>(nt);
+  const FusedLayout lay = fused_layout(T, E_local);
+  a.rows_per_tile = kRowsPerTile;
+  a.num_tiles = lay.num_tiles;
+  a.tiles_per_group = lay.tiles_per_group;
+  a.num_groups = lay.num_groups;
   a.topk_weights = topk_weights;
   a.topk_ids = topk_ids;
   a.counts = counts;
@@ -469,7 +536,9 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.inv_perm = inv_perm;
   a.status = static_cast<int32_t*>(workspace);
   a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 4);
-  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kWsHeaderBytes);
+  a.group_tickets = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + lay.group_tickets_off);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.tile_counts_off);
+  a.group_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.group_counts_off);
 
   // gating geometry: one warp per row, widest aligned vector that spreads the row over the warp
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;

@@ -64,17 +64,21 @@ class MoeRouter:
                                     self.dispatch_workspace, stream)
 
     def step(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
-        """gate + align + permute-gather (fused dispatch) + combine; expert_out stands in for the expert MLPs."""
-        self.dispatch(logits, hidden, stream)
-        return self.combine(expert_out, stream=stream)
-
-    def step_staged(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor,
-                    stream=None) -> torch.Tensor:
-        """The same step through the four stage entry points (four or five kernels)."""
+        """gate + align + permute-gather + combine through the four stage entry points (the fastest
+        path measured); expert_out stands in for the expert MLPs' output."""
         self.gate(logits, stream)
         self.align_permute(stream=stream)
         self.gather(hidden, stream, hidden_ready=True)  # hidden is an input of the step: ready before gating
         return self.combine(expert_out, stream=stream)
+
+    def step_fused(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor,
+                   stream=None) -> torch.Tensor:
+        """The same step with gating + align + gather fused into moe_route_dispatch (two kernels)."""
+        self.dispatch(logits, hidden, stream)
+        return self.combine(expert_out, stream=stream)
+
+    # the four-call path under its own name as well
+    step_staged = step
 
     def step_from_host(self, logits_host: torch.Tensor, hidden_host: torch.Tensor, expert_out: torch.Tensor,
                        out_host: torch.Tensor, stream=None) -> torch.Tensor:
