@@ -344,10 +344,10 @@ __global__ void __launch_bounds__(kAlignThreads) align_place_kernel(AlignArgs a)
 // which spread over every SM).  Global warp g = rank*32 + w owns the slot run [g*run, (g+1)*run).
 //   1. every warp counts its run into its own shared-memory row (shared atomics; the ids of up
 //      to 8 chunks are loaded at once and their experts kept for step 5);
-//   2. per expert, the CTA turns its warp rows into exclusive prefixes and writes its total to
-//      row `rank` of a table in the workspace;
-//   3. cluster barrier (release/acquire at cluster scope); each CTA scans the table: the sum
-//      over lower ranks is its base, the sum over all ranks is the expert's count;
+//   2. per expert, the CTA turns its warp rows into exclusive prefixes and its CTA total;
+//   3. every CTA pushes its totals into row `rank` of a table in the shared memory of every CTA
+//      (16-byte st.shared::cluster stores); cluster barrier; each CTA scans its own table: the
+//      sum over lower ranks is its base, the sum over all ranks is the expert's count;
 //   4. block-padded offsets (each CTA computes them; rank 0 writes counts/offsets/N_pad);
 //   5. every warp walks its run again and places its slots in order (peer masks from shared
 //      memory, rank = earlier peers in the chunk);
@@ -396,6 +396,9 @@ __device__ int block_exclusive_scan_1024(int* data, int n, int* warp_sums) {
 // expert column of 32 rows hit 32 different banks.
 __host__ __device__ inline int warp_row_stride(int E_local) { return E_local | 1; }
 
+// Row length of the cluster totals table: a multiple of 4 ints (16-byte rows for vector stores).
+__host__ __device__ inline int table_row_ints(int E_local) { return (E_local + 3) & ~3; }
+
 constexpr int kAlignBatch = 8;  // 32-slot chunks whose ids a warp loads at once
 
 // Local experts of one batch of a warp's run: slot base + 32*b + lane for b < kAlignBatch.  All
@@ -436,11 +439,13 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
   extern __shared__ int smem[];
   int* whist = smem;                                                          // [32][ES] counts, then prefixes
   unsigned* masks = reinterpret_cast<unsigned*>(whist + kClusterWarps * ES);  // [32][El] peer masks
-  int* s_cnt = reinterpret_cast<int*>(masks + kClusterWarps * El);            // [El] cluster counts
-  int* s_off = s_cnt + El;                                                    // [El+1] padded offsets
-  int* s_base = s_off + El + 1;                                               // [El] this CTA's first rows
-  int* warp_sums = s_base + El;                                               // [32]
-  int32_t* gtable = a.tile_counts;  // [nc][El] in the workspace: every CTA's totals
+  const int E4 = table_row_ints(El);
+  int* table = reinterpret_cast<int*>(masks + kClusterWarps * El);  // [kMaxClusterCtas][E4] totals of every rank
+  int* cta_cnt = table + kMaxClusterCtas * E4;                      // [E4] this CTA's totals
+  int* s_cnt = cta_cnt + E4;                                        // [El] cluster counts
+  int* s_off = s_cnt + El;                                          // [El+1] padded offsets
+  int* s_base = s_off + El + 1;                                     // [El] this CTA's first rows
+  int* warp_sums = s_base + El;                                     // [32]
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int64_t g = static_cast<int64_t>(rank) * kClusterWarps + warp;
@@ -452,6 +457,7 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
 
   for (int i = tid; i < kClusterWarps * ES; i += kClusterThreads) whist[i] = 0;
   for (int i = tid; i < kClusterWarps * El; i += kClusterThreads) masks[i] = 0u;
+  for (int i = El + tid; i < E4; i += kClusterThreads) cta_cnt[i] = 0;
   __syncthreads();
   moe::pdl_wait();  // topk_ids come from the previous kernel
   moe::pdl_launch_dependents();
@@ -465,8 +471,7 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
     }
   }
   __syncthreads();
-  // 2. per expert, exclusive prefix over this CTA's 32 warps (lane = warp index); the CTA total
-  //    goes to row `rank` of the cluster table
+  // 2. per expert, exclusive prefix over this CTA's 32 warps (lane = warp index) and the CTA total
   for (int e0 = warp; e0 < El; e0 += 4 * kClusterWarps) {
     int c[4], incl[4];
 #pragma unroll
@@ -488,24 +493,30 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
       const int e = e0 + q * kClusterWarps;
       if (e < El) {
         whist[lane * ES + e] = incl[q] - c[q];
-        if (lane == 31 && nc > 1) gtable[static_cast<int64_t>(rank) * El + e] = incl[q];
-        if (nc == 1 && lane == 31) {
-          s_base[e] = 0;
-          s_cnt[e] = incl[q];
-        }
+        if (lane == 31) cta_cnt[e] = incl[q];
       }
     }
   }
-  // 3. after the cluster barrier (release/acquire at cluster scope), each CTA scans the table:
-  //    lane = rank; the sum over lower ranks is its base, the sum over all ranks the count
+  // 3. every CTA pushes its totals into row `rank` of the table of every CTA of the cluster
+  //    (16-byte stores into distributed shared memory); after the cluster barrier each CTA scans
+  //    its own table with lane = rank: the sum over lower ranks is its base, the sum over all
+  //    ranks the count.  No CTA touches another's shared memory after that barrier.
+  __syncthreads();
   if (nc > 1) {
+    const int q4 = E4 / 4;
+    for (int i = tid; i < nc * q4; i += kClusterThreads) {
+      const int dst = i / q4;
+      const int q = i - dst * q4;
+      const uint4 v = *reinterpret_cast<const uint4*>(cta_cnt + 4 * q);
+      moe::st_cluster_v4(table + rank * E4 + 4 * q, static_cast<uint32_t>(dst), v);
+    }
     cluster.sync();
     for (int e0 = warp; e0 < El; e0 += 4 * kClusterWarps) {
       int c[4], incl[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int e = e0 + q * kClusterWarps;
-        c[q] = (e < El && lane < nc) ? __ldcg(gtable + static_cast<int64_t>(lane) * El + e) : 0;
+        c[q] = (e < El && lane < nc) ? table[lane * E4 + e] : 0;
         incl[q] = c[q];
       }
 #pragma unroll
@@ -527,6 +538,11 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
         }
       }
     }
+  } else {
+    for (int e = tid; e < El; e += kClusterThreads) {
+      s_base[e] = 0;
+      s_cnt[e] = cta_cnt[e];
+    }
   }
   __syncthreads();
   // 4. block-padded offsets
@@ -545,8 +561,10 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
   // 5. placement in slot order
   for (int64_t base = w0; base < w1; base += 32 * kAlignBatch) {
     if (!one_batch) load_batch(a, base, w1, lane, le);
+    const int nb = static_cast<int>((w1 - base + 31) / 32);  // chunks of this batch that hold slots
 #pragma unroll
     for (int b = 0; b < kAlignBatch; ++b) {
+      if (b >= nb) break;  // uniform over the warp
       const int64_t s = base + 32 * b + lane;
       const unsigned peers = peers_smem(my_masks, le[b], lane);
       if (le[b] >= 0) {
@@ -587,8 +605,9 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
 }
 
 __host__ inline size_t align_cluster_smem_bytes(int E_local) {
+  const int E4 = table_row_ints(E_local);
   return (static_cast<size_t>(kClusterWarps) * warp_row_stride(E_local) + static_cast<size_t>(kClusterWarps) * E_local +
-          3 * static_cast<size_t>(E_local) + 1 + 32) *
+          static_cast<size_t>(kMaxClusterCtas + 1) * E4 + 3 * static_cast<size_t>(E_local) + 1 + 32) *
          sizeof(int);
 }
 

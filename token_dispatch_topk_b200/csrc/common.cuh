@@ -100,19 +100,6 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return done != 0u;
 }
 
-// try_wait that may suspend the thread for up to `hint_ns` while the phase is incomplete.
-__device__ __forceinline__ bool mbar_try_wait_hint(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
-  uint32_t done;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(done)
-      : "r"(smem_addr(bar)), "r"(parity), "r"(hint_ns)
-      : "memory");
-  return done != 0u;
-}
-
 __device__ __forceinline__ uint64_t global_ns() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
@@ -121,12 +108,17 @@ __device__ __forceinline__ uint64_t global_ns() {
 
 // Bounded wait for the phase with the given parity: false if it has not completed after about
 // two seconds (every wait in this library completes in microseconds when the GPU is healthy).
+// Between polls the warp sleeps (__nanosleep, 32 ns doubling to 256 ns) so that waiting warps
+// take no issue slots from the warps doing the work.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
+  unsigned sleep_ns = 32;
   for (;;) {
-    if (mbar_try_wait_hint(bar, parity, 20000u)) return true;
+    __nanosleep(sleep_ns);
+    if (mbar_try_wait(bar, parity)) return true;
+    if (sleep_ns < 256) sleep_ns <<= 1;
     if (global_ns() - t0 > kWaitLimitNs) return false;
   }
 }
@@ -198,6 +190,14 @@ __device__ __forceinline__ void st_cluster_u32(const void* local_ptr, uint32_t r
   uint32_t raddr;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_addr(local_ptr)), "r"(rank));
   asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(raddr), "r"(v) : "memory");
+}
+
+// Store 16 bytes into the same shared-memory location of CTA `rank` of this cluster.
+__device__ __forceinline__ void st_cluster_v4(const void* local_ptr, uint32_t rank, const uint4& v) {
+  uint32_t raddr;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(raddr) : "r"(smem_addr(local_ptr)), "r"(rank));
+  asm volatile("st.shared::cluster.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(raddr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 }  // namespace moe

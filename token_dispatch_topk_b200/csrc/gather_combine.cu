@@ -185,9 +185,9 @@ struct CombineArgs {
 // of every local slot row of the unit into a stage of a shared-memory ring (mbarrier `full`), with
 // the slot weights and a validity mask beside it; one consumer thread waits for the stage and the
 // consumer warps are released together by a named barrier (waiting warps take no issue slots).
-// Consumers accumulate in fp32 (packed f32x2 fused multiply-adds: two independent correctly
-// rounded fmas, ascending slot order, from +0), store the bf16 result and release the stage
-// (mbarrier `empty`, one arrival per consumer warp).
+// Consumers accumulate in fp32 (fmaf, ascending slot order, from +0), store the bf16 result and
+// release the stage (mbarrier `empty`, one arrival per consumer warp).
+template <int KU>  // slot loop unrolled KU times (k rounded up to 2, 4 or 8; blocks of 8 beyond)
 __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_kernel(CombineArgs a) {
   extern __shared__ __align__(128) uint8_t smem[];
   const int k = a.k;
@@ -195,8 +195,8 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
   const int spu = a.tpu * k;  // slot rows per unit (<= 32)
   const uint32_t stage_bytes = static_cast<uint32_t>(spu) * a.chunk_bytes;
   uint8_t* buf = smem;
-  uint64_t* s_w2 = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(S) * stage_bytes);  // [S][32] {w, w}
-  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_w2 + S * 32);                              // [S]
+  float* s_w = reinterpret_cast<float*>(smem + static_cast<size_t>(S) * stage_bytes);  // [S][32] slot weights
+  uint32_t* s_mask = reinterpret_cast<uint32_t*>(s_w + S * 32);                          // [S]
   uint64_t* full = reinterpret_cast<uint64_t*>((reinterpret_cast<uintptr_t>(s_mask + S) + 7) & ~uintptr_t(7));
   uint64_t* empty = full + S;
   __shared__ int s_abort;
@@ -258,7 +258,7 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
       }
       const uint32_t mask = __ballot_sync(0xffffffffu, r_cur >= 0);
       const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
-      s_w2[s * 32 + lane] = moe::f32x2(w_cur, w_cur);
+      s_w[s * 32 + lane] = w_cur;
       if (lane == 0) s_mask[s] = mask;
       __threadfence_block();
       __syncwarp();
@@ -303,42 +303,44 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
     const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
     const uint32_t mask = s_mask[s];
     const uint8_t* stage = buf + static_cast<size_t>(s) * stage_bytes;
-    const uint64_t* w2 = s_w2 + s * 32;
     const int nvec = static_cast<int>(cb >> 4);
-    for (int item = ct; item < a.tpu * nvec; item += NCT) {
-      const int ti = item / nvec;
-      const int v = item - ti * nvec;
+    for (int ti = 0; ti < a.tpu; ++ti) {
       const int64_t t = grp * a.tpu + ti;
-      if (t >= a.T) break;  // items are in token order
-      uint64_t acc01 = 0ull, acc23 = 0ull, acc45 = 0ull, acc67 = 0ull;  // +0.0f pairs
-      const uint8_t* col = stage + static_cast<size_t>(ti) * k * a.chunk_bytes + static_cast<size_t>(v) * 16;
+      if (t >= a.T) break;
       const uint32_t tmask = mask >> (ti * k);
-      for (int j0 = 0; j0 < k; j0 += 8) {
+      const uint8_t* tok = stage + static_cast<size_t>(ti) * k * a.chunk_bytes;
+      const float* wt = s_w + s * 32 + ti * k;
+      uint8_t* dst = a.out + t * static_cast<int64_t>(a.row_bytes) + static_cast<int64_t>(c) * a.chunk_bytes;
+      for (int v = ct; v < nvec; v += NCT) {
+        float acc[8];
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        const uint8_t* col = tok + static_cast<size_t>(v) * 16;
+        for (int j0 = 0; j0 < k; j0 += KU) {
+#pragma unroll
+        for (int jj = 0; jj < KU; ++jj) {
           const int j = j0 + jj;
-          if (j < k && ((tmask >> j) & 1u)) {  // ascending j
+          if (j < k && ((tmask >> j) & 1u)) {  // ascending slot order
             const uint4 yv = moe::lds128(col + static_cast<size_t>(j) * a.chunk_bytes);
-            const uint64_t ww = moe::lds64(w2 + ti * k + j);
-            acc01 = moe::fma_bf16x2(ww, yv.x, acc01);
-            acc23 = moe::fma_bf16x2(ww, yv.y, acc23);
-            acc45 = moe::fma_bf16x2(ww, yv.z, acc45);
-            acc67 = moe::fma_bf16x2(ww, yv.w, acc67);
+            const float w = wt[j];
+            acc[0] = fmaf(w, moe::bf16_lo(yv.x), acc[0]);
+            acc[1] = fmaf(w, moe::bf16_hi(yv.x), acc[1]);
+            acc[2] = fmaf(w, moe::bf16_lo(yv.y), acc[2]);
+            acc[3] = fmaf(w, moe::bf16_hi(yv.y), acc[3]);
+            acc[4] = fmaf(w, moe::bf16_lo(yv.z), acc[4]);
+            acc[5] = fmaf(w, moe::bf16_hi(yv.z), acc[5]);
+            acc[6] = fmaf(w, moe::bf16_lo(yv.w), acc[6]);
+            acc[7] = fmaf(w, moe::bf16_hi(yv.w), acc[7]);
           }
         }
+        }
+        uint4 o;
+        o.x = moe::pack_bf16x2(acc[0], acc[1]);
+        o.y = moe::pack_bf16x2(acc[2], acc[3]);
+        o.z = moe::pack_bf16x2(acc[4], acc[5]);
+        o.w = moe::pack_bf16x2(acc[6], acc[7]);
+        moe::st_plain(reinterpret_cast<uint4*>(dst + static_cast<size_t>(v) * 16), o);
       }
-      float r[8];
-      moe::f32x2_split(acc01, r[0], r[1]);
-      moe::f32x2_split(acc23, r[2], r[3]);
-      moe::f32x2_split(acc45, r[4], r[5]);
-      moe::f32x2_split(acc67, r[6], r[7]);
-      uint4 o;
-      o.x = moe::pack_bf16x2(r[0], r[1]);
-      o.y = moe::pack_bf16x2(r[2], r[3]);
-      o.z = moe::pack_bf16x2(r[4], r[5]);
-      o.w = moe::pack_bf16x2(r[6], r[7]);
-      uint8_t* dst = a.out + t * static_cast<int64_t>(a.row_bytes) + static_cast<int64_t>(c) * a.chunk_bytes;
-      moe::st_plain(reinterpret_cast<uint4*>(dst + static_cast<size_t>(v) * 16), o);
     }
     __syncwarp();
     if (lane == 0) moe::mbar_arrive(&empty[s]);
@@ -456,7 +458,7 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   a.capacity = capacity;
   a.out = static_cast<uint8_t*>(out);
   a.status = device_status;
-  const size_t smem = static_cast<size_t>(stages) * stage_bytes + static_cast<size_t>(stages) * 32 * sizeof(uint64_t) +
+  const size_t smem = static_cast<size_t>(stages) * stage_bytes + static_cast<size_t>(stages) * 32 * sizeof(float) +
                       stages * sizeof(uint32_t) + 8 + 2 * stages * sizeof(uint64_t);
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -465,10 +467,10 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   int per_sm = static_cast<int>((200u * 1024u) / (smem + 1024));
   per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
   const int64_t grid = a.units < static_cast<int64_t>(sms) * per_sm ? a.units : static_cast<int64_t>(sms) * per_sm;
+  void (*kern)(CombineArgs) = k <= 2 ? combine_tma_kernel<2> : k <= 4 ? combine_tma_kernel<4> : combine_tma_kernel<8>;
   if (smem > 48 * 1024 &&
-      cudaFuncSetAttribute(combine_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=
-          cudaSuccess)
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return moe_host::launch_pdl(combine_tma_kernel, dim3(static_cast<unsigned>(grid)),
-                              dim3((1 + kCombineConsumerWarps) * 32), smem, static_cast<cudaStream_t>(stream), a);
+  return moe_host::launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3((1 + kCombineConsumerWarps) * 32), smem,
+                              static_cast<cudaStream_t>(stream), a);
 }
