@@ -8,7 +8,9 @@
 // warp-wide redux max; fp32 logits use a 64-bit key (ordered 32-bit value above, inverted index
 // below), reduced as its high word, then the low word among the lanes holding that high word.
 // Either way the round's maximum is the largest logit with the lowest index among equals, and the
-// winner is retired by zeroing its key (0 is below every real key).  Lane j keeps round j's key;
+// winner is retired (0 is below every real key).  With at most 8 keys per lane the keys are sorted
+// once (a sorting network) so that a round is one redux of the lanes' top keys and a shift in the
+// winning lane; with more, each round takes the lane maximum and zeroes the winner.  Lane j keeps round j's key;
 // after the rounds each of lanes 0..k-1 takes one exp, and a warp sum gives the renormalising
 // denominator (the full-row denominator Z is reduced in round 0 only when not renormalising).
 #pragma once
@@ -136,6 +138,41 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
+// Descending sorting networks for a lane's NV <= 8 keys (compare-exchange: larger key first).
+template <typename K>
+__device__ __forceinline__ void cas_desc(K& x, K& y) {
+  const K hi = x > y ? x : y;
+  const K lo = x > y ? y : x;
+  x = hi;
+  y = lo;
+}
+
+template <int NV, typename K>
+__device__ __forceinline__ void sort_desc(K (&k)[NV]) {
+  if constexpr (NV == 2) {
+    cas_desc(k[0], k[1]);
+  } else if constexpr (NV == 4) {
+    cas_desc(k[0], k[1]); cas_desc(k[2], k[3]);
+    cas_desc(k[0], k[2]); cas_desc(k[1], k[3]);
+    cas_desc(k[1], k[2]);
+  } else if constexpr (NV == 8) {  // Batcher odd-even merge sort, 19 comparators
+    cas_desc(k[0], k[1]); cas_desc(k[2], k[3]); cas_desc(k[4], k[5]); cas_desc(k[6], k[7]);
+    cas_desc(k[0], k[2]); cas_desc(k[1], k[3]); cas_desc(k[4], k[6]); cas_desc(k[5], k[7]);
+    cas_desc(k[1], k[2]); cas_desc(k[5], k[6]);
+    cas_desc(k[0], k[4]); cas_desc(k[1], k[5]); cas_desc(k[2], k[6]); cas_desc(k[3], k[7]);
+    cas_desc(k[2], k[4]); cas_desc(k[3], k[5]);
+    cas_desc(k[1], k[2]); cas_desc(k[3], k[4]); cas_desc(k[5], k[6]);
+  }
+}
+
+// Retire the lane's top key when it won the round: shift the sorted keys up by one.
+template <int NV, typename K>
+__device__ __forceinline__ void pop_front_if(K (&k)[NV], bool hit) {
+#pragma unroll
+  for (int i = 0; i + 1 < NV; ++i) k[i] = hit ? k[i + 1] : k[i];
+  k[NV - 1] = hit ? K(0) : k[NV - 1];
+}
+
 // Top-k of one row (all 32 lanes of the warp call it).  Lanes 0..k-1 return the expert of rank
 // `lane` in my_e and its weight in my_w; other lanes' outputs are unspecified.
 template <typename TIn, int VEC, int CPL>
@@ -162,10 +199,16 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
       }
     }
     uint32_t my_key = 0u, best0 = 0u;
+    constexpr bool kSorted = NV <= 8;  // few keys per lane: keep them sorted, the lane's top is key[0]
+    if constexpr (kSorted) sort_desc<NV>(key);
     for (int j = 0; j < k; ++j) {
       uint32_t best = 0u;
+      if constexpr (kSorted) {
+        best = key[0];
+      } else {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
+        for (int i = 0; i < NV; ++i) best = key[i] > best ? key[i] : best;
+      }
       best = __reduce_max_sync(0xffffffffu, best);
       if (j == 0) {
         best0 = best;
@@ -179,8 +222,12 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
           Z = warp_sum(z);
         }
       }
+      if constexpr (kSorted) {
+        pop_front_if<NV>(key, key[0] == best);
+      } else {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0u : key[i];
+        for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0u : key[i];
+      }
       if (lane == j) my_key = best;
     }
     m = ordered16_to_float(best0 >> 16);
@@ -206,10 +253,16 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
     }
     uint64_t my_key = 0ull;
     uint32_t hi0 = 0u;
+    constexpr bool kSorted = NV <= 8;
+    if constexpr (kSorted) sort_desc<NV>(key);
     for (int j = 0; j < k; ++j) {
       uint64_t mine = 0ull;
+      if constexpr (kSorted) {
+        mine = key[0];
+      } else {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) mine = key[i] > mine ? key[i] : mine;
+        for (int i = 0; i < NV; ++i) mine = key[i] > mine ? key[i] : mine;
+      }
       const uint32_t hi = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32));
       const uint32_t lo = __reduce_max_sync(0xffffffffu, static_cast<uint32_t>(mine >> 32) == hi
                                                              ? static_cast<uint32_t>(mine) : 0u);
@@ -226,8 +279,12 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
           Z = warp_sum(z);
         }
       }
+      if constexpr (kSorted) {
+        pop_front_if<NV>(key, key[0] == best);
+      } else {
 #pragma unroll
-      for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
+        for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
+      }
       if (lane == j) my_key = best;
     }
     m = ordered_to_float(hi0);
