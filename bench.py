@@ -3,9 +3,10 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = moe_topk_softmax -> moe_align_permute -> moe_gather -> moe_combine over one batch
-(the stand-in expert outputs replace the expert MLPs between gather and combine), replayed as
-one CUDA graph.  Inputs are resident in HBM; L2 is flushed (a 256 MiB write) between timed
+One step = MoeRouter.step over one batch: moe_topk_softmax -> moe_align_permute -> moe_gather ->
+moe_combine, or for decode-sized batches the single-kernel moe_route_dispatch -> moe_combine (the
+stand-in expert outputs replace the expert MLPs between gather and combine), replayed as one CUDA
+graph.  The decode workload also times every injected route pattern (routes given by the caller).  Inputs are resident in HBM; L2 is flushed (a 256 MiB write) between timed
 steps (then a 256 MiB read, so no dirty flush lines are written back inside a timed step);
 every step is timed with CUDA events on the launching stream and the K step times are
 summed; the result is the max over ranks.  N > 1 runs one independent batch per GPU (weak
@@ -44,6 +45,7 @@ KERNEL_SOURCES = {
     "gather_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "combine_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "gate_count_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "route_small_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
 }
 STAGE_KERNEL = {"topk": "topk_row_warp_kernel", "align": "align_cluster_kernel", "gather": "gather_tma_kernel",
                 "combine": "combine_tma_kernel", "dispatch": "gate_count_kernel+place_gather_kernel"}
@@ -290,9 +292,12 @@ def main():
     R = int(r.align.counts.sum().item())
     npad = int(r.align.num_tokens_post_pad.item())
     NB = r.align.expert_ids.numel()
-    launches_per_step = 4  # topk_row_warp_kernel, align_cluster_kernel (or 2 tile kernels), gather, combine
-    if wl.T * wl.k > 65536 or wl.experts_local > 512:
-        launches_per_step = 5
+    if r.small_batch:
+        launches_per_step = 2  # route_small_kernel, combine_tma_kernel
+    else:
+        launches_per_step = 4  # topk_row_warp_kernel, align_cluster_kernel (or 2 tile kernels), gather, combine
+        if wl.T * wl.k > 65536 or wl.experts_local > 512:
+            launches_per_step = 5
 
     use_graph = not args.no_graph
     graphs = {}
@@ -360,6 +365,10 @@ def main():
     abytes["dispatch"] = abytes["topk"] + abytes["align"] + abytes["gather"]
     st_iters = args.stage_steps or min(args.steps, 500)
 
+    stage_kernel = dict(STAGE_KERNEL)
+    if r.small_batch:
+        stage_kernel["dispatch"] = "route_small_kernel"
+
     def stage_times(names, calls):
         marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
 
@@ -392,7 +401,7 @@ def main():
         for j, name in enumerate(names):
             ms = sums[j] / st_iters
             out[name] = {"us": 1e3 * ms, "algorithmic_bytes": abytes[name],
-                         "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": STAGE_KERNEL[name],
+                         "achieved_gbs": abytes[name] / (ms * 1e-3) / 1e9, "kernel": stage_kernel[name],
                          "timing": "CUDA events between the stages of the step graph"}
         return out
 
@@ -400,13 +409,36 @@ def main():
                          [lambda: r.gate(logits), lambda: r.align_permute(),
                           lambda: r.gather(hidden, hidden_ready=True), lambda: r.combine(y)])
     stages_fused = stage_times(("dispatch", "combine"), [lambda: r.dispatch(logits, hidden), lambda: r.combine(y)])
-    dom = "combine"  # the dominant single kernel of the step (about half of its bytes)
-    ach = stages[dom]["achieved_gbs"]
+    # the dominant single kernel of the step: combine (about half of the bytes) on the four-call
+    # path; on the single-kernel dispatch path of small batches, the longer of its two kernels
+    in_step = stages_fused if r.small_batch else stages
+    dom = max(in_step, key=lambda n: in_step[n]["us"]) if r.small_batch else "combine"
+    ach = in_step[dom]["achieved_gbs"]
     total_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
     roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                "traffic": ncu_traffic(STAGE_KERNEL[dom], wl.name), "kernel": STAGE_KERNEL[dom],
+                "traffic": ncu_traffic(stage_kernel[dom], wl.name), "kernel": stage_kernel[dom],
                 "peak_source": peak_src,
                 "algorithmic_bytes_per_launch": abytes[dom]}
+
+    # ---- injected route patterns of the decode workload: the step for routes given by the caller
+    # (align + permute-gather + combine), one graph per pattern, same flush protocol; worst reported
+    patterns = None
+    if wl.name.startswith("ep_decode"):
+        w_inj = I.decode_pattern_weights(seed=seed).to(dev)
+        patterns = {}
+        for pname in I.DECODE_PATTERNS:
+            ids_p = I.decode_pattern_ids(pname).to(dev)
+            fn = (lambda ids_p=ids_p: r.step_routes(ids_p, w_inj, hidden, y))
+            if use_graph:
+                graphs["pattern"] = capture(fn)
+            stage_fns["pattern"] = fn
+            n_it = min(args.steps, 500)
+            patterns[pname] = 1e3 * timed("pattern", n_it, min(args.warmup, 10)) / n_it
+        patterns = {"us_per_step": patterns, "worst_us": max(patterns.values()),
+                    "worst": max(patterns, key=patterns.get),
+                    "path": "MoeRouter.step_routes: moe_route_dispatch (given routes) + moe_combine, one graph each"}
+        if r.device_status() != tdt.MOE_OK:
+            raise RuntimeError("device status after the route-pattern steps is not MOE_OK")
 
     # ---- end to end through the public API, from pinned host buffers
     e2e_steps = args.e2e_steps or min(args.steps, 200)
@@ -430,7 +462,8 @@ def main():
     d2h = out_h.numel() * out_h.element_size()
     e2e = {"value": ws * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-           "api": "MoeRouter.step_from_host (pinned H2D of logits+hidden, 4 C-ABI calls, D2H of out)"}
+           "api": f"MoeRouter.step_from_host (pinned H2D of logits+hidden, {launches_per_step if r.small_batch else 4} "
+                  f"C-ABI calls, D2H of out)"}
 
     if r.device_status() != tdt.MOE_OK:
         raise RuntimeError("device status after the timed steps is not MOE_OK")
@@ -455,7 +488,10 @@ def main():
             "algorithmic_bytes_per_step": total_bytes,
             "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
             "routed_slots_local": R, "num_tokens_post_pad": npad,
+            "step_path": "moe_route_dispatch (single kernel) + moe_combine" if r.small_batch else
+                         "moe_topk_softmax + moe_align_permute + moe_gather + moe_combine",
             "roofline": roofline, "stages": stages, "stages_fused_dispatch_path": stages_fused, "e2e": e2e,
+            "decode_route_patterns": patterns,
             "cpu_baseline": cpu,
             "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,
             "clocks": clocks,

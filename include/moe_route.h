@@ -85,6 +85,8 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 #define MOE_GATHER_HIDDEN_READY 4u /* moe_gather: `hidden` was complete before the previous kernel in
                                       the stream was launched, so it may be read before waiting for
                                       that kernel (true when hidden is an input of the routing step) */
+#define MOE_DISPATCH_GIVEN_IDS 8u /* moe_route_dispatch: topk_ids is an input (routes chosen by the
+                                     caller); no gating, logits and topk_weights are not accessed */
 
 /* Human-readable name of a status code (static string, never NULL). */
 MOE_API const char* moe_status_string(moe_status_t status);
@@ -242,11 +244,17 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
  *   topk_weights [T,k], topk_ids [T,k], counts [E_local], offsets [E_local+1],
  *   sorted_token_ids [C], expert_ids [NB], num_tokens_post_pad [1], inv_perm [T*k],
  *   permuted [C, H] (rows of local slots; pad rows untouched).
- * The first kernel gates tiles of tokens and counts each tile's slots per local expert with
- * their ranks inside the tile; the last of its CTAs to finish turns the tile counts into the
- * padded layout.  The second kernel gives every slot its row and copies the hidden rows there.
+ * For T > 32, T*k > 1024 or more than 160 KB of hidden rows: the first kernel gates tiles of
+ * tokens and counts each tile's slots per local expert with their ranks inside the tile; the
+ * last of its CTAs to finish turns the tile counts into the padded layout; the second kernel
+ * gives every slot its row and copies the hidden rows there.  Smaller batches (decode) take one
+ * kernel of one CTA that stages the hidden rows in shared memory, gates, aligns and stores the
+ * rows to their slots.
  *   logits [T, E] bf16/fp32 (dtype); hidden [T, H] bf16, 16-byte aligned, H % 8 == 0 and
  *   H <= 65536; expert_map and E_local as for moe_align_permute.
+ *   flags: MOE_RENORMALIZE; MOE_DISPATCH_GIVEN_IDS: the routes in topk_ids [T,k] are the
+ *   input (the align input of moe_align_permute), logits and topk_weights may be NULL and are
+ *   not read or written; every other output is as from moe_align_permute + moe_gather.
  *   workspace: >= moe_route_dispatch_workspace_bytes(T, k, E_local) bytes, zeroed before its
  *   first use and left ready by every call; its first 4 bytes are the device status word.
  *   Errors: as the three calls it replaces; UNSUPPORTED also for H > 65536.

@@ -115,3 +115,28 @@ def test_binding_rejects_cpu_tensors():
     import torch
     with pytest.raises(ValueError, match="CUDA tensor"):
         tdt.moe_topk_softmax(torch.zeros(4, 8, dtype=torch.bfloat16), 2, True)
+
+
+def test_flag_values_match_the_header():
+    text = open(HEADER).read()
+    defined = {m.group(1): int(m.group(2)) for m in re.finditer(r"^#define\s+(MOE_\w+)\s+(\d+)u", text, flags=re.M)}
+    for name in ("MOE_RENORMALIZE", "MOE_GATHER_ZERO_PAD", "MOE_GATHER_HIDDEN_READY", "MOE_DISPATCH_GIVEN_IDS"):
+        assert getattr(B, name) == defined[name], name
+
+
+def test_dispatch_validation_before_launch():
+    lib = B.load_library()
+    buf = ctypes.c_void_p(16)
+    d = lib.moe_route_dispatch
+
+    def call(logits, flags, weights, workspace=N, ws_bytes=0, H=16):
+        return d(logits, B.MOE_DTYPE_BF16, buf, 2, 160, 6, H, flags, buf, 40, 8, weights, buf, buf, buf, buf, buf,
+                 buf, buf, buf, workspace, ws_bytes, N)
+
+    given = B.MOE_DISPATCH_GIVEN_IDS
+    assert call(N, 0, buf) == B.MOE_ERR_INVALID_ARG                 # gating needs logits
+    assert call(buf, 0, N) == B.MOE_ERR_INVALID_ARG                 # and somewhere for the weights
+    assert call(N, given, N) == B.MOE_ERR_WORKSPACE                 # given routes: neither is needed
+    assert call(buf, 0x10, buf) == B.MOE_ERR_INVALID_ARG            # unknown flag
+    assert call(buf, B.MOE_GATHER_ZERO_PAD, buf) == B.MOE_ERR_INVALID_ARG
+    assert call(buf, B.MOE_RENORMALIZE | given, buf, H=12) == B.MOE_ERR_INVALID_ARG  # H % 8

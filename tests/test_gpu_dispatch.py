@@ -1,9 +1,12 @@
-"""GPU parity of the fused dispatch (moe_route_dispatch: gating + align + permute-gather in two
-kernels) against the CPU oracle pipeline, through the C ABI.
+"""GPU parity of the fused dispatch (moe_route_dispatch: gating + align + permute-gather) against
+the CPU oracle pipeline, through the C ABI.
 
-Shapes cover one and many gating tiles with a ragged last tile, maps with remote and out-of-range
-values, every gating vector width, k up to 32, 1024 experts, T = 0 and the decode size.  Bars as
-for the stage entry points: ids, align outputs and gathered rows bit-exact, weights within 2e-6.
+Two kernel paths sit behind the call: one CTA for small batches (T <= 32, T*k <= 1024, at most
+160 KB of hidden rows) and the tiled two-kernel path above that.  Shapes cover both sides of every
+one of those limits, one and many gating tiles with a ragged last tile, maps with remote and
+out-of-range values, every gating vector width, k up to 32, 1024 experts, T = 0 and the decode size,
+with logits-derived routes and with routes given by the caller.  Bars as for the stage entry points:
+ids, align outputs and gathered rows bit-exact, weights within 2e-6.
 """
 import math
 
@@ -32,6 +35,16 @@ CASES = [
     ("odd_e_bf16", 333, 61, 5, torch.bfloat16, True, None, 61, 3, 16),
     ("many_tiles_small_bs", 9000, 32, 2, torch.bfloat16, True, None, 32, 1, 8),
     ("zero_tokens", 0, 16, 4, torch.bfloat16, True, None, 16, 8, 64),
+    # single-CTA path and its limits
+    ("small_T1", 1, 64, 4, torch.bfloat16, True, None, 64, 16, 512),
+    ("small_T32_k32_fp32", 32, 64, 32, torch.float32, True, None, 64, 8, 128),
+    ("small_wide_1024_fp32", 8, 1024, 8, torch.float32, False, None, 1024, 4, 64),
+    ("small_wide_1024_bf16_map", 5, 1024, 8, torch.bfloat16, True, "strided", 256, 2, 64),
+    ("small_bad_map_values", 20, 64, 4, torch.bfloat16, True, "bad", 16, 16, 64),
+    ("small_odd_e_fp32", 31, 61, 5, torch.float32, True, None, 61, 3, 16),
+    ("small_rows_at_limit", 20, 64, 4, torch.bfloat16, True, None, 64, 8, 4096),
+    ("tile_rows_over_limit", 21, 64, 4, torch.bfloat16, True, None, 64, 8, 4096),
+    ("tile_T33_decode_map", 33, 160, 6, torch.bfloat16, True, "rank1", 40, 8, 4096),
 ]
 
 
@@ -101,3 +114,39 @@ def test_dispatch_matches_stage_entry_points():
     npad = int(a.align.num_tokens_post_pad.item())
     real = (a.align.sorted_token_ids[:npad] != wl.T * wl.k)
     assert torch.equal(a.permuted[:npad][real], b.permuted[:npad][real])
+
+
+GIVEN = [
+    # name, T, k, E, map kind, E_local, bs, H
+    ("small_decode_patterns", 2, 6, 160, "rank1", 40, 8, 4096),
+    ("tile_decode_patterns_tiled", 70, 6, 160, "rank1", 40, 8, 256),
+]
+
+
+@pytest.mark.parametrize("name,T,k,E,kind,E_local,bs,H", GIVEN, ids=[c[0] for c in GIVEN])
+def test_dispatch_given_routes(name, T, k, E, kind, E_local, bs, H):
+    """MOE_DISPATCH_GIVEN_IDS: every injected decode route pattern (rows repeated to T), plus a
+    pattern with out-of-range ids, through the small and the tiled path; topk_weights untouched."""
+    dev = require_gpu()
+    emap = _map(kind, E, E_local)
+    emap_d = torch.from_numpy(emap).to(dev)
+    hidden = torch.randn((T, H), generator=torch.Generator().manual_seed(5)).to(torch.bfloat16)
+    ws = tdt.alloc_dispatch_workspace(T, k, E_local, dev)
+    patterns = dict(I.DECODE_PATTERNS)
+    patterns["out_of_range"] = [[44, -1, 160, 3, 1000, 61], [-7, 44, 52, 52, 159, 0]]
+    for pname, rows in patterns.items():
+        ids = np.array([rows[t % 2] for t in range(T)], np.int32)
+        al = oracle.align_permute(ids, E, bs, emap, E_local)
+        npad = int(al["num_tokens_post_pad"][0])
+        perm_ref = oracle.gather(bf16_bits(hidden), k, al["sorted_token_ids"], npad, al["capacity"])
+        real = al["sorted_token_ids"][:npad] != T * k
+        sentinel = torch.full((T, k), -2.5, dtype=torch.float32, device=dev)
+        _, _, align, perm = tdt.moe_route_dispatch(None, hidden.to(dev), k, True, bs, emap_d, E_local,
+                                                   topk_weights=sentinel, topk_ids=torch.from_numpy(ids).to(dev),
+                                                   workspace=ws, given_ids=True, E=E)
+        torch.cuda.synchronize()
+        assert_align_equal(align, al, f"{name}/{pname}")
+        assert np.array_equal(bf16_bits(perm[:npad])[real], perm_ref[:npad][real]), (name, pname)
+        assert bool((sentinel == -2.5).all()), (name, pname)
+        status = tdt.moe_read_status(ws)
+        assert status == (tdt.MOE_ERR_BAD_EXPERT_ID if pname == "out_of_range" else tdt.MOE_OK), (name, pname)

@@ -64,7 +64,7 @@ def _check_all(r, wl, ref, what, y, y_bits):
 
 
 def _run(r, path, logits, hidden, y):
-    return r.step_fused(logits, hidden, y) if path == "fused" else r.step(logits, hidden, y)
+    return r.step_fused(logits, hidden, y) if path == "fused" else r.step_staged(logits, hidden, y)
 
 
 @pytest.mark.parametrize("path", ["fused", "staged"])
@@ -102,12 +102,15 @@ def test_ep_decode_every_route_pattern(path):
     w_inj = I.decode_pattern_weights()
     for name in I.DECODE_PATTERNS:
         ids = I.decode_pattern_ids(name)
-        r.gate(logits.to(dev))
-        r.topk_ids.copy_(ids.to(dev))
-        r.topk_weights.copy_(w_inj.to(dev))
-        r.align_permute()
-        r.gather(hidden.to(dev))
-        r.combine(y.to(dev))
+        if path == "fused":
+            r.step_routes(ids.to(dev), w_inj.to(dev), hidden.to(dev), y.to(dev))
+        else:
+            r.gate(logits.to(dev))
+            r.topk_ids.copy_(ids.to(dev))
+            r.topk_weights.copy_(w_inj.to(dev))
+            r.align_permute()
+            r.gather(hidden.to(dev))
+            r.combine(y.to(dev))
         torch.cuda.synchronize()
         w_ref, _, al, perm, out = _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y),
                                                    ids_override=ids.numpy(), w_override=w_inj.numpy())
@@ -165,15 +168,17 @@ def test_skewed_prefill_full_size_sampled(path):
     assert ulp_distance_bf16(got2, want).max() <= COMBINE_MAX_ULP
 
 
-def test_repeat_steps_are_bit_identical():
+@pytest.mark.parametrize("name", ["qwen3moe_prefill_T4096_E128_k8", "ep_decode_T2_E160_local40_k6"])
+def test_repeat_steps_are_bit_identical(name):
+    """Repeated steps, alternating the staged and the fused dispatch, give the same bits."""
     dev = require_gpu()
-    wl = I.WORKLOADS["qwen3moe_prefill_T4096_E128_k8"]
+    wl = I.WORKLOADS[name]
     logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)
     y = I.make_expert_out(wl.capacity, wl.H, device=dev)
     r = _router(wl, dev)
     first = None
     for i in range(6):
-        (r.step if i % 2 == 0 else r.step_fused)(logits, hidden, y)
+        (r.step_staged if i % 2 == 0 else r.step_fused)(logits, hidden, y)
         snap = [t.clone() for t in (r.topk_ids, r.topk_weights, r.align.sorted_token_ids, r.align.inv_perm,
                                     r.align.expert_ids, r.out)]
         if first is None:

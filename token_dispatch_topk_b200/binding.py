@@ -30,6 +30,7 @@ MOE_DTYPE_BF16 = 1
 MOE_RENORMALIZE = 1
 MOE_GATHER_ZERO_PAD = 2
 MOE_GATHER_HIDDEN_READY = 4
+MOE_DISPATCH_GIVEN_IDS = 8
 
 # Every symbol include/moe_route.h declares, with (restype, argtypes).
 _P, _I32, _I64, _U32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t
@@ -273,27 +274,39 @@ def alloc_dispatch_workspace(T: int, k: int, E_local: int, device) -> torch.Tens
     return torch.zeros((nbytes + 3) // 4, dtype=torch.int32, device=device)
 
 
-def moe_route_dispatch(logits: torch.Tensor, hidden: torch.Tensor, k: int, renormalize: bool, block_size: int,
-                       expert_map: Optional[torch.Tensor] = None, E_local: Optional[int] = None,
+def moe_route_dispatch(logits: Optional[torch.Tensor], hidden: torch.Tensor, k: int, renormalize: bool,
+                       block_size: int, expert_map: Optional[torch.Tensor] = None, E_local: Optional[int] = None,
                        topk_weights: Optional[torch.Tensor] = None, topk_ids: Optional[torch.Tensor] = None,
                        align: Optional[AlignResult] = None, permuted: Optional[torch.Tensor] = None,
-                       workspace: Optional[torch.Tensor] = None, stream=None):
-    """Gating + align + permute-gather in one call.  Returns (topk_weights, topk_ids, AlignResult, permuted)."""
-    T, E = logits.shape
-    H = hidden.shape[1]
-    if logits.dtype == torch.bfloat16:
+                       workspace: Optional[torch.Tensor] = None, stream=None, given_ids: bool = False,
+                       E: Optional[int] = None):
+    """Gating + align + permute-gather in one call.  Returns (topk_weights, topk_ids, AlignResult, permuted).
+
+    With ``given_ids`` the routes in ``topk_ids`` are the input (no gating): ``logits`` may be None (then
+    ``E`` gives the number of global experts) and ``topk_weights`` is neither read nor written."""
+    T, H = hidden.shape
+    if logits is not None:
+        assert logits.shape[0] == T
+        E = logits.shape[1]
+    if E is None:
+        raise ValueError("E is needed when logits is None")
+    if logits is None or logits.dtype == torch.bfloat16:
         dt = MOE_DTYPE_BF16
     elif logits.dtype == torch.float32:
         dt = MOE_DTYPE_F32
     else:
         raise ValueError(f"logits dtype {logits.dtype} unsupported (bf16 or fp32)")
+    if logits is None and not given_ids:
+        raise ValueError("logits are needed unless the routes are given")
     assert hidden.dtype == torch.bfloat16
     if E_local is None:
         E_local = E
-    dev = logits.device
-    if topk_weights is None:
+    dev = hidden.device
+    if topk_weights is None and not given_ids:
         topk_weights = torch.empty((T, k), dtype=torch.float32, device=dev)
     if topk_ids is None:
+        if given_ids:
+            raise ValueError("given_ids needs topk_ids")
         topk_ids = torch.empty((T, k), dtype=torch.int32, device=dev)
     if align is None:
         align = alloc_align_outputs(T, k, E_local, block_size, dev)
@@ -302,8 +315,9 @@ def moe_route_dispatch(logits: torch.Tensor, hidden: torch.Tensor, k: int, renor
     if workspace is None:
         workspace = alloc_dispatch_workspace(T, k, E_local, dev)
     assert expert_map is None or expert_map.dtype == torch.int32
+    flags = (MOE_RENORMALIZE if renormalize else 0) | (MOE_DISPATCH_GIVEN_IDS if given_ids else 0)
     st = load_library().moe_route_dispatch(
-        _dev(logits, "logits"), dt, _dev(hidden, "hidden"), T, E, k, H, MOE_RENORMALIZE if renormalize else 0,
+        _dev(logits, "logits"), dt, _dev(hidden, "hidden"), T, E, k, H, flags,
         _dev(expert_map, "expert_map"), E_local, block_size, _dev(topk_weights, "topk_weights"),
         _dev(topk_ids, "topk_ids"), _dev(align.counts, "counts"), _dev(align.offsets, "offsets"),
         _dev(align.sorted_token_ids, "sorted_token_ids"), _dev(align.expert_ids, "expert_ids"),

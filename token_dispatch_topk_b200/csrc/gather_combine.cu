@@ -162,6 +162,7 @@ constexpr int kCombineConsumerWarps = 8;
 constexpr int kCombineMaxStages = 8;
 constexpr uint32_t kCombineStageTarget = 32u * 1024u;  // bytes of slot rows per stage (about)
 constexpr uint32_t kCombineRingTarget = 96u * 1024u;   // bytes of stages per CTA (about)
+constexpr uint32_t kCombineMinChunk = 512u;            // narrowest chunk of a small batch
 
 struct CombineArgs {
   const uint8_t* y;         // expert_out [capacity, H] bf16
@@ -442,6 +443,10 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   a.T = T;
   a.k = k;
   a.row_bytes = static_cast<uint32_t>(H) * 2u;
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return MOE_ERR_CUDA;
   // a unit: `tpu` tokens x k slot rows x one chunk of each row, about 32 KB
   const uint32_t chunk_cap = k <= 8 ? 4096u : (k <= 16 ? 2048u : 1024u);
   a.chunk_bytes = a.row_bytes < chunk_cap ? a.row_bytes : chunk_cap;
@@ -449,6 +454,19 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   int tpu = static_cast<int>(kCombineStageTarget / (static_cast<uint32_t>(k) * a.chunk_bytes));
   if (tpu < 1) tpu = 1;
   if (tpu * k > 32) tpu = 32 / k;
+  if (((T + tpu - 1) / tpu) * a.nchunks < sms) {
+    // small batches (decode): one token per unit and narrower chunks, so that the units spread
+    // over the SMs instead of queueing behind a few producers
+    tpu = 1;
+    const int64_t want = (sms + T - 1) / T;  // chunks per row
+    uint32_t cb = static_cast<uint32_t>((a.row_bytes + want - 1) / want);
+    cb = (cb + 15u) & ~15u;
+    if (cb < kCombineMinChunk) cb = kCombineMinChunk;
+    if (cb < a.chunk_bytes) {
+      a.chunk_bytes = cb;
+      a.nchunks = static_cast<int>((a.row_bytes + cb - 1) / cb);
+    }
+  }
   a.tpu = tpu;
   const uint32_t stage_bytes = static_cast<uint32_t>(tpu * k) * a.chunk_bytes;
   int stages = static_cast<int>(kCombineRingTarget / stage_bytes);
@@ -460,10 +478,6 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   a.status = device_status;
   const size_t smem = static_cast<size_t>(stages) * stage_bytes + static_cast<size_t>(stages) * 32 * sizeof(float) +
                       stages * sizeof(uint32_t) + 8 + 2 * stages * sizeof(uint64_t);
-  int dev = 0, sms = 148;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
-    return MOE_ERR_CUDA;
   int per_sm = static_cast<int>((200u * 1024u) / (smem + 1024));
   per_sm = per_sm < 1 ? 1 : (per_sm > 4 ? 4 : per_sm);
   const int64_t grid = a.units < static_cast<int64_t>(sms) * per_sm ? a.units : static_cast<int64_t>(sms) * per_sm;

@@ -49,6 +49,7 @@ struct DispatchArgs {
   int E;
   int k;
   int renormalize;
+  int given_ids;  // topk_ids is an input: no gating, topk_weights untouched
   const int32_t* expert_map;
   int E_local;
   int bs;
@@ -217,9 +218,12 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   moe::pdl_wait();  // the logits may come from the previous kernel
   moe::pdl_launch_dependents();
 
-  // A. gating, one warp per row
+  // A. gating, one warp per row (or the routes the caller gave)
   const TIn* logits = static_cast<const TIn*>(a.logits);
-  for (int r = warp; r < rows; r += kGcWarps) {
+  if (a.given_ids) {
+    for (int i = tid; i < rows * k; i += kGcThreads) s_le[i] = to_local(a, a.topk_ids[row0 * k + i]);
+  }
+  for (int r = a.given_ids ? rows : warp; r < rows; r += kGcWarps) {
     const int64_t row = row0 + r;
     int my_e;
     float my_w;
@@ -405,44 +409,236 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
   if (n > 0) moe::bulk_wait_read_all();  // the staged rows must outlive the stores that read them
 }
 
-using GcKernel = void (*)(DispatchArgs);
+// ------------------------------------------------------------------------------------------
+// Small batches (decode): the whole dispatch in one CTA of kSmallThreads threads.
+//   1. the T hidden rows are bulk-loaded into shared memory, the expert map is read, and warp t
+//      gates row t, all at once (one memory latency for the three);
+//   2. every slot finds its stable rank among the slots of the same local expert by scanning
+//      the earlier slots in shared memory (P <= kSmallMaxSlots), the counts are rounded up to
+//      blocks and scanned across the CTA;
+//   3. counts, offsets, N_pad, expert_ids, sorted_token_ids (pads and tail included) and
+//      inv_perm are written, and each local slot bulk-stores its staged hidden row to its row.
+constexpr int kSmallThreads = 1024;
+constexpr int kSmallWarps = kSmallThreads / 32;
+constexpr int kSmallMaxTokens = kSmallWarps;
+constexpr int kSmallMaxSlots = kSmallThreads;
+constexpr uint32_t kSmallMaxRowBytes = 160u * 1024u;  // staged hidden bytes (T * H * 2)
 
+__host__ __device__ inline uint32_t small_rows_bytes(int64_t T, uint32_t row_bytes) {
+  return static_cast<uint32_t>(((static_cast<uint64_t>(T) * row_bytes) + 127u) & ~uint64_t{127});
+}
+__host__ __device__ inline int round4(int n) { return (n + 3) & ~3; }
+// Shared memory after the staged rows (ints): s_le[P] | s_map[E] | s_cnt[E_local] | s_off[E_local+1] | warp_sums[32]
+__host__ __device__ inline size_t small_smem_bytes(int64_t T, uint32_t row_bytes, int P, int E, int E_local) {
+  return small_rows_bytes(T, row_bytes) +
+         sizeof(int) * static_cast<size_t>(round4(P) + round4(E) + round4(E_local) + round4(E_local + 1) + 32);
+}
+
+template <typename TIn, int VEC, int CPL, bool kGivenIds>
+__global__ void __launch_bounds__(kSmallThreads)
+route_small_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t row_bytes,
+                   uint8_t* __restrict__ permuted) {
+  extern __shared__ __align__(128) uint8_t small_smem[];
+  __shared__ __align__(8) uint64_t bar;
+  const int T = static_cast<int>(a.T), k = a.k, E = a.E, El = a.E_local, P = T * k;
+  uint8_t* rows = small_smem;
+  int* s_le = reinterpret_cast<int*>(small_smem + small_rows_bytes(a.T, row_bytes));
+  int* s_map = s_le + round4(P);
+  int* s_cnt = s_map + round4(E);
+  int* s_off = s_cnt + round4(El);
+  int* warp_sums = s_off + round4(El + 1);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+
+  if (tid == 0) {
+    moe::mbar_init(&bar, 1);
+    moe::fence_barrier_init();
+  }
+  for (int e = tid; e < El; e += kSmallThreads) s_cnt[e] = 0;
+  __syncthreads();
+  moe::pdl_wait();  // logits, routes and hidden may come from the previous kernel
+  moe::pdl_launch_dependents();
+  if (tid == 0 && T > 0) {
+    moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(T) * row_bytes);
+    for (int t = 0; t < T; ++t)
+      moe::bulk_load(rows + static_cast<size_t>(t) * row_bytes, hidden + static_cast<int64_t>(t) * row_bytes,
+                     row_bytes, &bar);
+  }
+  // 1. expert map (E <= kSmallThreads) and gating, their loads in flight together
+  const int map_v = tid < E ? (a.expert_map != nullptr ? a.expert_map[tid] : tid) : 0;
+  int my_e = -1;
+  if constexpr (kGivenIds) {
+    if (warp < T && lane < k) my_e = a.topk_ids[warp * k + lane];
+  } else {
+    if (warp < T) {
+      float my_w;
+      int e;
+      moe_gate::gate_row<TIn, VEC, CPL>(static_cast<const TIn*>(a.logits) + static_cast<int64_t>(warp) * E, E, k,
+                                        a.renormalize, lane, e, my_w);
+      if (lane < k) {
+        my_e = e;
+        a.topk_weights[warp * k + lane] = my_w;
+        a.topk_ids[warp * k + lane] = e;
+      }
+    }
+  }
+  if (tid < E) s_map[tid] = map_v;
+  __syncthreads();
+  if (warp < T && lane < k) {
+    int le = -1;
+    if (static_cast<unsigned>(my_e) >= static_cast<unsigned>(E)) {
+      moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+    } else {
+      le = s_map[my_e];
+      if (le < -1 || le >= El) {
+        moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
+        le = -1;
+      }
+    }
+    s_le[warp * k + lane] = le;
+  }
+  __syncthreads();
+
+  // 2. stable rank of every slot among the earlier slots of its expert; counts
+  const int s = tid;
+  const int le = s < P ? s_le[s] : -1;
+  int rank = 0;
+  if (le >= 0) {
+    int j = 0;
+    for (; j + 4 <= s; j += 4) {
+      const int4 q = *reinterpret_cast<const int4*>(s_le + j);
+      rank += (q.x == le) + (q.y == le) + (q.z == le) + (q.w == le);
+    }
+    for (; j < s; ++j) rank += (s_le[j] == le);
+    atomicAdd(&s_cnt[le], 1);
+  }
+  __syncthreads();
+  // block-padded expert sizes, exclusive scan over the local experts (E_local <= kSmallThreads)
+  const int padded = tid < El ? ((s_cnt[tid] + a.bs - 1) / a.bs) * a.bs : 0;
+  int incl = padded;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) warp_sums[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = warp_sums[lane];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, w, off);
+      if (lane >= off) w += v;
+    }
+    warp_sums[lane] = w;
+  }
+  __syncthreads();
+  const int total = warp_sums[kSmallWarps - 1];
+  if (tid < El) s_off[tid] = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - padded;
+  if (tid == 0) s_off[El] = total;
+  __syncthreads();
+
+  // 3. layout, slot rows, pad rows and the tail past N_pad
+  if (tid < El) {
+    a.counts[tid] = s_cnt[tid];
+    a.offsets[tid] = s_off[tid];
+  }
+  if (tid == 0) {
+    a.offsets[El] = total;
+    a.n_pad[0] = total;
+  }
+  for (int b = tid; b < a.NB; b += kSmallThreads) {
+    const int64_t row = static_cast<int64_t>(b) * a.bs;
+    int e = -1;
+    if (row < total) {
+      int lo = 0, hi = El - 1;  // largest e with s_off[e] <= row (empty experts share offsets)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    a.expert_ids[b] = e;
+  }
+  const int32_t pad_value = P;
+  for (int e = warp; e < El; e += kSmallWarps) {
+    const int p1 = s_off[e + 1];
+    for (int p = s_off[e] + s_cnt[e] + lane; p < p1; p += 32) a.sorted_ids[p] = pad_value;
+  }
+  for (int64_t i = static_cast<int64_t>(total) + tid; i < a.C; i += kSmallThreads) a.sorted_ids[i] = pad_value;
+  int r = -1;
+  if (le >= 0) {
+    r = s_off[le] + rank;  // < s_off[le] + s_cnt[le] <= N_pad <= C
+    if (static_cast<int64_t>(r) >= a.C) {
+      moe::record_status(a.status, MOE_ERR_BAD_ROW);
+      r = -1;
+    } else {
+      a.sorted_ids[r] = s;
+    }
+  }
+  if (s < P) a.inv_perm[s] = r;
+  if (r >= 0) {
+    if (moe::mbar_wait(&bar, 0)) {
+      moe::bulk_store(permuted + static_cast<int64_t>(r) * row_bytes, rows + static_cast<size_t>(s / k) * row_bytes,
+                      row_bytes);
+      moe::bulk_commit();
+      moe::bulk_wait_read_all();  // the staged row must outlive the store that reads it
+    } else {
+      moe::record_status(a.status, MOE_ERR_TIMEOUT);
+    }
+  }
+  if (tid == 0 && T > 0) moe::mbar_wait(&bar, 0);  // never leave with loads in flight into shared memory
+}
+
+// Kernel families instantiated per gating geometry (logits type, vector width, chunks per lane).
 template <typename TIn, int VEC, int CPL>
-GcKernel gc_instance() {
+struct GateCountFamily {
+  using Fn = void (*)(DispatchArgs);
+  static Fn get() { return &gate_count_kernel<TIn, VEC, CPL>; }
+};
+template <typename TIn, int VEC, int CPL>
+struct SmallFamily {
+  using Fn = void (*)(DispatchArgs, const uint8_t*, uint32_t, uint8_t*);
+  static Fn get() { return &route_small_kernel<TIn, VEC, CPL, false>; }
+};
+using GcKernel = GateCountFamily<float, 1, 1>::Fn;
+using SmallKernel = SmallFamily<float, 1, 1>::Fn;
+
+template <template <typename, int, int> class F, typename TIn, int VEC, int CPL>
+typename F<float, 1, 1>::Fn family_instance() {
   if constexpr (VEC * CPL <= 32) {
-    return &gate_count_kernel<TIn, VEC, CPL>;
+    return F<TIn, VEC, CPL>::get();
   } else {
     return nullptr;
   }
 }
 
-template <typename TIn, int VEC>
-GcKernel gc_pick_cpl(int cpl) {
+template <template <typename, int, int> class F, typename TIn, int VEC>
+typename F<float, 1, 1>::Fn family_pick_cpl(int cpl) {
   switch (cpl) {
-    case 1: return gc_instance<TIn, VEC, 1>();
-    case 2: return gc_instance<TIn, VEC, 2>();
-    case 4: return gc_instance<TIn, VEC, 4>();
-    case 8: return gc_instance<TIn, VEC, 8>();
-    case 16: return gc_instance<TIn, VEC, 16>();
-    case 32: return gc_instance<TIn, VEC, 32>();
+    case 1: return family_instance<F, TIn, VEC, 1>();
+    case 2: return family_instance<F, TIn, VEC, 2>();
+    case 4: return family_instance<F, TIn, VEC, 4>();
+    case 8: return family_instance<F, TIn, VEC, 8>();
+    case 16: return family_instance<F, TIn, VEC, 16>();
+    case 32: return family_instance<F, TIn, VEC, 32>();
     default: return nullptr;
   }
 }
 
-template <typename TIn>
-GcKernel gc_pick(int vec, int cpl) {
+template <template <typename, int, int> class F, typename TIn>
+typename F<float, 1, 1>::Fn family_pick(int vec, int cpl) {
   if constexpr (sizeof(TIn) == 2) {
     switch (vec) {
-      case 8: return gc_pick_cpl<TIn, 8>(cpl);
-      case 4: return gc_pick_cpl<TIn, 4>(cpl);
-      case 2: return gc_pick_cpl<TIn, 2>(cpl);
-      default: return gc_pick_cpl<TIn, 1>(cpl);
+      case 8: return family_pick_cpl<F, TIn, 8>(cpl);
+      case 4: return family_pick_cpl<F, TIn, 4>(cpl);
+      case 2: return family_pick_cpl<F, TIn, 2>(cpl);
+      default: return family_pick_cpl<F, TIn, 1>(cpl);
     }
   } else {
     switch (vec) {
-      case 4: return gc_pick_cpl<TIn, 4>(cpl);
-      case 2: return gc_pick_cpl<TIn, 2>(cpl);
-      default: return gc_pick_cpl<TIn, 1>(cpl);
+      case 4: return family_pick_cpl<F, TIn, 4>(cpl);
+      case 2: return family_pick_cpl<F, TIn, 2>(cpl);
+      default: return family_pick_cpl<F, TIn, 1>(cpl);
     }
   }
 }
@@ -487,7 +683,8 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
                                            void* workspace, size_t workspace_bytes, void* stream) {
   if (T < 0 || E < 1 || k < 1 || k > E || H < 1 || E_local < 1 || block_size < 1) return MOE_ERR_INVALID_ARG;
   if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
-  if ((flags & ~MOE_RENORMALIZE) != 0u) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~(MOE_RENORMALIZE | MOE_DISPATCH_GIVEN_IDS)) != 0u) return MOE_ERR_INVALID_ARG;
+  const bool given_ids = (flags & MOE_DISPATCH_GIVEN_IDS) != 0u;
   if (E_local > E || (expert_map == nullptr && E_local != E)) return MOE_ERR_INVALID_ARG;
   if (E > 1024 || k > 32 || E_local > 1024) return MOE_ERR_UNSUPPORTED;
   if ((H % 8) != 0) return MOE_ERR_INVALID_ARG;
@@ -500,9 +697,9 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   if (counts == nullptr || offsets == nullptr || sorted_token_ids == nullptr || expert_ids == nullptr ||
       num_tokens_post_pad == nullptr)
     return MOE_ERR_INVALID_ARG;
-  if (T > 0 && (logits == nullptr || hidden == nullptr || topk_weights == nullptr || topk_ids == nullptr ||
-                inv_perm == nullptr || permuted == nullptr))
+  if (T > 0 && (hidden == nullptr || topk_ids == nullptr || inv_perm == nullptr || permuted == nullptr))
     return MOE_ERR_INVALID_ARG;
+  if (T > 0 && !given_ids && (logits == nullptr || topk_weights == nullptr)) return MOE_ERR_INVALID_ARG;
   if ((hidden && !moe_host::aligned16(hidden)) || (permuted && !moe_host::aligned16(permuted)))
     return MOE_ERR_INVALID_ARG;
   if (workspace == nullptr || workspace_bytes < moe_route_dispatch_workspace_bytes(T, k, E_local))
@@ -515,6 +712,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.E = E;
   a.k = k;
   a.renormalize = (flags & MOE_RENORMALIZE) ? 1 : 0;
+  a.given_ids = given_ids ? 1 : 0;
   a.expert_map = expert_map;
   a.E_local = E_local;
   a.bs = block_size;
@@ -556,10 +754,28 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   const int n_chunks = E / vec;
   int cpl = 1;
   while (cpl * 32 < n_chunks) cpl <<= 1;
-  GcKernel gk = dtype == MOE_DTYPE_BF16 ? gc_pick<__nv_bfloat16>(vec, cpl) : gc_pick<float>(vec, cpl);
-  if (gk == nullptr) return MOE_ERR_UNSUPPORTED;
-
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+
+  // small batches: the whole dispatch in one CTA
+  if (T <= kSmallMaxTokens && P <= kSmallMaxSlots && static_cast<uint64_t>(T) * row_bytes <= kSmallMaxRowBytes) {
+    SmallKernel sk = given_ids ? &route_small_kernel<float, 1, 1, true>
+                     : dtype == MOE_DTYPE_BF16 ? family_pick<SmallFamily, __nv_bfloat16>(vec, cpl)
+                                               : family_pick<SmallFamily, float>(vec, cpl);
+    if (sk == nullptr) return MOE_ERR_UNSUPPORTED;
+    const size_t smem = small_smem_bytes(T, row_bytes, static_cast<int>(P), E, E_local);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(sk), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    return moe_host::launch_pdl(sk, dim3(1), dim3(kSmallThreads), smem, st, a, static_cast<const uint8_t*>(hidden),
+                                row_bytes, static_cast<uint8_t*>(permuted));
+  }
+
+  // the gating geometry does not matter when the routes are given (no row is gated)
+  GcKernel gk = given_ids ? family_pick<GateCountFamily, float>(1, 1)
+                : dtype == MOE_DTYPE_BF16 ? family_pick<GateCountFamily, __nv_bfloat16>(vec, cpl)
+                                          : family_pick<GateCountFamily, float>(vec, cpl);
+  if (gk == nullptr) return MOE_ERR_UNSUPPORTED;
   const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
   if (smem1 > 48 * 1024 &&
       cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,

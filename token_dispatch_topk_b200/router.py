@@ -1,6 +1,7 @@
 """MoeRouter: the routing path for fixed sizes with every buffer preallocated on the device.
 
-One ``step`` runs the four library stages back to back on one stream:
+One ``step`` runs the routing path on one stream: for decode-sized batches the single-kernel
+moe_route_dispatch (gating + align + permute-gather) then moe_combine; above that the four stages
 moe_topk_softmax -> moe_align_permute -> moe_gather -> (caller's experts) -> moe_combine.
 No allocation, host synchronisation or Python-side arithmetic happens inside a step, so
 it can be captured in a CUDA graph.  ``step_from_host`` is the end-to-end form: it copies
@@ -57,15 +58,33 @@ class MoeRouter:
         return B.moe_combine(expert_out, w, self.align.inv_perm, self.out, device_status=self.workspace,
                              stream=stream)
 
-    def dispatch(self, logits: torch.Tensor, hidden: torch.Tensor, stream=None):
-        """gate + align + permute-gather through the fused entry point (two kernels)."""
-        return B.moe_route_dispatch(logits, hidden, self.k, self.renormalize, self.block_size, self.expert_map,
-                                    self.E_local, self.topk_weights, self.topk_ids, self.align, self.permuted,
-                                    self.dispatch_workspace, stream)
+    def dispatch(self, logits: Optional[torch.Tensor], hidden: torch.Tensor, stream=None,
+                 topk_ids: Optional[torch.Tensor] = None):
+        """gate + align + permute-gather through the fused entry point (one kernel for small batches,
+        two above).  With ``topk_ids`` given, those routes are aligned instead of gating ``logits``."""
+        given = topk_ids is not None
+        return B.moe_route_dispatch(None if given else logits, hidden, self.k, self.renormalize, self.block_size,
+                                    self.expert_map, self.E_local, None if given else self.topk_weights,
+                                    topk_ids if given else self.topk_ids, self.align, self.permuted,
+                                    self.dispatch_workspace, stream, given_ids=given, E=self.E)
+
+    @property
+    def small_batch(self) -> bool:
+        """True when moe_route_dispatch runs as a single kernel (decode-sized batches)."""
+        return self.T <= 32 and self.T * self.k <= 1024 and self.T * self.H * 2 <= 160 * 1024
 
     def step(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
-        """gate + align + permute-gather + combine through the four stage entry points (the fastest
-        path measured); expert_out stands in for the expert MLPs' output."""
+        """gate + align + permute-gather + combine; expert_out stands in for the expert MLPs' output.
+
+        Decode-sized batches take the single-kernel dispatch then combine (two kernels); larger ones
+        the four stage entry points, which measured faster there than the two-kernel dispatch."""
+        if self.small_batch:
+            return self.step_fused(logits, hidden, expert_out, stream)
+        return self.step_staged(logits, hidden, expert_out, stream)
+
+    def step_staged(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor,
+                    stream=None) -> torch.Tensor:
+        """The step through the four stage entry points."""
         self.gate(logits, stream)
         self.align_permute(stream=stream)
         self.gather(hidden, stream, hidden_ready=True)  # hidden is an input of the step: ready before gating
@@ -73,12 +92,15 @@ class MoeRouter:
 
     def step_fused(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor,
                    stream=None) -> torch.Tensor:
-        """The same step with gating + align + gather fused into moe_route_dispatch (two kernels)."""
+        """The step with gating + align + gather fused into moe_route_dispatch."""
         self.dispatch(logits, hidden, stream)
         return self.combine(expert_out, stream=stream)
 
-    # the four-call path under its own name as well
-    step_staged = step
+    def step_routes(self, topk_ids: torch.Tensor, topk_weights: torch.Tensor, hidden: torch.Tensor,
+                    expert_out: torch.Tensor, stream=None) -> torch.Tensor:
+        """The step for routes chosen by the caller (no gating): align + permute-gather + combine."""
+        self.dispatch(None, hidden, stream, topk_ids=topk_ids)
+        return self.combine(expert_out, topk_weights, stream=stream)
 
     def step_from_host(self, logits_host: torch.Tensor, hidden_host: torch.Tensor, expert_out: torch.Tensor,
                        out_host: torch.Tensor, stream=None) -> torch.Tensor:
