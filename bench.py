@@ -44,6 +44,7 @@ KERNEL_SOURCES = {
     "align_cluster_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
     "gather_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "combine_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
+    "combine_small_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "gate_count_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
     "route_small_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
 }
@@ -293,7 +294,7 @@ def main():
     npad = int(r.align.num_tokens_post_pad.item())
     NB = r.align.expert_ids.numel()
     if r.small_batch:
-        launches_per_step = 2  # route_small_kernel, combine_tma_kernel
+        launches_per_step = 2  # route_small_kernel, combine_small_kernel
     else:
         launches_per_step = 4  # topk_row_warp_kernel, align_cluster_kernel (or 2 tile kernels), gather, combine
         if wl.T * wl.k > 65536 or wl.experts_local > 512:
@@ -368,6 +369,9 @@ def main():
     stage_kernel = dict(STAGE_KERNEL)
     if r.small_batch:
         stage_kernel["dispatch"] = "route_small_kernel"
+    sms = torch.cuda.get_device_properties(dev).multi_processor_count
+    if wl.T * (-(-wl.H * 2 // 4096)) < sms:  # fewer 4 KB row chunks than SMs: the small-batch combine
+        stage_kernel["combine"] = "combine_small_kernel"
 
     def stage_times(names, calls):
         marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]

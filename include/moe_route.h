@@ -237,19 +237,19 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
                          int32_t k, int32_t H, int64_t capacity, void* out, int32_t* device_status, void* stream);
 
 /*
- * moe_route_dispatch -- gating, align and permute-gather in one call, as two kernels instead of
- * four ("Upstream Reference", "File Index": the gate -> topk -> expand part of the FusedMoE
+ * moe_route_dispatch -- gating, align and permute-gather in one call, as two kernels (one for
+ * small batches) instead of four ("Upstream Reference", "File Index": the gate -> topk -> expand part of the FusedMoE
  * pipeline).  Every output is the same as from moe_topk_softmax (flags: MOE_RENORMALIZE) then
  * moe_align_permute then moe_gather (without MOE_GATHER_ZERO_PAD), bit for bit:
  *   topk_weights [T,k], topk_ids [T,k], counts [E_local], offsets [E_local+1],
  *   sorted_token_ids [C], expert_ids [NB], num_tokens_post_pad [1], inv_perm [T*k],
  *   permuted [C, H] (rows of local slots; pad rows untouched).
- * For T > 32, T*k > 1024 or more than 160 KB of hidden rows: the first kernel gates tiles of
- * tokens and counts each tile's slots per local expert with their ranks inside the tile; the
- * last of its CTAs to finish turns the tile counts into the padded layout; the second kernel
- * gives every slot its row and copies the hidden rows there.  Smaller batches (decode) take one
- * kernel of one CTA that stages the hidden rows in shared memory, gates, aligns and stores the
- * rows to their slots.
+ * For T > 32 or T*k > 256: the first kernel gates tiles of tokens and counts each tile's slots
+ * per local expert with their ranks inside the tile; the last of its CTAs to finish turns the
+ * tile counts into the padded layout; the second kernel gives every slot its row and copies the
+ * hidden rows there.  Smaller batches (decode) take one kernel with one CTA per slot: each CTA
+ * routes the whole batch by itself, CTA 0 writes the routing outputs and every CTA copies the
+ * hidden row of its own slot.
  *   logits [T, E] bf16/fp32 (dtype); hidden [T, H] bf16, 16-byte aligned, H % 8 == 0 and
  *   H <= 65536; expert_map and E_local as for moe_align_permute.
  *   flags: MOE_RENORMALIZE; MOE_DISPATCH_GIVEN_IDS: the routes in topk_ids [T,k] are the

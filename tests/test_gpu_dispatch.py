@@ -1,8 +1,8 @@
 """GPU parity of the fused dispatch (moe_route_dispatch: gating + align + permute-gather) against
 the CPU oracle pipeline, through the C ABI.
 
-Two kernel paths sit behind the call: one CTA for small batches (T <= 32, T*k <= 1024, at most
-160 KB of hidden rows) and the tiled two-kernel path above that.  Shapes cover both sides of every
+Two kernel paths sit behind the call: one kernel with one CTA per slot for small batches
+(T <= 32 and T*k <= 256) and the tiled two-kernel path above that.  Shapes cover both sides of every
 one of those limits, one and many gating tiles with a ragged last tile, maps with remote and
 out-of-range values, every gating vector width, k up to 32, 1024 experts, T = 0 and the decode size,
 with logits-derived routes and with routes given by the caller.  Bars as for the stage entry points:
@@ -35,15 +35,18 @@ CASES = [
     ("odd_e_bf16", 333, 61, 5, torch.bfloat16, True, None, 61, 3, 16),
     ("many_tiles_small_bs", 9000, 32, 2, torch.bfloat16, True, None, 32, 1, 8),
     ("zero_tokens", 0, 16, 4, torch.bfloat16, True, None, 16, 8, 64),
-    # single-CTA path and its limits
+    # single-kernel path (one CTA per slot) and its limits
     ("small_T1", 1, 64, 4, torch.bfloat16, True, None, 64, 16, 512),
-    ("small_T32_k32_fp32", 32, 64, 32, torch.float32, True, None, 64, 8, 128),
+    ("small_T32_k8_fp32", 32, 64, 8, torch.float32, True, None, 64, 8, 128),
+    ("tile_T32_k9", 32, 64, 9, torch.bfloat16, True, None, 64, 8, 128),
+    ("tile_T9_k32_fp32", 9, 64, 32, torch.float32, True, None, 64, 8, 64),
+    ("small_T8_k32", 8, 64, 32, torch.bfloat16, False, None, 64, 4, 64),
     ("small_wide_1024_fp32", 8, 1024, 8, torch.float32, False, None, 1024, 4, 64),
     ("small_wide_1024_bf16_map", 5, 1024, 8, torch.bfloat16, True, "strided", 256, 2, 64),
     ("small_bad_map_values", 20, 64, 4, torch.bfloat16, True, "bad", 16, 16, 64),
     ("small_odd_e_fp32", 31, 61, 5, torch.float32, True, None, 61, 3, 16),
-    ("small_rows_at_limit", 20, 64, 4, torch.bfloat16, True, None, 64, 8, 4096),
-    ("tile_rows_over_limit", 21, 64, 4, torch.bfloat16, True, None, 64, 8, 4096),
+    ("small_long_rows", 3, 32, 2, torch.bfloat16, True, None, 32, 4, 65536),
+    ("small_rows_past_prefetch", 2, 160, 6, torch.bfloat16, True, "rank1", 40, 8, 8200),
     ("tile_T33_decode_map", 33, 160, 6, torch.bfloat16, True, "rank1", 40, 8, 4096),
 ]
 

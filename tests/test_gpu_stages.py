@@ -208,6 +208,12 @@ COMBINE_CASES = [
     (100, 8, 256, 128, 7168, True),
     (77, 32, 64, 8, 64, True),    # k = 32: four groups of eight loads
     (40, 5, 9, 3, 16, False),
+    (1, 1, 4, 2, 8, True),        # one vector per row
+    (3, 3, 10, 4, 65536, True),   # long rows, small batch
+    (73, 2, 16, 8, 4096, False),  # 146 row chunks of 4 KB: small-batch combine (148 SMs)
+    (74, 2, 16, 8, 4096, False),  # 148: streaming combine
+    (147, 2, 16, 8, 2048, False),
+    (148, 2, 16, 8, 2048, False),
 ]
 
 
@@ -227,10 +233,11 @@ def test_combine_parity(T, k, E, bs, H, renorm):
     assert d.max() == 0, f"expected bit-exact combine (same fma order), max ulp {d.max()}"
 
 
-def test_combine_remote_slots_and_partial_sums():
+@pytest.mark.parametrize("T", [64, 400])  # small-batch and streaming combine
+def test_combine_remote_slots_and_partial_sums(T):
     """Expert-parallel partial sums: remote slots (-1) add nothing; a token with none gets +0."""
     dev = require_gpu()
-    T, k, H = 64, 6, 512
+    k, H = 6, 512
     rng = np.random.default_rng(1)
     C = 200
     inv = rng.integers(-1, C, size=T * k).astype(np.int32)
@@ -244,10 +251,12 @@ def test_combine_remote_slots_and_partial_sums():
     assert (got[0] == 0).all()
 
 
-def test_bad_rows_are_skipped_and_flagged():
+@pytest.mark.parametrize("T", [8, 400])  # small-batch and streaming combine
+def test_bad_rows_are_skipped_and_flagged(T):
     dev = require_gpu()
-    T, k, H, C = 8, 2, 64, 10
-    inv = torch.tensor([0, 1, 2, 99, 4, 5, -7, 7, 8, 9, 1, 2, 3, 4, 5, 6], dtype=torch.int32)
+    k, H, C = 2, 64, 10
+    base = [0, 1, 2, 99, 4, 5, -7, 7, 8, 9, 1, 2, 3, 4, 5, 6]
+    inv = torch.tensor([base[i % 16] for i in range(T * k)], dtype=torch.int32)
     w = torch.full((T, k), 0.5)
     y = I.make_expert_out(C, H, seed=2)
     status = torch.zeros(1, dtype=torch.int32, device=dev)

@@ -185,6 +185,25 @@ __device__ __forceinline__ uint64_t lds64(const void* p) {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
+// Hold a value in a register from this point of the program on.  Kernel parameters are otherwise
+// read from the constant bank where they are first used, and in a latency-bound kernel every first
+// use of another parameter line is a constant-cache miss on the critical path; pinning them at
+// entry issues those reads together, before the kernel waits for anything.
+__device__ __forceinline__ int pin(int v) {
+  asm volatile("" : "+r"(v));
+  return v;
+}
+__device__ __forceinline__ int64_t pin(int64_t v) {
+  asm volatile("" : "+l"(v));
+  return v;
+}
+template <typename T>
+__device__ __forceinline__ T* pin(T* p) {
+  uint64_t u = reinterpret_cast<uint64_t>(p);
+  asm volatile("" : "+l"(u));
+  return reinterpret_cast<T*>(u);
+}
+
 // Store a 32-bit value into the same shared-memory variable of CTA `rank` of this cluster.
 __device__ __forceinline__ void st_cluster_u32(const void* local_ptr, uint32_t rank, uint32_t v) {
   uint32_t raddr;

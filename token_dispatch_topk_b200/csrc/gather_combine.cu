@@ -162,7 +162,6 @@ constexpr int kCombineConsumerWarps = 8;
 constexpr int kCombineMaxStages = 8;
 constexpr uint32_t kCombineStageTarget = 32u * 1024u;  // bytes of slot rows per stage (about)
 constexpr uint32_t kCombineRingTarget = 96u * 1024u;   // bytes of stages per CTA (about)
-constexpr uint32_t kCombineMinChunk = 512u;            // narrowest chunk of a small batch
 
 struct CombineArgs {
   const uint8_t* y;         // expert_out [capacity, H] bf16
@@ -352,6 +351,80 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
   }
 }
 
+// Small batches (decode): a batch of a few tokens is a chain of latencies (slot rows and weights,
+// then the k expert rows), not a stream.  Grid (ceil(nvec / kCombineSmallThreads), T): thread v of
+// token t reads the slot rows and weights of t (lane j holds slot j, passed around by shuffles),
+// issues the loads of its 16-byte column of all the token's local slot rows together, then
+// accumulates them in fp32 (fmaf, ascending slot order, from +0) and stores the bf16 result.
+constexpr int kCombineSmallThreads = 128;
+
+template <int KU>  // slots loaded together (k rounded up to 2, 4 or 8; blocks of 8 beyond)
+__global__ void __launch_bounds__(kCombineSmallThreads)
+combine_small_kernel(const uint4* __restrict__ y, const float* __restrict__ w, const int32_t* __restrict__ inv_perm,
+                     int k, int nvec, int64_t capacity, uint4* __restrict__ out, int32_t* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t t = blockIdx.y;
+  const int v = blockIdx.x * kCombineSmallThreads + threadIdx.x;
+  y = moe::pin(y);  // parameters into registers before waiting (moe::pin)
+  w = moe::pin(w);
+  inv_perm = moe::pin(inv_perm);
+  k = moe::pin(k);
+  nvec = moe::pin(nvec);
+  capacity = moe::pin(capacity);
+  out = moe::pin(out);
+  status = moe::pin(status);
+  moe::pdl_launch_dependents();
+  moe::pdl_wait();  // slot rows, weights and expert outputs come from earlier kernels
+  float acc[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+  for (int j0 = 0; j0 < k; j0 += 32) {
+    int r = -1;
+    float wj = 0.f;
+    if (j0 + lane < k) {
+      r = inv_perm[t * k + j0 + lane];
+      wj = w[t * k + j0 + lane];
+      if (r < -1 || static_cast<int64_t>(r) >= capacity) {
+        moe::record_status(status, MOE_ERR_BAD_ROW);
+        r = -1;
+      }
+    }
+    const int kb = (k - j0) < 32 ? (k - j0) : 32;
+    for (int j1 = 0; j1 < kb; j1 += KU) {
+      uint4 yv[KU];
+      int rr[KU];
+#pragma unroll
+      for (int jj = 0; jj < KU; ++jj) {
+        rr[jj] = __shfl_sync(0xffffffffu, r, (j1 + jj) & 31);
+        if (j1 + jj >= kb) rr[jj] = -1;
+        if (rr[jj] >= 0 && v < nvec) yv[jj] = __ldg(y + static_cast<int64_t>(rr[jj]) * nvec + v);
+      }
+#pragma unroll
+      for (int jj = 0; jj < KU; ++jj) {
+        const float wt = __shfl_sync(0xffffffffu, wj, (j1 + jj) & 31);
+        if (rr[jj] >= 0 && v < nvec) {  // ascending slot order
+          acc[0] = fmaf(wt, moe::bf16_lo(yv[jj].x), acc[0]);
+          acc[1] = fmaf(wt, moe::bf16_hi(yv[jj].x), acc[1]);
+          acc[2] = fmaf(wt, moe::bf16_lo(yv[jj].y), acc[2]);
+          acc[3] = fmaf(wt, moe::bf16_hi(yv[jj].y), acc[3]);
+          acc[4] = fmaf(wt, moe::bf16_lo(yv[jj].z), acc[4]);
+          acc[5] = fmaf(wt, moe::bf16_hi(yv[jj].z), acc[5]);
+          acc[6] = fmaf(wt, moe::bf16_lo(yv[jj].w), acc[6]);
+          acc[7] = fmaf(wt, moe::bf16_hi(yv[jj].w), acc[7]);
+        }
+      }
+    }
+  }
+  if (v < nvec) {
+    uint4 o;
+    o.x = moe::pack_bf16x2(acc[0], acc[1]);
+    o.y = moe::pack_bf16x2(acc[2], acc[3]);
+    o.z = moe::pack_bf16x2(acc[4], acc[5]);
+    o.w = moe::pack_bf16x2(acc[6], acc[7]);
+    out[t * nvec + v] = o;
+  }
+}
+
 // Split each token row into `seg` segments of `seg_len` 16-byte vectors so that small
 // batches still put enough warps on the GPU (about half its warp slots).
 void segment_rows(int64_t T, int NV, int* seg, int* seg_len) {
@@ -447,6 +520,16 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   if (cudaGetDevice(&dev) != cudaSuccess ||
       cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return MOE_ERR_CUDA;
+  const int nvec = static_cast<int>(a.row_bytes / 16u);
+  if (T * ((a.row_bytes + 4095u) / 4096u) < sms) {  // small batch: fewer 4 KB row chunks than SMs
+    void (*ks)(const uint4*, const float*, const int32_t*, int, int, int64_t, uint4*, int32_t*) =
+        k <= 2 ? combine_small_kernel<2> : k <= 4 ? combine_small_kernel<4> : combine_small_kernel<8>;
+    const dim3 grid(static_cast<unsigned>((nvec + kCombineSmallThreads - 1) / kCombineSmallThreads),
+                    static_cast<unsigned>(T));
+    return moe_host::launch_pdl(ks, grid, dim3(kCombineSmallThreads), 0, static_cast<cudaStream_t>(stream),
+                                static_cast<const uint4*>(expert_out), topk_weights, inv_perm, static_cast<int>(k),
+                                nvec, capacity, static_cast<uint4*>(out), device_status);
+  }
   // a unit: `tpu` tokens x k slot rows x one chunk of each row, about 32 KB
   const uint32_t chunk_cap = k <= 8 ? 4096u : (k <= 16 ? 2048u : 1024u);
   a.chunk_bytes = a.row_bytes < chunk_cap ? a.row_bytes : chunk_cap;
@@ -454,19 +537,6 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   int tpu = static_cast<int>(kCombineStageTarget / (static_cast<uint32_t>(k) * a.chunk_bytes));
   if (tpu < 1) tpu = 1;
   if (tpu * k > 32) tpu = 32 / k;
-  if (((T + tpu - 1) / tpu) * a.nchunks < sms) {
-    // small batches (decode): one token per unit and narrower chunks, so that the units spread
-    // over the SMs instead of queueing behind a few producers
-    tpu = 1;
-    const int64_t want = (sms + T - 1) / T;  // chunks per row
-    uint32_t cb = static_cast<uint32_t>((a.row_bytes + want - 1) / want);
-    cb = (cb + 15u) & ~15u;
-    if (cb < kCombineMinChunk) cb = kCombineMinChunk;
-    if (cb < a.chunk_bytes) {
-      a.chunk_bytes = cb;
-      a.nchunks = static_cast<int>((a.row_bytes + cb - 1) / cb);
-    }
-  }
   a.tpu = tpu;
   const uint32_t stage_bytes = static_cast<uint32_t>(tpu * k) * a.chunk_bytes;
   int stages = static_cast<int>(kCombineRingTarget / stage_bytes);

@@ -53,6 +53,7 @@ struct DispatchArgs {
   const int32_t* expert_map;
   int E_local;
   int bs;
+  int bs_shift;  // log2(bs) when bs is a power of two, else -1
   int64_t P;  // T * k
   int64_t C;  // capacity rows
   int NB;     // blocks
@@ -410,111 +411,156 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
 }
 
 // ------------------------------------------------------------------------------------------
-// Small batches (decode): the whole dispatch in one CTA of kSmallThreads threads.
-//   1. the T hidden rows are bulk-loaded into shared memory, the expert map is read, and warp t
-//      gates row t, all at once (one memory latency for the three);
-//   2. every slot finds its stable rank among the slots of the same local expert by scanning
-//      the earlier slots in shared memory (P <= kSmallMaxSlots), the counts are rounded up to
-//      blocks and scanned across the CTA;
-//   3. counts, offsets, N_pad, expert_ids, sorted_token_ids (pads and tail included) and
-//      inv_perm are written, and each local slot bulk-stores its staged hidden row to its row.
-constexpr int kSmallThreads = 1024;
+// Small batches (decode): one CTA per slot, each routing the whole batch by itself.
+// A decode batch is a handful of tokens: its routing is a short chain of dependent steps, and one
+// SM writing every hidden row to its slots would be bound by that SM's store bandwidth.  So the
+// grid has one CTA per slot s = t*k + j; every CTA gates all T rows, ranks the slots and scans the
+// local experts (no CTA waits for another); CTA 0 writes the routing outputs; CTA s copies the
+// hidden row of token t to the row of slot s when the slot is local.  The row is loaded into
+// registers at kernel entry, so its memory latency overlaps the gating loads.  The phases are
+// laid out for latency (few barriers, no serial searches):
+//   A. hidden row -> registers; expert map -> shared memory; warp w gates rows w, w + 8, ...
+//      (or reads the caller's routes);
+//   B. per warp of 32 slots: local expert, rank among the warp's earlier slots of the same expert
+//      and the warp's count of it (a 32-step shuffle loop); the first slot of each expert in the
+//      warp records the count in the warp's row of a histogram;
+//   C. per expert (one to four per thread): count = sum of the warp rows, blocks = ceil(count/bs),
+//      exclusive scan of the blocks over the experts; CTA 0 writes counts, offsets, the expert's
+//      expert_ids and its pad rows;
+//   D. row of slot s = offset of its expert + its expert's slots in earlier warps + its rank;
+//      CTA 0 writes sorted_token_ids, inv_perm and the tail past N_pad; CTA s copies its row.
+constexpr int kSmallThreads = 256;
 constexpr int kSmallWarps = kSmallThreads / 32;
-constexpr int kSmallMaxTokens = kSmallWarps;
-constexpr int kSmallMaxSlots = kSmallThreads;
-constexpr uint32_t kSmallMaxRowBytes = 160u * 1024u;  // staged hidden bytes (T * H * 2)
-
-__host__ __device__ inline uint32_t small_rows_bytes(int64_t T, uint32_t row_bytes) {
-  return static_cast<uint32_t>(((static_cast<uint64_t>(T) * row_bytes) + 127u) & ~uint64_t{127});
-}
-__host__ __device__ inline int round4(int n) { return (n + 3) & ~3; }
-// Shared memory after the staged rows (ints): s_le[P] | s_map[E] | s_cnt[E_local] | s_off[E_local+1] | warp_sums[32]
-__host__ __device__ inline size_t small_smem_bytes(int64_t T, uint32_t row_bytes, int P, int E, int E_local) {
-  return small_rows_bytes(T, row_bytes) +
-         sizeof(int) * static_cast<size_t>(round4(P) + round4(E) + round4(E_local) + round4(E_local + 1) + 32);
-}
+constexpr int kSmallMaxTokens = 32;
+constexpr int kSmallMaxSlots = kSmallThreads;  // one slot per thread
+constexpr int kSmallMaxExperts = 1024;
+constexpr int kSmallExpertsPerThread = kSmallMaxExperts / kSmallThreads;
+constexpr int kSmallPrefetch = 4;  // 16-byte vectors per thread of the row held in registers while routing
 
 template <typename TIn, int VEC, int CPL, bool kGivenIds>
 __global__ void __launch_bounds__(kSmallThreads)
-route_small_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t row_bytes,
-                   uint8_t* __restrict__ permuted) {
-  extern __shared__ __align__(128) uint8_t small_smem[];
-  __shared__ __align__(8) uint64_t bar;
-  const int T = static_cast<int>(a.T), k = a.k, E = a.E, El = a.E_local, P = T * k;
-  uint8_t* rows = small_smem;
-  int* s_le = reinterpret_cast<int*>(small_smem + small_rows_bytes(a.T, row_bytes));
-  int* s_map = s_le + round4(P);
-  int* s_cnt = s_map + round4(E);
-  int* s_off = s_cnt + round4(El);
-  int* warp_sums = s_off + round4(El + 1);
+route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, uint4* __restrict__ permuted) {
+  __shared__ int s_map[kSmallMaxExperts];
+  __shared__ int whist[kSmallWarps * kSmallMaxExperts];  // [warp][E_local]: the warp's slots per expert
+  __shared__ int s_off[kSmallMaxExperts];                // first row of each local expert
+  __shared__ int s_ge[kSmallMaxSlots];
+  __shared__ int s_le[kSmallMaxSlots];
+  __shared__ int s_rk[kSmallMaxSlots];
+  __shared__ int warp_sums[kSmallWarps];
+  // every parameter, read into registers at entry (moe::pin), before the kernel waits for anything
+  const int T = moe::pin(static_cast<int>(a.T)), k = moe::pin(a.k), E = moe::pin(a.E), El = moe::pin(a.E_local);
+  const int bs = moe::pin(a.bs), bs_shift = moe::pin(a.bs_shift), NB = moe::pin(a.NB);
+  const int renormalize = moe::pin(a.renormalize);
+  const int64_t C = moe::pin(a.C);
+  const TIn* logits = moe::pin(static_cast<const TIn*>(a.logits));
+  const int32_t* expert_map = moe::pin(a.expert_map);
+  int32_t* topk_ids = moe::pin(a.topk_ids);
+  float* topk_weights = moe::pin(a.topk_weights);
+  int32_t* counts = moe::pin(a.counts);
+  int32_t* offsets = moe::pin(a.offsets);
+  int32_t* sorted_ids = moe::pin(a.sorted_ids);
+  int32_t* expert_ids = moe::pin(a.expert_ids);
+  int32_t* n_pad = moe::pin(a.n_pad);
+  int32_t* inv_perm = moe::pin(a.inv_perm);
+  int32_t* status = moe::pin(a.status);
+  hidden = moe::pin(hidden);
+  permuted = moe::pin(permuted);
+  nvec = moe::pin(nvec);
+  const int P = T * k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nw = (P + 31) >> 5;  // warps holding slots
+  // grid (k, T): this CTA copies the row of slot tok * k + j (no CTA has a slot when P == 0)
+  const int tok = blockIdx.y, slot = tok * k + static_cast<int>(blockIdx.x);
+  const bool lead = blockIdx.x == 0 && blockIdx.y == 0;
+  for (int i = tid; i < nw * El; i += kSmallThreads) whist[i] = 0;
 
-  if (tid == 0) {
-    moe::mbar_init(&bar, 1);
-    moe::fence_barrier_init();
-  }
-  for (int e = tid; e < El; e += kSmallThreads) s_cnt[e] = 0;
-  __syncthreads();
   moe::pdl_wait();  // logits, routes and hidden may come from the previous kernel
   moe::pdl_launch_dependents();
-  if (tid == 0 && T > 0) {
-    moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(T) * row_bytes);
-    for (int t = 0; t < T; ++t)
-      moe::bulk_load(rows + static_cast<size_t>(t) * row_bytes, hidden + static_cast<int64_t>(t) * row_bytes,
-                     row_bytes, &bar);
+  // A. this CTA's hidden row, the expert map and the gating loads, in flight together
+  const uint4* src = hidden + static_cast<int64_t>(slot < P ? tok : 0) * nvec;
+  uint4 pre[kSmallPrefetch];
+#pragma unroll
+  for (int i = 0; i < kSmallPrefetch; ++i) {
+    const int v = tid + i * kSmallThreads;
+    if (slot < P && v < nvec) pre[i] = __ldg(src + v);
   }
-  // 1. expert map (E <= kSmallThreads) and gating, their loads in flight together
-  const int map_v = tid < E ? (a.expert_map != nullptr ? a.expert_map[tid] : tid) : 0;
-  int my_e = -1;
+  int mv[kSmallExpertsPerThread];
+#pragma unroll
+  for (int i = 0; i < kSmallExpertsPerThread; ++i) {
+    const int g = tid + i * kSmallThreads;
+    mv[i] = g < E ? (expert_map != nullptr ? __ldg(expert_map + g) : g) : 0;
+  }
   if constexpr (kGivenIds) {
-    if (warp < T && lane < k) my_e = a.topk_ids[warp * k + lane];
+    if (tid < P) s_ge[tid] = topk_ids[tid];
   } else {
-    if (warp < T) {
-      float my_w;
+    for (int row = warp; row < T; row += kSmallWarps) {
       int e;
-      moe_gate::gate_row<TIn, VEC, CPL>(static_cast<const TIn*>(a.logits) + static_cast<int64_t>(warp) * E, E, k,
-                                        a.renormalize, lane, e, my_w);
+      float w;
+      moe_gate::gate_row<TIn, VEC, CPL>(logits + static_cast<int64_t>(row) * E, E, k, renormalize, lane, e, w);
       if (lane < k) {
-        my_e = e;
-        a.topk_weights[warp * k + lane] = my_w;
-        a.topk_ids[warp * k + lane] = e;
+        s_ge[row * k + lane] = e;
+        if (lead) {
+          topk_weights[row * k + lane] = w;
+          topk_ids[row * k + lane] = e;
+        }
       }
     }
   }
-  if (tid < E) s_map[tid] = map_v;
-  __syncthreads();
-  if (warp < T && lane < k) {
-    int le = -1;
-    if (static_cast<unsigned>(my_e) >= static_cast<unsigned>(E)) {
-      moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
-    } else {
-      le = s_map[my_e];
-      if (le < -1 || le >= El) {
-        moe::record_status(a.status, MOE_ERR_BAD_EXPERT_ID);
-        le = -1;
-      }
-    }
-    s_le[warp * k + lane] = le;
+#pragma unroll
+  for (int i = 0; i < kSmallExpertsPerThread; ++i) {
+    const int g = tid + i * kSmallThreads;
+    if (g < E) s_map[g] = mv[i];
   }
   __syncthreads();
 
-  // 2. stable rank of every slot among the earlier slots of its expert; counts
-  const int s = tid;
-  const int le = s < P ? s_le[s] : -1;
-  int rank = 0;
-  if (le >= 0) {
-    int j = 0;
-    for (; j + 4 <= s; j += 4) {
-      const int4 q = *reinterpret_cast<const int4*>(s_le + j);
-      rank += (q.x == le) + (q.y == le) + (q.z == le) + (q.w == le);
+  // B. local expert, rank inside the warp and the warp's count per expert (thread s owns slot s)
+  int le = -1, rank = 0;
+  if (warp < nw) {
+    if (tid < P) {
+      const int g = s_ge[tid];
+      if (static_cast<unsigned>(g) >= static_cast<unsigned>(E)) {
+        if (lead) moe::record_status(status, MOE_ERR_BAD_EXPERT_ID);
+      } else {
+        le = s_map[g];
+        if (le < -1 || le >= El) {
+          if (lead) moe::record_status(status, MOE_ERR_BAD_EXPERT_ID);
+          le = -1;
+        }
+      }
     }
-    for (; j < s; ++j) rank += (s_le[j] == le);
-    atomicAdd(&s_cnt[le], 1);
+    int cnt = 0;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      const int lj = __shfl_sync(0xffffffffu, le, j);
+      const int same = (lj == le) ? 1 : 0;
+      cnt += same;
+      rank += (j < lane) ? same : 0;
+    }
+    if (le >= 0 && rank == 0) whist[warp * El + le] = cnt;
+    if (tid < P) {
+      s_le[tid] = le;
+      s_rk[tid] = rank;
+    }
   }
   __syncthreads();
-  // block-padded expert sizes, exclusive scan over the local experts (E_local <= kSmallThreads)
-  const int padded = tid < El ? ((s_cnt[tid] + a.bs - 1) / a.bs) * a.bs : 0;
-  int incl = padded;
+
+  // C. per expert: count, blocks, exclusive scan of the blocks; expert-owned outputs (CTA 0)
+  const int ept = (El + kSmallThreads - 1) / kSmallThreads;  // experts per thread, consecutive
+  const int e0 = tid * ept;
+  int cnt_e[kSmallExpertsPerThread], nb_e[kSmallExpertsPerThread];
+  int sum = 0;
+#pragma unroll
+  for (int i = 0; i < kSmallExpertsPerThread; ++i) {
+    const int e = e0 + i;
+    int c = 0;
+    if (i < ept && e < El) {
+      for (int w = 0; w < nw; ++w) c += whist[w * El + e];
+    }
+    cnt_e[i] = c;
+    nb_e[i] = c == 0 ? 0 : bs_shift >= 0 ? (c + bs - 1) >> bs_shift : (c + bs - 1) / bs;
+    sum += nb_e[i];
+  }
+  int incl = sum;
 #pragma unroll
   for (int off = 1; off < 32; off <<= 1) {
     const int v = __shfl_up_sync(0xffffffffu, incl, off);
@@ -522,71 +568,72 @@ route_small_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t 
   }
   if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
-  if (warp == 0) {
-    int w = warp_sums[lane];
+  int before = incl - sum;
+  int total_blocks = 0;
 #pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, w, off);
-      if (lane >= off) w += v;
-    }
-    warp_sums[lane] = w;
+  for (int w = 0; w < kSmallWarps; ++w) {
+    const int ws = warp_sums[w];
+    before += (w < warp) ? ws : 0;
+    total_blocks += ws;
   }
-  __syncthreads();
-  const int total = warp_sums[kSmallWarps - 1];
-  if (tid < El) s_off[tid] = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - padded;
-  if (tid == 0) s_off[El] = total;
+  const int total = total_blocks * bs;  // N_pad
+  const int32_t pad_value = P;
+#pragma unroll
+  for (int i = 0; i < kSmallExpertsPerThread; ++i) {
+    const int e = e0 + i;
+    if (i < ept && e < El) {
+      const int off = before * bs;
+      s_off[e] = off;
+      if (lead) {
+        counts[e] = cnt_e[i];
+        offsets[e] = off;
+        for (int b = 0; b < nb_e[i]; ++b) expert_ids[before + b] = e;
+        for (int p = off + cnt_e[i]; p < off + nb_e[i] * bs; ++p) sorted_ids[p] = pad_value;
+      }
+    }
+    before += nb_e[i];
+  }
+  if (lead && tid == 0) {
+    offsets[El] = total;
+    n_pad[0] = total;
+  }
   __syncthreads();
 
-  // 3. layout, slot rows, pad rows and the tail past N_pad
-  if (tid < El) {
-    a.counts[tid] = s_cnt[tid];
-    a.offsets[tid] = s_off[tid];
-  }
-  if (tid == 0) {
-    a.offsets[El] = total;
-    a.n_pad[0] = total;
-  }
-  for (int b = tid; b < a.NB; b += kSmallThreads) {
-    const int64_t row = static_cast<int64_t>(b) * a.bs;
-    int e = -1;
-    if (row < total) {
-      int lo = 0, hi = El - 1;  // largest e with s_off[e] <= row (empty experts share offsets)
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
+  // D. slot rows; the tail past N_pad (CTA 0); this CTA's hidden row to its slot row
+  if (lead) {
+    if (tid < P) {
+      int r = -1;
+      if (le >= 0) {
+        r = s_off[le] + rank;
+        for (int w = 0; w < warp; ++w) r += whist[w * El + le];
+        if (static_cast<int64_t>(r) >= C) {  // < N_pad <= C for consistent inputs
+          moe::record_status(status, MOE_ERR_BAD_ROW);
+          r = -1;
+        } else {
+          sorted_ids[r] = tid;
+        }
       }
-      e = lo;
+      inv_perm[tid] = r;
     }
-    a.expert_ids[b] = e;
+    for (int64_t i = static_cast<int64_t>(total) + tid; i < C; i += kSmallThreads) sorted_ids[i] = pad_value;
+    for (int b = total_blocks + tid; b < NB; b += kSmallThreads) expert_ids[b] = -1;
   }
-  const int32_t pad_value = P;
-  for (int e = warp; e < El; e += kSmallWarps) {
-    const int p1 = s_off[e + 1];
-    for (int p = s_off[e] + s_cnt[e] + lane; p < p1; p += 32) a.sorted_ids[p] = pad_value;
-  }
-  for (int64_t i = static_cast<int64_t>(total) + tid; i < a.C; i += kSmallThreads) a.sorted_ids[i] = pad_value;
-  int r = -1;
-  if (le >= 0) {
-    r = s_off[le] + rank;  // < s_off[le] + s_cnt[le] <= N_pad <= C
-    if (static_cast<int64_t>(r) >= a.C) {
-      moe::record_status(a.status, MOE_ERR_BAD_ROW);
-      r = -1;
-    } else {
-      a.sorted_ids[r] = s;
-    }
-  }
-  if (s < P) a.inv_perm[s] = r;
-  if (r >= 0) {
-    if (moe::mbar_wait(&bar, 0)) {
-      moe::bulk_store(permuted + static_cast<int64_t>(r) * row_bytes, rows + static_cast<size_t>(s / k) * row_bytes,
-                      row_bytes);
-      moe::bulk_commit();
-      moe::bulk_wait_read_all();  // the staged row must outlive the store that reads it
-    } else {
-      moe::record_status(a.status, MOE_ERR_TIMEOUT);
+  if (slot < P) {
+    const int le_s = s_le[slot];
+    if (le_s >= 0) {
+      int row = s_off[le_s] + s_rk[slot];
+      for (int w = 0; w < (slot >> 5); ++w) row += whist[w * El + le_s];
+      if (static_cast<int64_t>(row) < C) {
+        uint4* dst = permuted + static_cast<int64_t>(row) * nvec;
+#pragma unroll
+        for (int i = 0; i < kSmallPrefetch; ++i) {
+          const int v = tid + i * kSmallThreads;
+          if (v < nvec) dst[v] = pre[i];
+        }
+        for (int v = tid + kSmallPrefetch * kSmallThreads; v < nvec; v += kSmallThreads) dst[v] = __ldg(src + v);
+      }
     }
   }
-  if (tid == 0 && T > 0) moe::mbar_wait(&bar, 0);  // never leave with loads in flight into shared memory
 }
 
 // Kernel families instantiated per gating geometry (logits type, vector width, chunks per lane).
@@ -597,7 +644,7 @@ struct GateCountFamily {
 };
 template <typename TIn, int VEC, int CPL>
 struct SmallFamily {
-  using Fn = void (*)(DispatchArgs, const uint8_t*, uint32_t, uint8_t*);
+  using Fn = void (*)(DispatchArgs, const uint4*, int, uint4*);
   static Fn get() { return &route_small_kernel<TIn, VEC, CPL, false>; }
 };
 using GcKernel = GateCountFamily<float, 1, 1>::Fn;
@@ -716,6 +763,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.expert_map = expert_map;
   a.E_local = E_local;
   a.bs = block_size;
+  a.bs_shift = (block_size & (block_size - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(block_size)) : -1;
   a.P = P;
   a.C = C;
   a.NB = static_cast<int>((C + block_size - 1) / block_size);
@@ -756,19 +804,15 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   while (cpl * 32 < n_chunks) cpl <<= 1;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
-  // small batches: the whole dispatch in one CTA
-  if (T <= kSmallMaxTokens && P <= kSmallMaxSlots && static_cast<uint64_t>(T) * row_bytes <= kSmallMaxRowBytes) {
+  // small batches: one kernel, one CTA per slot
+  if (T <= kSmallMaxTokens && P <= kSmallMaxSlots && E <= kSmallMaxExperts) {
     SmallKernel sk = given_ids ? &route_small_kernel<float, 1, 1, true>
                      : dtype == MOE_DTYPE_BF16 ? family_pick<SmallFamily, __nv_bfloat16>(vec, cpl)
                                                : family_pick<SmallFamily, float>(vec, cpl);
     if (sk == nullptr) return MOE_ERR_UNSUPPORTED;
-    const size_t smem = small_smem_bytes(T, row_bytes, static_cast<int>(P), E, E_local);
-    if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(reinterpret_cast<const void*>(sk), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess)
-      return MOE_ERR_CUDA;
-    return moe_host::launch_pdl(sk, dim3(1), dim3(kSmallThreads), smem, st, a, static_cast<const uint8_t*>(hidden),
-                                row_bytes, static_cast<uint8_t*>(permuted));
+    const dim3 grid = P > 0 ? dim3(static_cast<unsigned>(k), static_cast<unsigned>(T)) : dim3(1, 1);  // (j, t)
+    return moe_host::launch_pdl(sk, grid, dim3(kSmallThreads), 0, st, a, static_cast<const uint4*>(hidden),
+                                static_cast<int>(row_bytes / 16u), static_cast<uint4*>(permuted));
   }
 
   // the gating geometry does not matter when the routes are given (no row is gated)
