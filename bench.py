@@ -3,16 +3,18 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
 
-One step = MoeRouter.step over one batch: moe_topk_softmax -> moe_align_permute -> moe_gather ->
-moe_combine, or for decode-sized batches the single-kernel moe_route_dispatch -> moe_combine (the
-stand-in expert outputs replace the expert MLPs between gather and combine), replayed as one CUDA
-graph.  The decode workload also times every injected route pattern (routes given by the caller).  Inputs are resident in HBM; L2 is flushed (a 256 MiB write) between timed
-steps (then a 256 MiB read, so no dirty flush lines are written back inside a timed step);
-every step is timed with CUDA events on the launching stream and the K step times are
-summed; the result is the max over ranks.  N > 1 runs one independent batch per GPU (weak
-scaling: the path has no cross-token exchange).  Rank 0 prints one JSON line.
+One step = MoeRouter.step over one batch: moe_route_dispatch (gating + align + permute-gather:
+three kernels, or one for decode-sized batches) -> moe_combine (the stand-in expert outputs replace
+the expert MLPs between gather and combine), replayed as one CUDA graph.  The decode workload also
+times every injected route pattern (routes given by the caller).  Inputs are resident in HBM; L2
+is flushed (a 256 MiB write) between timed steps (then a 256 MiB read, so no dirty flush lines
+are written back inside a timed step); every step is timed with CUDA events on the launching
+stream and the K step times are summed; the result is the max over ranks.  N > 1 runs one
+independent batch per GPU (weak scaling: the path has no cross-token exchange).  Rank 0 prints
+one JSON line.
 
-Also reported: per-stage device times and achieved HBM bandwidth from the algorithmic bytes,
+Also reported: per-stage device times and achieved HBM bandwidth from the algorithmic bytes (for
+the step's path and for the four stage entry points),
 the roofline of the dominant kernel against the measured copy peak, an end-to-end figure
 through MoeRouter.step_from_host (pinned host inputs copied in and the output copied back
 inside the timed region), SM clocks sampled during the timed region, and the CPU oracle
@@ -45,11 +47,12 @@ KERNEL_SOURCES = {
     "gather_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "combine_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "combine_small_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
-    "gate_count_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "gate_count_kernel+tile_scan_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "align_count_kernel+align_place_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
     "route_small_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
 }
 STAGE_KERNEL = {"topk": "topk_row_warp_kernel", "align": "align_cluster_kernel", "gather": "gather_tma_kernel",
-                "combine": "combine_tma_kernel", "dispatch": "gate_count_kernel+place_gather_kernel"}
+                "combine": "combine_tma_kernel", "dispatch": "gate_count_kernel+tile_scan_kernel+place_gather_kernel"}
 
 
 def parse_args():
@@ -296,9 +299,7 @@ def main():
     if r.small_batch:
         launches_per_step = 2  # route_small_kernel, combine_small_kernel
     else:
-        launches_per_step = 4  # topk_row_warp_kernel, align_cluster_kernel (or 2 tile kernels), gather, combine
-        if wl.T * wl.k > 65536 or wl.experts_local > 512:
-            launches_per_step = 5
+        launches_per_step = 4  # gate_count_kernel, tile_scan_kernel, place_gather_kernel, combine kernel
 
     use_graph = not args.no_graph
     graphs = {}
@@ -369,6 +370,8 @@ def main():
     stage_kernel = dict(STAGE_KERNEL)
     if r.small_batch:
         stage_kernel["dispatch"] = "route_small_kernel"
+    if wl.T * wl.k > 65536 or wl.experts_local > 512:  # beyond one cluster: the two-kernel align
+        stage_kernel["align"] = "align_count_kernel+align_place_kernel"
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     if wl.T * (-(-wl.H * 2 // 4096)) < sms:  # fewer 4 KB row chunks than SMs: the small-batch combine
         stage_kernel["combine"] = "combine_small_kernel"
@@ -413,9 +416,9 @@ def main():
                          [lambda: r.gate(logits), lambda: r.align_permute(),
                           lambda: r.gather(hidden, hidden_ready=True), lambda: r.combine(y)])
     stages_fused = stage_times(("dispatch", "combine"), [lambda: r.dispatch(logits, hidden), lambda: r.combine(y)])
-    # the dominant single kernel of the step: combine (about half of the bytes) on the four-call
-    # path; on the single-kernel dispatch path of small batches, the longer of its two kernels
-    in_step = stages_fused if r.small_batch else stages
+    # the dominant single kernel of the step: the combine (about half of the bytes) above the
+    # small-batch limits; for small batches the longer of the step's two kernels
+    in_step = stages_fused
     dom = max(in_step, key=lambda n: in_step[n]["us"]) if r.small_batch else "combine"
     ach = in_step[dom]["achieved_gbs"]
     total_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
@@ -466,8 +469,8 @@ def main():
     d2h = out_h.numel() * out_h.element_size()
     e2e = {"value": ws * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
            "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-           "api": f"MoeRouter.step_from_host (pinned H2D of logits+hidden, {launches_per_step if r.small_batch else 4} "
-                  f"C-ABI calls, D2H of out)"}
+           "api": "MoeRouter.step_from_host (pinned H2D of logits+hidden, moe_route_dispatch + moe_combine, "
+                  "D2H of out)"}
 
     if r.device_status() != tdt.MOE_OK:
         raise RuntimeError("device status after the timed steps is not MOE_OK")
@@ -493,8 +496,8 @@ def main():
             "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
             "routed_slots_local": R, "num_tokens_post_pad": npad,
             "step_path": "moe_route_dispatch (single kernel) + moe_combine" if r.small_batch else
-                         "moe_topk_softmax + moe_align_permute + moe_gather + moe_combine",
-            "roofline": roofline, "stages": stages, "stages_fused_dispatch_path": stages_fused, "e2e": e2e,
+                         "moe_route_dispatch (three kernels) + moe_combine",
+            "roofline": roofline, "stages": stages_fused, "stages_four_call_path": stages, "e2e": e2e,
             "decode_route_patterns": patterns,
             "cpu_baseline": cpu,
             "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,

@@ -459,8 +459,10 @@ __global__ void __launch_bounds__(kClusterThreads) align_cluster_kernel(AlignArg
   for (int i = tid; i < kClusterWarps * El; i += kClusterThreads) masks[i] = 0u;
   for (int i = El + tid; i < E4; i += kClusterThreads) cta_cnt[i] = 0;
   __syncthreads();
-  moe::pdl_wait();  // topk_ids come from the previous kernel
+  // let the next kernel start now: it waits for this one in turn, and the first kernel of the
+  // routing call has already waited for the producers of its inputs
   moe::pdl_launch_dependents();
+  moe::pdl_wait();  // topk_ids come from the previous kernel
   // 1. per-warp counts of the warp's own run
   int le[kAlignBatch];
   for (int64_t base = w0; base < w1; base += 32 * kAlignBatch) {

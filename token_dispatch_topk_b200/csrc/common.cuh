@@ -136,6 +136,12 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint3
                : "memory");
 }
 
+// Bring `bytes` of global memory into L2 ahead of use (no shared memory, nothing to wait for);
+// address and size 16-byte aligned.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
 // shared -> global bulk copy, tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src_smem)),
@@ -225,6 +231,29 @@ __device__ __forceinline__ void st_cluster_v4(const void* local_ptr, uint32_t ra
 namespace moe_host {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Dynamic shared memory to request so that at most `per_sm` CTAs of a kernel fit on one SM:
+// CTAs placed while other kernels still occupy SMs then spread evenly instead of piling onto the
+// idle SMs (a streaming kernel is as fast as its most loaded SM).  Returns 0 on a CUDA error.
+inline size_t smem_for_ctas_per_sm(size_t needed, int per_sm) {
+  int dev = 0, smem_sm = 0, rsv = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&rsv, cudaDevAttrReservedSharedMemoryPerBlock, dev) != cudaSuccess)
+    return 0;
+  // per_sm + 1 CTAs must not fit: (per_sm + 1) * (s + rsv) > smem_sm
+  size_t s = static_cast<size_t>(smem_sm) / static_cast<size_t>(per_sm + 1) + 1;
+  s = s > static_cast<size_t>(rsv) ? s - static_cast<size_t>(rsv) : 0;
+  s = (s + 15) & ~size_t{15};
+  return needed > s ? needed : s;
+}
+
+inline int sm_count() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return 0;
+  return sms;
+}
 
 inline moe_status_t launch_status() {
   cudaError_t e = cudaGetLastError();

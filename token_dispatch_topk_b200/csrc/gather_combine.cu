@@ -95,6 +95,7 @@ zero_pad_kernel(const int32_t* __restrict__ sorted_ids, const int32_t* __restric
 // ------------------------------------------------------------------------------------------
 constexpr int kGatherMaxTokensPerCta = 8;
 constexpr uint32_t kGatherCtaBytes = 32u * 1024u;  // hidden rows staged per CTA
+constexpr int kGatherCtasPerSm = 4;                 // gather_tma_kernel CTAs resident per SM
 
 // One warp per CTA: lane 0 bulk-loads the CTA's `tokens_per_cta` hidden rows into shared memory
 // while the lanes read the rows' destinations; then every lane bulk-stores the staged rows of its
@@ -461,11 +462,19 @@ extern "C" moe_status_t moe_gather(const void* hidden, int64_t T, int32_t H, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
   if (T > 0 && row_bytes <= kGatherCtaBytes * 4u) {
+    // tokens per CTA: at most kGatherMaxTokensPerCta (and kGatherCtaBytes of staged rows), and few
+    // enough that a batch fills kGatherCtasPerSm CTAs on every SM; shared memory sized so that no SM
+    // takes more (CTAs placed while the previous kernel runs would otherwise crowd its idle SMs)
     int tpc = static_cast<int>(kGatherCtaBytes / row_bytes);
     if (tpc < 1) tpc = 1;
     if (tpc > kGatherMaxTokensPerCta) tpc = kGatherMaxTokensPerCta;
+    const int sms = moe_host::sm_count();
+    if (sms <= 0) return MOE_ERR_CUDA;
+    const int64_t fill = (T + static_cast<int64_t>(sms) * kGatherCtasPerSm - 1) / (static_cast<int64_t>(sms) * kGatherCtasPerSm);
+    if (fill < tpc) tpc = fill < 1 ? 1 : static_cast<int>(fill);
     const int64_t blocks = (T + tpc - 1) / tpc;
-    const size_t smem = static_cast<size_t>(tpc) * row_bytes;
+    const size_t smem = moe_host::smem_for_ctas_per_sm(static_cast<size_t>(tpc) * row_bytes, kGatherCtasPerSm);
+    if (smem == 0) return MOE_ERR_CUDA;
     if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
     if (smem > 48 * 1024 &&
         cudaFuncSetAttribute(gather_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) !=

@@ -1,5 +1,5 @@
-// route_fused.cu -- fused dispatch: gating and expert counting in one kernel, placement and the
-// activation gather in the next.
+// route_fused.cu -- fused dispatch: gating, expert counting, the stable block-padded layout and the
+// activation gather, with the kernel boundaries placed for latency.
 //
 // Operations: the FusedMoE pipeline of "Upstream Reference: Deep-Spark xllm + vllm", "File
 // Index" (gate -> topk -> expand -> ...): topk_softmax (moe_topk_softmax_kernels.cuh), the
@@ -8,24 +8,24 @@
 // scheduler closure note.  The outputs are exactly those of moe_topk_softmax +
 // moe_align_permute + moe_gather; only the kernel boundaries move.
 //
-// gate_count_kernel (one CTA per tile of `rows_per_tile` tokens):
+// Batches above the small-batch limits take three kernels, chained by programmatic dependent
+// launch:
+// gate_count_kernel (one CTA per tile of kRowsPerTile tokens):
 //   A. each warp gates rows of the tile (gate_row: one warp per row) and writes topk_weights and
 //      topk_ids; the local expert of every slot of the tile goes to shared memory;
 //   B. stable ranks inside the tile: each warp owns a contiguous run of the tile's slots, counts
 //      it into its own shared-memory row, the rows are scanned across warps, and each slot's rank
 //      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm and the
-//      tile's per-expert counts go to the workspace;
-//   C. two-level scan with completion tickets (no spinning): the CTA that finishes last in its
-//      group of tiles scans the group's tile counters (staged through shared memory) into bases
-//      inside the group and publishes the group totals; the group that finishes last scans the
-//      group totals into group bases and writes counts, the block-padded offsets, N_pad and
-//      expert_ids.  Every ticket is reset by the CTA that used it last.
+//      tile's per-expert counts go to the workspace, expert-major ([E_local][tiles]).
+// tile_scan_kernel (one CTA per local expert): the expert's row of tile counts becomes the
+//   exclusive prefix over the tiles (the tile bases) and its total goes to the workspace.
+//   Nothing waits on another CTA: the kernel boundary is the only grid-wide step.
 // place_gather_kernel (one warp per CTA, up to 8 tokens, TMA staging as in gather_tma_kernel):
-//   each slot's row = offsets[e] + group base[e] + tile base[e] + rank (the rank and the expert
-//   were parked in inv_perm by the first kernel); the CTA writes sorted_token_ids and
-//   inv_perm for its slots, bulk-loads its hidden rows (before waiting for the previous kernel:
-//   hidden is an input of the call) and bulk-stores them to their rows; the pad rows, the tail
-//   rows past N_pad are spread over the CTAs.
+//   bulk-loads its hidden rows first (hidden is an input of the call, complete before the first
+//   kernel ran); scans the padded expert totals into the offsets itself (E_local values, in
+//   shared memory); each slot's row = offsets[e] + tile base[e] + rank; writes sorted_token_ids
+//   and inv_perm for its slots and bulk-stores the rows; the expert-owned outputs (counts,
+//   offsets, expert_ids, pad rows) and the tail past N_pad are spread over the CTAs.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -37,11 +37,13 @@ namespace {
 
 constexpr int kGcWarps = 16;
 constexpr int kGcThreads = kGcWarps * 32;
-constexpr int kWsHeaderBytes = 256;  // status word, ticket, padding
+constexpr int kWsHeaderBytes = 256;  // status word, padding
 constexpr int kRowsPerTile = 32;
-constexpr int kScanCap = 16384;  // ints of shared memory for staging a block of tile counters
+constexpr int kTsThreads = 128;  // tile_scan_kernel: threads per expert
 constexpr int kPgMaxTokens = 8;
 constexpr uint32_t kPgCtaBytes = 32u * 1024u;
+constexpr int kPgCtasPerSm = 4;  // place_gather_kernel CTAs resident per SM
+constexpr uint64_t kL2PrefetchMax = 48ull << 20;  // hidden bytes worth keeping in L2 through the routing
 
 struct DispatchArgs {
   const void* logits;
@@ -68,12 +70,11 @@ struct DispatchArgs {
   int32_t* n_pad;
   int32_t* inv_perm;
   int32_t* status;
-  unsigned int* ticket;
-  int32_t* tile_counts;         // [num_tiles][E_local]: tile counts, then bases inside the group
-  int tiles_per_group;
-  int num_groups;
-  unsigned int* group_tickets;  // [num_groups]
-  int32_t* group_counts;        // [num_groups][E_local]: group totals, then group bases
+  int32_t* tile_counts;  // [E_local][num_tiles]: tile counts, then tile bases
+  int32_t* totals;       // [E_local]
+  const uint8_t* hidden;  // prefetched into L2 by gate_count_kernel when prefetch_hidden
+  uint32_t row_bytes;
+  int prefetch_hidden;
 };
 
 // Local expert of global expert g (or -1: remote); out-of-range values are flagged.
@@ -102,95 +103,16 @@ __device__ __forceinline__ unsigned peers_of(unsigned* masks, int v, int lane) {
   return p;
 }
 
-// Exclusive scan of n <= 2 * kGcThreads ints in shared memory (block-wide, in place); returns the total.
-__device__ int scan_block(int* data, int n, int* warp_sums) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int i0 = 2 * tid, i1 = 2 * tid + 1;
-  const int x0 = i0 < n ? data[i0] : 0;
-  const int x1 = i1 < n ? data[i1] : 0;
-  int incl = x0 + x1;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const int v = __shfl_up_sync(0xffffffffu, incl, off);
-    if (lane >= off) incl += v;
-  }
-  if (lane == 31) warp_sums[warp] = incl;
-  __syncthreads();
-  if (warp == 0) {
-    int w = lane < kGcWarps ? warp_sums[lane] : 0;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, w, off);
-      if (lane >= off) w += v;
-    }
-    if (lane < kGcWarps) warp_sums[lane] = w;
-  }
-  __syncthreads();
-  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + incl - (x0 + x1);
-  const int total = warp_sums[kGcWarps - 1];
-  __syncthreads();
-  if (i0 < n) data[i0] = before;
-  if (i1 < n) data[i1] = before + x0;
-  __syncthreads();
-  return total;
+// Block-padded size of an expert with c slots: ceil(c / bs) * bs.
+__device__ __forceinline__ int padded_rows(int c, int bs, int bs_shift) {
+  if (c == 0) return 0;
+  return bs_shift >= 0 ? (((c + bs - 1) >> bs_shift) << bs_shift) : ((c + bs - 1) / bs) * bs;
 }
 
-// Shared memory of gate_count_kernel (ints):
-//   s_le[rows_per_tile * k] | work region: whist[kGcWarps][E_local] + masks[kGcWarps][E_local],
-//   later the staging buffer of the tile-counter scans | s_cnt[E_local] | s_off[E_local + 1] | warp_sums[32]
-__host__ __device__ inline size_t gc_work_ints(int E_local) {
-  const size_t w = 2 * static_cast<size_t>(kGcWarps) * E_local;
-  return w > static_cast<size_t>(kScanCap) ? w : static_cast<size_t>(kScanCap);
-}
+// Shared memory of gate_count_kernel (ints): s_le[rows_per_tile * k] | whist[kGcWarps][E_local] |
+// masks[kGcWarps][E_local]
 __host__ __device__ inline size_t gc_smem_ints(int rows_per_tile, int k, int E_local) {
-  return static_cast<size_t>(rows_per_tile) * k + gc_work_ints(E_local) + 2 * E_local + 1 + 32;
-}
-
-// In-place exclusive scan down the rows of a rows x cols int32 block in global memory (row
-// stride `cols`), column by column; column totals to `totals`.  The block is staged through
-// `buf` (cap ints of shared memory) in slices of columns, with coalesced, batched loads.
-// Block-wide (kGcThreads threads).
-__device__ void scan_columns(int32_t* g, int rows, int cols, int* buf, int cap, int* totals) {
-  const int tid = threadIdx.x;
-  int ec = cap / (rows > 0 ? rows : 1);
-  if (ec > cols) ec = cols;
-  if (ec < 1) ec = 1;
-  for (int c0 = 0; c0 < cols; c0 += ec) {
-    const int w = (cols - c0) < ec ? (cols - c0) : ec;
-    const int n = rows * w;
-    for (int i0 = tid; i0 < n; i0 += kGcThreads * 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * kGcThreads;
-        if (i < n) {
-          const int r = i / w;
-          v[u] = __ldcg(g + static_cast<int64_t>(r) * cols + c0 + (i - r * w));
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        const int i = i0 + u * kGcThreads;
-        if (i < n) buf[i] = v[u];
-      }
-    }
-    __syncthreads();
-    for (int j = tid; j < w; j += kGcThreads) {
-      int run = 0;
-      for (int r = 0; r < rows; ++r) {
-        const int x = buf[r * w + j];
-        buf[r * w + j] = run;
-        run += x;
-      }
-      totals[c0 + j] = run;
-    }
-    __syncthreads();
-    for (int i = tid; i < n; i += kGcThreads) {
-      const int r = i / w;
-      g[static_cast<int64_t>(r) * cols + c0 + (i - r * w)] = buf[i];
-    }
-    __syncthreads();
-  }
+  return static_cast<size_t>(rows_per_tile) * k + 2 * static_cast<size_t>(kGcWarps) * E_local;
 }
 
 template <typename TIn, int VEC, int CPL>
@@ -200,12 +122,6 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   int* s_le = smem;
   int* whist = s_le + RT * k;
   unsigned* masks = reinterpret_cast<unsigned*>(whist + kGcWarps * El);
-  int* work = whist;  // whist + masks, reused as the scan staging buffer
-  const int work_cap = static_cast<int>(gc_work_ints(El));
-  int* s_cnt = work + work_cap;
-  int* s_off = s_cnt + El;
-  int* warp_sums = s_off + El + 1;
-  __shared__ int s_is_last;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int tile = blockIdx.x;
@@ -218,6 +134,10 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   __syncthreads();
   moe::pdl_wait();  // the logits may come from the previous kernel
   moe::pdl_launch_dependents();
+  // the tile's hidden rows head for L2 while the tile is routed: the gather reads them from there
+  if (a.prefetch_hidden && tid < rows) {
+    moe::bulk_prefetch_l2(a.hidden + (row0 + tid) * static_cast<int64_t>(a.row_bytes), a.row_bytes);
+  }
 
   // A. gating, one warp per row (or the routes the caller gave)
   const TIn* logits = static_cast<const TIn*>(a.logits);
@@ -259,7 +179,7 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
       whist[w * El + e] = run;
       run += c;
     }
-    a.tile_counts[static_cast<int64_t>(tile) * El + e] = run;
+    a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = run;
   }
   __syncthreads();
   for (int c = c0; c < c1; ++c) {
@@ -276,68 +196,71 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
     if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
     __syncwarp();
   }
+}
 
-  // C. two-level scan of the tile counters.  The last CTA of each group of tiles turns the group's
-  //    tile counts into bases inside the group and publishes the group totals; the last group
-  //    to finish turns the group totals into group bases and writes the expert layout.
-  __threadfence();
-  __syncthreads();
-  const int grp = tile / a.tiles_per_group;
-  const int g0 = grp * a.tiles_per_group;
-  const int gt = (a.num_tiles - g0) < a.tiles_per_group ? (a.num_tiles - g0) : a.tiles_per_group;
-  if (tid == 0) s_is_last = (atomicAdd(&a.group_tickets[grp], 1u) == static_cast<unsigned>(gt - 1)) ? 1 : 0;
-  __syncthreads();
-  if (!s_is_last) return;
-  __threadfence();
-  scan_columns(a.tile_counts + static_cast<int64_t>(g0) * El, gt, El, work, work_cap, s_cnt);
-  for (int e = tid; e < El; e += kGcThreads) a.group_counts[static_cast<int64_t>(grp) * El + e] = s_cnt[e];
-  if (tid == 0) a.group_tickets[grp] = 0u;  // ready for the next call
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) s_is_last = (atomicAdd(a.ticket, 1u) == static_cast<unsigned>(a.num_groups - 1)) ? 1 : 0;
-  __syncthreads();
-  if (!s_is_last) return;
-  __threadfence();
-  scan_columns(a.group_counts, a.num_groups, El, work, work_cap, s_cnt);
-  __syncthreads();
-  for (int e = tid; e < El; e += kGcThreads) s_off[e] = ((s_cnt[e] + a.bs - 1) / a.bs) * a.bs;
-  __syncthreads();
-  const int total = scan_block(s_off, El, warp_sums);
-  if (tid == 0) {
-    s_off[El] = total;
-    a.offsets[El] = total;
-    a.n_pad[0] = total;
-    *a.ticket = 0u;  // ready for the next call
+// One CTA per local expert: its row of tile counts -> exclusive prefix over the tiles, in place;
+// the total to `totals`.  Thread i owns a contiguous run of tiles, read in unrolled batches so that
+// the loads of a run are in flight together.
+__global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
+  __shared__ int warp_sums[kTsThreads / 32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int e = blockIdx.x;
+  // let place_gather_kernel start now (it prefetches the hidden rows, then waits for this kernel,
+  // which completes after gate_count_kernel)
+  moe::pdl_launch_dependents();
+  moe::pdl_wait();  // tile counts come from gate_count_kernel
+  const int N = a.num_tiles;
+  int32_t* col = a.tile_counts + static_cast<int64_t>(e) * N;
+  const int per = (N + kTsThreads - 1) / kTsThreads;
+  const int t0 = tid * per < N ? tid * per : N;
+  const int t1 = t0 + per < N ? t0 + per : N;
+  int sum = 0;
+  for (int t = t0; t < t1; t += 8) {
+    int x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = t + u < t1 ? col[t + u] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) sum += x[u];
   }
-  for (int e = tid; e < El; e += kGcThreads) {
-    a.offsets[e] = s_off[e];
-    a.counts[e] = s_cnt[e];
+  int incl = sum;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
   }
+  if (lane == 31) warp_sums[warp] = incl;
   __syncthreads();
-  for (int b = tid; b < a.NB; b += kGcThreads) {
-    const int64_t row = static_cast<int64_t>(b) * a.bs;
-    int e = -1;
-    if (row < total) {
-      int lo = 0, hi = El - 1;  // largest e with s_off[e] <= row (empty experts share offsets)
-      while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
-      }
-      e = lo;
+  int run = incl - sum, total = 0;
+#pragma unroll
+  for (int w = 0; w < kTsThreads / 32; ++w) {
+    const int ws = warp_sums[w];
+    run += w < warp ? ws : 0;
+    total += ws;
+  }
+  for (int t = t0; t < t1; t += 8) {
+    int x[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) x[u] = t + u < t1 ? col[t + u] : 0;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (t + u < t1) col[t + u] = run;
+      run += x[u];
     }
-    a.expert_ids[b] = e;
   }
+  if (tid == 0) a.totals[e] = total;
 }
 
 // One warp per CTA: slots of tokens [t0, t0 + n) get their rows, the hidden rows are staged with
-// a bulk load and bulk-stored to every local row; then a share of the pad and tail rows.
+// a bulk load and bulk-stored to every local row; then a share of the expert-owned outputs, the
+// pad rows and the tail.  Shared memory: staged rows [tpc * row_bytes] | offsets [E_local + 1].
 __global__ void __launch_bounds__(32)
 place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t row_bytes, int tpc,
                     uint8_t* __restrict__ permuted) {
   extern __shared__ __align__(128) uint8_t rows[];
   __shared__ __align__(8) uint64_t bar;
+  int* s_off = reinterpret_cast<int*>(rows + static_cast<size_t>(tpc) * row_bytes);
   const int lane = threadIdx.x;
-  const int k = a.k, El = a.E_local;
+  const int k = a.k, El = a.E_local, bs = a.bs, bs_shift = a.bs_shift;
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * tpc;
   const int64_t left = a.T - t0;
   const int n = left <= 0 ? 0 : static_cast<int>(left < tpc ? left : tpc);
@@ -346,7 +269,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     moe::fence_barrier_init();
   }
   __syncwarp();
-  if (lane == 0 && n > 0) {  // hidden is an input of the call: complete before the previous kernel ran
+  if (lane == 0 && n > 0) {  // hidden is an input of the call: complete before the first kernel ran
     moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
     for (int i = 0; i < n; ++i) {
       moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes, hidden + (t0 + i) * static_cast<int64_t>(row_bytes),
@@ -354,7 +277,34 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     }
   }
   moe::pdl_launch_dependents();
-  moe::pdl_wait();  // ids, ranks, offsets and tile bases come from gate_count_kernel
+  moe::pdl_wait();  // ranks (gate_count_kernel), tile bases and totals (tile_scan_kernel)
+
+  // expert offsets: exclusive scan of the block-padded totals; lane l owns a contiguous run
+  {
+    const int per = (El + 31) >> 5;
+    const int e0 = lane * per < El ? lane * per : El;
+    const int e1 = e0 + per < El ? e0 + per : El;
+    int sum = 0;
+    for (int e = e0; e < e1; ++e) {
+      const int p = padded_rows(a.totals[e], bs, bs_shift);
+      s_off[e] = p;
+      sum += p;
+    }
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+    for (int e = e0; e < e1; ++e) {
+      const int p = s_off[e];
+      s_off[e] = run;
+      run += p;
+    }
+    if (lane == 31) s_off[El] = incl;
+    __syncwarp();
+  }
 
   const int nslots = n * k;  // <= kPgMaxTokens * 32
   int32_t dst[kPgMaxTokens];
@@ -367,9 +317,8 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
       const int v = a.inv_perm[s];  // (rank in the tile) << 10 | local expert, or -1
       if (v >= 0) {
         const int le = v & 1023;
-        const int64_t tile = (t0 + e / k) / a.rows_per_tile;
-        const int64_t grp = tile / a.tiles_per_group;
-        r = a.offsets[le] + a.group_counts[grp * El + le] + a.tile_counts[tile * El + le] + (v >> 10);
+        const int64_t tile = (t0 + e / k) / kRowsPerTile;
+        r = s_off[le] + a.tile_counts[static_cast<int64_t>(le) * a.num_tiles + tile] + (v >> 10);
         if (r < 0 || static_cast<int64_t>(r) >= a.C) {  // cannot happen for consistent inputs
           moe::record_status(a.status, MOE_ERR_BAD_ROW);
           r = -1;
@@ -397,16 +346,39 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     }
     moe::bulk_commit();
   }
-  // pad rows of every expert and the tail past N_pad hold the pad value
-  const int32_t pad_value = static_cast<int32_t>(a.P);
-  const int npad = a.offsets[El];
-  for (int e = blockIdx.x; e < El; e += gridDim.x) {
-    const int p1 = a.offsets[e + 1];
-    for (int p = a.offsets[e] + a.counts[e] + lane; p < p1; p += 32) a.sorted_ids[p] = pad_value;
+
+  // a share of the expert-owned outputs, the pad rows and the tail past N_pad
+  const int G = gridDim.x, b = blockIdx.x;
+  const int total = s_off[El];
+  for (int e = b * 32 + lane; e < El; e += G * 32) {
+    a.counts[e] = a.totals[e];
+    a.offsets[e] = s_off[e];
   }
-  const int64_t tail = a.C - npad;
-  for (int64_t i = static_cast<int64_t>(blockIdx.x) * 32 + lane; i < tail; i += static_cast<int64_t>(gridDim.x) * 32)
-    a.sorted_ids[npad + i] = pad_value;
+  if (b == 0 && lane == 0) {
+    a.offsets[El] = total;
+    a.n_pad[0] = total;
+  }
+  for (int64_t blk = static_cast<int64_t>(b) * 32 + lane; blk < a.NB; blk += static_cast<int64_t>(G) * 32) {
+    const int64_t row = blk * bs;
+    int e = -1;
+    if (row < total) {
+      int lo = 0, hi = El - 1;  // largest e with s_off[e] <= row (empty experts share offsets)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_off[mid] <= row) lo = mid; else hi = mid - 1;
+      }
+      e = lo;
+    }
+    a.expert_ids[blk] = e;
+  }
+  const int32_t pad_value = static_cast<int32_t>(a.P);
+  for (int e = b; e < El; e += G) {
+    const int p1 = s_off[e + 1];
+    for (int p = s_off[e] + a.totals[e] + lane; p < p1; p += 32) a.sorted_ids[p] = pad_value;
+  }
+  const int64_t tail = a.C - total;
+  for (int64_t i = static_cast<int64_t>(b) * 32 + lane; i < tail; i += static_cast<int64_t>(G) * 32)
+    a.sorted_ids[total + i] = pad_value;
   if (n > 0) moe::bulk_wait_read_all();  // the staged rows must outlive the stores that read them
 }
 
@@ -690,27 +662,18 @@ typename F<float, 1, 1>::Fn family_pick(int vec, int cpl) {
   }
 }
 
-// Tiles per group: a group's block of tile counters fits the shared-memory scan buffer.
-int tiles_per_group_for(int E_local) {
-  int g = kScanCap / E_local;
-  return g < 2 ? 2 : (g > 64 ? 64 : g);
-}
-
 struct FusedLayout {
-  int num_tiles, tiles_per_group, num_groups;
-  size_t group_tickets_off, tile_counts_off, group_counts_off, bytes;
+  int num_tiles;
+  size_t tile_counts_off, totals_off, bytes;
 };
 
 FusedLayout fused_layout(int64_t T, int E_local) {
   FusedLayout l{};
   const int64_t nt = (T + kRowsPerTile - 1) / kRowsPerTile;
   l.num_tiles = nt < 1 ? 1 : static_cast<int>(nt);
-  l.tiles_per_group = tiles_per_group_for(E_local);
-  l.num_groups = (l.num_tiles + l.tiles_per_group - 1) / l.tiles_per_group;
-  l.group_tickets_off = kWsHeaderBytes;
-  l.tile_counts_off = l.group_tickets_off + ((static_cast<size_t>(l.num_groups) * 4 + 255) & ~size_t{255});
-  l.group_counts_off = l.tile_counts_off + static_cast<size_t>(l.num_tiles) * E_local * 4;
-  l.bytes = l.group_counts_off + static_cast<size_t>(l.num_groups) * E_local * 4;
+  l.tile_counts_off = kWsHeaderBytes;
+  l.totals_off = l.tile_counts_off + ((static_cast<size_t>(l.num_tiles) * E_local * 4 + 255) & ~size_t{255});
+  l.bytes = l.totals_off + static_cast<size_t>(E_local) * 4;
   return l;
 }
 
@@ -770,8 +733,6 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   const FusedLayout lay = fused_layout(T, E_local);
   a.rows_per_tile = kRowsPerTile;
   a.num_tiles = lay.num_tiles;
-  a.tiles_per_group = lay.tiles_per_group;
-  a.num_groups = lay.num_groups;
   a.topk_weights = topk_weights;
   a.topk_ids = topk_ids;
   a.counts = counts;
@@ -781,10 +742,11 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.n_pad = num_tokens_post_pad;
   a.inv_perm = inv_perm;
   a.status = static_cast<int32_t*>(workspace);
-  a.ticket = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + 4);
-  a.group_tickets = reinterpret_cast<unsigned int*>(static_cast<char*>(workspace) + lay.group_tickets_off);
+  a.hidden = static_cast<const uint8_t*>(hidden);
+  a.row_bytes = row_bytes;
+  a.prefetch_hidden = static_cast<uint64_t>(T) * row_bytes <= kL2PrefetchMax ? 1 : 0;
   a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.tile_counts_off);
-  a.group_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.group_counts_off);
+  a.totals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.totals_off);
 
   // gating geometry: one warp per row, widest aligned vector that spreads the row over the warp
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
@@ -827,13 +789,24 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     return MOE_ERR_CUDA;
   if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
     return MOE_ERR_CUDA;
+  if (moe_host::launch_pdl(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
+      MOE_OK)
+    return MOE_ERR_CUDA;
 
+  // tokens per CTA: at most kPgMaxTokens (and kPgCtaBytes of staged rows), and few enough that a
+  // batch fills kPgCtasPerSm CTAs on every SM; shared memory sized so that no SM takes more
   int tpc = static_cast<int>(kPgCtaBytes / row_bytes);
   tpc = tpc < 1 ? 1 : (tpc > kPgMaxTokens ? kPgMaxTokens : tpc);
+  const int sms = moe_host::sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  const int64_t fill = (T + static_cast<int64_t>(sms) * kPgCtasPerSm - 1) / (static_cast<int64_t>(sms) * kPgCtasPerSm);
+  if (fill < tpc) tpc = fill < 1 ? 1 : static_cast<int>(fill);
   int64_t blocks = (T + tpc - 1) / tpc;
   if (blocks < 1) blocks = 1;
   if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
-  const size_t smem2 = static_cast<size_t>(tpc) * row_bytes;
+  const size_t smem2 = moe_host::smem_for_ctas_per_sm(
+      static_cast<size_t>(tpc) * row_bytes + static_cast<size_t>(E_local + 1) * sizeof(int), kPgCtasPerSm);
+  if (smem2 == 0) return MOE_ERR_CUDA;
   if (smem2 > 48 * 1024 &&
       cudaFuncSetAttribute(place_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2)) !=
           cudaSuccess)

@@ -1,8 +1,9 @@
 """MoeRouter: the routing path for fixed sizes with every buffer preallocated on the device.
 
-One ``step`` runs the routing path on one stream: for decode-sized batches the single-kernel
-moe_route_dispatch (gating + align + permute-gather) then moe_combine; above that the four stages
-moe_topk_softmax -> moe_align_permute -> moe_gather -> (caller's experts) -> moe_combine.
+One ``step`` runs the routing path on one stream: moe_route_dispatch (gating + align +
+permute-gather; one kernel for decode-sized batches, three above) -> (caller's experts) ->
+moe_combine.  ``step_staged`` runs the same path through the four stage entry points
+moe_topk_softmax -> moe_align_permute -> moe_gather -> moe_combine.
 No allocation, host synchronisation or Python-side arithmetic happens inside a step, so
 it can be captured in a CUDA graph.  ``step_from_host`` is the end-to-end form: it copies
 the step's inputs from (pinned) host memory, runs the step and copies the result back.
@@ -76,11 +77,9 @@ class MoeRouter:
     def step(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
         """gate + align + permute-gather + combine; expert_out stands in for the expert MLPs' output.
 
-        Decode-sized batches take the single-kernel dispatch then combine (two kernels); larger ones
-        the four stage entry points, which measured faster there than the two-kernel dispatch."""
-        if self.small_batch:
-            return self.step_fused(logits, hidden, expert_out, stream)
-        return self.step_staged(logits, hidden, expert_out, stream)
+        Runs the fused dispatch (one kernel for decode-sized batches, three above) then the combine;
+        it measured faster than the four stage entry points at every size."""
+        return self.step_fused(logits, hidden, expert_out, stream)
 
     def step_staged(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor,
                     stream=None) -> torch.Tensor:
