@@ -248,6 +248,15 @@ inline size_t smem_for_ctas_per_sm(size_t needed, int per_sm) {
   return needed > s ? needed : s;
 }
 
+// Tokens per CTA for a one-pass kernel over T tokens with `slots` CTAs resident at a time and at
+// most tpc_max tokens per CTA: the fewest full waves, each as evenly filled as possible.
+inline int tokens_per_cta(int64_t T, int tpc_max, int64_t slots) {
+  if (T <= 0 || slots <= 0) return tpc_max;
+  const int64_t waves = (T + slots * tpc_max - 1) / (slots * tpc_max);
+  const int64_t tpc = (T + slots * waves - 1) / (slots * waves);
+  return tpc < 1 ? 1 : static_cast<int>(tpc);
+}
+
 inline int sm_count() {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)

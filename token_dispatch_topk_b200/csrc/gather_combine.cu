@@ -162,7 +162,7 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
 constexpr int kCombineConsumerWarps = 8;
 constexpr int kCombineMaxStages = 8;
 constexpr uint32_t kCombineStageTarget = 32u * 1024u;  // bytes of slot rows per stage (about)
-constexpr uint32_t kCombineRingTarget = 96u * 1024u;   // bytes of stages per CTA (about)
+constexpr uint32_t kCombineRingTarget = 64u * 1024u;   // bytes of stages per CTA (about)
 
 struct CombineArgs {
   const uint8_t* y;         // expert_out [capacity, H] bf16
@@ -462,16 +462,15 @@ extern "C" moe_status_t moe_gather(const void* hidden, int64_t T, int32_t H, int
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const uint32_t row_bytes = static_cast<uint32_t>(H) * 2u;
   if (T > 0 && row_bytes <= kGatherCtaBytes * 4u) {
-    // tokens per CTA: at most kGatherMaxTokensPerCta (and kGatherCtaBytes of staged rows), and few
-    // enough that a batch fills kGatherCtasPerSm CTAs on every SM; shared memory sized so that no SM
+    // tokens per CTA: at most kGatherMaxTokensPerCta (and kGatherCtaBytes of staged rows), chosen so
+    // that the CTAs fill whole waves of kGatherCtasPerSm per SM; shared memory sized so that no SM
     // takes more (CTAs placed while the previous kernel runs would otherwise crowd its idle SMs)
     int tpc = static_cast<int>(kGatherCtaBytes / row_bytes);
     if (tpc < 1) tpc = 1;
     if (tpc > kGatherMaxTokensPerCta) tpc = kGatherMaxTokensPerCta;
     const int sms = moe_host::sm_count();
     if (sms <= 0) return MOE_ERR_CUDA;
-    const int64_t fill = (T + static_cast<int64_t>(sms) * kGatherCtasPerSm - 1) / (static_cast<int64_t>(sms) * kGatherCtasPerSm);
-    if (fill < tpc) tpc = fill < 1 ? 1 : static_cast<int>(fill);
+    tpc = moe_host::tokens_per_cta(T, tpc, static_cast<int64_t>(sms) * kGatherCtasPerSm);
     const int64_t blocks = (T + tpc - 1) / tpc;
     const size_t smem = moe_host::smem_for_ctas_per_sm(static_cast<size_t>(tpc) * row_bytes, kGatherCtasPerSm);
     if (smem == 0) return MOE_ERR_CUDA;

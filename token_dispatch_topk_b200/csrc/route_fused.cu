@@ -793,14 +793,13 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
       MOE_OK)
     return MOE_ERR_CUDA;
 
-  // tokens per CTA: at most kPgMaxTokens (and kPgCtaBytes of staged rows), and few enough that a
-  // batch fills kPgCtasPerSm CTAs on every SM; shared memory sized so that no SM takes more
+  // tokens per CTA: at most kPgMaxTokens (and kPgCtaBytes of staged rows), chosen so that the CTAs
+  // fill whole waves of kPgCtasPerSm per SM; shared memory sized so that no SM takes more
   int tpc = static_cast<int>(kPgCtaBytes / row_bytes);
   tpc = tpc < 1 ? 1 : (tpc > kPgMaxTokens ? kPgMaxTokens : tpc);
   const int sms = moe_host::sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
-  const int64_t fill = (T + static_cast<int64_t>(sms) * kPgCtasPerSm - 1) / (static_cast<int64_t>(sms) * kPgCtasPerSm);
-  if (fill < tpc) tpc = fill < 1 ? 1 : static_cast<int>(fill);
+  tpc = moe_host::tokens_per_cta(T, tpc, static_cast<int64_t>(sms) * kPgCtasPerSm);
   int64_t blocks = (T + tpc - 1) / tpc;
   if (blocks < 1) blocks = 1;
   if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
