@@ -6,12 +6,14 @@
 One step = MoeRouter.step over one batch: moe_route_dispatch (gating + align + permute-gather:
 three kernels, or one for decode-sized batches) -> moe_combine (the stand-in expert outputs replace
 the expert MLPs between gather and combine), replayed as one CUDA graph.  The decode workload also
-times every injected route pattern (routes given by the caller).  Inputs are resident in HBM; L2
-is flushed (a 256 MiB write) between timed steps (then a 256 MiB read, so no dirty flush lines
-are written back inside a timed step); every step is timed with CUDA events on the launching
-stream and the K step times are summed; the result is the max over ranks.  N > 1 runs one
-independent batch per GPU (weak scaling: the path has no cross-token exchange).  Rank 0 prints
-one JSON line.
+times every injected route pattern (routes given by the caller).  Inputs are resident in HBM.
+When one step moves more bytes than L2 holds (the prefill workloads), the K steps are replayed
+back to back between one pair of CUDA events on the launching stream; otherwise L2 is flushed (a
+256 MiB write, then a 256 MiB read, so no dirty flush lines are written back inside a timed step)
+before each step and every step is timed with its own pair of events (``--flush-always`` forces
+this mode; the flushed figure is reported beside the other).  The result is the max over ranks.
+N > 1 runs one independent batch per GPU (weak scaling: the path has no cross-token exchange).
+Rank 0 prints one JSON line.
 
 Also reported: per-stage device times and achieved HBM bandwidth from the algorithmic bytes (for
 the step's path and for the four stage entry points),
@@ -63,7 +65,9 @@ def parse_args():
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
     p.add_argument("--workload", default=None, help="workload name (default: the Qwen3-MoE-like prefill)")
     p.add_argument("--seed", type=int, default=0)
-    p.add_argument("--no-graph", action="store_true", help="launch the four calls directly instead of a graph")
+    p.add_argument("--no-graph", action="store_true", help="launch the calls directly instead of a graph")
+    p.add_argument("--flush-always", action="store_true",
+                   help="flush L2 before every timed step even when a step moves more bytes than L2 holds")
     p.add_argument("--stage-steps", type=int, default=None,
                    help="instrumented steps for the per-stage breakdown (default: min(steps, 500))")
     p.add_argument("--e2e-steps", type=int, default=None, help="timed end-to-end steps (default: min(steps, 200))")
@@ -333,6 +337,26 @@ def main():
         stream.synchronize()
         return sum(a.elapsed_time(b) for a, b in evs)
 
+    def timed_back_to_back(name, iters, warm):
+        """Time (ms) of `iters` steps replayed back to back between one pair of events (no flush:
+        used when one step's bytes exceed L2, so no step finds its inputs left there by the last)."""
+        with torch.cuda.stream(stream):
+            for i in range(warm):
+                run(name)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for i in range(iters):
+                run(name)
+            b.record(stream)
+        stream.synchronize()
+        return a.elapsed_time(b)
+
+    abytes = algorithmic_bytes(wl, R, r.capacity, NB)
+    step_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
+    l2_bytes = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20))
+    back_to_back = step_bytes > l2_bytes and not args.flush_always
+
     # ---- the timed region: K steps
     uuid = None
     try:
@@ -346,7 +370,10 @@ def main():
     if sampler:
         sampler.start()
         time.sleep(0.4)
-    total_ms = timed("step", args.steps, args.warmup)
+    if back_to_back:
+        total_ms = timed_back_to_back("step", args.steps, args.warmup)
+    else:
+        total_ms = timed("step", args.steps, args.warmup)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
     if ws > 1:
@@ -356,6 +383,10 @@ def main():
         dist.barrier()
     ms_per_step = total_ms / args.steps
     value = ws * wl.T * args.steps / (total_ms / 1e3)
+    # the same step with L2 flushed before each step and events around each step (adds the
+    # launch-to-event latency of a lone graph, about 5 us, to every step)
+    n_fl = min(args.steps, 200)
+    flushed_ms_per_step = (timed("step", n_fl, 3) / n_fl) if back_to_back else ms_per_step
 
     # ---- per-stage times inside the step, and roofline
     # The step is captured once more with external event records between its stages, so each
@@ -363,7 +394,6 @@ def main():
     # fused step has two stages (dispatch = gate_count + place_gather kernels, then combine); the
     # four stage entry points are timed the same way for comparison.
     peak, peak_src = measured_peaks()
-    abytes = algorithmic_bytes(wl, R, r.capacity, NB)
     abytes["dispatch"] = abytes["topk"] + abytes["align"] + abytes["gather"]
     st_iters = args.stage_steps or min(args.steps, 500)
 
@@ -417,14 +447,55 @@ def main():
                           lambda: r.gather(hidden, hidden_ready=True), lambda: r.combine(y)])
     stages_fused = stage_times(("dispatch", "combine"), [lambda: r.dispatch(logits, hidden), lambda: r.combine(y)])
     # the dominant single kernel of the step: the combine (about half of the bytes) above the
-    # small-batch limits; for small batches the longer of the step's two kernels
+    # small-batch limits; for small batches the longer of the step's two kernels.  Its launch time
+    # is measured without the per-step event floor: a graph of n x [L2 flush, launch] minus a graph
+    # of n x [L2 flush], both replayed between one pair of events on the launching stream.
+    def launch_us(fn, n=20, reps=5):
+        def cap(body):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                body()
+            return g
+
+        def both():
+            for i in range(n):
+                flush(i)
+                fn()
+
+        def flush_only():
+            for i in range(n):
+                flush(i)
+
+        ga, gb = cap(both), cap(flush_only)
+        res = []
+        with torch.cuda.stream(stream):
+            for g in (ga, gb):
+                g.replay()
+                ts = []
+                for _ in range(reps):
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record(stream)
+                    g.replay()
+                    e1.record(stream)
+                    ts.append((e0, e1))
+                stream.synchronize()
+                res.append(statistics.median(a.elapsed_time(b) for a, b in ts))
+        del ga, gb
+        return 1e3 * (res[0] - res[1]) / n
+
     in_step = stages_fused
-    dom = max(in_step, key=lambda n: in_step[n]["us"]) if r.small_batch else "combine"
-    ach = in_step[dom]["achieved_gbs"]
+    if r.small_batch:
+        dom = max(in_step, key=lambda n: in_step[n]["us"])
+    else:
+        dom = "combine"
+    dom_fn = (lambda: r.combine(y)) if dom == "combine" else (lambda: r.dispatch(logits, hidden))
+    dom_us = launch_us(dom_fn)
+    ach = abytes[dom] / (dom_us * 1e-6) / 1e9
     total_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
     roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": ncu_traffic(stage_kernel[dom], wl.name), "kernel": stage_kernel[dom],
-                "peak_source": peak_src,
+                "peak_source": peak_src, "launch_us": dom_us,
+                "timing": "graph of 20 x [L2 flush, launch] minus graph of 20 x [L2 flush], per launch",
                 "algorithmic_bytes_per_launch": abytes[dom]}
 
     # ---- injected route patterns of the decode workload: the step for routes given by the caller
@@ -487,14 +558,17 @@ def main():
             "dtype_detail": "bf16 activations, fp32 gating math and combine accumulation, int32 indices",
             "data": "synthetic (seeded; see token_dispatch_topk_b200/inputs.py)",
             "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
-                       "l2": f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write + "
-                             f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)",
+                       "l2": (f"not flushed: steps replayed back to back, each moving {step_bytes / 2**20:.0f} MiB "
+                              f"> L2 ({l2_bytes >> 20} MiB)") if back_to_back else
+                             (f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write + "
+                              f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)"),
                        "cuda_graph": use_graph,
                        "parallelism": "one independent batch per GPU" if ws > 1 else "single GPU"},
             "achieved_hbm_gbs": total_bytes / (ms_per_step * 1e-3) / 1e9,
             "algorithmic_bytes_per_step": total_bytes,
             "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
             "routed_slots_local": R, "num_tokens_post_pad": npad,
+            "flushed_ms_per_step": flushed_ms_per_step,
             "step_path": "moe_route_dispatch (single kernel) + moe_combine" if r.small_batch else
                          "moe_route_dispatch (three kernels) + moe_combine",
             "roofline": roofline, "stages": stages_fused, "stages_four_call_path": stages, "e2e": e2e,

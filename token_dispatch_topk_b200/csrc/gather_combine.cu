@@ -235,19 +235,19 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
         }
       }
     };
-    int64_t cur = u0 / a.nchunks;  // token group
+    int64_t grp = u0 / a.nchunks;  // token group of unit u (advanced without dividing)
+    int c = static_cast<int>(u0 - grp * a.nchunks);
     int r_cur, r_next;
     float w_cur, w_next;
-    load_meta(cur, r_cur, w_cur);
-    load_meta(cur + 1, r_next, w_next);
+    load_meta(grp, r_cur, w_cur);
+    load_meta(grp + 1, r_next, w_next);
     int s = 0;
     uint32_t round = 0;  // completed passes over the ring
     int64_t issued = 0;
     for (int64_t u = u0; u < u1; ++u, ++issued) {
-      const int64_t grp = u / a.nchunks;
-      const int c = static_cast<int>(u - grp * a.nchunks);
-      if (grp != cur) {  // units are in group order: advance one group and prefetch the next
-        cur = grp;
+      if (u != u0 && ++c == a.nchunks) {  // units are in group order: next group, prefetch the one after
+        c = 0;
+        ++grp;
         r_cur = r_next;
         w_cur = w_next;
         load_meta(grp + 1, r_next, w_next);
@@ -290,7 +290,13 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
   constexpr int NCT = kCombineConsumerWarps * 32;
   int s = 0;
   uint32_t round = 0;
+  int64_t grp = u0 / a.nchunks;  // token group of unit u (advanced without dividing)
+  int c = static_cast<int>(u0 - grp * a.nchunks) - 1;
   for (int64_t u = u0; u < u1; ++u) {
+    if (++c == a.nchunks) {
+      c = 0;
+      ++grp;
+    }
     if (ct == 0 && !moe::mbar_wait(&full[s], round & 1u)) {
       moe::record_status(a.status, MOE_ERR_TIMEOUT);
       s_abort = 1;
@@ -299,8 +305,6 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
     if (s_abort) break;
     while (!moe::mbar_try_wait(&full[s], round & 1u)) {
     }  // completed already: gives this thread its own acquire of the stage
-    const int64_t grp = u / a.nchunks;
-    const int c = static_cast<int>(u - grp * a.nchunks);
     const uint32_t cb = (c == a.nchunks - 1) ? a.row_bytes - static_cast<uint32_t>(c) * a.chunk_bytes : a.chunk_bytes;
     const uint32_t mask = s_mask[s];
     const uint8_t* stage = buf + static_cast<size_t>(s) * stage_bytes;
