@@ -503,7 +503,7 @@ def main():
     patterns = None
     if wl.name.startswith("ep_decode"):
         w_inj = I.decode_pattern_weights(seed=seed).to(dev)
-        patterns = {}
+        patterns, device = {}, {}
         for pname in I.DECODE_PATTERNS:
             ids_p = I.decode_pattern_ids(pname).to(dev)
             fn = (lambda ids_p=ids_p: r.step_routes(ids_p, w_inj, hidden, y))
@@ -512,8 +512,13 @@ def main():
             stage_fns["pattern"] = fn
             n_it = min(args.steps, 500)
             patterns[pname] = 1e3 * timed("pattern", n_it, min(args.warmup, 10)) / n_it
+            device[pname] = launch_us(fn)
+        device["logits"] = launch_us(lambda: r.step(logits, hidden, y))
         patterns = {"us_per_step": patterns, "worst_us": max(patterns.values()),
                     "worst": max(patterns, key=patterns.get),
+                    "device_us_per_step": device, "device_worst_us": max(device.values()),
+                    "device_timing": "graph of 20 x [L2 flush, step] minus graph of 20 x [L2 flush], per step "
+                                     "(kernels and the gaps between them, without the per-step event latency)",
                     "path": "MoeRouter.step_routes: moe_route_dispatch (given routes) + moe_combine, one graph each"}
         if r.device_status() != tdt.MOE_OK:
             raise RuntimeError("device status after the route-pattern steps is not MOE_OK")
