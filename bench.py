@@ -79,10 +79,8 @@ def parse_args():
 
 # ------------------------------------------------------------------------- helpers --
 def dist_env():
-    ws = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    return ws, rank, local
+    from token_dispatch_topk_b200.dist import rank_env
+    return rank_env()
 
 
 def measured_peaks():
@@ -262,6 +260,7 @@ def main():
     import torch
     import torch.distributed as dist
     import token_dispatch_topk_b200 as tdt
+    from token_dispatch_topk_b200.dist import max_over_ranks, rank_seed
 
     ws, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -269,7 +268,7 @@ def main():
     if ws > 1:
         from datetime import timedelta
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
-    seed = args.seed + rank  # an independent batch per rank
+    seed = rank_seed(args.seed, rank)  # an independent batch per rank
     tdt.load_library()
 
     # ---- inputs resident in HBM
@@ -376,10 +375,8 @@ def main():
         total_ms = timed("step", args.steps, args.warmup)
     torch.cuda.synchronize()
     clocks = sampler.stop() if sampler else None
+    total_ms = max_over_ranks(total_ms, dev)
     if ws > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
         dist.barrier()
     ms_per_step = total_ms / args.steps
     value = ws * wl.T * args.steps / (total_ms / 1e3)
@@ -537,10 +534,7 @@ def main():
             b.record(stream)
     stream.synchronize()
     e2e_ms = sum(a.elapsed_time(b) for a, b in evs)
-    if ws > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, dev)
     h2d = lp.numel() * lp.element_size() + hp.numel() * hp.element_size()
     d2h = out_h.numel() * out_h.element_size()
     e2e = {"value": ws * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,

@@ -1,0 +1,129 @@
+"""The multi-process path on the CPU: two gloo ranks (world size 2), no GPU.
+
+  * data parallel: each rank gets its own seed, and the timing reduction returns the maximum
+    over the ranks;
+  * expert parallel: each rank owns a contiguous block of experts (``ep_expert_map``), routes the
+    same tokens with its map (the oracle stands in for the rank's kernels here), combines its
+    local slots into a bf16 partial, and ``ep_reduce_partials`` sums the partials over the ranks.
+    The result must match the oracle's single-rank combine of all slots within the rounding of
+    the two partials and the final sum; the expert outputs are a function of (global expert,
+    token) so that every rank builds its own expert-grouped rows consistently.
+"""
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import oracle
+from token_dispatch_topk_b200 import dist as D
+from token_dispatch_topk_b200 import inputs as I
+
+from oracle_pins import bf16_bits_to_f32, f32_to_bf16_bits
+
+
+def _free_port() -> int:
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _expert_rows(ids_rows_experts, tokens, H):
+    """Expert output row of (global expert e, token t): bf16 values from a fixed formula."""
+    e = np.asarray(ids_rows_experts, np.float64)[:, None]
+    t = np.asarray(tokens, np.float64)[:, None]
+    h = np.arange(H, dtype=np.float64)[None, :]
+    v = np.sin(0.37 * e + 0.11 * h) * np.cos(0.23 * t - 0.05 * h) * 3.0
+    return f32_to_bf16_bits(v.astype(np.float32))
+
+
+def _rank_partial(logits_bits, T, E, k, H, bs, world, rank):
+    """One expert-parallel rank: route with its map, build its expert-grouped rows, combine its slots."""
+    w, ids = oracle.topk_softmax(logits_bits, k, True)
+    emap, El = D.ep_expert_map(E, world, rank)
+    al = oracle.align_permute(ids, E, bs, emap.numpy(), El)
+    C = al["capacity"]
+    inv = al["inv_perm"]
+    y = np.zeros((C, H), np.uint16)
+    rows = np.nonzero(inv >= 0)[0]
+    if rows.size:
+        y[inv[rows]] = _expert_rows(ids.reshape(-1)[rows], rows // k, H)
+    return w, ids, oracle.combine(y, w, inv)
+
+
+def _worker(rank, world, port, q):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        out = {"seed": D.rank_seed(5, rank), "max": D.max_over_ranks(1.5 + rank)}
+        wl = I.WORKLOADS["tiny_T64_E8_k2"]
+        T, E, k, H, bs = 24, 16, 4, 64, 8
+        logits = I.make_logits(wl, T=T)  # bf16 [T, 8]: widen to 16 experts deterministically
+        logits = torch.cat([logits, logits.flip(1) * 0.5], dim=1).contiguous()
+        bits = logits.view(torch.int16).numpy().view(np.uint16)
+        _, _, partial = _rank_partial(bits, T, E, k, H, bs, world, rank)
+        summed = D.ep_reduce_partials(torch.from_numpy(partial.view(np.int16)).view(torch.bfloat16))
+        out["partial"] = partial
+        out["summed"] = summed.view(torch.int16).numpy().view(np.uint16)
+        out["bits"] = bits
+        q.put((rank, out))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.fixture(scope="module")
+def two_ranks():
+    oracle.default()
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict(q.get(timeout=180) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    return res
+
+
+def test_data_parallel_seeds_and_max_over_ranks(two_ranks):
+    assert two_ranks[0]["seed"] != two_ranks[1]["seed"]
+    assert two_ranks[0]["max"] == two_ranks[1]["max"] == 2.5
+
+
+def test_expert_parallel_partials_sum_to_the_full_combine(two_ranks):
+    T, E, k, H, bs = 24, 16, 4, 64, 8
+    bits = two_ranks[0]["bits"]
+    assert np.array_equal(bits, two_ranks[1]["bits"])
+    s0, s1 = two_ranks[0]["summed"], two_ranks[1]["summed"]
+    assert np.array_equal(s0, s1), "every rank holds the same reduced output"
+    # single rank owning every expert
+    w, ids, full = _rank_partial(bits, T, E, k, H, bs, 1, 0)
+    p0 = bf16_bits_to_f32(two_ranks[0]["partial"]).astype(np.float64)
+    p1 = bf16_bits_to_f32(two_ranks[1]["partial"]).astype(np.float64)
+    got = bf16_bits_to_f32(s0).astype(np.float64)
+    want = bf16_bits_to_f32(full).astype(np.float64)
+
+    def ulp(x):  # one bf16 ulp at |x| (normal range)
+        e = np.floor(np.log2(np.maximum(np.abs(x), 2.0 ** -120)))
+        return 2.0 ** (e - 7)
+
+    # each partial and the final sum are rounded once to bf16, the full combine once
+    bound = 0.5 * (ulp(p0) + ulp(p1) + ulp(got) + ulp(want)) + 1e-6 * (np.abs(p0) + np.abs(p1))
+    assert (np.abs(got - want) <= bound).all(), np.max(np.abs(got - want) - bound)
+    # and the partials cover disjoint expert blocks: each slot is local on exactly one rank
+    lo0, hi0 = D.ep_expert_range(E, 2, 0)
+    lo1, hi1 = D.ep_expert_range(E, 2, 1)
+    assert (lo0, hi0, lo1, hi1) == (0, 8, 8, 16)
+
+
+def test_ep_expert_range_splits_evenly():
+    assert [D.ep_expert_range(10, 4, r) for r in range(4)] == [(0, 3), (3, 6), (6, 8), (8, 10)]
+    m, El = D.ep_expert_map(160, 4, 1)
+    assert El == 40 and m[40].item() == 0 and m[79].item() == 39 and m[39].item() == -1 and m[80].item() == -1
+    with pytest.raises(ValueError):
+        D.ep_expert_range(3, 4, 0)
