@@ -69,6 +69,8 @@ class Oracle:
         lib = ctypes.CDLL(lib_path)
         lib.oracle_topk_softmax.argtypes = [_P, ctypes.c_int, _I64, _I32, _I32, ctypes.c_int, _P, _P]
         lib.oracle_topk_softmax.restype = ctypes.c_int
+        lib.oracle_topk_sigmoid.argtypes = [_P, ctypes.c_int, _I64, _I32, _I32, ctypes.c_int, _P, _P]
+        lib.oracle_topk_sigmoid.restype = ctypes.c_int
         lib.oracle_align_capacity.argtypes = [_I64, _I32, _I32, _I32]
         lib.oracle_align_capacity.restype = _I64
         lib.oracle_align_permute.argtypes = [_P, _I64, _I32, _I32, _P, _I32, _I32, _P, _P, _P, _P, _P, _P]
@@ -94,6 +96,22 @@ class Oracle:
         ids = np.empty((T, k), np.int32)
         _check(self._lib.oracle_topk_softmax(_ptr(logits), dtype, T, E, k, int(bool(renormalize)),
                                              _ptr(w), _ptr(ids)), "topk_softmax")
+        return w, ids
+
+    def topk_sigmoid(self, logits: np.ndarray, k: int, renormalize: bool):
+        """Sigmoid-scored top-k: the same selection, weights 1/(1+exp(-x)) (optionally renormalised)."""
+        logits = np.ascontiguousarray(logits)
+        if logits.dtype == np.uint16:
+            dtype = 1
+        elif logits.dtype == np.float32:
+            dtype = 0
+        else:
+            raise TypeError(f"logits must be float32 or bf16 bits (uint16), got {logits.dtype}")
+        T, E = logits.shape
+        w = np.empty((T, k), np.float32)
+        ids = np.empty((T, k), np.int32)
+        _check(self._lib.oracle_topk_sigmoid(_ptr(logits), dtype, T, E, k, int(bool(renormalize)),
+                                             _ptr(w), _ptr(ids)), "topk_sigmoid")
         return w, ids
 
     def align_capacity(self, T: int, k: int, E_local: int, block_size: int) -> int:
@@ -169,6 +187,10 @@ def default() -> Oracle:
 
 def topk_softmax(logits, k, renormalize):
     return default().topk_softmax(logits, k, renormalize)
+
+
+def topk_sigmoid(logits, k, renormalize):
+    return default().topk_sigmoid(logits, k, renormalize)
 
 
 def align_capacity(T, k, E_local, block_size):

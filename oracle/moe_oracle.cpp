@@ -60,6 +60,23 @@ double logit_as_double(const void* logits, int dtype, int64_t idx) {
     return static_cast<double>(static_cast<const float*>(logits)[idx]);
 }
 
+/* k rounds of "first maximum among the experts not yet taken": the largest logit, the lowest
+ * expert index among equal logits (reading: lowest-index tie-break, selection made on the
+ * logits themselves). */
+void select_topk(const std::vector<double>& x, int32_t E, int32_t k, std::vector<char>& taken,
+                 std::vector<int32_t>& sel) {
+    for (int32_t e = 0; e < E; ++e) taken[e] = 0;
+    for (int32_t j = 0; j < k; ++j) {
+        int32_t best = -1;
+        for (int32_t e = 0; e < E; ++e) {
+            if (taken[e]) continue;
+            if (best < 0 || x[e] > x[best]) best = e; /* strict '>' keeps the lowest index */
+        }
+        taken[best] = 1;
+        sel[j] = best;
+    }
+}
+
 }  // namespace
 
 extern "C" {
@@ -92,20 +109,9 @@ int oracle_topk_softmax(const void* logits, int dtype, int64_t T, int32_t E, int
     std::vector<int32_t> sel(static_cast<size_t>(k));
 
     for (int64_t t = 0; t < T; ++t) {
-        for (int32_t e = 0; e < E; ++e) {
-            x[e] = logit_as_double(logits, dtype, t * E + e);
-            taken[e] = 0;
-        }
+        for (int32_t e = 0; e < E; ++e) x[e] = logit_as_double(logits, dtype, t * E + e);
         /* step 1: k rounds of "first maximum among the experts not yet taken" */
-        for (int32_t j = 0; j < k; ++j) {
-            int32_t best = -1;
-            for (int32_t e = 0; e < E; ++e) {
-                if (taken[e]) continue;
-                if (best < 0 || x[e] > x[best]) best = e; /* strict '>' keeps the lowest index */
-            }
-            taken[best] = 1;
-            sel[j] = best;
-        }
+        select_topk(x, E, k, taken, sel);
         /* step 2: softmax denominator over all E experts */
         double m = x[0];
         for (int32_t e = 1; e < E; ++e) {
@@ -123,6 +129,46 @@ int oracle_topk_softmax(const void* logits, int dtype, int64_t T, int32_t E, int
         /* step 4: one rounding to fp32 */
         for (int32_t j = 0; j < k; ++j) {
             double wj = std::exp(x[sel[j]] - m) / denom;
+            topk_weights[t * k + j] = static_cast<float>(wj);
+            topk_ids[t * k + j] = sel[j];
+        }
+    }
+    return 0;
+}
+
+/*
+ * Sigmoid scoring variant of the gating ("Upstream Reference: Deep-Spark xllm + vllm", "File
+ * Index": moe_topk_sigmoid_kernels.cuh, "sigmoid variant for DeepSeek-style routing", chosen by
+ * the sigmoid/softmax top-k dispatcher moe_fused_topk.cu).  The page gives no formula; the
+ * plainest reading, taken here:
+ *   1. select k experts exactly as oracle_topk_softmax does (on the logits; the logistic
+ *      function is increasing, so this is also the order of the scores);
+ *   2. score_j = 1 / (1 + exp(-x_sel_j)) in double, each expert on its own (no normalisation
+ *      across experts);
+ *   3. weight_j = score_j, or score_j / sum_j score_j when renormalize != 0 (1/k when that sum
+ *      is 0, which needs every selected logit below about -745);
+ *   4. round the weight once to fp32; ids are stored in selection order.
+ */
+int oracle_topk_sigmoid(const void* logits, int dtype, int64_t T, int32_t E, int32_t k,
+                        int renormalize, float* topk_weights, int32_t* topk_ids) {
+    if (T < 0 || E < 1 || k < 1 || k > E || (dtype != 0 && dtype != 1)) return 1;
+    if (T > 0 && (logits == nullptr || topk_weights == nullptr || topk_ids == nullptr)) return 1;
+
+    std::vector<double> x(static_cast<size_t>(E));
+    std::vector<char> taken(static_cast<size_t>(E));
+    std::vector<int32_t> sel(static_cast<size_t>(k));
+    std::vector<double> score(static_cast<size_t>(k));
+
+    for (int64_t t = 0; t < T; ++t) {
+        for (int32_t e = 0; e < E; ++e) x[e] = logit_as_double(logits, dtype, t * E + e);
+        select_topk(x, E, k, taken, sel);
+        double S = 0.0;
+        for (int32_t j = 0; j < k; ++j) {
+            score[j] = 1.0 / (1.0 + std::exp(-x[sel[j]]));
+            S += score[j];
+        }
+        for (int32_t j = 0; j < k; ++j) {
+            const double wj = renormalize ? (S > 0.0 ? score[j] / S : 1.0 / k) : score[j];
             topk_weights[t * k + j] = static_cast<float>(wj);
             topk_ids[t * k + j] = sel[j];
         }

@@ -195,6 +195,79 @@ TOPK_PINS = [pin_topk_hand_example, pin_topk_equal_logits, pin_topk_two_expert_l
              pin_topk_selects_on_logits, pin_topk_overflow_and_shift, pin_topk_invariants]
 
 
+# ------------------------------------------------------------ sigmoid topk --
+def _sigmoid_tanh(x: float) -> float:
+    """The logistic function through tanh: (1 + tanh(x/2)) / 2 (an independent evaluation)."""
+    return (1.0 + math.tanh(x / 2.0)) / 2.0
+
+
+def pin_sigmoid_closed_forms(orc) -> None:
+    # sigmoid(0) = 1/2 and sigmoid(ln 3) = 3/4; an expert alone with renormalisation weighs 1
+    x = np.array([[0.0, -2.0, -3.0], [math.log(3.0), 0.0, -1.0]], np.float32)
+    w, ids = orc.topk_sigmoid(x, 1, renormalize=False)
+    assert ids[:, 0].tolist() == [0, 0]
+    assert w[0, 0] == np.float32(0.5)
+    assert abs(int(ordered_int32(w[1:2, 0])[0]) - int(ordered_int32(np.float32(_sigmoid_tanh(float(x[1, 0]))))))<= 1
+    w, _ = orc.topk_sigmoid(x, 1, renormalize=True)
+    assert (w == np.float32(1.0)).all(), w
+    # far tails: no NaN, 0 and 1
+    x = np.array([[-1000.0, 1000.0, 0.0]], np.float32)
+    w, ids = orc.topk_sigmoid(x, 3, renormalize=False)
+    assert ids[0].tolist() == [1, 2, 0] and w[0].tolist() == [1.0, 0.5, 0.0], w
+
+
+def pin_sigmoid_tanh_identity(orc) -> None:
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((40, 24)) * 4).astype(np.float32)
+    for bits in (False, True):
+        xin = f32_to_bf16_bits(x) if bits else x
+        vals = bf16_bits_to_f32(xin) if bits else x
+        w, ids = orc.topk_sigmoid(xin, 5, renormalize=False)
+        for t in range(x.shape[0]):
+            for j in range(5):
+                want = np.float32(_sigmoid_tanh(float(vals[t, ids[t, j]])))
+                assert abs(int(ordered_int32(w[t:t + 1, j])[0]) - int(ordered_int32(want))) <= 1, (t, j)
+        wr, idr = orc.topk_sigmoid(xin, 5, renormalize=True)
+        assert np.array_equal(ids, idr)
+        # renormalised: the ratio of two weights is the ratio of their scores
+        for t in range(x.shape[0]):
+            s = np.array([_sigmoid_tanh(float(vals[t, e])) for e in ids[t]])
+            want = (s / s.sum()).astype(np.float32)
+            assert (np.abs(ordered_int32(wr[t]) - ordered_int32(want)) <= 2).all(), (wr[t], want)
+
+
+def pin_sigmoid_symmetry_and_equal_logits(orc) -> None:
+    # sigmoid(d) + sigmoid(-d) = 1: with k = 2 over [d, -d] the raw and renormalised weights agree
+    for d in (0.25, 1.0, 3.5, 7.0):
+        x = np.array([[d, -d], [-d, d]], np.float32)
+        wn, idn = orc.topk_sigmoid(x, 2, renormalize=False)
+        wr, idr = orc.topk_sigmoid(x, 2, renormalize=True)
+        assert idn.tolist() == [[0, 1], [1, 0]] and np.array_equal(idn, idr)
+        assert (np.abs(ordered_int32(wn) - ordered_int32(wr)) <= 1).all(), (wn, wr)
+        assert abs(float(wn[0].astype(np.float64).sum()) - 1.0) <= 2.0 ** -23
+    for E, k in ((8, 2), (60, 4), (160, 6)):
+        x = np.full((2, E), -1.25, np.float32)
+        w, ids = orc.topk_sigmoid(x, k, renormalize=True)
+        assert (ids == np.arange(k)).all() and (w == np.float32(1.0 / k)).all(), w
+
+
+def pin_sigmoid_selection_is_the_softmax_selection(orc) -> None:
+    rng = np.random.default_rng(23)
+    for E in range(1, 9):
+        for k in range(1, E + 1):
+            rows = np.concatenate([rng.integers(0, 4, size=(8, E)).astype(np.float32),
+                                   rng.standard_normal((4, E)).astype(np.float32)])
+            bits = f32_to_bf16_bits(rows)
+            vals = bf16_bits_to_f32(bits)
+            _, ids = orc.topk_sigmoid(bits, k, renormalize=False)
+            for t in range(rows.shape[0]):
+                assert ids[t].tolist() == brute_force_topk(vals[t], k), (vals[t], k, ids[t])
+
+
+SIGMOID_PINS = [pin_sigmoid_closed_forms, pin_sigmoid_tanh_identity, pin_sigmoid_symmetry_and_equal_logits,
+                pin_sigmoid_selection_is_the_softmax_selection]
+
+
 # ------------------------------------------------------------------- align --
 def _resolve_map(spec, E_global, E_local):
     if spec is None:
@@ -499,4 +572,4 @@ GATHER_COMBINE_PINS = [pin_gather_hand_example, pin_gather_rows_and_pads, pin_co
                        pin_combine_identity, pin_combine_error_bound, pin_combine_remote_dropped,
                        pin_combine_fma_sequence]
 
-ALL_PINS = TOPK_PINS + ALIGN_PINS + GATHER_COMBINE_PINS
+ALL_PINS = TOPK_PINS + SIGMOID_PINS + ALIGN_PINS + GATHER_COMBINE_PINS

@@ -64,6 +64,13 @@ MUTANTS = [
      "u += 0x7fffu + lsb;", "u += 0u * lsb;"),
     ("combine ignores the remote marker",
      "if (r < 0) continue;", "if (r < 0) r = 0;"),
+    ("sigmoid with the sign of the exponent flipped",
+     "score[j] = 1.0 / (1.0 + std::exp(-x[sel[j]]));", "score[j] = 1.0 / (1.0 + std::exp(x[sel[j]]));"),
+    ("sigmoid renormalise flag ignored",
+     "const double wj = renormalize ? (S > 0.0 ? score[j] / S : 1.0 / k) : score[j];",
+     "const double wj = score[j];"),
+    ("sigmoid weight taken from the wrong expert",
+     "score[j] = 1.0 / (1.0 + std::exp(-x[sel[j]]));", "score[j] = 1.0 / (1.0 + std::exp(-x[j]));"),
 ]
 
 
