@@ -85,6 +85,9 @@ typedef enum { MOE_DTYPE_F32 = 0, MOE_DTYPE_BF16 = 1 } moe_dtype_t;
 #define MOE_GATHER_HIDDEN_READY 4u /* moe_gather: `hidden` was complete before the previous kernel in
                                       the stream was launched, so it may be read before waiting for
                                       that kernel (true when hidden is an input of the routing step) */
+#define MOE_SCORING_SIGMOID 16u /* moe_topk_softmax, moe_route_dispatch: score each selected expert
+                                   with the logistic function 1/(1+exp(-x)) instead of the softmax
+                                   (the sigmoid variant of the gating); the selection is the same */
 #define MOE_DISPATCH_GIVEN_IDS 8u /* moe_route_dispatch: topk_ids is an input (routes chosen by the
                                      caller); no gating, logits and topk_weights are not accessed */
 
@@ -103,8 +106,12 @@ MOE_API int32_t moe_version(void);
  *   topk_weights  [T, k] fp32 out: softmax over all E logits of the selected
  *                 experts; with MOE_RENORMALIZE divided by their sum instead
  *                 (equivalently exp(x_j - max) / sum over the k selected).
+ *                 With MOE_SCORING_SIGMOID ("File Index": moe_topk_sigmoid_kernels.cuh,
+ *                 the sigmoid variant, chosen by the moe_fused_topk.cu dispatcher):
+ *                 1 / (1 + exp(-x_j)) per selected expert, with MOE_RENORMALIZE
+ *                 divided by their sum (1/k if that sum is 0).
  *   Computed in fp32 on the device (exp, sums, one division); within 2e-6 of the
- *   double-precision softmax.  Selection compares the logits exactly.
+ *   double-precision result.  Selection compares the logits exactly.
  *   Preconditions: finite logits (NaN/inf give unspecified ids).
  *   Errors: INVALID_ARG (T < 0; E < 1; k < 1 or k > E; null pointers with T > 0;
  *   unknown dtype or flags), UNSUPPORTED (E > 1024 or k > 32).  T == 0 is a no-op.
@@ -252,7 +259,8 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
  * hidden row of its own slot.
  *   logits [T, E] bf16/fp32 (dtype); hidden [T, H] bf16, 16-byte aligned, H % 8 == 0 and
  *   H <= 65536; expert_map and E_local as for moe_align_permute.
- *   flags: MOE_RENORMALIZE; MOE_DISPATCH_GIVEN_IDS: the routes in topk_ids [T,k] are the
+ *   flags: MOE_RENORMALIZE, MOE_SCORING_SIGMOID (as for moe_topk_softmax);
+ *   MOE_DISPATCH_GIVEN_IDS: the routes in topk_ids [T,k] are the
  *   input (the align input of moe_align_permute), logits and topk_weights may be NULL and are
  *   not read or written; every other output is as from moe_align_permute + moe_gather.
  *   workspace: >= moe_route_dispatch_workspace_bytes(T, k, E_local) bytes, zeroed before its

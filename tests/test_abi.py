@@ -68,7 +68,8 @@ def test_topk_validation_before_launch():
     assert f(N, B.MOE_DTYPE_BF16, 4, 8, 0, 0, N, N, N) == B.MOE_ERR_INVALID_ARG       # k < 1
     assert f(N, B.MOE_DTYPE_BF16, -1, 8, 2, 0, N, N, N) == B.MOE_ERR_INVALID_ARG      # T < 0
     assert f(N, 7, 4, 8, 2, 0, N, N, N) == B.MOE_ERR_INVALID_ARG                      # dtype
-    assert f(N, B.MOE_DTYPE_F32, 4, 8, 2, 0x10, N, N, N) == B.MOE_ERR_INVALID_ARG     # flags
+    assert f(N, B.MOE_DTYPE_F32, 4, 8, 2, 0x20, N, N, N) == B.MOE_ERR_INVALID_ARG     # flags
+    assert f(N, B.MOE_DTYPE_F32, 0, 8, 2, B.MOE_SCORING_SIGMOID | B.MOE_RENORMALIZE, N, N, N) == B.MOE_OK
     assert f(N, B.MOE_DTYPE_F32, 4, 2048, 2, 0, N, N, N) == B.MOE_ERR_UNSUPPORTED     # E > 1024
     assert f(N, B.MOE_DTYPE_F32, 4, 64, 33, 0, N, N, N) == B.MOE_ERR_UNSUPPORTED      # k > 32
     assert f(N, B.MOE_DTYPE_F32, 4, 64, 8, 0, N, N, N) == B.MOE_ERR_INVALID_ARG       # null pointers
@@ -120,7 +121,8 @@ def test_binding_rejects_cpu_tensors():
 def test_flag_values_match_the_header():
     text = open(HEADER).read()
     defined = {m.group(1): int(m.group(2)) for m in re.finditer(r"^#define\s+(MOE_\w+)\s+(\d+)u", text, flags=re.M)}
-    for name in ("MOE_RENORMALIZE", "MOE_GATHER_ZERO_PAD", "MOE_GATHER_HIDDEN_READY", "MOE_DISPATCH_GIVEN_IDS"):
+    for name in ("MOE_RENORMALIZE", "MOE_GATHER_ZERO_PAD", "MOE_GATHER_HIDDEN_READY", "MOE_DISPATCH_GIVEN_IDS",
+                 "MOE_SCORING_SIGMOID"):
         assert getattr(B, name) == defined[name], name
 
 
@@ -137,6 +139,7 @@ def test_dispatch_validation_before_launch():
     assert call(N, 0, buf) == B.MOE_ERR_INVALID_ARG                 # gating needs logits
     assert call(buf, 0, N) == B.MOE_ERR_INVALID_ARG                 # and somewhere for the weights
     assert call(N, given, N) == B.MOE_ERR_WORKSPACE                 # given routes: neither is needed
-    assert call(buf, 0x10, buf) == B.MOE_ERR_INVALID_ARG            # unknown flag
+    assert call(buf, 0x20, buf) == B.MOE_ERR_INVALID_ARG            # unknown flag
+    assert call(buf, B.MOE_SCORING_SIGMOID, buf) == B.MOE_ERR_WORKSPACE  # sigmoid scoring accepted
     assert call(buf, B.MOE_GATHER_ZERO_PAD, buf) == B.MOE_ERR_INVALID_ARG
     assert call(buf, B.MOE_RENORMALIZE | given, buf, H=12) == B.MOE_ERR_INVALID_ARG  # H % 8

@@ -153,3 +153,28 @@ def test_dispatch_given_routes(name, T, k, E, kind, E_local, bs, H):
         assert bool((sentinel == -2.5).all()), (name, pname)
         status = tdt.moe_read_status(ws)
         assert status == (tdt.MOE_ERR_BAD_EXPERT_ID if pname == "out_of_range" else tdt.MOE_OK), (name, pname)
+
+
+@pytest.mark.parametrize("T,E,k,dtype,renorm,E_local,bs,H", [
+    (2, 160, 6, torch.bfloat16, True, 160, 8, 512),       # single-kernel path
+    (20, 64, 4, torch.float32, False, 64, 16, 64),
+    (300, 128, 8, torch.bfloat16, True, 128, 64, 256),    # three-kernel path
+    (777, 60, 4, torch.float32, False, 60, 64, 128),
+], ids=["small_bf16", "small_fp32", "tile_bf16", "tile_fp32"])
+def test_dispatch_sigmoid_scoring(T, E, k, dtype, renorm, E_local, bs, H):
+    """moe_route_dispatch with MOE_SCORING_SIGMOID: weights from the sigmoid reading, the rest as for softmax."""
+    dev = require_gpu()
+    g = torch.Generator().manual_seed(T * 13 + E)
+    x = torch.randn((T, E), generator=g).to(dtype)
+    hidden = torch.randn((T, H), generator=g).to(torch.bfloat16)
+    w_ref, ids_ref = oracle.topk_sigmoid(logits_for_oracle(x), k, renorm)
+    al = oracle.align_permute(ids_ref, E, bs)
+    npad = int(al["num_tokens_post_pad"][0])
+    perm_ref = oracle.gather(bf16_bits(hidden), k, al["sorted_token_ids"], npad, al["capacity"])
+    real = al["sorted_token_ids"][:npad] != T * k
+    w, ids, align, perm = tdt.moe_route_dispatch(x.to(dev), hidden.to(dev), k, renorm, bs, scoring="sigmoid")
+    torch.cuda.synchronize()
+    assert np.array_equal(np_i32(ids), ids_ref)
+    assert np.abs(w.cpu().numpy() - w_ref).max() <= TOPK_WEIGHT_ATOL
+    assert_align_equal(align, al, "sigmoid dispatch")
+    assert np.array_equal(bf16_bits(perm[:npad])[real], perm_ref[:npad][real])

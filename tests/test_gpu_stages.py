@@ -65,6 +65,32 @@ def test_topk_softmax_parity(T, E, k, dtype, renorm, sigma, ties):
     assert err.max() <= TOPK_WEIGHT_ATOL, err.max()
 
 
+SIGMOID_CASES = [
+    # T, E, k, dtype, renormalize, sigma, ties  (sub-warp rows, one warp per row, fp32, wide, tie-heavy, tails)
+    (64, 8, 2, torch.bfloat16, True, 1.0, False),
+    (37, 7, 3, torch.float32, False, 1.0, False),
+    (4096, 128, 8, torch.bfloat16, True, 1.0, False),
+    (2000, 60, 4, torch.float32, False, math.sqrt(2.0), False),
+    (2, 160, 6, torch.bfloat16, False, 1.0, False),
+    (50, 1000, 8, torch.float32, True, 3.0, False),
+    (999, 256, 8, torch.bfloat16, True, 1.0, True),
+    (300, 64, 8, torch.float32, False, 30.0, False),       # far tails: scores near 0 and 1
+]
+
+
+@pytest.mark.parametrize("T,E,k,dtype,renorm,sigma,ties", SIGMOID_CASES)
+def test_topk_sigmoid_parity(T, E, k, dtype, renorm, sigma, ties):
+    """The sigmoid scoring variant (MOE_SCORING_SIGMOID) against the oracle's reading of it."""
+    dev = require_gpu()
+    x = _logits(T, E, dtype, sigma, seed=3 * T + E, ties=ties)
+    w, ids = tdt.moe_topk_softmax(x.to(dev), k, renorm, scoring="sigmoid")
+    torch.cuda.synchronize()
+    w_ref, ids_ref = oracle.topk_sigmoid(logits_for_oracle(x), k, renorm)
+    assert np.array_equal(np_i32(ids), ids_ref), np.nonzero(np_i32(ids) != ids_ref)
+    err = np.abs(w.cpu().numpy().astype(np.float64) - w_ref.astype(np.float64))
+    assert err.max() <= TOPK_WEIGHT_ATOL, err.max()
+
+
 def test_topk_softmax_misaligned_rows():
     """A logits view that starts 2 bytes past a 16-byte boundary takes the narrow-load path."""
     dev = require_gpu()

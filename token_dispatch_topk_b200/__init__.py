@@ -8,7 +8,7 @@ The Python layer only marshals arguments (``binding``) and preallocates buffers
 from .binding import (  # noqa: F401
     MOE_DTYPE_BF16, MOE_DTYPE_F32, MOE_ERR_BAD_EXPERT_ID, MOE_ERR_BAD_ROW, MOE_ERR_CUDA, MOE_ERR_INVALID_ARG,
     MOE_ERR_TIMEOUT, MOE_ERR_UNSUPPORTED, MOE_ERR_WORKSPACE, MOE_GATHER_HIDDEN_READY, MOE_GATHER_ZERO_PAD, MOE_OK,
-    MOE_RENORMALIZE, MOE_DISPATCH_GIVEN_IDS,
+    MOE_RENORMALIZE, MOE_DISPATCH_GIVEN_IDS, MOE_SCORING_SIGMOID,
     AlignResult, MoeError, alloc_align_outputs, alloc_workspace, load_library, moe_align_capacity,
     moe_align_num_blocks, moe_align_permute, moe_align_permute_noalloc, moe_align_workspace_bytes, moe_combine, moe_gather, moe_read_status,
     moe_route_dispatch, moe_route_dispatch_workspace_bytes, moe_topk_softmax, moe_version, moe_workspace_init,

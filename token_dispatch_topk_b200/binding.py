@@ -31,6 +31,7 @@ MOE_RENORMALIZE = 1
 MOE_GATHER_ZERO_PAD = 2
 MOE_GATHER_HIDDEN_READY = 4
 MOE_DISPATCH_GIVEN_IDS = 8
+MOE_SCORING_SIGMOID = 16
 
 # Every symbol include/moe_route.h declares, with (restype, argtypes).
 _P, _I32, _I64, _U32, _SZ = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_uint32, ctypes.c_size_t
@@ -136,9 +137,19 @@ def alloc_workspace(T: int, k: int, E_local: int, device) -> torch.Tensor:
     return torch.zeros((nbytes + 3) // 4, dtype=torch.int32, device=device)
 
 
+def _scoring_flag(scoring: str) -> int:
+    if scoring == "softmax":
+        return 0
+    if scoring == "sigmoid":
+        return MOE_SCORING_SIGMOID
+    raise ValueError(f"scoring must be 'softmax' or 'sigmoid', got {scoring!r}")
+
+
 def moe_topk_softmax(logits: torch.Tensor, k: int, renormalize: bool, topk_weights: Optional[torch.Tensor] = None,
-                     topk_ids: Optional[torch.Tensor] = None, stream=None):
-    """logits [T, E] bf16/fp32 -> (topk_weights [T, k] fp32, topk_ids [T, k] int32)."""
+                     topk_ids: Optional[torch.Tensor] = None, stream=None, scoring: str = "softmax"):
+    """logits [T, E] bf16/fp32 -> (topk_weights [T, k] fp32, topk_ids [T, k] int32).
+
+    ``scoring``: "softmax" (default) or "sigmoid" (each selected expert weighs 1/(1+exp(-x)))."""
     if logits.dim() != 2:
         raise ValueError("logits must be [T, E]")
     T, E = logits.shape
@@ -155,7 +166,7 @@ def moe_topk_softmax(logits: torch.Tensor, k: int, renormalize: bool, topk_weigh
     assert topk_weights.dtype == torch.float32 and topk_ids.dtype == torch.int32
     assert topk_weights.numel() == T * k and topk_ids.numel() == T * k
     st = load_library().moe_topk_softmax(_dev(logits, "logits"), dt, T, E, k,
-                                         MOE_RENORMALIZE if renormalize else 0,
+                                         (MOE_RENORMALIZE if renormalize else 0) | _scoring_flag(scoring),
                                          _dev(topk_weights, "topk_weights"), _dev(topk_ids, "topk_ids"),
                                          _stream(stream))
     _check(st, "moe_topk_softmax")
@@ -279,7 +290,7 @@ def moe_route_dispatch(logits: Optional[torch.Tensor], hidden: torch.Tensor, k: 
                        topk_weights: Optional[torch.Tensor] = None, topk_ids: Optional[torch.Tensor] = None,
                        align: Optional[AlignResult] = None, permuted: Optional[torch.Tensor] = None,
                        workspace: Optional[torch.Tensor] = None, stream=None, given_ids: bool = False,
-                       E: Optional[int] = None):
+                       E: Optional[int] = None, scoring: str = "softmax"):
     """Gating + align + permute-gather in one call.  Returns (topk_weights, topk_ids, AlignResult, permuted).
 
     With ``given_ids`` the routes in ``topk_ids`` are the input (no gating): ``logits`` may be None (then
@@ -315,7 +326,8 @@ def moe_route_dispatch(logits: Optional[torch.Tensor], hidden: torch.Tensor, k: 
     if workspace is None:
         workspace = alloc_dispatch_workspace(T, k, E_local, dev)
     assert expert_map is None or expert_map.dtype == torch.int32
-    flags = (MOE_RENORMALIZE if renormalize else 0) | (MOE_DISPATCH_GIVEN_IDS if given_ids else 0)
+    flags = (MOE_RENORMALIZE if renormalize else 0) | (MOE_DISPATCH_GIVEN_IDS if given_ids else 0) | \
+        _scoring_flag(scoring)
     st = load_library().moe_route_dispatch(
         _dev(logits, "logits"), dt, _dev(hidden, "hidden"), T, E, k, H, flags,
         _dev(expert_map, "expert_map"), E_local, block_size, _dev(topk_weights, "topk_weights"),

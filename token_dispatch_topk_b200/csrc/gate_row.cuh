@@ -23,6 +23,10 @@
 
 namespace moe_gate {
 
+// Scoring mode bits of gate_row and the gating kernels.
+constexpr int kGateRenorm = 1;   // renormalise the k weights to sum to 1
+constexpr int kGateSigmoid = 2;  // score each expert with the logistic function instead of the softmax
+
 __device__ __forceinline__ uint32_t ordered_bits(float x) {
   uint32_t u = __float_as_uint(x);
   if ((u & 0x7fffffffu) == 0u) u = 0u;  // -0 and +0 compare equal
@@ -174,12 +178,16 @@ __device__ __forceinline__ void pop_front_if(K (&k)[NV], bool hit) {
 }
 
 // Top-k of one row (all 32 lanes of the warp call it).  Lanes 0..k-1 return the expert of rank
-// `lane` in my_e and its weight in my_w; other lanes' outputs are unspecified.
+// `lane` in my_e and its weight in my_w; other lanes' outputs are unspecified.  `mode`: bits
+// kGateRenorm and kGateSigmoid.  Softmax weights are exp(x - m) over the full-row sum (or over the
+// k selected); sigmoid weights are 1 / (1 + exp(-x)) each (or over their sum, 1/k if it is 0).
 template <typename TIn, int VEC, int CPL>
-__device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int k, int renormalize, int lane,
+__device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int k, int mode, int lane,
                                          int& my_e, float& my_w) {
   constexpr int NV = CPL * VEC;
   const int n_chunks = E / VEC;
+  const bool renormalize = (mode & kGateRenorm) != 0;
+  const bool sigmoid = (mode & kGateSigmoid) != 0;
   float m = 0.f, Z = 0.f, S = 0.f, my_p = 0.f;
   my_e = 0;
 
@@ -212,7 +220,7 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
       best = __reduce_max_sync(0xffffffffu, best);
       if (j == 0) {
         best0 = best;
-        if (!renormalize) {  // full-row denominator, from the keys before any is retired
+        if (!renormalize && !sigmoid) {  // full-row denominator, from the keys before any is retired
           m = ordered16_to_float(best >> 16);
           float z = 0.f;
 #pragma unroll
@@ -232,7 +240,8 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
     }
     m = ordered16_to_float(best0 >> 16);
     if (lane < k) {
-      my_p = expf(ordered16_to_float(my_key >> 16) - m);
+      const float xj = ordered16_to_float(my_key >> 16);
+      my_p = sigmoid ? 1.f / (1.f + expf(-xj)) : expf(xj - m);
       my_e = static_cast<int>(0xffffu - (my_key & 0xffffu));
     }
     if (renormalize) S = warp_sum(my_p);
@@ -269,7 +278,7 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
       const uint64_t best = (static_cast<uint64_t>(hi) << 32) | lo;
       if (j == 0) {
         hi0 = hi;
-        if (!renormalize) {
+        if (!renormalize && !sigmoid) {
           m = ordered_to_float(hi);
           float z = 0.f;
 #pragma unroll
@@ -289,13 +298,17 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
     }
     m = ordered_to_float(hi0);
     if (lane < k) {
-      my_p = expf(ordered_to_float(static_cast<uint32_t>(my_key >> 32)) - m);
+      const float xj = ordered_to_float(static_cast<uint32_t>(my_key >> 32));
+      my_p = sigmoid ? 1.f / (1.f + expf(-xj)) : expf(xj - m);
       my_e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(my_key));
     }
     if (renormalize) S = warp_sum(my_p);
   }
-  const float den = renormalize ? S : Z;
-  my_w = my_p / den;
+  if (sigmoid) {
+    my_w = renormalize ? (S > 0.f ? my_p / S : 1.f / static_cast<float>(k)) : my_p;
+  } else {
+    my_w = my_p / (renormalize ? S : Z);
+  }
 }
 
 }  // namespace moe_gate

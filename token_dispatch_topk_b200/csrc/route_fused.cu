@@ -50,7 +50,7 @@ struct DispatchArgs {
   int64_t T;
   int E;
   int k;
-  int renormalize;
+  int renormalize;  // scoring mode bits: moe_gate::kGateRenorm, moe_gate::kGateSigmoid
   int given_ids;  // topk_ids is an input: no gating, topk_weights untouched
   const int32_t* expert_map;
   int E_local;
@@ -693,7 +693,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
                                            void* workspace, size_t workspace_bytes, void* stream) {
   if (T < 0 || E < 1 || k < 1 || k > E || H < 1 || E_local < 1 || block_size < 1) return MOE_ERR_INVALID_ARG;
   if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
-  if ((flags & ~(MOE_RENORMALIZE | MOE_DISPATCH_GIVEN_IDS)) != 0u) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~(MOE_RENORMALIZE | MOE_DISPATCH_GIVEN_IDS | MOE_SCORING_SIGMOID)) != 0u) return MOE_ERR_INVALID_ARG;
   const bool given_ids = (flags & MOE_DISPATCH_GIVEN_IDS) != 0u;
   if (E_local > E || (expert_map == nullptr && E_local != E)) return MOE_ERR_INVALID_ARG;
   if (E > 1024 || k > 32 || E_local > 1024) return MOE_ERR_UNSUPPORTED;
@@ -721,7 +721,8 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.T = T;
   a.E = E;
   a.k = k;
-  a.renormalize = (flags & MOE_RENORMALIZE) ? 1 : 0;
+  a.renormalize = ((flags & MOE_RENORMALIZE) ? moe_gate::kGateRenorm : 0) |
+                  ((flags & MOE_SCORING_SIGMOID) ? moe_gate::kGateSigmoid : 0);
   a.given_ids = given_ids ? 1 : 0;
   a.expert_map = expert_map;
   a.E_local = E_local;

@@ -79,6 +79,7 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
     }
   }
 
+  const bool renorm = (renormalize & kGateRenorm) != 0, sigmoid = (renormalize & kGateSigmoid) != 0;
   float m = 0.f, Z = 0.f, S = 0.f;
   for (int j = 0; j < k; ++j) {
     uint64_t best = 0ull;
@@ -89,7 +90,7 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
       best = o > best ? o : best;
     }
     const float xj = ordered_to_float(static_cast<uint32_t>(best >> 32));
-    if (j == 0) {
+    if (j == 0 && !sigmoid) {
       // the first winner is the row maximum; reduce Z = sum over the row of exp(x - m)
       m = xj;
       float z = 0.f;
@@ -102,14 +103,14 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
     }
 #pragma unroll
     for (int i = 0; i < NV; ++i) key[i] = (key[i] == best) ? 0ull : key[i];
-    const float p = expf(xj - m);
+    const float p = sigmoid ? 1.f / (1.f + expf(-xj)) : expf(xj - m);
     S += p;
     if (g == 0) {
       s_id[sub * k + j] = static_cast<int32_t>(0xffffffffu - static_cast<uint32_t>(best));
       s_p[sub * k + j] = p;
     }
   }
-  if (g == 0) s_den[sub] = renormalize ? S : Z;
+  if (g == 0) s_den[sub] = renorm ? S : (sigmoid ? 1.f : Z);
   __syncwarp();
 
   const int64_t rows_here = (T - row0) < rows_per_warp ? (T - row0) : rows_per_warp;
@@ -118,7 +119,8 @@ topk_softmax_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, int
   int32_t* idst = topk_ids + row0 * k;
   for (int idx = lane; idx < n_out; idx += 32) {
     const int r = idx / k;
-    wdst[idx] = s_p[idx] / s_den[r];
+    const float den = s_den[r];
+    wdst[idx] = den > 0.f ? s_p[idx] / den : 1.f / static_cast<float>(k);  // 0 only for sigmoid sums
     idst[idx] = s_id[idx];
   }
 }
@@ -283,14 +285,16 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
                                          uint32_t flags, float* topk_weights, int32_t* topk_ids, void* stream) {
   if (T < 0 || E < 1 || k < 1 || k > E) return MOE_ERR_INVALID_ARG;
   if (dtype != MOE_DTYPE_F32 && dtype != MOE_DTYPE_BF16) return MOE_ERR_INVALID_ARG;
-  if ((flags & ~MOE_RENORMALIZE) != 0u) return MOE_ERR_INVALID_ARG;
+  if ((flags & ~(MOE_RENORMALIZE | MOE_SCORING_SIGMOID)) != 0u) return MOE_ERR_INVALID_ARG;
   if (E > 1024 || k > 32) return MOE_ERR_UNSUPPORTED;
   if (T == 0) return MOE_OK;
   if (logits == nullptr || topk_weights == nullptr || topk_ids == nullptr) return MOE_ERR_INVALID_ARG;
   if (T > (int64_t{1} << 40)) return MOE_ERR_INVALID_ARG;
 
   const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
-  int renorm_flag = (flags & MOE_RENORMALIZE) ? 1 : 0;
+  // scoring mode bits of the kernels (moe_gate::kGateRenorm, moe_gate::kGateSigmoid)
+  int renorm_flag = ((flags & MOE_RENORMALIZE) ? moe_gate::kGateRenorm : 0) |
+                    ((flags & MOE_SCORING_SIGMOID) ? moe_gate::kGateSigmoid : 0);
   if (E >= 16) {
     // one warp per row: the widest aligned vector that still spreads the row over all 32 lanes
     int vec_max = 16 / elem;

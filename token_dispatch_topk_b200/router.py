@@ -20,8 +20,9 @@ from . import binding as B
 class MoeRouter:
     def __init__(self, T: int, E: int, k: int, H: int, block_size: int, renormalize: bool,
                  E_local: Optional[int] = None, expert_map: Optional[torch.Tensor] = None,
-                 logits_dtype: torch.dtype = torch.bfloat16, device="cuda"):
+                 logits_dtype: torch.dtype = torch.bfloat16, device="cuda", scoring: str = "softmax"):
         B.load_library()
+        self.scoring = scoring
         self.T, self.E, self.k, self.H, self.block_size = T, E, k, H, block_size
         self.renormalize = renormalize
         self.E_local = E if E_local is None else E_local
@@ -42,7 +43,8 @@ class MoeRouter:
 
     # ------------------------------------------------------------------ stages --
     def gate(self, logits: torch.Tensor, stream=None):
-        return B.moe_topk_softmax(logits, self.k, self.renormalize, self.topk_weights, self.topk_ids, stream)
+        return B.moe_topk_softmax(logits, self.k, self.renormalize, self.topk_weights, self.topk_ids, stream,
+                                  scoring=self.scoring)
 
     def align_permute(self, topk_ids: Optional[torch.Tensor] = None, stream=None) -> B.AlignResult:
         ids = self.topk_ids if topk_ids is None else topk_ids
@@ -67,7 +69,8 @@ class MoeRouter:
         return B.moe_route_dispatch(None if given else logits, hidden, self.k, self.renormalize, self.block_size,
                                     self.expert_map, self.E_local, None if given else self.topk_weights,
                                     topk_ids if given else self.topk_ids, self.align, self.permuted,
-                                    self.dispatch_workspace, stream, given_ids=given, E=self.E)
+                                    self.dispatch_workspace, stream, given_ids=given, E=self.E,
+                                    scoring=self.scoring)
 
     @property
     def small_batch(self) -> bool:
