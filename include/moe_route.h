@@ -251,7 +251,7 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
  *   topk_weights [T,k], topk_ids [T,k], counts [E_local], offsets [E_local+1],
  *   sorted_token_ids [C], expert_ids [NB], num_tokens_post_pad [1], inv_perm [T*k],
  *   permuted [C, H] (rows of local slots; pad rows untouched).
- * For T > 32 or T*k > 256: the first kernel gates tiles of tokens and counts each tile's slots
+ * For T > 32, T*k > 256 or E > 256: the first kernel gates tiles of tokens and counts each tile's slots
  * per local expert with their ranks inside the tile; the last of its CTAs to finish turns the
  * tile counts into the padded layout; the second kernel gives every slot its row and copies the
  * hidden rows there.  Smaller batches (decode) take one kernel with one CTA per slot: each CTA

@@ -2,7 +2,7 @@
 the CPU oracle pipeline, through the C ABI.
 
 Two kernel paths sit behind the call: one kernel with one CTA per slot for small batches
-(T <= 32 and T*k <= 256) and the tiled two-kernel path above that.  Shapes cover both sides of every
+(T <= 32, T*k <= 256 and E <= 256) and the tiled three-kernel path above that.  Shapes cover both sides of every
 one of those limits, one and many gating tiles with a ragged last tile, maps with remote and
 out-of-range values, every gating vector width, k up to 32, 1024 experts, T = 0 and the decode size,
 with logits-derived routes and with routes given by the caller.  Bars as for the stage entry points:
@@ -41,8 +41,11 @@ CASES = [
     ("tile_T32_k9", 32, 64, 9, torch.bfloat16, True, None, 64, 8, 128),
     ("tile_T9_k32_fp32", 9, 64, 32, torch.float32, True, None, 64, 8, 64),
     ("small_T8_k32", 8, 64, 32, torch.bfloat16, False, None, 64, 4, 64),
-    ("small_wide_1024_fp32", 8, 1024, 8, torch.float32, False, None, 1024, 4, 64),
-    ("small_wide_1024_bf16_map", 5, 1024, 8, torch.bfloat16, True, "strided", 256, 2, 64),
+    ("tile_small_T_wide_1024_fp32", 8, 1024, 8, torch.float32, False, None, 1024, 4, 64),
+    ("tile_small_T_wide_1024_bf16_map", 5, 1024, 8, torch.bfloat16, True, "strided", 256, 2, 64),
+    ("small_E256_fp32", 8, 256, 8, torch.float32, False, None, 256, 4, 64),
+    ("small_E256_bf16_map", 5, 256, 8, torch.bfloat16, True, "strided", 64, 2, 64),
+    ("tile_E257", 4, 257, 8, torch.bfloat16, True, None, 257, 4, 64),
     ("small_bad_map_values", 20, 64, 4, torch.bfloat16, True, "bad", 16, 16, 64),
     ("small_odd_e_fp32", 31, 61, 5, torch.float32, True, None, 61, 3, 16),
     ("small_long_rows", 3, 32, 2, torch.bfloat16, True, None, 32, 4, 65536),

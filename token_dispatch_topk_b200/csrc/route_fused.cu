@@ -396,7 +396,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
 //   B. per warp of 32 slots: local expert, rank among the warp's earlier slots of the same expert
 //      and the warp's count of it (a 32-step shuffle loop); the first slot of each expert in the
 //      warp records the count in the warp's row of a histogram;
-//   C. per expert (one to four per thread): count = sum of the warp rows, blocks = ceil(count/bs),
+//   C. per expert (one per thread): count = sum of the warp rows, blocks = ceil(count/bs),
 //      exclusive scan of the blocks over the experts; CTA 0 writes counts, offsets, the expert's
 //      expert_ids and its pad rows;
 //   D. row of slot s = offset of its expert + its expert's slots in earlier warps + its rank;
@@ -405,7 +405,7 @@ constexpr int kSmallThreads = 256;
 constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallMaxTokens = 32;
 constexpr int kSmallMaxSlots = kSmallThreads;  // one slot per thread
-constexpr int kSmallMaxExperts = 1024;
+constexpr int kSmallMaxExperts = 256;  // one expert per thread in every per-expert loop
 constexpr int kSmallExpertsPerThread = kSmallMaxExperts / kSmallThreads;
 constexpr int kSmallPrefetch = 4;  // 16-byte vectors per thread of the row held in registers while routing
 

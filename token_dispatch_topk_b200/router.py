@@ -75,7 +75,7 @@ class MoeRouter:
     @property
     def small_batch(self) -> bool:
         """True when moe_route_dispatch runs as a single kernel (decode-sized batches)."""
-        return self.T <= 32 and self.T * self.k <= 256 and self.E <= 1024
+        return self.T <= 32 and self.T * self.k <= 256 and self.E <= 256
 
     def step(self, logits: torch.Tensor, hidden: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
         """gate + align + permute-gather + combine; expert_out stands in for the expert MLPs' output.
