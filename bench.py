@@ -196,6 +196,20 @@ def host_inputs_numpy(wl, seed: int, T_max: int):
     return logits_np, hidden_bits, y_bits, None if emap is None else emap.numpy()
 
 
+def host_cpu() -> dict:
+    """CPU model and logical core count of this host (for the CPU-baseline record)."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"model": model, "logical_cores": os.cpu_count()}
+
+
 def cpu_oracle_rate(wl, seed: int, budget_s: float, T_max: int = 4096):
     """Tokens/s of the oracle on this host over a bounded sample (single-threaded)."""
     import oracle as oracle_mod
@@ -211,7 +225,8 @@ def cpu_oracle_rate(wl, seed: int, budget_s: float, T_max: int = 4096):
         if el >= budget_s or reps >= 1000:
             break
     return {"value": done / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{reps} oracle passes over the first {T} tokens of the workload ({el:.1f} s, single thread)"}
+            "sample": f"{reps} oracle passes over the first {T} tokens of the workload ({el:.1f} s, single thread)",
+            "host": host_cpu()}
 
 
 def run_reference(args, wl):
@@ -243,7 +258,8 @@ def run_reference(args, wl):
             "vs_baseline": None, "dtype": "f64 softmax, fp32 combine", "data": "synthetic",
             "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"}},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                             "sample": f"{n} tokens of the workload per step, single-threaded C++ oracle"},
+                             "sample": f"{n} tokens of the workload per step, single-threaded C++ oracle",
+                             "host": host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
@@ -334,7 +350,11 @@ def main():
                 run(name)
                 b.record(stream)
         stream.synchronize()
-        return sum(a.elapsed_time(b) for a, b in evs)
+        per_step = [a.elapsed_time(b) for a, b in evs]
+        step_samples[name] = per_step
+        return sum(per_step)
+
+    step_samples = {}
 
     def timed_back_to_back(name, iters, warm):
         """Time (ms) of `iters` steps replayed back to back between one pair of events (no flush:
@@ -384,6 +404,9 @@ def main():
     # launch-to-event latency of a lone graph, about 5 us, to every step)
     n_fl = min(args.steps, 200)
     flushed_ms_per_step = (timed("step", n_fl, 3) / n_fl) if back_to_back else ms_per_step
+    qs = statistics.quantiles(step_samples["step"], n=10) if len(step_samples.get("step", [])) >= 10 else None
+    flushed_pct_us = None if qs is None else {"p10": 1e3 * qs[0], "p50": 1e3 * statistics.median(step_samples["step"]),
+                                              "p90": 1e3 * qs[-1], "steps": len(step_samples["step"])}
 
     # ---- per-stage times inside the step, and roofline
     # The step is captured once more with external event records between its stages, so each
@@ -567,7 +590,7 @@ def main():
             "algorithmic_bytes_per_step": total_bytes,
             "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
             "routed_slots_local": R, "num_tokens_post_pad": npad,
-            "flushed_ms_per_step": flushed_ms_per_step,
+            "flushed_ms_per_step": flushed_ms_per_step, "flushed_step_us_percentiles": flushed_pct_us,
             "step_path": "moe_route_dispatch (single kernel) + moe_combine" if r.small_batch else
                          "moe_route_dispatch (three kernels) + moe_combine",
             "roofline": roofline, "stages": stages_fused, "stages_four_call_path": stages, "e2e": e2e,
