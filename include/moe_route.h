@@ -131,7 +131,7 @@ MOE_API int64_t moe_align_num_blocks(int64_t T, int32_t k, int32_t E_local, int3
 
 /*
  * Bytes of device workspace moe_align_permute needs for these sizes (a status
- * word, a completion ticket and per-tile expert counters).  Host-only.
+ * word, a completion ticket, per-tile expert counters and the expert totals).  Host-only.
  * The workspace must be zero-filled once before its first use (see
  * moe_workspace_init); every call leaves it ready for the next one.  The first
  * 4 bytes are the device status word that moe_read_status reads; pass the
@@ -188,7 +188,8 @@ MOE_API moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32
  *   Same arguments, outputs, ordering and errors as moe_align_permute, except:
  *   - no workspace: the completion ticket and the per-tile expert counters live in a fixed
  *     1 MiB array inside the library, one per GPU that loads it, held until the process exits;
- *   - sizes whose scratch would exceed that array (moe_align_workspace_bytes(T, k, E_local)
+ *   - it always runs the count + place tile kernels; sizes whose scratch would exceed that
+ *     array (a 256-byte header plus 4 bytes per local expert per tile of up to 8192 slots,
  *     > 1 MiB, e.g. E_local = 1024 with more than about 1M slots) return MOE_ERR_UNSUPPORTED
  *     before anything is enqueued;
  *   - device_status: a caller device int32 that collects device-side errors, or NULL.

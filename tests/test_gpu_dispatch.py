@@ -51,6 +51,12 @@ CASES = [
     ("small_long_rows", 3, 32, 2, torch.bfloat16, True, None, 32, 4, 65536),
     ("small_rows_past_prefetch", 2, 160, 6, torch.bfloat16, True, "rank1", 40, 8, 8200),
     ("tile_T33_decode_map", 33, 160, 6, torch.bfloat16, True, "rank1", 40, 8, 4096),
+    # degenerate shapes on both paths
+    ("tile_k1_bs1_H8", 100, 16, 1, torch.bfloat16, True, None, 16, 1, 8),
+    ("tile_one_local_expert", 200, 32, 4, torch.bfloat16, True, "one_local", 1, 8, 64),
+    ("small_one_local_expert", 3, 32, 4, torch.float32, False, "one_local", 1, 8, 64),
+    ("small_k1_bs1_H8", 1, 4, 1, torch.bfloat16, False, None, 4, 1, 8),
+    ("tile_all_remote", 64, 32, 4, torch.bfloat16, True, "none_local", 8, 16, 32),
 ]
 
 
@@ -63,6 +69,14 @@ def _map(kind, E, E_local):
         return m
     if kind == "strided":
         return I.strided_expert_map(E, 4, 1).numpy()
+    if kind == "one_local":  # a single local expert: global 5
+        m = np.full(E, -1, np.int32)
+        m[5] = 0
+        return m
+    if kind == "none_local":  # a rank whose experts the router never picks (map covers only the last 8)
+        m = np.full(E, -1, np.int32)
+        m[E - E_local:] = np.arange(E_local)
+        return m
     if kind == "bad":  # some globals map past E_local or below -1: those slots are dropped and flagged
         m = np.full(E, -1, np.int32)
         m[:E_local] = np.arange(E_local)
@@ -77,6 +91,8 @@ def test_dispatch_parity(name, T, E, k, dtype, renorm, kind, E_local, bs, H):
     dev = require_gpu()
     g = torch.Generator().manual_seed(T + 7 * E + k)
     x = torch.randn((T, E), generator=g).to(dtype)
+    if kind == "none_local":  # the last E_local experts never make the top k
+        x[:, E - E_local:] -= 50.0
     if kind == "bad":  # make the flagged globals win often
         x[:, E_local] += 3.0
         x[:, E_local + 1] += 3.0

@@ -41,7 +41,8 @@ def sources():
 
 
 def _deps():
-    return sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + [os.path.join(INCLUDE, "moe_route.h")]
+    return (sources() + sorted(glob.glob(os.path.join(CSRC, "*.cuh"))) + sorted(glob.glob(os.path.join(CSRC, "*.h")))
+            + [os.path.join(INCLUDE, "moe_route.h")])
 
 
 def is_stale() -> bool:

@@ -23,11 +23,15 @@
 //     the tail rows past N_pad, and expert_ids.
 // When all slots fit one tile (decode, small batches), the count kernel does
 // everything in one CTA and the place kernel is not launched.
+// moe_align_permute takes these kernels above 65 536 slots (or 512 local experts), one
+// thread-block cluster (align_cluster_kernel, below) up to 4096 slots, and between the two
+// the tile kernels of the fused dispatch (route_fused.cu, moe_internal::align_tiles).
 #include <cooperative_groups.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
 #include "common.cuh"
+#include "route_internal.h"
 
 namespace {
 
@@ -360,6 +364,7 @@ constexpr int kClusterThreads = 1024;
 constexpr int kClusterWarps = kClusterThreads / 32;
 constexpr int kMaxClusterCtas = 16;
 constexpr int64_t kClusterMaxSlots = 65536;
+constexpr int64_t kAlignTilesMinSlots = 4096;  // above this (up to kClusterMaxSlots): the tile kernels
 constexpr int kClusterMaxExperts = 512;
 
 // Exclusive scan of n <= 1024 ints in shared memory, one per thread of a 1024-thread block.
@@ -701,14 +706,24 @@ extern "C" int64_t moe_align_num_blocks(int64_t T, int32_t k, int32_t E_local, i
   return (C + block_size - 1) / block_size;
 }
 
-extern "C" size_t moe_align_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
-  if (T < 0 || k < 1 || E_local < 1) return 0;
+namespace {
+// Scratch of the count + place kernels and of the cluster kernel: header + per-tile (or per
+// cluster rank) expert counters.
+size_t count_place_scratch_bytes(int64_t T, int32_t k, int32_t E_local) {
   const int64_t P = T * k;
   const int ts = tile_slots_for(P);
   const int nt = num_tiles_for(P, ts);
   size_t rows = nt > 1 ? static_cast<size_t>(nt) : 0;  // per-tile counters of the tile kernels
   if (P > 4096 && rows < static_cast<size_t>(kMaxClusterCtas)) rows = kMaxClusterCtas;  // cluster table
   return kWsHeaderBytes + rows * static_cast<size_t>(E_local) * sizeof(int32_t);
+}
+}  // namespace
+
+extern "C" size_t moe_align_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
+  if (T < 0 || k < 1 || E_local < 1) return 0;
+  const size_t own = count_place_scratch_bytes(T, k, E_local);
+  const size_t tiles = moe_internal::align_tiles_workspace_bytes(T, E_local);  // the fused path's tile kernels
+  return own > tiles ? own : tiles;
 }
 
 extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
@@ -753,6 +768,12 @@ extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, in
   a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + kWsHeaderBytes);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  // mid-size batches: the tile kernels of the fused dispatch (per-tile ranks, a per-expert tile
+  // scan, placement), measured faster there than the single cluster; small batches: one cluster;
+  // above: count + place tile kernels over every SM
+  if (P > kAlignTilesMinSlots && P <= kClusterMaxSlots)
+    return moe_internal::align_tiles(topk_ids, T, k, E_global, expert_map, E_local, block_size, counts, offsets,
+                                     sorted_token_ids, expert_ids, num_tokens_post_pad, inv_perm, workspace, st);
   if (P <= kClusterMaxSlots && E_local <= kClusterMaxExperts) return launch_align_cluster(a, st);
   // large batches or many local experts: count + place tile kernels over every SM
   const size_t smem = align_smem_ints(E_local, a.tile_slots) * sizeof(int);
@@ -826,7 +847,7 @@ extern "C" moe_status_t moe_align_permute_noalloc(const int32_t* topk_ids, int64
     return MOE_ERR_INVALID_ARG;
   if (P > 0 && (topk_ids == nullptr || inv_perm == nullptr)) return MOE_ERR_INVALID_ARG;
   // the scratch these sizes need must fit the fixed array
-  if (moe_align_workspace_bytes(T, k, E_local) > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
+  if (count_place_scratch_bytes(T, k, E_local) > kNoAllocScratchBytes) return MOE_ERR_UNSUPPORTED;
 
   void* scratch = nullptr;
   const moe_status_t st_scratch = noalloc_scratch(&scratch);

@@ -32,6 +32,7 @@
 
 #include "common.cuh"
 #include "gate_row.cuh"
+#include "route_internal.h"
 
 namespace {
 
@@ -253,6 +254,7 @@ __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
 // One warp per CTA: slots of tokens [t0, t0 + n) get their rows, the hidden rows are staged with
 // a bulk load and bulk-stored to every local row; then a share of the expert-owned outputs, the
 // pad rows and the tail.  Shared memory: staged rows [tpc * row_bytes] | offsets [E_local + 1].
+template <bool kGather>  // false: placement only (moe_align_permute), no hidden rows
 __global__ void __launch_bounds__(32)
 place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t row_bytes, int tpc,
                     uint8_t* __restrict__ permuted) {
@@ -264,12 +266,12 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * tpc;
   const int64_t left = a.T - t0;
   const int n = left <= 0 ? 0 : static_cast<int>(left < tpc ? left : tpc);
-  if (lane == 0) {
+  if (kGather && lane == 0) {
     moe::mbar_init(&bar, 1);
     moe::fence_barrier_init();
   }
   __syncwarp();
-  if (lane == 0 && n > 0) {  // hidden is an input of the call: complete before the first kernel ran
+  if (kGather && lane == 0 && n > 0) {  // hidden is an input of the call: complete before the first kernel ran
     moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
     for (int i = 0; i < n; ++i) {
       moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes, hidden + (t0 + i) * static_cast<int64_t>(row_bytes),
@@ -315,7 +317,11 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     if (e < nslots) {
       const int64_t s = t0 * k + e;
       const int v = a.inv_perm[s];  // (rank in the tile) << 10 | local expert, or -1
-      if (v >= 0) {
+      // a parked value names a local expert; anything else (buffers shared with a concurrent call)
+      // is flagged and skipped, never used as an index
+      if (v >= 0 && (v & 1023) >= El) {
+        moe::record_status(a.status, MOE_ERR_BAD_ROW);
+      } else if (v >= 0) {
         const int le = v & 1023;
         const int64_t tile = (t0 + e / k) / kRowsPerTile;
         r = s_off[le] + a.tile_counts[static_cast<int64_t>(le) * a.num_tiles + tile] + (v >> 10);
@@ -330,7 +336,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     }
     dst[m] = r;
   }
-  if (n > 0) {
+  if (kGather && n > 0) {
     if (!moe::mbar_wait(&bar, 0)) {
       moe::record_status(a.status, MOE_ERR_TIMEOUT);
       moe::mbar_wait(&bar, 0);  // one more bounded wait for the loads in flight before leaving
@@ -379,7 +385,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
   const int64_t tail = a.C - total;
   for (int64_t i = static_cast<int64_t>(b) * 32 + lane; i < tail; i += static_cast<int64_t>(G) * 32)
     a.sorted_ids[total + i] = pad_value;
-  if (n > 0) moe::bulk_wait_read_all();  // the staged rows must outlive the stores that read them
+  if (kGather && n > 0) moe::bulk_wait_read_all();  // the staged rows must outlive the stores that read them
 }
 
 // ------------------------------------------------------------------------------------------
@@ -808,9 +814,68 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
       static_cast<size_t>(tpc) * row_bytes + static_cast<size_t>(E_local + 1) * sizeof(int), kPgCtasPerSm);
   if (smem2 == 0) return MOE_ERR_CUDA;
   if (smem2 > 48 * 1024 &&
-      cudaFuncSetAttribute(place_gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2)) !=
+      cudaFuncSetAttribute(place_gather_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2)) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
-  return moe_host::launch_pdl(place_gather_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st, a,
+  return moe_host::launch_pdl(place_gather_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st, a,
                               static_cast<const uint8_t*>(hidden), row_bytes, tpc, static_cast<uint8_t*>(permuted));
+}
+
+// ---------------------------------------------------------------------------------------------
+// moe_align_permute through the tile kernels above (given routes, no gather).
+// ---------------------------------------------------------------------------------------------
+size_t moe_internal::align_tiles_workspace_bytes(int64_t T, int32_t E_local) { return fused_layout(T, E_local).bytes; }
+
+moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
+                                       const int32_t* expert_map, int32_t E_local, int32_t block_size,
+                                       int32_t* counts, int32_t* offsets, int32_t* sorted_token_ids,
+                                       int32_t* expert_ids, int32_t* num_tokens_post_pad, int32_t* inv_perm,
+                                       void* workspace, cudaStream_t st) {
+  DispatchArgs a{};
+  a.T = T;
+  a.E = E_global;
+  a.k = k;
+  a.given_ids = 1;
+  a.expert_map = expert_map;
+  a.E_local = E_local;
+  a.bs = block_size;
+  a.bs_shift = (block_size & (block_size - 1)) == 0 ? __builtin_ctz(static_cast<unsigned>(block_size)) : -1;
+  a.P = T * k;
+  a.C = moe_align_capacity(T, k, E_local, block_size);
+  a.NB = static_cast<int>((a.C + block_size - 1) / block_size);
+  const FusedLayout lay = fused_layout(T, E_local);
+  a.rows_per_tile = kRowsPerTile;
+  a.num_tiles = lay.num_tiles;
+  a.topk_ids = const_cast<int32_t*>(topk_ids);  // read only: given_ids
+  a.counts = counts;
+  a.offsets = offsets;
+  a.sorted_ids = sorted_token_ids;
+  a.expert_ids = expert_ids;
+  a.n_pad = num_tokens_post_pad;
+  a.inv_perm = inv_perm;
+  a.status = static_cast<int32_t*>(workspace);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.tile_counts_off);
+  a.totals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.totals_off);
+
+  GcKernel gk = family_pick<GateCountFamily, float>(1, 1);  // no row is gated
+  const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
+  if (smem1 > 48 * 1024 &&
+      cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem1)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
+    return MOE_ERR_CUDA;
+  if (moe_host::launch_pdl(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
+      MOE_OK)
+    return MOE_ERR_CUDA;
+  // placement only: up to kPgMaxTokens tokens per one-warp CTA, the CTAs filling whole waves
+  const int sms = moe_host::sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  const int tpc = moe_host::tokens_per_cta(T, kPgMaxTokens, static_cast<int64_t>(sms) * 16);
+  int64_t blocks = (T + tpc - 1) / tpc;
+  if (blocks < 1) blocks = 1;
+  if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
+  const size_t smem2 = static_cast<size_t>(E_local + 1) * sizeof(int);
+  return moe_host::launch_pdl(place_gather_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st,
+                              a, static_cast<const uint8_t*>(nullptr), 0u, tpc, static_cast<uint8_t*>(nullptr));
 }
