@@ -57,6 +57,14 @@ CASES = [
     ("small_one_local_expert", 3, 32, 4, torch.float32, False, "one_local", 1, 8, 64),
     ("small_k1_bs1_H8", 1, 4, 1, torch.bfloat16, False, None, 4, 1, 8),
     ("tile_all_remote", 64, 32, 4, torch.bfloat16, True, "none_local", 8, 16, 32),
+    # one thread per row (T >= 1024, E <= 64 in whole 16-byte chunks, k <= 8): maps, ties, k == E,
+    # ragged last tiles
+    ("lanes_bf16_E64_k8_strided_map", 1500, 64, 8, torch.bfloat16, True, "strided", 16, 16, 64),
+    ("lanes_fp32_E8_k8_k_equals_E", 1100, 8, 8, torch.float32, False, None, 8, 4, 32),
+    ("lanes_bf16_E16_k1_ties", 2049, 16, 1, torch.bfloat16, True, None, 16, 8, 16),
+    ("lanes_fp32_E12_k3_one_local", 1030, 12, 3, torch.float32, True, "one_local", 1, 2, 16),
+    ("lanes_bf16_bad_map_values", 1200, 64, 4, torch.bfloat16, True, "bad", 16, 16, 64),
+    ("lanes_fp32_E48_k6_ties", 2077, 48, 6, torch.float32, False, None, 48, 32, 48),
 ]
 
 
@@ -91,6 +99,8 @@ def test_dispatch_parity(name, T, E, k, dtype, renorm, kind, E_local, bs, H):
     dev = require_gpu()
     g = torch.Generator().manual_seed(T + 7 * E + k)
     x = torch.randn((T, E), generator=g).to(dtype)
+    if name.endswith("_ties"):  # integer logits: equal values at the k boundary in most rows
+        x = torch.randint(0, 4, (T, E), generator=g).to(dtype)
     if kind == "none_local":  # the last E_local experts never make the top k
         x[:, E - E_local:] -= 50.0
     if kind == "bad":  # make the flagged globals win often
@@ -118,13 +128,15 @@ def test_dispatch_parity(name, T, E, k, dtype, renorm, kind, E_local, bs, H):
         assert status == (tdt.MOE_ERR_BAD_EXPERT_ID if kind == "bad" else tdt.MOE_OK), (name, status)
 
 
-def test_dispatch_matches_stage_entry_points():
-    """The fused dispatch and the three stage calls it replaces give identical outputs."""
+@pytest.mark.parametrize("workload", ["qwen3moe_prefill_T4096_E128_k8", "nonpow2_T16384_E60_k4"])
+def test_dispatch_matches_stage_entry_points(workload):
+    """The fused dispatch and the three stage calls it replaces give identical outputs (one warp per
+    row on the prefill workload, one thread per row on the non-power-of-2 one)."""
     dev = require_gpu()
-    wl = I.WORKLOADS["qwen3moe_prefill_T4096_E128_k8"]
+    wl = I.WORKLOADS[workload]
     logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)
-    a = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, device=dev)
-    b = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, device=dev)
+    a = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, logits_dtype=logits.dtype, device=dev)
+    b = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, logits_dtype=logits.dtype, device=dev)
     a.dispatch(logits, hidden)
     b.gate(logits)
     b.align_permute()
@@ -179,7 +191,9 @@ def test_dispatch_given_routes(name, T, k, E, kind, E_local, bs, H):
     (20, 64, 4, torch.float32, False, 64, 16, 64),
     (300, 128, 8, torch.bfloat16, True, 128, 64, 256),    # three-kernel path
     (777, 60, 4, torch.float32, False, 60, 64, 128),
-], ids=["small_bf16", "small_fp32", "tile_bf16", "tile_fp32"])
+    (2500, 60, 4, torch.float32, True, 60, 64, 128),     # one thread per row
+    (1300, 64, 8, torch.bfloat16, False, 64, 16, 64),
+], ids=["small_bf16", "small_fp32", "tile_bf16", "tile_fp32", "lanes_fp32", "lanes_bf16"])
 def test_dispatch_sigmoid_scoring(T, E, k, dtype, renorm, E_local, bs, H):
     """moe_route_dispatch with MOE_SCORING_SIGMOID: weights from the sigmoid reading, the rest as for softmax."""
     dev = require_gpu()

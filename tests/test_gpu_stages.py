@@ -50,6 +50,13 @@ TOPK_CASES = [
     (999, 128, 8, torch.bfloat16, True, 1.0, True),        # tie-heavy: integer logits
     (999, 256, 8, torch.bfloat16, False, 1.0, True),
     (333, 8, 8, torch.bfloat16, True, 1.0, True),          # k == E
+    # one thread per row (T >= 1024, E <= 64 in whole 16-byte chunks, k <= 8)
+    (1500, 64, 8, torch.bfloat16, True, 1.0, True),        # tie-heavy
+    (1024, 32, 1, torch.float32, False, 1.0, False),
+    (4097, 16, 2, torch.bfloat16, False, 1.0, True),       # ragged last tile, ties
+    (2048, 48, 6, torch.float32, True, 2.0, True),
+    (1025, 8, 8, torch.bfloat16, True, 1.0, False),        # k == E
+    (1100, 60, 7, torch.float32, False, 8.0, False),       # wide logits: tiny weights
 ]
 
 
@@ -75,6 +82,8 @@ SIGMOID_CASES = [
     (50, 1000, 8, torch.float32, True, 3.0, False),
     (999, 256, 8, torch.bfloat16, True, 1.0, True),
     (300, 64, 8, torch.float32, False, 30.0, False),       # far tails: scores near 0 and 1
+    (1500, 64, 8, torch.bfloat16, True, 1.0, True),        # one thread per row, tie-heavy
+    (1100, 24, 3, torch.float32, False, 30.0, False),      # one thread per row, far tails
 ]
 
 

@@ -669,6 +669,8 @@ moe_status_t launch_align_cluster(const AlignArgs& a, cudaStream_t st) {
   if (cudaFuncSetAttribute(align_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
+  if (moe_host::prefer_max_shared(reinterpret_cast<const void*>(align_cluster_kernel)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   const int nc = align_cluster_ctas(a.P, smem);
   const int64_t warps = static_cast<int64_t>(nc) * kClusterWarps;
   int64_t run = (a.P + warps - 1) / warps;
@@ -784,6 +786,9 @@ extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, in
                              static_cast<int>(smem)) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
+  if (moe_host::prefer_max_shared(reinterpret_cast<const void*>(align_count_kernel)) != cudaSuccess ||
+      moe_host::prefer_max_shared(reinterpret_cast<const void*>(align_place_kernel)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   align_count_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   if (a.num_tiles > 1) {
@@ -885,6 +890,9 @@ extern "C" moe_status_t moe_align_permute_noalloc(const int32_t* topk_ids, int64
                              static_cast<int>(smem)) != cudaSuccess)
       return MOE_ERR_CUDA;
   }
+  if (moe_host::prefer_max_shared(reinterpret_cast<const void*>(align_count_kernel)) != cudaSuccess ||
+      moe_host::prefer_max_shared(reinterpret_cast<const void*>(align_place_kernel)) != cudaSuccess)
+    return MOE_ERR_CUDA;
   align_count_kernel<<<a.num_tiles, kAlignThreads, smem, st>>>(a);
   if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
   if (a.num_tiles > 1) {

@@ -269,11 +269,21 @@ inline moe_status_t launch_status() {
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
+// Every kernel of the library asks for the same split of each SM's L1 / shared memory (the most
+// shared memory).  An SM changes its split only when it is idle, so kernels with different splits
+// chained by programmatic dependent launch would leave SMs unable to take the next kernel's CTAs
+// until every CTA of the previous ones has left them.
+inline cudaError_t prefer_max_shared(const void* kernel) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                              static_cast<int>(cudaSharedmemCarveoutMaxShared));
+}
+
 // Launch with programmatic stream serialisation (the kernel may start while the previous kernel
 // in the stream finishes; it calls moe::pdl_wait before reading that kernel's outputs).
 template <typename... KArgs, typename... Args>
 inline moe_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                                Args&&... args) {
+  if (prefer_max_shared(reinterpret_cast<const void*>(kernel)) != cudaSuccess) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;

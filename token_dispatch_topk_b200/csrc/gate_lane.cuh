@@ -1,0 +1,207 @@
+// gate_lane.cuh -- fused softmax + top-k of short router-logit rows, one thread per row.
+//
+// Operation: the fused softmax+topk of "Upstream Reference: Deep-Spark xllm + vllm", "File Index"
+// (moe_topk_softmax_kernels.cuh; vLLM topk_softmax_kernels.cu), with the same selection order and
+// weights as gate_row.cuh: the k largest logits, larger first, the lower expert index first among
+// equal logits; softmax over the whole row (or over the k with renormalisation), or the logistic
+// scores of the sigmoid variant (moe_topk_sigmoid_kernels.cuh).
+//
+// gate_row.cuh spends a warp on each row: k rounds of warp-wide reductions, a few hundred
+// instructions per row, which makes gating of many short rows (say E = 60 experts, T = 16K tokens)
+// bound by instruction issue.  Here a CTA stages 32 rows in shared memory and G lanes (up to 4)
+// scan each row once, inserting every logit into a register-resident list of the K largest (about
+// 5 * K instructions per logit); the G lists are merged with two shuffle rounds.  Several times
+// fewer instructions per row than the warp-per-row kernel.
+//
+// Order: logits arrive in ascending expert order and a logit moves ahead only of kept logits it
+// strictly exceeds, so among equal logits the lower index stays ahead (+0 and -0 compare equal).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "gate_row.cuh"
+
+namespace moe_gate {
+
+constexpr int kLaneGateMaxK = 8;      // K is a template parameter: 1..8
+constexpr int kLaneGateMaxE = 64;     // logits one thread scans
+constexpr int64_t kLaneGateMinRows = 1024;  // below this, the warp-per-row kernels have lower latency
+
+// Whether a batch of rows takes the one-thread-per-row gating (the same rule for every entry point,
+// so that moe_topk_softmax and moe_route_dispatch choose the same arithmetic for the same batch).
+// Rows must be whole 16-byte chunks and the logits 16-byte aligned.
+inline bool lane_gating_fits(int64_t T, int E, int k, int elem_bytes, const void* logits) {
+  return T >= kLaneGateMinRows && k <= kLaneGateMaxK && E <= kLaneGateMaxE && (E * elem_bytes) % 16 == 0 &&
+         (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
+}
+
+// Shared-memory layout of a staged tile: row r starts at chunk r * stride, stride = chunks per row
+// rounded up to odd, so 32 lanes each reading 16 bytes of their own row hit distinct bank groups.
+__host__ __device__ inline int lane_tile_stride(int cpr) { return cpr | 1; }
+
+// Copy rows [0, rows) of a tile (contiguous in global memory, 16-byte aligned, cpr chunks a row)
+// into shared memory with coalesced 16-byte loads, kLaneLoadBatch of them in flight per thread
+// before the first store (the kernels stage at most 4 chunks per thread: one batch).
+// Chunk c of the tile belongs to row c / cpr, computed as floor((c + 0.5) / cpr) in fp32: exact
+// for the tile sizes here (c < 2^12, cpr <= 16).
+constexpr int kLaneLoadBatch = 4;
+__device__ __forceinline__ void lane_tile_load(const uint4* __restrict__ g, int rows, int cpr, int stride,
+                                               uint4* __restrict__ s, int tid, int nthreads) {
+  const int n = rows * cpr;
+  const float inv = 1.f / static_cast<float>(cpr);
+  for (int c0 = tid; c0 < n; c0 += kLaneLoadBatch * nthreads) {
+    uint4 v[kLaneLoadBatch];
+#pragma unroll
+    for (int u = 0; u < kLaneLoadBatch; ++u) {
+      const int c = c0 + u * nthreads;
+      if (c < n) v[u] = __ldcs(g + c);
+    }
+#pragma unroll
+    for (int u = 0; u < kLaneLoadBatch; ++u) {
+      const int c = c0 + u * nthreads;
+      if (c < n) {
+        const int r = static_cast<int>((static_cast<float>(c) + 0.5f) * inv);
+        s[r * stride + (c - r * cpr)] = v[u];
+      }
+    }
+  }
+}
+
+// The K largest logits seen so far, larger first (v), with their experts (e).
+template <int K>
+struct LaneTopK {
+  float v[K];
+  int e[K];
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int p = 0; p < K; ++p) {
+      v[p] = -INFINITY;
+      e[p] = 0;
+    }
+  }
+
+  // Logit x of expert i, experts arriving in ascending order.
+  __device__ __forceinline__ void insert(float x, int i) {
+    bool gt[K];
+#pragma unroll
+    for (int p = 0; p < K; ++p) gt[p] = x > v[p];
+#pragma unroll
+    for (int p = K - 1; p > 0; --p) {
+      v[p] = gt[p - 1] ? v[p - 1] : (gt[p] ? x : v[p]);
+      e[p] = gt[p - 1] ? e[p - 1] : (gt[p] ? i : e[p]);
+    }
+    v[0] = gt[0] ? x : v[0];
+    e[0] = gt[0] ? i : e[0];
+  }
+};
+
+// Insert the logits of one 16-byte chunk (chunk j of the row) in ascending expert order.
+template <typename TIn, int K>
+__device__ __forceinline__ void lane_insert_chunk(LaneTopK<K>& t, const uint4 q, int j) {
+  if constexpr (sizeof(TIn) == 4) {
+    const int i = 4 * j;
+    t.insert(__uint_as_float(q.x), i);
+    t.insert(__uint_as_float(q.y), i + 1);
+    t.insert(__uint_as_float(q.z), i + 2);
+    t.insert(__uint_as_float(q.w), i + 3);
+  } else {
+    const int i = 8 * j;
+    t.insert(moe::bf16_lo(q.x), i);
+    t.insert(moe::bf16_hi(q.x), i + 1);
+    t.insert(moe::bf16_lo(q.y), i + 2);
+    t.insert(moe::bf16_hi(q.y), i + 3);
+    t.insert(moe::bf16_lo(q.z), i + 4);
+    t.insert(moe::bf16_hi(q.z), i + 5);
+    t.insert(moe::bf16_lo(q.w), i + 6);
+    t.insert(moe::bf16_hi(q.w), i + 7);
+  }
+}
+
+// Lanes per row: G lanes share a row, lane g scanning chunks [g * cpr / G, (g + 1) * cpr / G) (at
+// least one chunk each).  More lanes per row put more warps in flight for the same instructions
+// per row: the scan is a chain of dependent inserts, and one lane per row leaves too few warps.
+__host__ __device__ inline int lane_gate_lanes(int cpr) { return cpr >= 4 ? 4 : (cpr >= 2 ? 2 : 1); }
+
+// Gate one staged row (cpr 16-byte chunks of TIn logits; E = cpr * 16 / sizeof(TIn)) with the G
+// lanes g = lane % G of a row group (consecutive lanes; every lane of the warp calls this).
+// `mode`: kGateRenorm, kGateSigmoid.  Every lane of the group returns the K experts in selection
+// order and their weights.
+// Merge: after each lane's scan, lists are merged pairwise (shuffle distance 1, then 2): the list of
+// the lower chunks is the base and the other is inserted into it in its own order.  Every expert of
+// the inserted list has a higher index than every expert of the base, and among equal logits the
+// inserted list keeps the lower index ahead, so the merged list is the one a single scan in expert
+// order would give.
+template <typename TIn, int K, int G>
+__device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, int cpr, int mode, int g,
+                                              float (&w)[K], int (&ids)[K]) {
+  LaneTopK<K> t;
+  t.init();
+  const int j0 = (g * cpr) / G, j1 = ((g + 1) * cpr) / G;
+  for (int j = j0; j < j1; ++j) lane_insert_chunk<TIn, K>(t, srow[j], j);
+#pragma unroll
+  for (int d = 1; d < G; d <<= 1) {
+    LaneTopK<K> o;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      o.v[q] = __shfl_xor_sync(0xffffffffu, t.v[q], d);
+      o.e[q] = __shfl_xor_sync(0xffffffffu, t.e[q], d);
+    }
+    const bool upper = (g & d) != 0;  // this lane's chunks come after the partner's
+    LaneTopK<K> base, add;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      base.v[q] = upper ? o.v[q] : t.v[q];
+      base.e[q] = upper ? o.e[q] : t.e[q];
+      add.v[q] = upper ? t.v[q] : o.v[q];
+      add.e[q] = upper ? t.e[q] : o.e[q];
+    }
+#pragma unroll
+    for (int q = 0; q < K; ++q) base.insert(add.v[q], add.e[q]);
+    t = base;
+  }
+  const bool renormalize = (mode & kGateRenorm) != 0;
+  const bool sigmoid = (mode & kGateSigmoid) != 0;
+  const float m = t.v[0];
+  float p[K];
+  float den = 0.f;
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    p[q] = sigmoid ? 1.f / (1.f + expf(-t.v[q])) : expf(t.v[q] - m);
+    den += p[q];
+  }
+  if (!renormalize && !sigmoid) {  // full-row denominator: each lane sums its chunks, then the group
+    float z[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (short dependency chains)
+    for (int j = j0; j < j1; ++j) {
+      const uint4 q = srow[j];
+      if constexpr (sizeof(TIn) == 4) {
+        z[0] += expf(__uint_as_float(q.x) - m);
+        z[1] += expf(__uint_as_float(q.y) - m);
+        z[2] += expf(__uint_as_float(q.z) - m);
+        z[3] += expf(__uint_as_float(q.w) - m);
+      } else {
+        z[0] += expf(moe::bf16_lo(q.x) - m) + expf(moe::bf16_hi(q.x) - m);
+        z[1] += expf(moe::bf16_lo(q.y) - m) + expf(moe::bf16_hi(q.y) - m);
+        z[2] += expf(moe::bf16_lo(q.z) - m) + expf(moe::bf16_hi(q.z) - m);
+        z[3] += expf(moe::bf16_lo(q.w) - m) + expf(moe::bf16_hi(q.w) - m);
+      }
+    }
+    den = (z[0] + z[1]) + (z[2] + z[3]);
+#pragma unroll
+    for (int d = 1; d < G; d <<= 1) den += __shfl_xor_sync(0xffffffffu, den, d);
+  }
+#pragma unroll
+  for (int q = 0; q < K; ++q) {
+    if (sigmoid) {
+      w[q] = renormalize ? (den > 0.f ? p[q] / den : 1.f / static_cast<float>(K)) : p[q];
+    } else {
+      w[q] = p[q] / den;
+    }
+    ids[q] = t.e[q];
+  }
+}
+
+}  // namespace moe_gate

@@ -203,9 +203,10 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
   __shared__ int s_abort;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int64_t per = (a.units + gridDim.x - 1) / gridDim.x;
-  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * per;
-  const int64_t u1 = (u0 + per < a.units) ? u0 + per : a.units;
+  // an even share of the units (floor(b * units / G) up to floor((b + 1) * units / G)): every CTA
+  // of the grid works, and the SMs, each holding the same number of CTAs, get the same bytes
+  const int64_t u0 = static_cast<int64_t>(blockIdx.x) * a.units / gridDim.x;
+  const int64_t u1 = static_cast<int64_t>(blockIdx.x + 1) * a.units / gridDim.x;
   if (tid == 0) {
     for (int s = 0; s < S; ++s) {
       moe::mbar_init(&full[s], 1);

@@ -10,13 +10,16 @@
 //
 // Batches above the small-batch limits take three kernels, chained by programmatic dependent
 // launch:
-// gate_count_kernel (one CTA per tile of kRowsPerTile tokens):
+// gate_count_kernel (one CTA per tile of 16 or 32 tokens; 16 when the tiles of a batch fit on
+// the SMs at once, so that each warp gates one row):
 //   A. each warp gates rows of the tile (gate_row: one warp per row) and writes topk_weights and
 //      topk_ids; the local expert of every slot of the tile goes to shared memory;
 //   B. stable ranks inside the tile: each warp owns a contiguous run of the tile's slots, counts
 //      it into its own shared-memory row, the rows are scanned across warps, and each slot's rank
 //      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm and the
 //      tile's per-expert counts go to the workspace, expert-major ([E_local][tiles]).
+//   gate_count_lanes_kernel replaces it for many short rows (moe_gate::lane_gating_fits): one
+//   CTA per tile of 32 tokens, up to four lanes per row (gate_lane.cuh), the same ranks and counts.
 // tile_scan_kernel (one CTA per local expert): the expert's row of tile counts becomes the
 //   exclusive prefix over the tiles (the tile bases) and its total goes to the workspace.
 //   Nothing waits on another CTA: the kernel boundary is the only grid-wide step.
@@ -31,6 +34,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "gate_lane.cuh"
 #include "gate_row.cuh"
 #include "route_internal.h"
 
@@ -39,12 +43,13 @@ namespace {
 constexpr int kGcWarps = 16;
 constexpr int kGcThreads = kGcWarps * 32;
 constexpr int kWsHeaderBytes = 256;  // status word, padding
-constexpr int kRowsPerTile = 32;
+constexpr int kRowsPerTile = 32;       // tile height of the lane kernel and of the align entry point
+constexpr int kRowsPerTileSmall = 16;  // tile height of gate_count_kernel when all tiles fit at once
+constexpr int kGcCtasPerSm = 4;        // gate_count_kernel CTAs resident per SM (2048 threads)
 constexpr int kTsThreads = 128;  // tile_scan_kernel: threads per expert
 constexpr int kPgMaxTokens = 8;
 constexpr uint32_t kPgCtaBytes = 32u * 1024u;
 constexpr int kPgCtasPerSm = 4;  // place_gather_kernel CTAs resident per SM
-constexpr uint64_t kL2PrefetchMax = 48ull << 20;  // hidden bytes worth keeping in L2 through the routing
 
 struct DispatchArgs {
   const void* logits;
@@ -61,6 +66,7 @@ struct DispatchArgs {
   int64_t C;  // capacity rows
   int NB;     // blocks
   int rows_per_tile;
+  int rt_shift;  // log2(rows_per_tile)
   int num_tiles;
   float* topk_weights;
   int32_t* topk_ids;
@@ -73,9 +79,6 @@ struct DispatchArgs {
   int32_t* status;
   int32_t* tile_counts;  // [E_local][num_tiles]: tile counts, then tile bases
   int32_t* totals;       // [E_local]
-  const uint8_t* hidden;  // prefetched into L2 by gate_count_kernel when prefetch_hidden
-  uint32_t row_bytes;
-  int prefetch_hidden;
 };
 
 // Local expert of global expert g (or -1: remote); out-of-range values are flagged.
@@ -135,10 +138,6 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   __syncthreads();
   moe::pdl_wait();  // the logits may come from the previous kernel
   moe::pdl_launch_dependents();
-  // the tile's hidden rows head for L2 while the tile is routed: the gather reads them from there
-  if (a.prefetch_hidden && tid < rows) {
-    moe::bulk_prefetch_l2(a.hidden + (row0 + tid) * static_cast<int64_t>(a.row_bytes), a.row_bytes);
-  }
 
   // A. gating, one warp per row (or the routes the caller gave)
   const TIn* logits = static_cast<const TIn*>(a.logits);
@@ -199,6 +198,93 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   }
 }
 
+
+// One CTA of G warps per tile of kRowsPerTile tokens, G lanes per row: the tile's logits are staged
+// in shared memory and each group of G lanes gates one row (moe_gate::lane_gate_row); then warp 0
+// computes the stable ranks inside the tile (the slots in order, 32 at a time: rank = the expert's
+// count so far + earlier peers in the chunk), parked in inv_perm as in gate_count_kernel, and the
+// tile's per-expert counts.
+// Shared memory: staged rows [kRowsPerTile * stride chunks] | hist [E_local] | s_le [kRowsPerTile * K].
+template <typename TIn, int K, int G>
+__global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a, int cpr) {
+  constexpr int NT = 32 * G;
+  extern __shared__ __align__(16) uint4 s_rows[];
+  const int El = a.E_local;
+  const int stride = moe_gate::lane_tile_stride(cpr);
+  int* hist = reinterpret_cast<int*>(s_rows + kRowsPerTile * stride);
+  int* s_le = hist + El;
+  const int tid = threadIdx.x, lane = tid & 31;
+  const int tile = blockIdx.x;
+  const int64_t row0 = static_cast<int64_t>(tile) * kRowsPerTile;
+  const int rows = static_cast<int>((a.T - row0) < kRowsPerTile ? (a.T - row0) : kRowsPerTile);  // >= 1
+  for (int e = tid; e < El; e += NT) hist[e] = 0;
+  moe::pdl_wait();  // the logits may come from the previous kernel
+  moe::pdl_launch_dependents();
+  moe_gate::lane_tile_load(static_cast<const uint4*>(a.logits) + row0 * cpr, rows, cpr, stride, s_rows, tid, NT);
+  __syncthreads();
+  {
+    const int r = tid / G, g = tid % G;
+    const int rr = r < rows ? r : rows - 1;  // every lane takes part in the group's shuffles
+    float w[K];
+    int ids[K];
+    moe_gate::lane_gate_row<TIn, K, G>(s_rows + rr * stride, cpr, a.renormalize, g, w, ids);
+    if (r < rows && g == 0) {
+      const int64_t o = (row0 + r) * K;
+#pragma unroll
+      for (int q = 0; q < K; ++q) {
+        a.topk_weights[o + q] = w[q];
+        a.topk_ids[o + q] = ids[q];
+        s_le[r * K + q] = to_local(a, ids[q]);
+      }
+    }
+  }
+  __syncthreads();
+  if (tid >= 32) return;
+  const int nslots = rows * K;
+  for (int c = 0; c < nslots; c += 32) {
+    const int i = c + lane;
+    const int le = i < nslots ? s_le[i] : -1;
+    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    if (le >= 0) {
+      // parked until place_gather_kernel: (rank in the tile) << 10 | local expert
+      a.inv_perm[row0 * K + i] = ((hist[le] + __popc(peers & moe::lanemask_lt())) << 10) | le;
+    } else if (i < nslots) {
+      a.inv_perm[row0 * K + i] = -1;
+    }
+    __syncwarp();
+    if (le >= 0 && lane == __ffs(peers) - 1) hist[le] += __popc(peers);
+    __syncwarp();
+  }
+  for (int e = lane; e < El; e += 32) a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = hist[e];
+}
+
+using LanesKernel = void (*)(DispatchArgs, int);
+
+template <typename TIn, int K>
+LanesKernel lanes_kernel_g(int G) {
+  switch (G) {
+    case 1: return &gate_count_lanes_kernel<TIn, K, 1>;
+    case 2: return &gate_count_lanes_kernel<TIn, K, 2>;
+    case 4: return &gate_count_lanes_kernel<TIn, K, 4>;
+    default: return nullptr;
+  }
+}
+
+template <typename TIn>
+LanesKernel lanes_kernel_for(int k, int G) {
+  switch (k) {
+    case 1: return lanes_kernel_g<TIn, 1>(G);
+    case 2: return lanes_kernel_g<TIn, 2>(G);
+    case 3: return lanes_kernel_g<TIn, 3>(G);
+    case 4: return lanes_kernel_g<TIn, 4>(G);
+    case 5: return lanes_kernel_g<TIn, 5>(G);
+    case 6: return lanes_kernel_g<TIn, 6>(G);
+    case 7: return lanes_kernel_g<TIn, 7>(G);
+    case 8: return lanes_kernel_g<TIn, 8>(G);
+    default: return nullptr;
+  }
+}
+
 // One CTA per local expert: its row of tile counts -> exclusive prefix over the tiles, in place;
 // the total to `totals`.  Thread i owns a contiguous run of tiles, read in unrolled batches so that
 // the loads of a run are in flight together.
@@ -206,7 +292,7 @@ __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
   __shared__ int warp_sums[kTsThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int e = blockIdx.x;
-  // let place_gather_kernel start now (it prefetches the hidden rows, then waits for this kernel,
+  // let place_gather_kernel start now (it loads its hidden rows, then waits for this kernel,
   // which completes after gate_count_kernel)
   moe::pdl_launch_dependents();
   moe::pdl_wait();  // tile counts come from gate_count_kernel
@@ -323,7 +409,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
         moe::record_status(a.status, MOE_ERR_BAD_ROW);
       } else if (v >= 0) {
         const int le = v & 1023;
-        const int64_t tile = (t0 + e / k) / kRowsPerTile;
+        const int64_t tile = (t0 + e / k) >> a.rt_shift;
         r = s_off[le] + a.tile_counts[static_cast<int64_t>(le) * a.num_tiles + tile] + (v >> 10);
         if (r < 0 || static_cast<int64_t>(r) >= a.C) {  // cannot happen for consistent inputs
           moe::record_status(a.status, MOE_ERR_BAD_ROW);
@@ -673,9 +759,9 @@ struct FusedLayout {
   size_t tile_counts_off, totals_off, bytes;
 };
 
-FusedLayout fused_layout(int64_t T, int E_local) {
+FusedLayout fused_layout(int64_t T, int E_local, int rows_per_tile) {
   FusedLayout l{};
-  const int64_t nt = (T + kRowsPerTile - 1) / kRowsPerTile;
+  const int64_t nt = (T + rows_per_tile - 1) / rows_per_tile;
   l.num_tiles = nt < 1 ? 1 : static_cast<int>(nt);
   l.tile_counts_off = kWsHeaderBytes;
   l.totals_off = l.tile_counts_off + ((static_cast<size_t>(l.num_tiles) * E_local * 4 + 255) & ~size_t{255});
@@ -687,7 +773,7 @@ FusedLayout fused_layout(int64_t T, int E_local) {
 
 extern "C" size_t moe_route_dispatch_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
   if (T < 0 || k < 1 || E_local < 1) return 0;
-  return fused_layout(T, E_local).bytes;
+  return fused_layout(T, E_local, kRowsPerTileSmall).bytes;  // the larger of the two tile heights' layouts
 }
 
 extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, const void* hidden, int64_t T,
@@ -737,8 +823,20 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.P = P;
   a.C = C;
   a.NB = static_cast<int>((C + block_size - 1) / block_size);
-  const FusedLayout lay = fused_layout(T, E_local);
-  a.rows_per_tile = kRowsPerTile;
+  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  const int sms = moe_host::sm_count();
+  if (sms <= 0) return MOE_ERR_CUDA;
+  // the gating kernel and its tile height: one thread per row for many short rows (32-row tiles);
+  // else one warp per row, in 16-row tiles when all of them fit on the SMs at once (then each warp
+  // gates one row), 32-row tiles above
+  const bool small_batch = T <= kSmallMaxTokens && P <= kSmallMaxSlots && E <= kSmallMaxExperts;
+  const bool lanes = !small_batch && !given_ids && moe_gate::lane_gating_fits(T, E, k, elem, logits);
+  int rt = kRowsPerTile;
+  if (!lanes && (T + kRowsPerTileSmall - 1) / kRowsPerTileSmall <= static_cast<int64_t>(sms) * kGcCtasPerSm)
+    rt = kRowsPerTileSmall;
+  const FusedLayout lay = fused_layout(T, E_local, rt);
+  a.rows_per_tile = rt;
+  a.rt_shift = rt == kRowsPerTileSmall ? 4 : 5;
   a.num_tiles = lay.num_tiles;
   a.topk_weights = topk_weights;
   a.topk_ids = topk_ids;
@@ -749,14 +847,10 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.n_pad = num_tokens_post_pad;
   a.inv_perm = inv_perm;
   a.status = static_cast<int32_t*>(workspace);
-  a.hidden = static_cast<const uint8_t*>(hidden);
-  a.row_bytes = row_bytes;
-  a.prefetch_hidden = static_cast<uint64_t>(T) * row_bytes <= kL2PrefetchMax ? 1 : 0;
   a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.tile_counts_off);
   a.totals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.totals_off);
 
-  // gating geometry: one warp per row, widest aligned vector that spreads the row over the warp
-  const int elem = dtype == MOE_DTYPE_BF16 ? 2 : 4;
+  // gating geometry of the warp-per-row kernels: widest aligned vector that spreads the row over the warp
   int vec_max = 16 / elem;
   while (vec_max > 1 && ((E % vec_max) != 0 || (reinterpret_cast<uintptr_t>(logits) % (vec_max * elem)) != 0))
     vec_max >>= 1;
@@ -774,7 +868,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   cudaStream_t st = static_cast<cudaStream_t>(stream);
 
   // small batches: one kernel, one CTA per slot
-  if (T <= kSmallMaxTokens && P <= kSmallMaxSlots && E <= kSmallMaxExperts) {
+  if (small_batch) {
     SmallKernel sk = given_ids ? &route_small_kernel<float, 1, 1, true>
                      : dtype == MOE_DTYPE_BF16 ? family_pick<SmallFamily, __nv_bfloat16>(vec, cpl)
                                                : family_pick<SmallFamily, float>(vec, cpl);
@@ -784,18 +878,29 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
                                 static_cast<int>(row_bytes / 16u), static_cast<uint4*>(permuted));
   }
 
-  // the gating geometry does not matter when the routes are given (no row is gated)
-  GcKernel gk = given_ids ? family_pick<GateCountFamily, float>(1, 1)
-                : dtype == MOE_DTYPE_BF16 ? family_pick<GateCountFamily, __nv_bfloat16>(vec, cpl)
-                                          : family_pick<GateCountFamily, float>(vec, cpl);
-  if (gk == nullptr) return MOE_ERR_UNSUPPORTED;
-  const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
-  if (smem1 > 48 * 1024 &&
-      cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           static_cast<int>(smem1)) != cudaSuccess)
-    return MOE_ERR_CUDA;
-  if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
-    return MOE_ERR_CUDA;
+  if (lanes) {
+    const int cpr = E * elem / 16;
+    const int G = moe_gate::lane_gate_lanes(cpr);
+    LanesKernel lk = dtype == MOE_DTYPE_BF16 ? lanes_kernel_for<__nv_bfloat16>(k, G) : lanes_kernel_for<float>(k, G);
+    if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
+    const size_t smem1 = static_cast<size_t>(kRowsPerTile) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4) +
+                         (static_cast<size_t>(E_local) + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
+    if (moe_host::launch_pdl(lk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(32 * G), smem1, st, a, cpr) != MOE_OK)
+      return MOE_ERR_CUDA;
+  } else {
+    // the gating geometry does not matter when the routes are given (no row is gated)
+    GcKernel gk = given_ids ? family_pick<GateCountFamily, float>(1, 1)
+                  : dtype == MOE_DTYPE_BF16 ? family_pick<GateCountFamily, __nv_bfloat16>(vec, cpl)
+                                            : family_pick<GateCountFamily, float>(vec, cpl);
+    if (gk == nullptr) return MOE_ERR_UNSUPPORTED;
+    const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
+    if (smem1 > 48 * 1024 &&
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem1)) != cudaSuccess)
+      return MOE_ERR_CUDA;
+    if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
+      return MOE_ERR_CUDA;
+  }
   if (moe_host::launch_pdl(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
       MOE_OK)
     return MOE_ERR_CUDA;
@@ -804,8 +909,6 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   // fill whole waves of kPgCtasPerSm per SM; shared memory sized so that no SM takes more
   int tpc = static_cast<int>(kPgCtaBytes / row_bytes);
   tpc = tpc < 1 ? 1 : (tpc > kPgMaxTokens ? kPgMaxTokens : tpc);
-  const int sms = moe_host::sm_count();
-  if (sms <= 0) return MOE_ERR_CUDA;
   tpc = moe_host::tokens_per_cta(T, tpc, static_cast<int64_t>(sms) * kPgCtasPerSm);
   int64_t blocks = (T + tpc - 1) / tpc;
   if (blocks < 1) blocks = 1;
@@ -824,7 +927,9 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
 // ---------------------------------------------------------------------------------------------
 // moe_align_permute through the tile kernels above (given routes, no gather).
 // ---------------------------------------------------------------------------------------------
-size_t moe_internal::align_tiles_workspace_bytes(int64_t T, int32_t E_local) { return fused_layout(T, E_local).bytes; }
+size_t moe_internal::align_tiles_workspace_bytes(int64_t T, int32_t E_local) {
+  return fused_layout(T, E_local, kRowsPerTile).bytes;
+}
 
 moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
                                        const int32_t* expert_map, int32_t E_local, int32_t block_size,
@@ -843,8 +948,9 @@ moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32
   a.P = T * k;
   a.C = moe_align_capacity(T, k, E_local, block_size);
   a.NB = static_cast<int>((a.C + block_size - 1) / block_size);
-  const FusedLayout lay = fused_layout(T, E_local);
+  const FusedLayout lay = fused_layout(T, E_local, kRowsPerTile);
   a.rows_per_tile = kRowsPerTile;
+  a.rt_shift = 5;
   a.num_tiles = lay.num_tiles;
   a.topk_ids = const_cast<int32_t*>(topk_ids);  // read only: given_ids
   a.counts = counts;

@@ -4,9 +4,10 @@
 // (moe_topk_softmax_kernels.cuh: fused softmax+topk; vLLM topk_softmax_kernels.cu),
 // placed by "Call Chain: MoE topk_softmax on BI-V100" between the router and the experts.
 //
-// Design (sm_100a).  Rows of E >= 16 experts: one warp per row (topk_row_warp_kernel below),
-// one warp-wide redux.sync max per selection round.  Short rows (E < 16): the sub-warp kernel
-// described here.
+// Design (sm_100a).  Many rows of at most 64 experts and k <= 8 (moe_gate::lane_gating_fits): up
+// to four lanes per row (topk_lane_kernel below, gate_lane.cuh).  Otherwise rows of E >= 16 experts: one
+// warp per row (topk_row_warp_kernel below), one warp-wide redux.sync max per selection round;
+// short rows (E < 16): the sub-warp kernel described here.
 // Sub-warp kernel: a sub-warp of G lanes (G a power of two, 1..32) owns one row.
 // Each lane loads its share of the row with 16-byte vector loads (8-, 4- or
 // 2-byte, or scalar, when the row length or base pointer does not allow 16),
@@ -25,6 +26,7 @@
 #include <stdint.h>
 
 #include "common.cuh"
+#include "gate_lane.cuh"
 #include "gate_row.cuh"
 
 namespace {
@@ -155,11 +157,77 @@ topk_row_warp_kernel(const TIn* __restrict__ logits, int64_t T, int E, int k, in
   }
 }
 
+// ------------------------------------------------------------------------------------------
+// G lanes per row (moe_gate::lane_gate_row): a CTA stages kLaneThreads / G consecutive rows in
+// shared memory with coalesced 16-byte loads, then each group of G lanes gates one row and its
+// first lane writes the K weights and ids.
+// ------------------------------------------------------------------------------------------
+constexpr int kLaneThreads = 128;
+
+template <typename TIn, int K, int G>
+__global__ void __launch_bounds__(kLaneThreads)
+topk_lane_kernel(const TIn* __restrict__ logits, int64_t T, int cpr, int mode, float* __restrict__ topk_weights,
+                 int32_t* __restrict__ topk_ids) {
+  constexpr int kRows = kLaneThreads / G;
+  extern __shared__ __align__(16) uint4 s_rows[];
+  const int tid = threadIdx.x;
+  const int stride = moe_gate::lane_tile_stride(cpr);
+  moe::pdl_wait();  // the logits may come from the previous kernel (the router projection)
+  moe::pdl_launch_dependents();
+  const int64_t row0 = static_cast<int64_t>(blockIdx.x) * kRows;
+  const int rows = (T - row0) < kRows ? static_cast<int>(T - row0) : kRows;  // >= 1
+  moe_gate::lane_tile_load(reinterpret_cast<const uint4*>(logits) + row0 * cpr, rows, cpr, stride, s_rows, tid,
+                           kLaneThreads);
+  __syncthreads();
+  const int r = tid / G, g = tid % G;
+  const int rr = r < rows ? r : rows - 1;  // every lane takes part in the group's shuffles
+  float w[K];
+  int ids[K];
+  moe_gate::lane_gate_row<TIn, K, G>(s_rows + rr * stride, cpr, mode, g, w, ids);
+  if (r < rows && g == 0) {
+    const int64_t o = (row0 + r) * K;
+#pragma unroll
+    for (int q = 0; q < K; ++q) {
+      topk_weights[o + q] = w[q];
+      topk_ids[o + q] = ids[q];
+    }
+  }
+}
+
+using LaneKernel = void (*)(const void*, int64_t, int, int, float*, int32_t*);
+
+template <typename TIn, int K>
+LaneKernel lane_kernel_g(int G) {
+  switch (G) {
+    case 1: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 1>);
+    case 2: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 2>);
+    case 4: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 4>);
+    default: return nullptr;
+  }
+}
+
+template <typename TIn>
+LaneKernel lane_kernel_for(int k, int G) {
+  switch (k) {
+    case 1: return lane_kernel_g<TIn, 1>(G);
+    case 2: return lane_kernel_g<TIn, 2>(G);
+    case 3: return lane_kernel_g<TIn, 3>(G);
+    case 4: return lane_kernel_g<TIn, 4>(G);
+    case 5: return lane_kernel_g<TIn, 5>(G);
+    case 6: return lane_kernel_g<TIn, 6>(G);
+    case 7: return lane_kernel_g<TIn, 7>(G);
+    case 8: return lane_kernel_g<TIn, 8>(G);
+    default: return nullptr;
+  }
+}
+
 using TopkKernel = void (*)(const void*, int64_t, int, int, int, int, float*, int32_t*);
 
 // Launch a gating kernel (any instance, arguments as a void* array) with programmatic stream
 // serialisation.
 cudaError_t launch_topk(TopkKernel kern, int64_t grid, int block, size_t smem, cudaStream_t st, void** args) {
+  const cudaError_t e = moe_host::prefer_max_shared(reinterpret_cast<const void*>(kern));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(block);
@@ -295,6 +363,20 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
   // scoring mode bits of the kernels (moe_gate::kGateRenorm, moe_gate::kGateSigmoid)
   int renorm_flag = ((flags & MOE_RENORMALIZE) ? moe_gate::kGateRenorm : 0) |
                     ((flags & MOE_SCORING_SIGMOID) ? moe_gate::kGateSigmoid : 0);
+  if (moe_gate::lane_gating_fits(T, E, k, elem, logits)) {
+    // G lanes per row
+    const int cpr = E * elem / 16;
+    const int G = moe_gate::lane_gate_lanes(cpr);
+    LaneKernel lk = dtype == MOE_DTYPE_BF16 ? lane_kernel_for<__nv_bfloat16>(k, G) : lane_kernel_for<float>(k, G);
+    if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
+    const int64_t rows_per_cta = kLaneThreads / G;
+    const int64_t grid = (T + rows_per_cta - 1) / rows_per_cta;
+    if (grid > 0x7fffffff) return MOE_ERR_INVALID_ARG;
+    const size_t smem = static_cast<size_t>(rows_per_cta) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4);
+    return moe_host::launch_pdl(lk, dim3(static_cast<unsigned>(grid)), dim3(kLaneThreads), smem,
+                                static_cast<cudaStream_t>(stream), logits, T, cpr, renorm_flag, topk_weights,
+                                topk_ids);
+  }
   if (E >= 16) {
     // one warp per row: the widest aligned vector that still spreads the row over all 32 lanes
     int vec_max = 16 / elem;
