@@ -121,10 +121,11 @@ __device__ __forceinline__ void lane_insert_chunk(LaneTopK<K>& t, const uint4 q,
   }
 }
 
-// Lanes per row: G lanes share a row, lane g scanning chunks [g * cpr / G, (g + 1) * cpr / G) (at
-// least one chunk each).  More lanes per row put more warps in flight for the same instructions
+// Lanes per row: G lanes share a row (G = 1, 2 or 4), lane g scanning chunks
+// [g * cpr / G, (g + 1) * cpr / G) (one to four chunks each, read into registers once).  More lanes per row put more warps in flight for the same instructions
 // per row: the scan is a chain of dependent inserts, and one lane per row leaves too few warps.
 __host__ __device__ inline int lane_gate_lanes(int cpr) { return cpr >= 4 ? 4 : (cpr >= 2 ? 2 : 1); }
+constexpr int kLaneMaxChunks = 4;  // chunks one lane holds: ceil(cpr / G) <= 4 for cpr <= 16
 
 // Gate one staged row (cpr 16-byte chunks of TIn logits; E = cpr * 16 / sizeof(TIn)) with the G
 // lanes g = lane % G of a row group (consecutive lanes; every lane of the warp calls this).
@@ -141,7 +142,15 @@ __device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, in
   LaneTopK<K> t;
   t.init();
   const int j0 = (g * cpr) / G, j1 = ((g + 1) * cpr) / G;
-  for (int j = j0; j < j1; ++j) lane_insert_chunk<TIn, K>(t, srow[j], j);
+  uint4 q[kLaneMaxChunks];
+#pragma unroll
+  for (int u = 0; u < kLaneMaxChunks; ++u) {
+    if (j0 + u < j1) q[u] = srow[j0 + u];
+  }
+#pragma unroll
+  for (int u = 0; u < kLaneMaxChunks; ++u) {
+    if (j0 + u < j1) lane_insert_chunk<TIn, K>(t, q[u], j0 + u);
+  }
 #pragma unroll
   for (int d = 1; d < G; d <<= 1) {
     LaneTopK<K> o;
@@ -175,18 +184,20 @@ __device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, in
   }
   if (!renormalize && !sigmoid) {  // full-row denominator: each lane sums its chunks, then the group
     float z[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (short dependency chains)
-    for (int j = j0; j < j1; ++j) {
-      const uint4 q = srow[j];
-      if constexpr (sizeof(TIn) == 4) {
-        z[0] += expf(__uint_as_float(q.x) - m);
-        z[1] += expf(__uint_as_float(q.y) - m);
-        z[2] += expf(__uint_as_float(q.z) - m);
-        z[3] += expf(__uint_as_float(q.w) - m);
-      } else {
-        z[0] += expf(moe::bf16_lo(q.x) - m) + expf(moe::bf16_hi(q.x) - m);
-        z[1] += expf(moe::bf16_lo(q.y) - m) + expf(moe::bf16_hi(q.y) - m);
-        z[2] += expf(moe::bf16_lo(q.z) - m) + expf(moe::bf16_hi(q.z) - m);
-        z[3] += expf(moe::bf16_lo(q.w) - m) + expf(moe::bf16_hi(q.w) - m);
+#pragma unroll
+    for (int u = 0; u < kLaneMaxChunks; ++u) {
+      if (j0 + u < j1) {
+        if constexpr (sizeof(TIn) == 4) {
+          z[0] += expf(__uint_as_float(q[u].x) - m);
+          z[1] += expf(__uint_as_float(q[u].y) - m);
+          z[2] += expf(__uint_as_float(q[u].z) - m);
+          z[3] += expf(__uint_as_float(q[u].w) - m);
+        } else {
+          z[0] += expf(moe::bf16_lo(q[u].x) - m) + expf(moe::bf16_hi(q[u].x) - m);
+          z[1] += expf(moe::bf16_lo(q[u].y) - m) + expf(moe::bf16_hi(q[u].y) - m);
+          z[2] += expf(moe::bf16_lo(q[u].z) - m) + expf(moe::bf16_hi(q[u].z) - m);
+          z[3] += expf(moe::bf16_lo(q[u].w) - m) + expf(moe::bf16_hi(q[u].w) - m);
+        }
       }
     }
     den = (z[0] + z[1]) + (z[2] + z[3]);

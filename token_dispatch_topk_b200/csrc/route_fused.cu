@@ -286,8 +286,10 @@ LanesKernel lanes_kernel_for(int k, int G) {
 }
 
 // One CTA per local expert: its row of tile counts -> exclusive prefix over the tiles, in place;
-// the total to `totals`.  Thread i owns a contiguous run of tiles, read in unrolled batches so that
-// the loads of a run are in flight together.
+// the total to `totals`.  Thread i owns a contiguous run of tiles; runs of up to kTsCache tiles
+// (batches of tiles up to 2048) are read once into registers, longer ones are read again for the
+// second pass.
+constexpr int kTsCache = 16;
 __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
   __shared__ int warp_sums[kTsThreads / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -301,13 +303,22 @@ __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
   const int per = (N + kTsThreads - 1) / kTsThreads;
   const int t0 = tid * per < N ? tid * per : N;
   const int t1 = t0 + per < N ? t0 + per : N;
+  const bool cached = per <= kTsCache;
+  int x[kTsCache];
   int sum = 0;
-  for (int t = t0; t < t1; t += 8) {
-    int x[8];
+  if (cached) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = t + u < t1 ? col[t + u] : 0;
+    for (int u = 0; u < kTsCache; ++u) x[u] = t0 + u < t1 ? col[t0 + u] : 0;
 #pragma unroll
-    for (int u = 0; u < 8; ++u) sum += x[u];
+    for (int u = 0; u < kTsCache; ++u) sum += x[u];
+  } else {
+    for (int t = t0; t < t1; t += 8) {
+      int y[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) y[u] = t + u < t1 ? col[t + u] : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += y[u];
+    }
   }
   int incl = sum;
 #pragma unroll
@@ -324,14 +335,22 @@ __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
     run += w < warp ? ws : 0;
     total += ws;
   }
-  for (int t = t0; t < t1; t += 8) {
-    int x[8];
+  if (cached) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) x[u] = t + u < t1 ? col[t + u] : 0;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      if (t + u < t1) col[t + u] = run;
+    for (int u = 0; u < kTsCache; ++u) {
+      if (t0 + u < t1) col[t0 + u] = run;
       run += x[u];
+    }
+  } else {
+    for (int t = t0; t < t1; t += 8) {
+      int y[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) y[u] = t + u < t1 ? col[t + u] : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (t + u < t1) col[t + u] = run;
+        run += y[u];
+      }
     }
   }
   if (tid == 0) a.totals[e] = total;
@@ -367,6 +386,26 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
   moe::pdl_launch_dependents();
   moe::pdl_wait();  // ranks (gate_count_kernel), tile bases and totals (tile_scan_kernel)
 
+  // the slots' parked values (rank in the tile << 10 | local expert, or -1) and their tiles' bases
+  // are loaded first, so that these loads are in flight during the offsets scan
+  const int nslots = n * k;  // <= kPgMaxTokens * 32
+  int pv[kPgMaxTokens];
+  int base[kPgMaxTokens];
+#pragma unroll
+  for (int m = 0; m < kPgMaxTokens; ++m) {
+    const int e = lane + 32 * m;
+    pv[m] = e < nslots ? a.inv_perm[t0 * k + e] : -1;
+  }
+#pragma unroll
+  for (int m = 0; m < kPgMaxTokens; ++m) {
+    const int e = lane + 32 * m;
+    base[m] = 0;
+    if (pv[m] >= 0 && (pv[m] & 1023) < El) {
+      const int64_t tile = (t0 + e / k) >> a.rt_shift;
+      base[m] = a.tile_counts[static_cast<int64_t>(pv[m] & 1023) * a.num_tiles + tile];
+    }
+  }
+
   // expert offsets: exclusive scan of the block-padded totals; lane l owns a contiguous run
   {
     const int per = (El + 31) >> 5;
@@ -394,30 +433,25 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     __syncwarp();
   }
 
-  const int nslots = n * k;  // <= kPgMaxTokens * 32
   int32_t dst[kPgMaxTokens];
 #pragma unroll
   for (int m = 0; m < kPgMaxTokens; ++m) {
     const int e = lane + 32 * m;
     int r = -1;
-    if (e < nslots) {
+    const int v = pv[m];
+    // a parked value names a local expert; anything else (buffers shared with a concurrent call)
+    // is flagged and skipped, never used as an index
+    if (v >= 0 && (v & 1023) >= El) {
+      moe::record_status(a.status, MOE_ERR_BAD_ROW);
+    } else if (v >= 0) {
       const int64_t s = t0 * k + e;
-      const int v = a.inv_perm[s];  // (rank in the tile) << 10 | local expert, or -1
-      // a parked value names a local expert; anything else (buffers shared with a concurrent call)
-      // is flagged and skipped, never used as an index
-      if (v >= 0 && (v & 1023) >= El) {
+      r = s_off[v & 1023] + base[m] + (v >> 10);
+      if (r < 0 || static_cast<int64_t>(r) >= a.C) {  // cannot happen for consistent inputs
         moe::record_status(a.status, MOE_ERR_BAD_ROW);
-      } else if (v >= 0) {
-        const int le = v & 1023;
-        const int64_t tile = (t0 + e / k) >> a.rt_shift;
-        r = s_off[le] + a.tile_counts[static_cast<int64_t>(le) * a.num_tiles + tile] + (v >> 10);
-        if (r < 0 || static_cast<int64_t>(r) >= a.C) {  // cannot happen for consistent inputs
-          moe::record_status(a.status, MOE_ERR_BAD_ROW);
-          r = -1;
-        } else {
-          a.sorted_ids[r] = static_cast<int32_t>(s);
-          a.inv_perm[s] = r;
-        }
+        r = -1;
+      } else {
+        a.sorted_ids[r] = static_cast<int32_t>(s);
+        a.inv_perm[s] = r;
       }
     }
     dst[m] = r;
