@@ -65,6 +65,8 @@ CASES = [
     ("lanes_fp32_E12_k3_one_local", 1030, 12, 3, torch.float32, True, "one_local", 1, 2, 16),
     ("lanes_bf16_bad_map_values", 1200, 64, 4, torch.bfloat16, True, "bad", 16, 16, 64),
     ("lanes_fp32_E48_k6_ties", 2077, 48, 6, torch.float32, False, None, 48, 32, 48),
+    ("lanes_bf16_E64_k8_ties", 2100, 64, 8, torch.bfloat16, True, None, 64, 64, 64),
+    ("lanes_bf16_E56_k7_strided_map", 1111, 56, 7, torch.bfloat16, False, "strided", 14, 16, 32),
 ]
 
 

@@ -57,6 +57,8 @@ TOPK_CASES = [
     (2048, 48, 6, torch.float32, True, 2.0, True),
     (1025, 8, 8, torch.bfloat16, True, 1.0, False),        # k == E
     (1100, 60, 7, torch.float32, False, 8.0, False),       # wide logits: tiny weights
+    (1500, 64, 8, torch.bfloat16, False, 1.0, True),       # bf16 keys, tie-heavy, full-row denominator
+    (2049, 56, 5, torch.bfloat16, True, 1.0, True),        # ragged last tile, ties
 ]
 
 

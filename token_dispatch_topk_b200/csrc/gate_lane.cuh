@@ -9,9 +9,10 @@
 // gate_row.cuh spends a warp on each row: k rounds of warp-wide reductions, a few hundred
 // instructions per row, which makes gating of many short rows (say E = 60 experts, T = 16K tokens)
 // bound by instruction issue.  Here a CTA stages 32 rows in shared memory and G lanes (up to 4)
-// scan each row once, inserting every logit into a register-resident list of the K largest (about
-// 5 * K instructions per logit); the G lists are merged with two shuffle rounds.  Several times
-// fewer instructions per row than the warp-per-row kernel.
+// scan each row once, inserting every logit into a register-resident list of the K largest (2 * K
+// instructions per bf16 logit, as unique 32-bit keys; about 5 * K per fp32 logit, as value and
+// index); the G lists are merged with two shuffle rounds.  Several times fewer instructions per
+// row than the warp-per-row kernel.
 //
 // Order: logits arrive in ascending expert order and a logit moves ahead only of kept logits it
 // strictly exceeds, so among equal logits the lower index stays ahead (+0 and -0 compare equal).
@@ -26,13 +27,15 @@
 
 namespace moe_gate {
 
-constexpr int kLaneGateMaxK = 8;      // K is a template parameter: 1..8
-constexpr int kLaneGateMaxE = 64;     // logits one thread scans
+constexpr int kLaneGateMaxK = 8;            // K is a template parameter: 1..8
+constexpr int kLaneGateMaxE = 64;           // at most 16 chunks a row: 4 lanes x 4 chunks
 constexpr int64_t kLaneGateMinRows = 1024;  // below this, the warp-per-row kernels have lower latency
 
-// Whether a batch of rows takes the one-thread-per-row gating (the same rule for every entry point,
-// so that moe_topk_softmax and moe_route_dispatch choose the same arithmetic for the same batch).
-// Rows must be whole 16-byte chunks and the logits 16-byte aligned.
+// Whether a batch of rows takes the lane gating (the same rule for every entry point, so that
+// moe_topk_softmax and moe_route_dispatch choose the same arithmetic for the same batch).
+// Rows must be whole 16-byte chunks and the logits 16-byte aligned.  (bf16 rows of up to 128
+// experts would fit the lane kernels too; measured in back-to-back steps of the 4096 x 128
+// prefill batch they were slower than one warp per row, so the bound is 64 experts.)
 inline bool lane_gating_fits(int64_t T, int E, int k, int elem_bytes, const void* logits) {
   return T >= kLaneGateMinRows && k <= kLaneGateMaxK && E <= kLaneGateMaxE && (E * elem_bytes) % 16 == 0 &&
          (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
@@ -99,6 +102,46 @@ struct LaneTopK {
   }
 };
 
+// bf16 logits: the ordered 16-bit value above, 0xFFFF - expert below, so the keys of a row are
+// unique and their order is the selection order (0 is below every key of a finite logit).  The K
+// largest keys are kept sorted descending: a key bubbles down the list with one max and one min
+// per entry.  Keys being unique, the list holds the K largest keys whatever order they arrive in.
+template <int K>
+struct LaneTopKey {
+  uint32_t v[K];
+
+  __device__ __forceinline__ void init() {
+#pragma unroll
+    for (int p = 0; p < K; ++p) v[p] = 0u;
+  }
+
+  __device__ __forceinline__ void insert(uint32_t x) {
+#pragma unroll
+    for (int p = 0; p < K; ++p) {
+      const uint32_t hi = v[p] > x ? v[p] : x;
+      x = v[p] > x ? x : v[p];
+      v[p] = hi;
+    }
+  }
+};
+
+__device__ __forceinline__ uint32_t bf16_key(uint32_t bits16, int e) {
+  return (ordered16(bits16) << 16) | (0xffffu - static_cast<uint32_t>(e));
+}
+
+template <int K>
+__device__ __forceinline__ void lane_insert_chunk_keys(LaneTopKey<K>& t, const uint4 q, int j) {
+  const int i = 8 * j;
+  t.insert(bf16_key(q.x & 0xffffu, i));
+  t.insert(bf16_key(q.x >> 16, i + 1));
+  t.insert(bf16_key(q.y & 0xffffu, i + 2));
+  t.insert(bf16_key(q.y >> 16, i + 3));
+  t.insert(bf16_key(q.z & 0xffffu, i + 4));
+  t.insert(bf16_key(q.z >> 16, i + 5));
+  t.insert(bf16_key(q.w & 0xffffu, i + 6));
+  t.insert(bf16_key(q.w >> 16, i + 7));
+}
+
 // Insert the logits of one 16-byte chunk (chunk j of the row) in ascending expert order.
 template <typename TIn, int K>
 __device__ __forceinline__ void lane_insert_chunk(LaneTopK<K>& t, const uint4 q, int j) {
@@ -125,52 +168,75 @@ __device__ __forceinline__ void lane_insert_chunk(LaneTopK<K>& t, const uint4 q,
 // [g * cpr / G, (g + 1) * cpr / G) (one to four chunks each, read into registers once).  More lanes per row put more warps in flight for the same instructions
 // per row: the scan is a chain of dependent inserts, and one lane per row leaves too few warps.
 __host__ __device__ inline int lane_gate_lanes(int cpr) { return cpr >= 4 ? 4 : (cpr >= 2 ? 2 : 1); }
-constexpr int kLaneMaxChunks = 4;  // chunks one lane holds: ceil(cpr / G) <= 4 for cpr <= 16
+constexpr int kLaneMaxChunks = 4;  // chunks one lane holds: cpr / G rounded up, <= 4 for cpr <= 16
 
 // Gate one staged row (cpr 16-byte chunks of TIn logits; E = cpr * 16 / sizeof(TIn)) with the G
 // lanes g = lane % G of a row group (consecutive lanes; every lane of the warp calls this).
 // `mode`: kGateRenorm, kGateSigmoid.  Every lane of the group returns the K experts in selection
 // order and their weights.
-// Merge: after each lane's scan, lists are merged pairwise (shuffle distance 1, then 2): the list of
-// the lower chunks is the base and the other is inserted into it in its own order.  Every expert of
-// the inserted list has a higher index than every expert of the base, and among equal logits the
-// inserted list keeps the lower index ahead, so the merged list is the one a single scan in expert
-// order would give.
+// Merge, after each lane's scan, pairwise over shuffle distance 1, then 2:
+//   bf16: the keys are unique, so inserting the partner's K keys gives the K largest of both.
+//   fp32: the list of the lower chunks is the base and the other is inserted into it in its own
+//   order.  Every expert of the inserted list has a higher index than every expert of the base,
+//   and among equal logits the inserted list keeps the lower index ahead, so the merged list is
+//   the one a single scan in expert order would give.
 template <typename TIn, int K, int G>
 __device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, int cpr, int mode, int g,
                                               float (&w)[K], int (&ids)[K]) {
-  LaneTopK<K> t;
-  t.init();
   const int j0 = (g * cpr) / G, j1 = ((g + 1) * cpr) / G;
   uint4 q[kLaneMaxChunks];
 #pragma unroll
   for (int u = 0; u < kLaneMaxChunks; ++u) {
     if (j0 + u < j1) q[u] = srow[j0 + u];
   }
+  LaneTopK<K> t;
+  if constexpr (sizeof(TIn) == 2) {
+    LaneTopKey<K> kt;
+    kt.init();
 #pragma unroll
-  for (int u = 0; u < kLaneMaxChunks; ++u) {
-    if (j0 + u < j1) lane_insert_chunk<TIn, K>(t, q[u], j0 + u);
-  }
-#pragma unroll
-  for (int d = 1; d < G; d <<= 1) {
-    LaneTopK<K> o;
-#pragma unroll
-    for (int q = 0; q < K; ++q) {
-      o.v[q] = __shfl_xor_sync(0xffffffffu, t.v[q], d);
-      o.e[q] = __shfl_xor_sync(0xffffffffu, t.e[q], d);
-    }
-    const bool upper = (g & d) != 0;  // this lane's chunks come after the partner's
-    LaneTopK<K> base, add;
-#pragma unroll
-    for (int q = 0; q < K; ++q) {
-      base.v[q] = upper ? o.v[q] : t.v[q];
-      base.e[q] = upper ? o.e[q] : t.e[q];
-      add.v[q] = upper ? t.v[q] : o.v[q];
-      add.e[q] = upper ? t.e[q] : o.e[q];
+    for (int u = 0; u < kLaneMaxChunks; ++u) {
+      if (j0 + u < j1) lane_insert_chunk_keys<K>(kt, q[u], j0 + u);
     }
 #pragma unroll
-    for (int q = 0; q < K; ++q) base.insert(add.v[q], add.e[q]);
-    t = base;
+    for (int d = 1; d < G; d <<= 1) {
+      uint32_t o[K];
+#pragma unroll
+      for (int r = 0; r < K; ++r) o[r] = __shfl_xor_sync(0xffffffffu, kt.v[r], d);
+#pragma unroll
+      for (int r = 0; r < K; ++r) kt.insert(o[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < K; ++r) {
+      t.v[r] = ordered16_to_float(kt.v[r] >> 16);
+      t.e[r] = static_cast<int>(0xffffu - (kt.v[r] & 0xffffu));
+    }
+  } else {
+    t.init();
+#pragma unroll
+    for (int u = 0; u < kLaneMaxChunks; ++u) {
+      if (j0 + u < j1) lane_insert_chunk<TIn, K>(t, q[u], j0 + u);
+    }
+#pragma unroll
+    for (int d = 1; d < G; d <<= 1) {
+      LaneTopK<K> o;
+#pragma unroll
+      for (int r = 0; r < K; ++r) {
+        o.v[r] = __shfl_xor_sync(0xffffffffu, t.v[r], d);
+        o.e[r] = __shfl_xor_sync(0xffffffffu, t.e[r], d);
+      }
+      const bool upper = (g & d) != 0;  // this lane's chunks come after the partner's
+      LaneTopK<K> base, add;
+#pragma unroll
+      for (int r = 0; r < K; ++r) {
+        base.v[r] = upper ? o.v[r] : t.v[r];
+        base.e[r] = upper ? o.e[r] : t.e[r];
+        add.v[r] = upper ? t.v[r] : o.v[r];
+        add.e[r] = upper ? t.e[r] : o.e[r];
+      }
+#pragma unroll
+      for (int r = 0; r < K; ++r) base.insert(add.v[r], add.e[r]);
+      t = base;
+    }
   }
   const bool renormalize = (mode & kGateRenorm) != 0;
   const bool sigmoid = (mode & kGateSigmoid) != 0;
@@ -178,9 +244,9 @@ __device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, in
   float p[K];
   float den = 0.f;
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
-    p[q] = sigmoid ? 1.f / (1.f + expf(-t.v[q])) : expf(t.v[q] - m);
-    den += p[q];
+  for (int r = 0; r < K; ++r) {
+    p[r] = sigmoid ? 1.f / (1.f + expf(-t.v[r])) : expf(t.v[r] - m);
+    den += p[r];
   }
   if (!renormalize && !sigmoid) {  // full-row denominator: each lane sums its chunks, then the group
     float z[4] = {0.f, 0.f, 0.f, 0.f};  // four partial sums (short dependency chains)
@@ -205,13 +271,13 @@ __device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, in
     for (int d = 1; d < G; d <<= 1) den += __shfl_xor_sync(0xffffffffu, den, d);
   }
 #pragma unroll
-  for (int q = 0; q < K; ++q) {
+  for (int r = 0; r < K; ++r) {
     if (sigmoid) {
-      w[q] = renormalize ? (den > 0.f ? p[q] / den : 1.f / static_cast<float>(K)) : p[q];
+      w[r] = renormalize ? (den > 0.f ? p[r] / den : 1.f / static_cast<float>(K)) : p[r];
     } else {
-      w[q] = p[q] / den;
+      w[r] = p[r] / den;
     }
-    ids[q] = t.e[q];
+    ids[r] = t.e[r];
   }
 }
 

@@ -204,7 +204,8 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
 // computes the stable ranks inside the tile (the slots in order, 32 at a time: rank = the expert's
 // count so far + earlier peers in the chunk), parked in inv_perm as in gate_count_kernel, and the
 // tile's per-expert counts.
-// Shared memory: staged rows [kRowsPerTile * stride chunks] | hist [E_local] | s_le [kRowsPerTile * K].
+// Shared memory: staged rows [kRowsPerTile * stride chunks] | hist [E_local] | peer masks [E_local] |
+// s_le [kRowsPerTile * K].
 template <typename TIn, int K, int G>
 __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a, int cpr) {
   constexpr int NT = 32 * G;
@@ -212,12 +213,16 @@ __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a
   const int El = a.E_local;
   const int stride = moe_gate::lane_tile_stride(cpr);
   int* hist = reinterpret_cast<int*>(s_rows + kRowsPerTile * stride);
-  int* s_le = hist + El;
+  unsigned* masks = reinterpret_cast<unsigned*>(hist + El);
+  int* s_le = reinterpret_cast<int*>(masks + El);
   const int tid = threadIdx.x, lane = tid & 31;
   const int tile = blockIdx.x;
   const int64_t row0 = static_cast<int64_t>(tile) * kRowsPerTile;
   const int rows = static_cast<int>((a.T - row0) < kRowsPerTile ? (a.T - row0) : kRowsPerTile);  // >= 1
-  for (int e = tid; e < El; e += NT) hist[e] = 0;
+  for (int e = tid; e < El; e += NT) {
+    hist[e] = 0;
+    masks[e] = 0u;
+  }
   moe::pdl_wait();  // the logits may come from the previous kernel
   moe::pdl_launch_dependents();
   moe_gate::lane_tile_load(static_cast<const uint4*>(a.logits) + row0 * cpr, rows, cpr, stride, s_rows, tid, NT);
@@ -244,7 +249,7 @@ __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a
   for (int c = 0; c < nslots; c += 32) {
     const int i = c + lane;
     const int le = i < nslots ? s_le[i] : -1;
-    const unsigned peers = __match_any_sync(0xffffffffu, le);
+    const unsigned peers = peers_of(masks, le, lane);
     if (le >= 0) {
       // parked until place_gather_kernel: (rank in the tile) << 10 | local expert
       a.inv_perm[row0 * K + i] = ((hist[le] + __popc(peers & moe::lanemask_lt())) << 10) | le;
@@ -918,7 +923,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     LanesKernel lk = dtype == MOE_DTYPE_BF16 ? lanes_kernel_for<__nv_bfloat16>(k, G) : lanes_kernel_for<float>(k, G);
     if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
     const size_t smem1 = static_cast<size_t>(kRowsPerTile) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4) +
-                         (static_cast<size_t>(E_local) + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
+                         (2 * static_cast<size_t>(E_local) + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
     if (moe_host::launch_pdl(lk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(32 * G), smem1, st, a, cpr) != MOE_OK)
       return MOE_ERR_CUDA;
   } else {
