@@ -269,10 +269,12 @@ inline moe_status_t launch_status() {
   return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
-// Every kernel of the library asks for the same split of each SM's L1 / shared memory (the most
-// shared memory).  An SM changes its split only when it is idle, so kernels with different splits
-// chained by programmatic dependent launch would leave SMs unable to take the next kernel's CTAs
-// until every CTA of the previous ones has left them.
+// The kernels of the large-batch chains (gating with the tile counts, tile scan, placement and
+// gather, the TMA gather and combine, align) ask for the same split of each SM's L1 / shared
+// memory: the most shared memory, which the staging kernels need.  An SM changes its split only
+// when it is idle, so kernels with different splits chained by programmatic dependent launch would
+// leave SMs unable to take the next kernel's CTAs until every CTA of the previous ones has left
+// them.  The decode-sized kernels keep the default split, the one of the kernels around them.
 inline cudaError_t prefer_max_shared(const void* kernel) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
                               static_cast<int>(cudaSharedmemCarveoutMaxShared));
@@ -283,7 +285,6 @@ inline cudaError_t prefer_max_shared(const void* kernel) {
 template <typename... KArgs, typename... Args>
 inline moe_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
                                Args&&... args) {
-  if (prefer_max_shared(reinterpret_cast<const void*>(kernel)) != cudaSuccess) return MOE_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
@@ -295,6 +296,14 @@ inline moe_status_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, 
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...) == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// launch_pdl for the kernels of the large-batch chains (the most shared memory, see above).
+template <typename... KArgs, typename... Args>
+inline moe_status_t launch_pdl_max_shared(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                                          cudaStream_t st, Args&&... args) {
+  if (prefer_max_shared(reinterpret_cast<const void*>(kernel)) != cudaSuccess) return MOE_ERR_CUDA;
+  return launch_pdl(kernel, grid, block, smem, st, std::forward<Args>(args)...);
 }
 
 }  // namespace moe_host

@@ -485,7 +485,7 @@ extern "C" moe_status_t moe_gather(const void* hidden, int64_t T, int32_t H, int
             cudaSuccess)
       return MOE_ERR_CUDA;
     const int ready = (flags & MOE_GATHER_HIDDEN_READY) ? 1 : 0;
-    if (moe_host::launch_pdl(gather_tma_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32), smem, st,
+    if (moe_host::launch_pdl_max_shared(gather_tma_kernel, dim3(static_cast<unsigned>(blocks)), dim3(32), smem, st,
                              static_cast<const uint8_t*>(hidden), T, row_bytes, k, tpc, inv_perm, capacity,
                              static_cast<uint8_t*>(permuted), device_status, ready) != MOE_OK)
       return MOE_ERR_CUDA;
@@ -568,6 +568,6 @@ extern "C" moe_status_t moe_combine(const void* expert_out, const float* topk_we
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  return moe_host::launch_pdl(kern, dim3(static_cast<unsigned>(grid)), dim3((1 + kCombineConsumerWarps) * 32), smem,
+  return moe_host::launch_pdl_max_shared(kern, dim3(static_cast<unsigned>(grid)), dim3((1 + kCombineConsumerWarps) * 32), smem,
                               static_cast<cudaStream_t>(stream), a);
 }

@@ -924,7 +924,8 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
     const size_t smem1 = static_cast<size_t>(kRowsPerTile) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4) +
                          (2 * static_cast<size_t>(E_local) + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
-    if (moe_host::launch_pdl(lk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(32 * G), smem1, st, a, cpr) != MOE_OK)
+    if (moe_host::launch_pdl_max_shared(lk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(32 * G), smem1, st, a, cpr) !=
+        MOE_OK)
       return MOE_ERR_CUDA;
   } else {
     // the gating geometry does not matter when the routes are given (no row is gated)
@@ -937,10 +938,10 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
         cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem1)) != cudaSuccess)
       return MOE_ERR_CUDA;
-    if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
+    if (moe_host::launch_pdl_max_shared(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
       return MOE_ERR_CUDA;
   }
-  if (moe_host::launch_pdl(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
+  if (moe_host::launch_pdl_max_shared(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
       MOE_OK)
     return MOE_ERR_CUDA;
 
@@ -959,7 +960,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
       cudaFuncSetAttribute(place_gather_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem2)) !=
           cudaSuccess)
     return MOE_ERR_CUDA;
-  return moe_host::launch_pdl(place_gather_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st, a,
+  return moe_host::launch_pdl_max_shared(place_gather_kernel<true>, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st, a,
                               static_cast<const uint8_t*>(hidden), row_bytes, tpc, static_cast<uint8_t*>(permuted));
 }
 
@@ -1008,9 +1009,9 @@ moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32
       cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem1)) != cudaSuccess)
     return MOE_ERR_CUDA;
-  if (moe_host::launch_pdl(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
+  if (moe_host::launch_pdl_max_shared(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
     return MOE_ERR_CUDA;
-  if (moe_host::launch_pdl(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
+  if (moe_host::launch_pdl_max_shared(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
       MOE_OK)
     return MOE_ERR_CUDA;
   // placement only: up to kPgMaxTokens tokens per one-warp CTA, the CTAs filling whole waves
@@ -1021,6 +1022,6 @@ moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32
   if (blocks < 1) blocks = 1;
   if (blocks > 0x7fffffff) return MOE_ERR_INVALID_ARG;
   const size_t smem2 = static_cast<size_t>(E_local + 1) * sizeof(int);
-  return moe_host::launch_pdl(place_gather_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st,
+  return moe_host::launch_pdl_max_shared(place_gather_kernel<false>, dim3(static_cast<unsigned>(blocks)), dim3(32), smem2, st,
                               a, static_cast<const uint8_t*>(nullptr), 0u, tpc, static_cast<uint8_t*>(nullptr));
 }

@@ -226,8 +226,6 @@ using TopkKernel = void (*)(const void*, int64_t, int, int, int, int, float*, in
 // Launch a gating kernel (any instance, arguments as a void* array) with programmatic stream
 // serialisation.
 cudaError_t launch_topk(TopkKernel kern, int64_t grid, int block, size_t smem, cudaStream_t st, void** args) {
-  const cudaError_t e = moe_host::prefer_max_shared(reinterpret_cast<const void*>(kern));
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(block);
@@ -373,7 +371,7 @@ extern "C" moe_status_t moe_topk_softmax(const void* logits, moe_dtype_t dtype, 
     const int64_t grid = (T + rows_per_cta - 1) / rows_per_cta;
     if (grid > 0x7fffffff) return MOE_ERR_INVALID_ARG;
     const size_t smem = static_cast<size_t>(rows_per_cta) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4);
-    return moe_host::launch_pdl(lk, dim3(static_cast<unsigned>(grid)), dim3(kLaneThreads), smem,
+    return moe_host::launch_pdl_max_shared(lk, dim3(static_cast<unsigned>(grid)), dim3(kLaneThreads), smem,
                                 static_cast<cudaStream_t>(stream), logits, T, cpr, renorm_flag, topk_weights,
                                 topk_ids);
   }
