@@ -136,12 +136,6 @@ __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint3
                : "memory");
 }
 
-// Bring `bytes` of global memory into L2 ahead of use (no shared memory, nothing to wait for);
-// address and size 16-byte aligned.
-__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
-
 // shared -> global bulk copy, tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
   asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src_smem)),

@@ -11,7 +11,7 @@
 //   gather_tma_kernel:  each hidden row is bulk-loaded once and bulk-stored to every
 //                       local destination row of its token.
 //   combine_tma_kernel: a producer warp bulk-loads the local slot rows of each (token,
-//                       column chunk) into a 3-stage ring; consumer warps run the fp32
+//                       column chunk) into a ring of stages; consumer warps run the fp32
 //                       fused multiply-adds in ascending slot order from +0 and store one
 //                       bf16 round-to-nearest-even result.
 // The register-staged gather_kernel (one warp per token or row segment, lane j < k holding
