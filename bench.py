@@ -50,6 +50,9 @@ KERNEL_SOURCES = {
     "combine_tma_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "combine_small_kernel": "token_dispatch_topk_b200/csrc/gather_combine.cu",
     "gate_count_kernel+tile_scan_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "gate_count_lanes_kernel+tile_scan_kernel+place_gather_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "gate_count_kernel+tile_scan_kernel+place_gather_kernel<false>": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "topk_lane_kernel": "token_dispatch_topk_b200/csrc/topk_softmax.cu",
     "align_count_kernel+align_place_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
     "route_small_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
 }
@@ -418,9 +421,19 @@ def main():
     st_iters = args.stage_steps or min(args.steps, 500)
 
     stage_kernel = dict(STAGE_KERNEL)
+    # the kernels each entry point launches for this workload (the library's selection rules)
+    elem = 2 if wl.logits_dtype == "bf16" else 4
+    lanes = wl.T >= 1024 and wl.k <= 8 and wl.E <= 64 and (wl.E * elem) % 16 == 0
     if r.small_batch:
         stage_kernel["dispatch"] = "route_small_kernel"
-    if wl.T * wl.k > 65536 or wl.experts_local > 512:  # beyond one cluster: the two-kernel align
+    elif lanes:
+        stage_kernel["dispatch"] = "gate_count_lanes_kernel+tile_scan_kernel+place_gather_kernel"
+    if lanes:
+        stage_kernel["topk"] = "topk_lane_kernel"
+    P = wl.T * wl.k
+    if 4096 < P <= 65536:  # the fused path's tile kernels, placement only
+        stage_kernel["align"] = "gate_count_kernel+tile_scan_kernel+place_gather_kernel<false>"
+    elif P > 65536 or wl.experts_local > 512:  # beyond one cluster: the two-kernel align
         stage_kernel["align"] = "align_count_kernel+align_place_kernel"
     sms = torch.cuda.get_device_properties(dev).multi_processor_count
     if wl.T * (-(-wl.H * 2 // 4096)) < sms:  # fewer 4 KB row chunks than SMs: the small-batch combine

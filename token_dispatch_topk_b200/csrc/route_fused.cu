@@ -119,6 +119,55 @@ __host__ __device__ inline size_t gc_smem_ints(int rows_per_tile, int k, int E_l
   return static_cast<size_t>(rows_per_tile) * k + 2 * static_cast<size_t>(kGcWarps) * E_local;
 }
 
+// Stable ranks inside a tile, by the CTA's `nwarps` warps (all threads call this, after s_le is
+// complete): warp w owns a contiguous run of the tile's 32-slot chunks and counts it into its row of
+// `whist` ([nwarps][E_local], zero on entry); the rows are scanned across warps per expert (the
+// tile's counts go to the workspace, expert-major); each slot's rank = earlier warps' count of its
+// expert + the warp's running count + earlier peers in its chunk.  The rank is parked in inv_perm
+// as (rank << 10) | local expert for place_gather_kernel; remote slots get -1.  `masks`
+// ([nwarps][E_local]) is zero on entry and left zero.
+__device__ __forceinline__ void rank_tile_slots(const DispatchArgs& a, const int* s_le, int nslots, int64_t row0,
+                                                int tile, int* whist, unsigned* masks, int nwarps) {
+  const int El = a.E_local, k = a.k;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nthreads = nwarps * 32;
+  const int nch = (nslots + 31) / 32;
+  const int cpw = (nch + nwarps - 1) / nwarps;
+  const int c0 = warp * cpw;
+  const int c1 = (c0 + cpw < nch) ? c0 + cpw : nch;
+  int* my_hist = whist + warp * El;
+  unsigned* my_masks = masks + warp * El;
+  for (int c = c0; c < c1; ++c) {
+    const int i = c * 32 + lane;
+    const int le = i < nslots ? s_le[i] : -1;
+    if (le >= 0) atomicAdd(&my_hist[le], 1);
+  }
+  __syncthreads();
+  for (int e = tid; e < El; e += nthreads) {
+    int run = 0;
+    for (int w = 0; w < nwarps; ++w) {
+      const int c = whist[w * El + e];
+      whist[w * El + e] = run;
+      run += c;
+    }
+    a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = run;
+  }
+  __syncthreads();
+  for (int c = c0; c < c1; ++c) {
+    const int i = c * 32 + lane;
+    const int le = i < nslots ? s_le[i] : -1;
+    const unsigned peers = peers_of(my_masks, le, lane);
+    if (le >= 0) {
+      a.inv_perm[row0 * k + i] = ((my_hist[le] + __popc(peers & moe::lanemask_lt())) << 10) | le;
+    } else if (i < nslots) {
+      a.inv_perm[row0 * k + i] = -1;
+    }
+    __syncwarp();
+    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
+    __syncwarp();
+  }
+}
+
 template <typename TIn, int VEC, int CPL>
 __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) {
   extern __shared__ int smem[];
@@ -159,68 +208,29 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   __syncthreads();
 
   // B. stable ranks inside the tile
-  const int nslots = rows * k;
-  const int nch = (nslots + 31) / 32;
-  const int cpw = (nch + kGcWarps - 1) / kGcWarps;
-  const int c0 = warp * cpw;
-  const int c1 = (c0 + cpw < nch) ? c0 + cpw : nch;
-  int* my_hist = whist + warp * El;
-  unsigned* my_masks = masks + warp * El;
-  for (int c = c0; c < c1; ++c) {
-    const int i = c * 32 + lane;
-    const int le = i < nslots ? s_le[i] : -1;
-    if (le >= 0) atomicAdd(&my_hist[le], 1);
-  }
-  __syncthreads();
-  for (int e = tid; e < El; e += kGcThreads) {
-    int run = 0;
-    for (int w = 0; w < kGcWarps; ++w) {
-      const int c = whist[w * El + e];
-      whist[w * El + e] = run;
-      run += c;
-    }
-    a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = run;
-  }
-  __syncthreads();
-  for (int c = c0; c < c1; ++c) {
-    const int i = c * 32 + lane;
-    const int le = i < nslots ? s_le[i] : -1;
-    const unsigned peers = peers_of(my_masks, le, lane);
-    if (le >= 0) {
-      // parked until place_gather_kernel: (rank in the tile) << 10 | local expert
-      a.inv_perm[row0 * k + i] = ((my_hist[le] + __popc(peers & moe::lanemask_lt())) << 10) | le;
-    } else if (i < nslots) {
-      a.inv_perm[row0 * k + i] = -1;
-    }
-    __syncwarp();
-    if (le >= 0 && lane == __ffs(peers) - 1) my_hist[le] += __popc(peers);
-    __syncwarp();
-  }
+  rank_tile_slots(a, s_le, rows * k, row0, tile, whist, masks, kGcWarps);
 }
 
-
 // One CTA of G warps per tile of kRowsPerTile tokens, G lanes per row: the tile's logits are staged
-// in shared memory and each group of G lanes gates one row (moe_gate::lane_gate_row); then warp 0
-// computes the stable ranks inside the tile (the slots in order, 32 at a time: rank = the expert's
-// count so far + earlier peers in the chunk), parked in inv_perm as in gate_count_kernel, and the
-// tile's per-expert counts.
-// Shared memory: staged rows [kRowsPerTile * stride chunks] | hist [E_local] | peer masks [E_local] |
-// s_le [kRowsPerTile * K].
+// in shared memory and each group of G lanes gates one row (moe_gate::lane_gate_row); then the G
+// warps rank the tile's slots and write its per-expert counts (rank_tile_slots, as gate_count_kernel).
+// Shared memory: staged rows [kRowsPerTile * stride chunks] | whist [G][E_local] | peer masks
+// [G][E_local] | s_le [kRowsPerTile * K].
 template <typename TIn, int K, int G>
 __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a, int cpr) {
   constexpr int NT = 32 * G;
   extern __shared__ __align__(16) uint4 s_rows[];
   const int El = a.E_local;
   const int stride = moe_gate::lane_tile_stride(cpr);
-  int* hist = reinterpret_cast<int*>(s_rows + kRowsPerTile * stride);
-  unsigned* masks = reinterpret_cast<unsigned*>(hist + El);
-  int* s_le = reinterpret_cast<int*>(masks + El);
-  const int tid = threadIdx.x, lane = tid & 31;
+  int* whist = reinterpret_cast<int*>(s_rows + kRowsPerTile * stride);
+  unsigned* masks = reinterpret_cast<unsigned*>(whist + G * El);
+  int* s_le = reinterpret_cast<int*>(masks + G * El);
+  const int tid = threadIdx.x;
   const int tile = blockIdx.x;
   const int64_t row0 = static_cast<int64_t>(tile) * kRowsPerTile;
   const int rows = static_cast<int>((a.T - row0) < kRowsPerTile ? (a.T - row0) : kRowsPerTile);  // >= 1
-  for (int e = tid; e < El; e += NT) {
-    hist[e] = 0;
+  for (int e = tid; e < G * El; e += NT) {
+    whist[e] = 0;
     masks[e] = 0u;
   }
   moe::pdl_wait();  // the logits may come from the previous kernel
@@ -244,23 +254,7 @@ __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a
     }
   }
   __syncthreads();
-  if (tid >= 32) return;
-  const int nslots = rows * K;
-  for (int c = 0; c < nslots; c += 32) {
-    const int i = c + lane;
-    const int le = i < nslots ? s_le[i] : -1;
-    const unsigned peers = peers_of(masks, le, lane);
-    if (le >= 0) {
-      // parked until place_gather_kernel: (rank in the tile) << 10 | local expert
-      a.inv_perm[row0 * K + i] = ((hist[le] + __popc(peers & moe::lanemask_lt())) << 10) | le;
-    } else if (i < nslots) {
-      a.inv_perm[row0 * K + i] = -1;
-    }
-    __syncwarp();
-    if (le >= 0 && lane == __ffs(peers) - 1) hist[le] += __popc(peers);
-    __syncwarp();
-  }
-  for (int e = lane; e < El; e += 32) a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = hist[e];
+  rank_tile_slots(a, s_le, rows * K, row0, tile, whist, masks, G);
 }
 
 using LanesKernel = void (*)(DispatchArgs, int);
@@ -923,7 +917,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     LanesKernel lk = dtype == MOE_DTYPE_BF16 ? lanes_kernel_for<__nv_bfloat16>(k, G) : lanes_kernel_for<float>(k, G);
     if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
     const size_t smem1 = static_cast<size_t>(kRowsPerTile) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4) +
-                         (2 * static_cast<size_t>(E_local) + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
+                         (2 * static_cast<size_t>(G) * E_local + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
     if (moe_host::launch_pdl_max_shared(lk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(32 * G), smem1, st, a, cpr) !=
         MOE_OK)
       return MOE_ERR_CUDA;
