@@ -67,6 +67,8 @@ CASES = [
     ("lanes_fp32_E48_k6_ties", 2077, 48, 6, torch.float32, False, None, 48, 32, 48),
     ("lanes_bf16_E64_k8_ties", 2100, 64, 8, torch.bfloat16, True, None, 64, 64, 64),
     ("lanes_bf16_E56_k7_strided_map", 1111, 56, 7, torch.bfloat16, False, "strided", 14, 16, 32),
+    ("lanes_wide_bf16_E256_k8_strided_map", 16500, 256, 8, torch.bfloat16, True, "strided", 64, 128, 16),
+    ("lanes_wide_bf16_E192_k5_ties", 16401, 192, 5, torch.bfloat16, False, None, 192, 32, 8),
 ]
 
 
@@ -130,10 +132,11 @@ def test_dispatch_parity(name, T, E, k, dtype, renorm, kind, E_local, bs, H):
         assert status == (tdt.MOE_ERR_BAD_EXPERT_ID if kind == "bad" else tdt.MOE_OK), (name, status)
 
 
-@pytest.mark.parametrize("workload", ["qwen3moe_prefill_T4096_E128_k8", "nonpow2_T16384_E60_k4"])
+@pytest.mark.parametrize("workload", ["qwen3moe_prefill_T4096_E128_k8", "nonpow2_T16384_E60_k4",
+                                      "zipf_prefill_T65536_E256_k8_H7168"])
 def test_dispatch_matches_stage_entry_points(workload):
     """The fused dispatch and the three stage calls it replaces give identical outputs (one warp per
-    row on the prefill workload, one thread per row on the non-power-of-2 one)."""
+    row on the prefill workload, lanes per row on the non-power-of-2 and skewed ones)."""
     dev = require_gpu()
     wl = I.WORKLOADS[workload]
     logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)

@@ -59,6 +59,8 @@ TOPK_CASES = [
     (1100, 60, 7, torch.float32, False, 8.0, False),       # wide logits: tiny weights
     (1500, 64, 8, torch.bfloat16, False, 1.0, True),       # bf16 keys, tie-heavy, full-row denominator
     (2049, 56, 5, torch.bfloat16, True, 1.0, True),        # ragged last tile, ties
+    (16400, 256, 8, torch.bfloat16, True, 1.0, True),      # wide bf16 rows, eight lanes per row, ties
+    (16500, 192, 6, torch.bfloat16, False, 1.0, False),    # wide bf16 rows, three chunks per lane
 ]
 
 
@@ -86,6 +88,7 @@ SIGMOID_CASES = [
     (300, 64, 8, torch.float32, False, 30.0, False),       # far tails: scores near 0 and 1
     (1500, 64, 8, torch.bfloat16, True, 1.0, True),        # one thread per row, tie-heavy
     (1100, 24, 3, torch.float32, False, 30.0, False),      # one thread per row, far tails
+    (16400, 256, 8, torch.bfloat16, True, 1.0, False),     # wide bf16 rows, eight lanes per row
 ]
 
 

@@ -8,10 +8,10 @@
 //
 // gate_row.cuh spends a warp on each row: k rounds of warp-wide reductions, a few hundred
 // instructions per row, which makes gating of many short rows (say E = 60 experts, T = 16K tokens)
-// bound by instruction issue.  Here a CTA stages 32 rows in shared memory and G lanes (up to 4)
+// bound by instruction issue.  Here a CTA stages 32 rows in shared memory and G lanes (up to 8)
 // scan each row once, inserting every logit into a register-resident list of the K largest (2 * K
 // instructions per bf16 logit, as unique 32-bit keys; about 5 * K per fp32 logit, as value and
-// index); the G lists are merged with two shuffle rounds.  Several times fewer instructions per
+// index); the G lists are merged with log2(G) shuffle rounds.  Several times fewer instructions per
 // row than the warp-per-row kernel.
 //
 // Order: logits arrive in ascending expert order and a logit moves ahead only of kept logits it
@@ -28,17 +28,22 @@
 namespace moe_gate {
 
 constexpr int kLaneGateMaxK = 8;            // K is a template parameter: 1..8
-constexpr int kLaneGateMaxE = 64;           // at most 16 chunks a row: 4 lanes x 4 chunks
+constexpr int kLaneGateMaxE = 64;           // rows of up to 64 logits: from 1024 rows on
 constexpr int64_t kLaneGateMinRows = 1024;  // below this, the warp-per-row kernels have lower latency
+constexpr int kLaneGateWideMaxE = 256;      // bf16 rows of up to 256 logits: from 16384 rows on
+constexpr int64_t kLaneGateWideMinRows = 16384;
 
 // Whether a batch of rows takes the lane gating (the same rule for every entry point, so that
 // moe_topk_softmax and moe_route_dispatch choose the same arithmetic for the same batch).
-// Rows must be whole 16-byte chunks and the logits 16-byte aligned.  (bf16 rows of up to 128
-// experts would fit the lane kernels too; measured in back-to-back steps of the 4096 x 128
-// prefill batch they were slower than one warp per row, so the bound is 64 experts.)
+// Rows must be whole 16-byte chunks and the logits 16-byte aligned.  Short rows take it from 1024
+// rows on.  Wider bf16 rows take it only for large batches, where gating is bound by instruction
+// issue: measured in back-to-back steps of the 4096 x 128 prefill batch, the lane kernel was
+// slower than one warp per row there (65.9 against 63.6 us a step).
 inline bool lane_gating_fits(int64_t T, int E, int k, int elem_bytes, const void* logits) {
-  return T >= kLaneGateMinRows && k <= kLaneGateMaxK && E <= kLaneGateMaxE && (E * elem_bytes) % 16 == 0 &&
-         (reinterpret_cast<uintptr_t>(logits) & 15u) == 0;
+  if (k > kLaneGateMaxK || (E * elem_bytes) % 16 != 0 || (reinterpret_cast<uintptr_t>(logits) & 15u) != 0)
+    return false;
+  if (E <= kLaneGateMaxE) return T >= kLaneGateMinRows;
+  return elem_bytes == 2 && E <= kLaneGateWideMaxE && T >= kLaneGateWideMinRows;
 }
 
 // Shared-memory layout of a staged tile: row r starts at chunk r * stride, stride = chunks per row
@@ -164,17 +169,20 @@ __device__ __forceinline__ void lane_insert_chunk(LaneTopK<K>& t, const uint4 q,
   }
 }
 
-// Lanes per row: G lanes share a row (G = 1, 2 or 4), lane g scanning chunks
-// [g * cpr / G, (g + 1) * cpr / G) (one to four chunks each, read into registers once).  More lanes per row put more warps in flight for the same instructions
-// per row: the scan is a chain of dependent inserts, and one lane per row leaves too few warps.
-__host__ __device__ inline int lane_gate_lanes(int cpr) { return cpr >= 4 ? 4 : (cpr >= 2 ? 2 : 1); }
-constexpr int kLaneMaxChunks = 4;  // chunks one lane holds: cpr / G rounded up, <= 4 for cpr <= 16
+// Lanes per row: G lanes share a row (G = 1, 2, 4, or 8 for rows of more than 16 chunks), lane g
+// scanning chunks [g * cpr / G, (g + 1) * cpr / G) (one to four chunks each, read into registers
+// once).  More lanes per row put more warps in flight for the same instructions per row: the scan
+// is a chain of dependent inserts, and one lane per row leaves too few warps.
+__host__ __device__ inline int lane_gate_lanes(int cpr) {
+  return cpr > 16 ? 8 : (cpr >= 4 ? 4 : (cpr >= 2 ? 2 : 1));
+}
+constexpr int kLaneMaxChunks = 4;  // chunks one lane holds: cpr / G rounded up, <= 4 for cpr <= 32
 
 // Gate one staged row (cpr 16-byte chunks of TIn logits; E = cpr * 16 / sizeof(TIn)) with the G
 // lanes g = lane % G of a row group (consecutive lanes; every lane of the warp calls this).
 // `mode`: kGateRenorm, kGateSigmoid.  Every lane of the group returns the K experts in selection
 // order and their weights.
-// Merge, after each lane's scan, pairwise over shuffle distance 1, then 2:
+// Merge, after each lane's scan, pairwise over shuffle distance 1, 2, then 4:
 //   bf16: the keys are unique, so inserting the partner's K keys gives the K largest of both.
 //   fp32: the list of the lower chunks is the base and the other is inserted into it in its own
 //   order.  Every expert of the inserted list has a higher index than every expert of the base,

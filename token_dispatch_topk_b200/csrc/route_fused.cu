@@ -19,7 +19,7 @@
 //      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm and the
 //      tile's per-expert counts go to the workspace, expert-major ([E_local][tiles]).
 //   gate_count_lanes_kernel replaces it for many short rows (moe_gate::lane_gating_fits): one
-//   CTA per tile of 32 tokens, up to four lanes per row (gate_lane.cuh), the same ranks and counts.
+//   CTA per tile of 32 tokens, up to eight lanes per row (gate_lane.cuh), the same ranks and counts.
 // tile_scan_kernel (one CTA per local expert): the expert's row of tile counts becomes the
 //   exclusive prefix over the tiles (the tile bases) and its total goes to the workspace.
 //   Nothing waits on another CTA: the kernel boundary is the only grid-wide step.
@@ -46,7 +46,9 @@ constexpr int kWsHeaderBytes = 256;  // status word, padding
 constexpr int kRowsPerTile = 32;       // tile height of the lane kernel and of the align entry point
 constexpr int kRowsPerTileSmall = 16;  // tile height of gate_count_kernel when all tiles fit at once
 constexpr int kGcCtasPerSm = 4;        // gate_count_kernel CTAs resident per SM (2048 threads)
-constexpr int kTsThreads = 128;  // tile_scan_kernel: threads per expert
+constexpr int kTsThreadsSmall = 128;  // tile_scan_kernel: threads per expert up to kTsWideTiles tiles
+constexpr int kTsThreadsWide = 512;   // and above
+constexpr int kTsWideTiles = 1024;
 constexpr int kPgMaxTokens = 8;
 constexpr uint32_t kPgCtaBytes = 32u * 1024u;
 constexpr int kPgCtasPerSm = 4;  // place_gather_kernel CTAs resident per SM
@@ -265,6 +267,7 @@ LanesKernel lanes_kernel_g(int G) {
     case 1: return &gate_count_lanes_kernel<TIn, K, 1>;
     case 2: return &gate_count_lanes_kernel<TIn, K, 2>;
     case 4: return &gate_count_lanes_kernel<TIn, K, 4>;
+    case 8: return &gate_count_lanes_kernel<TIn, K, 8>;
     default: return nullptr;
   }
 }
@@ -286,11 +289,13 @@ LanesKernel lanes_kernel_for(int k, int G) {
 
 // One CTA per local expert: its row of tile counts -> exclusive prefix over the tiles, in place;
 // the total to `totals`.  Thread i owns a contiguous run of tiles; runs of up to kTsCache tiles
-// (batches of tiles up to 2048) are read once into registers, longer ones are read again for the
-// second pass.
-constexpr int kTsCache = 16;
-__global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
-  __shared__ int warp_sums[kTsThreads / 32];
+// are read once into registers (NT threads: up to 8 * NT tiles), longer ones are read again for the
+// second pass.  The launcher takes 128 threads up to kTsWideTiles tiles: resident early (programmatic
+// dependent launch), wider CTAs take SM room from the gating kernel.
+constexpr int kTsCache = 8;
+template <int NT>
+__global__ void __launch_bounds__(NT) tile_scan_kernel(DispatchArgs a) {
+  __shared__ int warp_sums[NT / 32];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int e = blockIdx.x;
   // let place_gather_kernel start now (it loads its hidden rows, then waits for this kernel,
@@ -299,7 +304,7 @@ __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
   moe::pdl_wait();  // tile counts come from gate_count_kernel
   const int N = a.num_tiles;
   int32_t* col = a.tile_counts + static_cast<int64_t>(e) * N;
-  const int per = (N + kTsThreads - 1) / kTsThreads;
+  const int per = (N + NT - 1) / NT;
   const int t0 = tid * per < N ? tid * per : N;
   const int t1 = t0 + per < N ? t0 + per : N;
   const bool cached = per <= kTsCache;
@@ -329,7 +334,7 @@ __global__ void __launch_bounds__(kTsThreads) tile_scan_kernel(DispatchArgs a) {
   __syncthreads();
   int run = incl - sum, total = 0;
 #pragma unroll
-  for (int w = 0; w < kTsThreads / 32; ++w) {
+  for (int w = 0; w < NT / 32; ++w) {
     const int ws = warp_sums[w];
     run += w < warp ? ws : 0;
     total += ws;
@@ -787,6 +792,14 @@ typename F<float, 1, 1>::Fn family_pick(int vec, int cpl) {
   }
 }
 
+moe_status_t launch_tile_scan(const DispatchArgs& a, int E_local, cudaStream_t st) {
+  if (a.num_tiles > kTsWideTiles)
+    return moe_host::launch_pdl_max_shared(tile_scan_kernel<kTsThreadsWide>, dim3(static_cast<unsigned>(E_local)),
+                                           dim3(kTsThreadsWide), 0, st, a);
+  return moe_host::launch_pdl_max_shared(tile_scan_kernel<kTsThreadsSmall>, dim3(static_cast<unsigned>(E_local)),
+                                         dim3(kTsThreadsSmall), 0, st, a);
+}
+
 struct FusedLayout {
   int num_tiles;
   size_t tile_counts_off, totals_off, bytes;
@@ -918,6 +931,10 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
     const size_t smem1 = static_cast<size_t>(kRowsPerTile) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4) +
                          (2 * static_cast<size_t>(G) * E_local + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
+    if (smem1 > 48 * 1024 &&
+        cudaFuncSetAttribute(reinterpret_cast<const void*>(lk), cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem1)) != cudaSuccess)
+      return MOE_ERR_CUDA;
     if (moe_host::launch_pdl_max_shared(lk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(32 * G), smem1, st, a, cpr) !=
         MOE_OK)
       return MOE_ERR_CUDA;
@@ -935,9 +952,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     if (moe_host::launch_pdl_max_shared(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
       return MOE_ERR_CUDA;
   }
-  if (moe_host::launch_pdl_max_shared(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
-      MOE_OK)
-    return MOE_ERR_CUDA;
+  if (launch_tile_scan(a, E_local, st) != MOE_OK) return MOE_ERR_CUDA;
 
   // tokens per CTA: at most kPgMaxTokens (and kPgCtaBytes of staged rows), chosen so that the CTAs
   // fill whole waves of kPgCtasPerSm per SM; shared memory sized so that no SM takes more
@@ -1005,9 +1020,7 @@ moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32
     return MOE_ERR_CUDA;
   if (moe_host::launch_pdl_max_shared(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
     return MOE_ERR_CUDA;
-  if (moe_host::launch_pdl_max_shared(tile_scan_kernel, dim3(static_cast<unsigned>(E_local)), dim3(kTsThreads), 0, st, a) !=
-      MOE_OK)
-    return MOE_ERR_CUDA;
+  if (launch_tile_scan(a, E_local, st) != MOE_OK) return MOE_ERR_CUDA;
   // placement only: up to kPgMaxTokens tokens per one-warp CTA, the CTAs filling whole waves
   const int sms = moe_host::sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;

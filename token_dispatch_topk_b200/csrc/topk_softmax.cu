@@ -4,8 +4,8 @@
 // (moe_topk_softmax_kernels.cuh: fused softmax+topk; vLLM topk_softmax_kernels.cu),
 // placed by "Call Chain: MoE topk_softmax on BI-V100" between the router and the experts.
 //
-// Design (sm_100a).  Many rows of at most 64 experts and k <= 8 (moe_gate::lane_gating_fits): up
-// to four lanes per row (topk_lane_kernel below, gate_lane.cuh).  Otherwise rows of E >= 16 experts: one
+// Design (sm_100a).  Many rows of short logit rows and k <= 8 (moe_gate::lane_gating_fits): up
+// to eight lanes per row (topk_lane_kernel below, gate_lane.cuh).  Otherwise rows of E >= 16 experts: one
 // warp per row (topk_row_warp_kernel below), one warp-wide redux.sync max per selection round;
 // short rows (E < 16): the sub-warp kernel described here.
 // Sub-warp kernel: a sub-warp of G lanes (G a power of two, 1..32) owns one row.
@@ -202,6 +202,7 @@ LaneKernel lane_kernel_g(int G) {
     case 1: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 1>);
     case 2: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 2>);
     case 4: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 4>);
+    case 8: return reinterpret_cast<LaneKernel>(&topk_lane_kernel<TIn, K, 8>);
     default: return nullptr;
   }
 }
