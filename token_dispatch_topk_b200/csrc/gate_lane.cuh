@@ -1,4 +1,4 @@
-// gate_lane.cuh -- fused softmax + top-k of short router-logit rows, one thread per row.
+// gate_lane.cuh -- fused softmax + top-k of router-logit rows, a few lanes per row.
 //
 // Operation: the fused softmax+topk of "Upstream Reference: Deep-Spark xllm + vllm", "File Index"
 // (moe_topk_softmax_kernels.cuh; vLLM topk_softmax_kernels.cu), with the same selection order and
@@ -47,14 +47,16 @@ inline bool lane_gating_fits(int64_t T, int E, int k, int elem_bytes, const void
 }
 
 // Shared-memory layout of a staged tile: row r starts at chunk r * stride, stride = chunks per row
-// rounded up to odd, so 32 lanes each reading 16 bytes of their own row hit distinct bank groups.
+// rounded up to odd, so lanes reading 16 bytes of different rows at the same offset hit distinct
+// bank groups.
 __host__ __device__ inline int lane_tile_stride(int cpr) { return cpr | 1; }
 
 // Copy rows [0, rows) of a tile (contiguous in global memory, 16-byte aligned, cpr chunks a row)
 // into shared memory with coalesced 16-byte loads, kLaneLoadBatch of them in flight per thread
 // before the first store (the kernels stage at most 4 chunks per thread: one batch).
 // Chunk c of the tile belongs to row c / cpr, computed as floor((c + 0.5) / cpr) in fp32: exact
-// for the tile sizes here (c < 2^12, cpr <= 16).
+// for the tile sizes here (c < 2^12, cpr <= 32: the fraction stays at least 1/64 from an integer,
+// far above the rounding error).
 constexpr int kLaneLoadBatch = 4;
 __device__ __forceinline__ void lane_tile_load(const uint4* __restrict__ g, int rows, int cpr, int stride,
                                                uint4* __restrict__ s, int tid, int nthreads) {
