@@ -128,18 +128,31 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
+// Every bulk copy of this library moves data used once (hidden rows read by the gathers,
+// expert-output rows read by the combine, gathered rows written for the expert GEMMs), so loads and
+// stores carry an L2 evict-first policy: those lines are the first to leave L2, ahead of lines that
+// are still to be used.  Measured on one GPU, back-to-back steps: the 4096 x 128 prefill step takes
+// 60.4 us with both hints, 63.3 with the loads' alone, 63.2 with the stores' alone, 63.5 with
+// neither; the 16384 x 60 step 123.0 us with both and with neither.
+__device__ __forceinline__ uint64_t evict_first_policy() {
+  uint64_t policy;
+  asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
+  return policy;
+}
+
 // global -> shared bulk copy; `bytes` and both addresses 16-byte aligned.
 __device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-                   smem_addr(dst_smem)),
-               "l"(src), "r"(bytes), "r"(smem_addr(bar))
-               : "memory");
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
+          smem_addr(dst_smem)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(evict_first_policy())
+      : "memory");
 }
 
 // shared -> global bulk copy, tracked by this thread's bulk groups.
 __device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src_smem)),
-               "r"(bytes)
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+               "r"(smem_addr(src_smem)), "r"(bytes), "l"(evict_first_policy())
                : "memory");
 }
 
