@@ -128,12 +128,16 @@ __device__ __forceinline__ void named_barrier(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Every bulk copy of this library moves data used once (hidden rows read by the gathers,
-// expert-output rows read by the combine, gathered rows written for the expert GEMMs), so loads and
-// stores carry an L2 evict-first policy: those lines are the first to leave L2, ahead of lines that
-// are still to be used.  Measured on one GPU, back-to-back steps: the 4096 x 128 prefill step takes
-// 60.4 us with both hints, 63.3 with the loads' alone, 63.2 with the stores' alone, 63.5 with
-// neither; the 16384 x 60 step 123.0 us with both and with neither.
+// Bulk copies of rows used once (hidden rows read by the gathers, expert-output rows read by the
+// combine, gathered rows written for the expert GEMMs) may carry an L2 evict-first policy: those
+// lines are the first to leave L2, ahead of lines that are still to be used.  The kernels ask for it
+// when a row is at most kEvictFirstMaxRowBytes (one bulk copy per row).  Measured on one GPU in
+// back-to-back steps: the 4096 x 128 prefill step (4 KB rows) takes 60.4 us with the policy on loads
+// and stores, 63.3 with loads only, 63.2 with stores only, 63.5 without; the 16384 x 60 step (4 KB
+// rows) 123.0 us with and without; the 65536 x 256 step (14 KB rows, which the combine copies in
+// 4 KB pieces) 2672 us with and 2600 us without.
+constexpr uint32_t kEvictFirstMaxRowBytes = 4096;
+
 __device__ __forceinline__ uint64_t evict_first_policy() {
   uint64_t policy;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(policy));
@@ -141,19 +145,33 @@ __device__ __forceinline__ uint64_t evict_first_policy() {
 }
 
 // global -> shared bulk copy; `bytes` and both addresses 16-byte aligned.
-__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], %4;" ::"r"(
-          smem_addr(dst_smem)),
-      "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(evict_first_policy())
-      : "memory");
+__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar,
+                                          bool evict_first) {
+  if (evict_first) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1], %2, [%3], "
+        "%4;" ::"r"(smem_addr(dst_smem)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar)), "l"(evict_first_policy())
+        : "memory");
+  } else {
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                     smem_addr(dst_smem)),
+                 "l"(src), "r"(bytes), "r"(smem_addr(bar))
+                 : "memory");
+  }
 }
 
 // shared -> global bulk copy, tracked by this thread's bulk groups.
-__device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes) {
-  asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
-               "r"(smem_addr(src_smem)), "r"(bytes), "l"(evict_first_policy())
-               : "memory");
+__device__ __forceinline__ void bulk_store(void* dst, const void* src_smem, uint32_t bytes, bool evict_first) {
+  if (evict_first) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group.L2::cache_hint [%0], [%1], %2, %3;" ::"l"(dst),
+                 "r"(smem_addr(src_smem)), "r"(bytes), "l"(evict_first_policy())
+                 : "memory");
+  } else {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(dst), "r"(smem_addr(src_smem)),
+                 "r"(bytes)
+                 : "memory");
+  }
 }
 
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }

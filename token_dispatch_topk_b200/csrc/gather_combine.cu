@@ -114,12 +114,13 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
     moe::fence_barrier_init();
   }
   __syncwarp();
+  const bool evict_first = row_bytes <= moe::kEvictFirstMaxRowBytes;
   auto load_rows = [&]() {
     if (lane == 0) {
       moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
       for (int i = 0; i < n; ++i) {
         moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes,
-                       hidden + (t0 + i) * static_cast<int64_t>(row_bytes), row_bytes, &bar);
+                       hidden + (t0 + i) * static_cast<int64_t>(row_bytes), row_bytes, &bar, evict_first);
       }
     }
   };
@@ -152,7 +153,7 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
     const int e = lane + 32 * m;
     if (e < nslots && dst[m] >= 0) {
       moe::bulk_store(permuted + static_cast<int64_t>(dst[m]) * row_bytes, rows + static_cast<size_t>(e / k) * row_bytes,
-                      row_bytes);
+                      row_bytes, evict_first);
     }
   }
   moe::bulk_commit();
@@ -222,6 +223,7 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
 
   if (warp == 0) {
     // ---- producer: lane l < spu handles slot l of the unit (token t0 + l / k, rank l % k)
+    const bool evict_first = a.row_bytes <= moe::kEvictFirstMaxRowBytes;
     auto load_meta = [&](int64_t grp, int& r, float& w) {
       r = -1;
       w = 0.f;
@@ -269,7 +271,7 @@ __global__ void __launch_bounds__((1 + kCombineConsumerWarps) * 32) combine_tma_
       if (r_cur >= 0) {
         moe::bulk_load(buf + static_cast<size_t>(s) * stage_bytes + static_cast<size_t>(lane) * a.chunk_bytes,
                        a.y + static_cast<int64_t>(r_cur) * a.row_bytes + static_cast<int64_t>(c) * a.chunk_bytes, cb,
-                       &full[s]);
+                       &full[s], evict_first);
       }
       if (++s == S) {
         s = 0;

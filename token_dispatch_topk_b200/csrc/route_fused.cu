@@ -384,7 +384,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
     for (int i = 0; i < n; ++i) {
       moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes, hidden + (t0 + i) * static_cast<int64_t>(row_bytes),
-                     row_bytes, &bar);
+                     row_bytes, &bar, row_bytes <= moe::kEvictFirstMaxRowBytes);
     }
   }
   moe::pdl_launch_dependents();
@@ -471,7 +471,8 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
       const int e = lane + 32 * m;
       if (e < nslots && dst[m] >= 0) {
         moe::bulk_store(permuted + static_cast<int64_t>(dst[m]) * row_bytes,
-                        rows + static_cast<size_t>(e / k) * row_bytes, row_bytes);
+                        rows + static_cast<size_t>(e / k) * row_bytes, row_bytes,
+                        row_bytes <= moe::kEvictFirstMaxRowBytes);
       }
     }
     moe::bulk_commit();
