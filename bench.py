@@ -421,9 +421,11 @@ def main():
     st_iters = args.stage_steps or min(args.steps, 500)
 
     stage_kernel = dict(STAGE_KERNEL)
-    # the kernels each entry point launches for this workload (the library's selection rules)
+    # the kernels each entry point launches for this workload (the library's selection rules; the
+    # lane-gating rule is moe_gate::lane_gating_fits in csrc/gate_lane.cuh)
     elem = 2 if wl.logits_dtype == "bf16" else 4
-    lanes = wl.T >= 1024 and wl.k <= 8 and wl.E <= 64 and (wl.E * elem) % 16 == 0
+    lanes = wl.k <= 8 and (wl.E * elem) % 16 == 0 and (
+        (wl.E <= 64 and wl.T >= 1024) or (elem == 2 and wl.E <= 256 and wl.T >= 16384))
     if r.small_batch:
         stage_kernel["dispatch"] = "route_small_kernel"
     elif lanes:
