@@ -8,7 +8,7 @@ Every function takes and returns numpy arrays; bf16 tensors travel as their raw
 ``uint16`` bit patterns.  The arithmetic lives in ``moe_oracle.cpp``; this file
 only allocates output arrays and marshals pointers.
 
-Parity pins: all four functions are pinned by ``tests/test_oracle_*.py``
+Parity pins: every function is pinned by ``tests/test_oracle_*.py``
 (hand-worked examples under ``tests/golden/``, closed forms, brute force over
 all subsets, a stable library sort, exact rational accumulation, invariants),
 and ``tests/test_oracle_mutants.py`` shows that planted mistakes fail them.
@@ -63,7 +63,7 @@ def _check(rc: int, what: str) -> None:
 
 
 class Oracle:
-    """The four oracle functions bound to one compiled copy of moe_oracle.cpp."""
+    """The oracle functions bound to one compiled copy of moe_oracle.cpp."""
 
     def __init__(self, lib_path: str):
         lib = ctypes.CDLL(lib_path)
@@ -79,6 +79,8 @@ class Oracle:
         lib.oracle_gather.restype = ctypes.c_int
         lib.oracle_combine.argtypes = [_P, _P, _P, _I64, _I32, _I32, _P]
         lib.oracle_combine.restype = ctypes.c_int
+        lib.oracle_reduce_partials.argtypes = [_P, _I32, _I64, _I32, _P]
+        lib.oracle_reduce_partials.restype = ctypes.c_int
         self._lib = lib
         self.path = lib_path
 
@@ -174,6 +176,16 @@ class Oracle:
         return out
 
 
+    def reduce_partials(self, partials: np.ndarray) -> np.ndarray:
+        """partials: [n, rows, H] uint16 (bf16 bits), one partial combine per rank.  Returns [rows, H]
+        uint16: the fp32 sum in ascending rank order from +0, rounded once to bf16."""
+        p = np.ascontiguousarray(partials, dtype=np.uint16)
+        n, rows, H = p.shape
+        out = np.empty((rows, H), np.uint16)
+        _check(self._lib.oracle_reduce_partials(_ptr(p), n, rows, H, _ptr(out)), "reduce_partials")
+        return out
+
+
 _default: Optional[Oracle] = None
 
 
@@ -207,3 +219,7 @@ def gather(hidden, k, sorted_token_ids, num_tokens_post_pad, capacity, zero_pad=
 
 def combine(expert_out, topk_weights, inv_perm):
     return default().combine(expert_out, topk_weights, inv_perm)
+
+
+def reduce_partials(partials):
+    return default().reduce_partials(partials)

@@ -308,4 +308,19 @@ int oracle_combine(const uint16_t* expert_out, const float* topk_weights, const 
     return 0;
 }
 
+/* The exchange after an expert-parallel combine: each of n ranks holds a bf16 partial [rows, H] (the
+ * combine over its local slots, remote slots dropped); the layer output is the sum of the partials.
+ * Reading (the closure note leaves the collective out): widened to fp32, summed in ascending rank
+ * order starting from +0, rounded once to bf16.  partials: [n][rows][H] bf16 bits, rank-major. */
+int oracle_reduce_partials(const uint16_t* partials, int32_t n, int64_t rows, int32_t H, uint16_t* out) {
+    if (n < 1 || rows < 0 || H < 1) return 1;
+    const int64_t m = rows * static_cast<int64_t>(H);
+    for (int64_t i = 0; i < m; ++i) {
+        float acc = 0.0f;
+        for (int32_t r = 0; r < n; ++r) acc = acc + bf16_to_float(partials[r * m + i]);
+        out[i] = float_to_bf16_rne(acc);
+    }
+    return 0;
+}
+
 }  // extern "C"

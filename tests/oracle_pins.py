@@ -572,4 +572,89 @@ GATHER_COMBINE_PINS = [pin_gather_hand_example, pin_gather_rows_and_pads, pin_co
                        pin_combine_identity, pin_combine_error_bound, pin_combine_remote_dropped,
                        pin_combine_fma_sequence]
 
-ALL_PINS = TOPK_PINS + SIGMOID_PINS + ALIGN_PINS + GATHER_COMBINE_PINS
+
+# ----------------------------------------------------------------------------------------------
+# The expert-parallel exchange: the sum of the ranks' bf16 partial combines, widened to fp32 and
+# added in ascending rank order from +0, rounded once to bf16 (the reading the oracle takes where
+# the closure note leaves the collective out).
+# ----------------------------------------------------------------------------------------------
+def _partials(values) -> np.ndarray:
+    """[n] values -> [n, 1, 1] bf16 bits (each value must be a bf16 number)."""
+    b = f32_to_bf16_bits(np.array(values, np.float32).reshape(-1, 1, 1))
+    assert np.array_equal(bf16_bits_to_f32(b).reshape(-1), np.array(values, np.float32))
+    return b
+
+
+def pin_reduce_hand_examples(orc) -> None:
+    # fp32 accumulation: 1 + 2^-8 + 2^-8 = 1 + 2^-7, a bf16 number; bf16 accumulation would give 1
+    assert float(bf16_bits_to_f32(orc.reduce_partials(_partials([1.0, 2.0 ** -8, 2.0 ** -8])))[0, 0]) == 1.0 + 2.0 ** -7
+    # ascending rank order: 2^24 + 1 rounds to 2^24 in fp32, so (2^24, 1, -2^24) gives 0 and
+    # (2^24, -2^24, 1) gives 1
+    assert float(bf16_bits_to_f32(orc.reduce_partials(_partials([2.0 ** 24, 1.0, -2.0 ** 24])))[0, 0]) == 0.0
+    assert float(bf16_bits_to_f32(orc.reduce_partials(_partials([2.0 ** 24, -2.0 ** 24, 1.0])))[0, 0]) == 1.0
+    # x + (-x) is +0 (bits 0), as is a lone -0 (0 + -0 = +0)
+    assert int(orc.reduce_partials(_partials([3.5, -3.5]))[0, 0]) == 0
+    assert int(orc.reduce_partials(np.full((1, 1, 1), 0x8000, np.uint16))[0, 0]) == 0
+    # one rank: its partial, bit for bit (no -0 among them)
+    rng = np.random.default_rng(23)
+    one = f32_to_bf16_bits(rng.standard_normal((1, 7, 24)).astype(np.float32))
+    one[one == 0x8000] = 0
+    assert np.array_equal(orc.reduce_partials(one), one[0])
+    # a sum that needs rounding: 1 + 2^-8 + 2^-9 = 1.005859375 lies between the bf16 numbers 1 and
+    # 1.0078125, nearer the second (truncation would give 1)
+    assert float(bf16_bits_to_f32(orc.reduce_partials(_partials([1.0, 2.0 ** -8, 2.0 ** -9])))[0, 0]) == 1.0078125
+
+
+def pin_reduce_fp32_chain(orc) -> None:
+    """Each element is a chain of correctly rounded fp32 additions in ascending rank order from +0,
+    then one bf16 round-to-nearest-even; emulated here with exact rationals."""
+    rng = np.random.default_rng(29)
+    for n in (2, 3, 5, 8):
+        mags = np.float32(2.0) ** rng.integers(-12, 13, size=(n, 9, 8)).astype(np.float32)
+        p = f32_to_bf16_bits(rng.standard_normal((n, 9, 8)).astype(np.float32) * mags)
+        pv = bf16_bits_to_f32(p)
+        want = np.empty((9, 8), np.float32)
+        for i in range(9):
+            for h in range(8):
+                acc = Fraction(0)
+                for r in range(n):
+                    acc = round_to_f32(acc + Fraction(float(pv[r, i, h])))
+                want[i, h] = np.float32(float(acc))
+        got = orc.reduce_partials(p)
+        assert np.array_equal(got, f32_to_bf16_bits(want)), n
+
+
+def pin_reduce_of_rank_partials(orc) -> None:
+    """Expert-parallel decomposition: each of 4 ranks combines over its own block of experts; the
+    reduce of the 4 partials agrees with the single-rank combine within the rounding of the
+    partials (each is rounded to bf16 once) and of the sums."""
+    rng = np.random.default_rng(31)
+    T, E, k, H, bs, n = 20, 16, 4, 24, 4, 4
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    w, ids = orc.topk_softmax(logits, k, True)
+    full = orc.align_permute(ids, E, bs)
+    y_full = f32_to_bf16_bits(rng.standard_normal((full["capacity"], H)).astype(np.float32))
+    ref = bf16_bits_to_f32(orc.combine(y_full, w, full["inv_perm"]))
+    # the rank-local expert-output rows are the same rows of the full layout, relaid per rank
+    parts, bound = [], np.zeros((T, H))
+    for r in range(n):
+        m = np.full(E, -1, np.int32)
+        m[r * 4:(r + 1) * 4] = np.arange(4)
+        loc = orc.align_permute(ids, E, bs, m, 4)
+        y = np.zeros((loc["capacity"], H), np.uint16)
+        for s in range(T * k):
+            if loc["inv_perm"][s] >= 0:
+                y[loc["inv_perm"][s]] = y_full[full["inv_perm"][s]]
+        part = orc.combine(y, w, loc["inv_perm"])
+        parts.append(part)
+        pv = np.abs(bf16_bits_to_f32(part).astype(np.float64))
+        bound += 2.0 ** (np.floor(np.log2(np.maximum(pv, 2.0 ** -126))) - 8)
+    got = bf16_bits_to_f32(orc.reduce_partials(np.stack(parts))).astype(np.float64)
+    mag = np.abs(ref.astype(np.float64))
+    bound += 2.0 ** (np.floor(np.log2(np.maximum(mag + bound, 2.0 ** -126))) - 7) + 1e-6
+    assert (np.abs(got - ref) <= bound).all(), float(np.max(np.abs(got - ref) - bound))
+
+
+REDUCE_PINS = [pin_reduce_hand_examples, pin_reduce_fp32_chain, pin_reduce_of_rank_partials]
+
+ALL_PINS = TOPK_PINS + SIGMOID_PINS + ALIGN_PINS + GATHER_COMBINE_PINS + REDUCE_PINS

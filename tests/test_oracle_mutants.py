@@ -71,6 +71,15 @@ MUTANTS = [
      "const double wj = score[j];"),
     ("sigmoid weight taken from the wrong expert",
      "score[j] = 1.0 / (1.0 + std::exp(-x[sel[j]]));", "score[j] = 1.0 / (1.0 + std::exp(-x[j]));"),
+    ("reduce adds the ranks in descending order",
+     "for (int32_t r = 0; r < n; ++r) acc = acc + bf16_to_float(partials[r * m + i]);",
+     "for (int32_t r = n - 1; r >= 0; --r) acc = acc + bf16_to_float(partials[r * m + i]);"),
+    ("reduce accumulates in bf16",
+     "for (int32_t r = 0; r < n; ++r) acc = acc + bf16_to_float(partials[r * m + i]);",
+     "for (int32_t r = 0; r < n; ++r) acc = bf16_to_float(float_to_bf16_rne(acc + bf16_to_float(partials[r * m + i])));"),
+    ("reduce drops the last rank",
+     "for (int32_t r = 0; r < n; ++r) acc = acc + bf16_to_float(partials[r * m + i]);",
+     "for (int32_t r = 0; r + 1 < n; ++r) acc = acc + bf16_to_float(partials[r * m + i]);"),
 ]
 
 
