@@ -8,7 +8,8 @@
  *   moe_gather         activation permute-gather into the expert-grouped layout
  *   moe_combine        top-k weighted combine back to token order
  * Between moe_gather and moe_combine the caller runs its expert MLPs on the
- * expert-grouped rows; they are not part of this library.
+ * expert-grouped rows; they are not part of this library.  Under expert
+ * parallelism, moe_reduce_partials sums the ranks' partial combines.
  *
  * Sources (web pages, by title and section):
  *   "project_6/upstream_ref -- Upstream Reference: Deep-Spark xllm + vllm":
@@ -33,7 +34,8 @@
  *   k experts per token, H hidden size, bs block size.  Slot s = t*k + j is the
  *   j-th routed choice of token t (P = T*k slots).
  *   Memory: every pointer argument is DEVICE memory owned by the caller, except
- *   the host out-parameter of moe_read_status.  All arrays are dense row-major.
+ *   the host out-parameter of moe_read_status and the host pointer array of
+ *   moe_reduce_partials.  All arrays are dense row-major.
  *   The library allocates nothing, keeps no global state and never synchronises
  *   the stream except in moe_read_status.
  *   Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
@@ -276,6 +278,31 @@ MOE_API moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, c
                                         int32_t* counts, int32_t* offsets, int32_t* sorted_token_ids,
                                         int32_t* expert_ids, int32_t* num_tokens_post_pad, int32_t* inv_perm,
                                         void* permuted, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * moe_reduce_partials -- the exchange after an expert-parallel combine: the sum of
+ * the ranks' partial combines ("b70-optimization-lab: 2026-07-16 MTP1 M=2 compact
+ * scheduler closure note", scheduler paragraph: each rank keeps the slots of its own
+ * experts through expert_map, so its moe_combine is a partial sum over its local
+ * slots; the note leaves the collective that sums them out).
+ *   partials    HOST array of n_partials DEVICE pointers, the partials in rank order,
+ *               each [rows, H] bf16, 16-byte aligned.  A pointer may address another
+ *               GPU's memory (peer access enabled): it is read with plain 16-byte loads.
+ *               The array itself is read during the call only.
+ *   n_partials  1..16.
+ *   out         [rows, H] bf16 out: each element is the fp32 sum of the partials'
+ *               elements in ascending rank order from +0, rounded once to bf16
+ *               (round-to-nearest-even).  out may be one of the partials (every
+ *               element is read before it is written).
+ *   For a reduce-scatter, rank r's moe_combine writes owner o's token range of its
+ *   partial into owner o's receive buffer (`out` pointing into the owner's memory, with
+ *   topk_weights and inv_perm advanced to the range's first token); once every rank has
+ *   written (the caller's barrier), owner o calls moe_reduce_partials on its buffers.
+ *   Errors: INVALID_ARG (rows < 0, H % 8 != 0, null or misaligned pointers),
+ *   UNSUPPORTED (n_partials > 16).
+ */
+MOE_API moe_status_t moe_reduce_partials(const void* const* partials, int32_t n_partials, int64_t rows, int32_t H,
+                                         void* out, void* stream);
 
 /*
  * Read the device status word (first 4 bytes of an align workspace, or any

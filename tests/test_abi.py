@@ -143,3 +143,20 @@ def test_dispatch_validation_before_launch():
     assert call(buf, B.MOE_SCORING_SIGMOID, buf) == B.MOE_ERR_WORKSPACE  # sigmoid scoring accepted
     assert call(buf, B.MOE_GATHER_ZERO_PAD, buf) == B.MOE_ERR_INVALID_ARG
     assert call(buf, B.MOE_RENORMALIZE | given, buf, H=12) == B.MOE_ERR_INVALID_ARG  # H % 8
+
+
+def test_reduce_partials_host_validation():
+    """moe_reduce_partials rejects bad arguments before any CUDA call (no GPU needed)."""
+    lib = B.load_library()
+    aligned = ctypes.c_void_p(1 << 20)
+    arr = (ctypes.c_void_p * 17)(*([aligned] * 17))
+    p = ctypes.cast(arr, ctypes.c_void_p)
+    assert lib.moe_reduce_partials(p, 0, 4, 8, aligned, None) == B.MOE_ERR_INVALID_ARG      # no partial
+    assert lib.moe_reduce_partials(p, 17, 4, 8, aligned, None) == B.MOE_ERR_UNSUPPORTED     # more than 16
+    assert lib.moe_reduce_partials(p, 2, 4, 12, aligned, None) == B.MOE_ERR_INVALID_ARG     # H % 8 != 0
+    assert lib.moe_reduce_partials(p, 2, -1, 8, aligned, None) == B.MOE_ERR_INVALID_ARG     # rows < 0
+    assert lib.moe_reduce_partials(p, 2, 0, 8, aligned, None) == B.MOE_OK                   # nothing to do
+    assert lib.moe_reduce_partials(p, 2, 4, 8, ctypes.c_void_p(0x1002), None) == B.MOE_ERR_INVALID_ARG  # out
+    bad = (ctypes.c_void_p * 2)(aligned, ctypes.c_void_p(0x1008))
+    assert lib.moe_reduce_partials(ctypes.cast(bad, ctypes.c_void_p), 2, 4, 8, aligned, None) == B.MOE_ERR_INVALID_ARG
+    assert lib.moe_reduce_partials(None, 2, 4, 8, aligned, None) == B.MOE_ERR_INVALID_ARG

@@ -127,3 +127,35 @@ def test_ep_expert_range_splits_evenly():
     assert El == 40 and m[40].item() == 0 and m[79].item() == 39 and m[39].item() == -1 and m[80].item() == -1
     with pytest.raises(ValueError):
         D.ep_expert_range(3, 4, 0)
+
+
+def test_ep_token_range_partitions_the_tokens():
+    """The owners' token ranges of the reduce-scatter form cover [0, T) in order, without overlap,
+    sizes differing by at most one (owners past T get empty ranges)."""
+    for T in (0, 1, 2, 3, 7, 64, 4097):
+        for world in (1, 2, 3, 4, 8):
+            ranges = [D.ep_token_range(T, world, o) for o in range(world)]
+            assert ranges[0][0] == 0 and ranges[-1][1] == T
+            for (lo, hi), (lo2, _) in zip(ranges, ranges[1:]):
+                assert hi == lo2
+            sizes = [hi - lo for lo, hi in ranges]
+            assert max(sizes) - min(sizes) <= 1 and min(sizes) >= 0
+    with pytest.raises(ValueError):
+        D.ep_token_range(10, 4, 4)
+    with pytest.raises(ValueError):
+        D.ep_token_range(-1, 2, 0)
+
+
+def test_reduce_scatter_of_the_oracle_partials_is_the_reduce():
+    """The reduce-scatter form gives each owner the rows of the full reduce: reducing each owner's
+    token range of the partials and concatenating equals reducing the whole partials (per element
+    the same sum in the same rank order)."""
+    rng = np.random.default_rng(5)
+    world, T, H = 4, 11, 16
+    parts = f32_to_bf16_bits(rng.standard_normal((world, T, H)).astype(np.float32))
+    full = oracle.reduce_partials(parts)
+    pieces = []
+    for o in range(world):
+        lo, hi = D.ep_token_range(T, world, o)
+        pieces.append(oracle.reduce_partials(parts[:, lo:hi]) if hi > lo else np.zeros((0, H), np.uint16))
+    assert np.array_equal(np.concatenate(pieces), full)

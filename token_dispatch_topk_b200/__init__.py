@@ -11,6 +11,7 @@ from .binding import (  # noqa: F401
     MOE_RENORMALIZE, MOE_DISPATCH_GIVEN_IDS, MOE_SCORING_SIGMOID,
     AlignResult, MoeError, alloc_align_outputs, alloc_workspace, load_library, moe_align_capacity,
     moe_align_num_blocks, moe_align_permute, moe_align_permute_noalloc, moe_align_workspace_bytes, moe_combine, moe_gather, moe_read_status,
+    moe_reduce_partials,
     moe_route_dispatch, moe_route_dispatch_workspace_bytes, moe_topk_softmax, moe_version, moe_workspace_init,
     status_string, alloc_dispatch_workspace,
 )

@@ -52,6 +52,7 @@ SIGNATURES = {
     "moe_route_dispatch_workspace_bytes": (_SZ, [_I64, _I32, _I32]),
     "moe_route_dispatch": (ctypes.c_int, [_P, ctypes.c_int, _P, _I64, _I32, _I32, _I32, _U32, _P, _I32, _I32, _P, _P,
                                           _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P]),
+    "moe_reduce_partials": (ctypes.c_int, [_P, _I32, _I64, _I32, _P, _P]),
 }
 
 _lib: Optional[ctypes.CDLL] = None
@@ -272,6 +273,24 @@ def moe_combine(expert_out: torch.Tensor, topk_weights: torch.Tensor, inv_perm: 
                                     _dev(inv_perm, "inv_perm"), T, k, H, capacity, _dev(out, "out"),
                                     _dev(device_status, "device_status"), _stream(stream))
     _check(st, "moe_combine")
+    return out
+
+
+def moe_reduce_partials(partials, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """partials: the ranks' bf16 partial combines [rows, H] in rank order (tensors on this GPU or,
+    with peer access, on others) -> out [rows, H] bf16: their fp32 sum in rank order, rounded once."""
+    partials = list(partials)
+    if not partials:
+        raise ValueError("moe_reduce_partials needs at least one partial")
+    rows, H = partials[0].shape
+    for p in partials:
+        assert p.dtype == torch.bfloat16 and tuple(p.shape) == (rows, H), "partials must all be bf16 [rows, H]"
+    if out is None:
+        out = torch.empty((rows, H), dtype=torch.bfloat16, device=partials[0].device)
+    ptrs = (ctypes.c_void_p * len(partials))(*[_dev(p, "partial") for p in partials])
+    st = load_library().moe_reduce_partials(ctypes.cast(ptrs, ctypes.c_void_p), len(partials), rows, H,
+                                            _dev(out, "out"), _stream(stream))
+    _check(st, "moe_reduce_partials")
     return out
 
 
