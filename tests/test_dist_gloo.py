@@ -159,3 +159,33 @@ def test_reduce_scatter_of_the_oracle_partials_is_the_reduce():
         lo, hi = D.ep_token_range(T, world, o)
         pieces.append(oracle.reduce_partials(parts[:, lo:hi]) if hi > lo else np.zeros((0, H), np.uint16))
     assert np.array_equal(np.concatenate(pieces), full)
+
+
+def test_combine_to_owners_slices_each_owner_range(monkeypatch):
+    """Host logic of the reduce-scatter form on the CPU: ep_combine_to_owners hands moe_combine each
+    owner's token range (weights, slot rows and destination); the oracle's combine stands in for the
+    kernel here, so each owner's slot must hold exactly that range of the rank's partial, owners
+    without tokens included."""
+    from token_dispatch_topk_b200 import binding as B
+
+    def oracle_combine(expert_out, topk_weights, inv_perm, out=None, device_status=None, stream=None):
+        bits = expert_out.contiguous().view(torch.int16).numpy().view(np.uint16)
+        res = oracle.combine(bits, topk_weights.numpy(), inv_perm.numpy())
+        out.copy_(torch.from_numpy(res.view(np.int16)).view(torch.bfloat16))
+        return out
+
+    monkeypatch.setattr(B, "moe_combine", oracle_combine)
+    rng = np.random.default_rng(3)
+    for T, E, k, H, bs, world in [(50, 32, 4, 16, 4, 4), (2, 160, 6, 8, 8, 4), (7, 12, 2, 8, 2, 3)]:
+        w, ids = oracle.topk_softmax(rng.standard_normal((T, E)).astype(np.float32), k, True)
+        ranges = [D.ep_token_range(T, world, o) for o in range(world)]
+        for r in range(world):
+            m, El = D.ep_expert_map(E, world, r)
+            al = oracle.align_permute(ids, E, bs, m.numpy(), El)
+            y = f32_to_bf16_bits(rng.standard_normal((al["capacity"], H)).astype(np.float32))
+            dests = [torch.full((hi - lo, H), 7.0, dtype=torch.bfloat16) for lo, hi in ranges]
+            D.ep_combine_to_owners(torch.from_numpy(y.view(np.int16)).view(torch.bfloat16), torch.from_numpy(w),
+                                   torch.from_numpy(al["inv_perm"]), dests)
+            full = oracle.combine(y, w, al["inv_perm"])
+            for (lo, hi), d in zip(ranges, dests):
+                assert np.array_equal(d.view(torch.int16).numpy().view(np.uint16), full[lo:hi]), (T, r, lo)
