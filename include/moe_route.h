@@ -298,8 +298,8 @@ MOE_API moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, c
  *   partial into owner o's receive buffer (`out` pointing into the owner's memory, with
  *   topk_weights and inv_perm advanced to the range's first token); once every rank has
  *   written (the caller's barrier), owner o calls moe_reduce_partials on its buffers.
- *   Errors: INVALID_ARG (rows < 0, H % 8 != 0, null or misaligned pointers),
- *   UNSUPPORTED (n_partials > 16).
+ *   Errors: INVALID_ARG (rows < 0, H % 8 != 0, rows * H beyond 2^47, null or misaligned
+ *   pointers), UNSUPPORTED (n_partials > 16).
  */
 MOE_API moe_status_t moe_reduce_partials(const void* const* partials, int32_t n_partials, int64_t rows, int32_t H,
                                          void* out, void* stream);
