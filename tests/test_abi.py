@@ -161,3 +161,4 @@ def test_reduce_partials_host_validation():
     assert lib.moe_reduce_partials(ctypes.cast(bad, ctypes.c_void_p), 2, 4, 8, aligned, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_reduce_partials(None, 2, 4, 8, aligned, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_reduce_partials(p, 2, 1 << 40, 1 << 20, aligned, None) == B.MOE_ERR_INVALID_ARG  # rows * H too large
+    assert lib.moe_reduce_partials(p, 2, 1 << 40, (1 << 31) - 8, aligned, None) == B.MOE_ERR_INVALID_ARG

@@ -72,7 +72,7 @@ extern "C" moe_status_t moe_reduce_partials(const void* const* partials, int32_t
                                             void* out, void* stream) {
   if (n_partials < 1 || rows < 0 || H < 1 || (H % 8) != 0) return MOE_ERR_INVALID_ARG;
   if (n_partials > kMaxPartials) return MOE_ERR_UNSUPPORTED;
-  if (rows > (int64_t{1} << 40) || rows * static_cast<int64_t>(H / 8) > (int64_t{1} << 44)) return MOE_ERR_INVALID_ARG;
+  if (rows > (int64_t{1} << 40) || rows > (int64_t{1} << 44) / (H / 8)) return MOE_ERR_INVALID_ARG;  // H >= 8
   if (rows == 0) return MOE_OK;
   if (partials == nullptr || out == nullptr || !moe_host::aligned16(out)) return MOE_ERR_INVALID_ARG;
   ReduceArgs a{};
