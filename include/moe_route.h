@@ -70,7 +70,7 @@ extern "C" {
 typedef enum {
   MOE_OK = 0,
   MOE_ERR_INVALID_ARG = 1,   /* null pointer, negative size, k > E, misalignment, ... */
-  MOE_ERR_UNSUPPORTED = 2,   /* valid but beyond this build: E > 1024, k > 32, E_local > 1024 */
+  MOE_ERR_UNSUPPORTED = 2,   /* valid but beyond the library's limits: E > 1024, k > 32, E_local > 1024 */
   MOE_ERR_WORKSPACE = 3,     /* workspace null or smaller than moe_align_workspace_bytes() */
   MOE_ERR_CUDA = 4,          /* a CUDA launch or copy failed */
   MOE_ERR_TIMEOUT = 5,       /* device: a bounded wait ran out (recorded in the status word) */

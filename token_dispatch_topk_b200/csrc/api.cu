@@ -8,7 +8,7 @@ extern "C" const char* moe_status_string(moe_status_t status) {
   switch (status) {
     case MOE_OK: return "MOE_OK";
     case MOE_ERR_INVALID_ARG: return "MOE_ERR_INVALID_ARG: invalid argument";
-    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: size beyond this build (E or E_local > 1024, k > 32)";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: size beyond the library's limits (E or E_local > 1024, k > 32)";
     case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace missing or too small";
     case MOE_ERR_CUDA: return "MOE_ERR_CUDA: a CUDA launch or copy failed";
     case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: a bounded device wait ran out";
