@@ -1,6 +1,7 @@
 """B200 (sm_100a) MoE token routing: fused softmax+top-k gating, expert align/permute,
-activation permute-gather and top-k weighted combine, as hand-written CUDA kernels
-behind the C ABI of libmoe_route.so (include/moe_route.h).
+activation permute-gather, top-k weighted combine and the expert-parallel sum of the
+ranks' partial combines, as hand-written CUDA kernels behind the C ABI of
+libmoe_route.so (include/moe_route.h).
 
 The Python layer only marshals arguments (``binding``) and preallocates buffers
 (``router.MoeRouter``); synthetic workloads live in ``inputs``.
