@@ -36,8 +36,10 @@
  *   Memory: every pointer argument is DEVICE memory owned by the caller, except
  *   the host out-parameter of moe_read_status and the host pointer array of
  *   moe_reduce_partials.  All arrays are dense row-major.
- *   The library allocates nothing, keeps no global state and never synchronises
- *   the stream except in moe_read_status.
+ *   The library allocates nothing and never synchronises the stream except in
+ *   moe_read_status.  It keeps no global state, with one exception:
+ *   moe_align_permute_noalloc keeps its scratch in a fixed 1 MiB device array per
+ *   GPU and the array's device address per CUDA context (see that entry point).
  *   Streams: `stream` is a cudaStream_t passed as void* (NULL = legacy default
  *   stream).  Every call only enqueues work on it and returns.
  *   Errors: arguments are validated on the host before anything is enqueued;
@@ -195,9 +197,11 @@ MOE_API moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32
  *     > 1 MiB, e.g. E_local = 1024 with more than about 1M slots) return MOE_ERR_UNSUPPORTED
  *     before anything is enqueued;
  *   - device_status: a caller device int32 that collects device-side errors, or NULL.
- *   It calls no cudaMalloc, cudaFree or other allocating routine.  The first call on each
- *   device looks up the array's device address (cudaGetSymbolAddress) with that device
- *   current; make that first call before any stream capture.  Each call clears the ticket
+ *   It calls no cudaMalloc, cudaFree or other allocating routine.  The first call in each
+ *   CUDA context (the device's primary context; again after a device reset, which makes a new
+ *   one) looks up the array's device address (cudaGetSymbolAddress) with that device current
+ *   and caches it under the context's id; make that first call before any stream capture.
+ *   Each call clears the ticket
  *   with an asynchronous 4-byte memset on `stream`; the counters are rewritten before they
  *   are read.  All calls on a device share the one array and it keeps the last call's
  *   contents, so calls that overlap on the GPU (different streams, concurrent graphs) race

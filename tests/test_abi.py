@@ -162,3 +162,16 @@ def test_reduce_partials_host_validation():
     assert lib.moe_reduce_partials(None, 2, 4, 8, aligned, None) == B.MOE_ERR_INVALID_ARG
     assert lib.moe_reduce_partials(p, 2, 1 << 40, 1 << 20, aligned, None) == B.MOE_ERR_INVALID_ARG  # rows * H too large
     assert lib.moe_reduce_partials(p, 2, 1 << 40, (1 << 31) - 8, aligned, None) == B.MOE_ERR_INVALID_ARG
+
+
+def test_noalloc_rejects_sizes_beyond_its_scratch_on_the_host():
+    """moe_align_permute_noalloc checks the size of its fixed scratch before any CUDA call: 255 tiles
+    of 8192 slots with 1024 local experts fit the 1 MiB array, 256 tiles do not."""
+    lib = B.load_library()
+    buf = (ctypes.c_int32 * 16)()
+    p = ctypes.addressof(buf)  # never dereferenced: every call below is rejected on the host
+    f = lib.moe_align_permute_noalloc
+    assert f(p, 522241, 4, 1024, N, 1024, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED
+    assert f(p, 1 << 18, 4, 1024, N, 1024, 64, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED
+    assert f(p, 4, 4, 2048, N, 2048, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED  # E_local > 1024
+    assert f(p, 4, 4, 8, N, 4, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_INVALID_ARG  # identity map, E_local != E

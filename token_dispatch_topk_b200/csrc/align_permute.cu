@@ -803,6 +803,8 @@ extern "C" moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, in
 // and per-tile expert counters) in a file-scope device array instead of a caller workspace.
 // For callers that cannot allocate device memory at all (see the header).
 // ---------------------------------------------------------------------------------------------
+#include <cuda.h>  // CUcontext and CUresult for the two driver calls below (reached through the runtime)
+
 #include <mutex>
 
 namespace {
@@ -811,25 +813,62 @@ constexpr int kNoAllocMaxDevices = 64;
 }  // namespace
 
 // Host code may not use this name as an address: it is a host-side stand-in.  The device address
-// comes from cudaGetSymbolAddress, fetched once per device below.
+// comes from cudaGetSymbolAddress, looked up once per CUDA context below.
 static __device__ __align__(256) unsigned char g_align_noalloc_scratch[kNoAllocScratchBytes];
 
 namespace {
-std::mutex g_noalloc_mutex;
-void* g_noalloc_scratch_addr[kNoAllocMaxDevices] = {};
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of the scratch array on the current device (looked up on first use).
+std::mutex g_noalloc_mutex;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+struct NoAllocSlot {
+  unsigned long long ctx_id;  // the context the address belongs to (ids are unique within a process)
+  void* addr;
+};
+NoAllocSlot g_noalloc_slot[kNoAllocMaxDevices] = {};
+
+// Unique id of the context current on this thread (the device's primary context once the runtime
+// has made it current).  Caller holds g_noalloc_mutex.
+moe_status_t current_context_id(unsigned long long* id) {
+  if (g_ctx_get_current == nullptr || g_ctx_get_id == nullptr) {
+    void* f1 = nullptr;
+    void* f2 = nullptr;
+    cudaDriverEntryPointQueryResult q1 = cudaDriverEntryPointSymbolNotFound, q2 = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPointByVersion("cuCtxGetCurrent", &f1, 12000, cudaEnableDefault, &q1) != cudaSuccess ||
+        cudaGetDriverEntryPointByVersion("cuCtxGetId", &f2, 12000, cudaEnableDefault, &q2) != cudaSuccess ||
+        q1 != cudaDriverEntryPointSuccess || q2 != cudaDriverEntryPointSuccess || f1 == nullptr || f2 == nullptr)
+      return MOE_ERR_CUDA;
+    g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(f1);
+    g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(f2);
+  }
+  CUcontext ctx = nullptr;
+  if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return MOE_ERR_CUDA;
+  return g_ctx_get_id(ctx, id) == CUDA_SUCCESS ? MOE_OK : MOE_ERR_CUDA;
+}
+
+// Device address of the scratch array in the current device's context.  Looked up with
+// cudaGetSymbolAddress on the first call in each context and cached under the context's id, so
+// that a reset device (a new primary context, where the module and the array may sit elsewhere)
+// gets a fresh lookup instead of a stale address.
 moe_status_t noalloc_scratch(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
   if (dev < 0 || dev >= kNoAllocMaxDevices) return MOE_ERR_UNSUPPORTED;
+  if (cudaSetDevice(dev) != cudaSuccess) return MOE_ERR_CUDA;  // the device's primary context, current here
   std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-  if (g_noalloc_scratch_addr[dev] == nullptr) {
+  unsigned long long id = 0;
+  const moe_status_t s = current_context_id(&id);
+  if (s != MOE_OK) return s;
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  if (slot.addr == nullptr || slot.ctx_id != id) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_align_noalloc_scratch) != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-    g_noalloc_scratch_addr[dev] = p;
+    slot.ctx_id = id;
+    slot.addr = p;
   }
-  *out = g_noalloc_scratch_addr[dev];
+  *out = slot.addr;
   return MOE_OK;
 }
 }  // namespace
