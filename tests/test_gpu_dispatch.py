@@ -139,7 +139,7 @@ def test_dispatch_matches_stage_entry_points(workload):
     row on the prefill workload, lanes per row on the non-power-of-2 and skewed ones)."""
     dev = require_gpu()
     wl = I.WORKLOADS[workload]
-    logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)
+    logits, hidden = I.make_logits(wl, device=dev), I.make_hidden(wl, device=dev)
     a = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, logits_dtype=logits.dtype, device=dev)
     b = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, logits_dtype=logits.dtype, device=dev)
     a.dispatch(logits, hidden)

@@ -1,10 +1,12 @@
 """End-to-end GPU parity on the five routing workloads, at their full sizes, through
 MoeRouter.step (the four C-ABI calls the bench times) against the CPU oracle pipeline.
 
-The tiny, prefill, decode and non-power-of-2 workloads are compared in full.  The
-skewed 65 536-token workload (about 17 GB on the device) is compared in full for gating
-and align, and on sampled rows for gather and combine: the oracle computes those rows one
-by one from the same inputs, the expert outputs being read back for the sampled rows only.
+Every workload is compared in full.  The skewed 65 536-token workload (about 17 GB on the
+device) is compared in chunks: every gathered row below N_pad against the oracle's gather of
+that chunk's slot ids, and every combined token against the oracle's combine of that chunk of
+tokens, the expert-output rows they read being copied back from the device.  The large inputs
+are generated on the device by the counter-based generator (the same bits as on the host, which
+tests/test_gpu_inputs.py checks) and copied back for the oracle.
 """
 import numpy as np
 import pytest
@@ -73,10 +75,10 @@ def test_workload_full_size(name, path):
     dev = require_gpu()
     wl = I.WORKLOADS[name]
     logits = I.make_logits(wl)
-    hidden = I.make_hidden(wl)
-    y = I.make_expert_out(wl.capacity, wl.H)
+    hidden = I.make_hidden(wl, device=dev).cpu()
+    yd = I.make_expert_out(wl.capacity, wl.H, device=dev)
+    y = yd.cpu()
     r = _router(wl, dev)
-    yd = y.to(dev)
     _run(r, path, logits.to(dev), hidden.to(dev), yd)
     torch.cuda.synchronize()
     ref = _oracle_pipeline(wl, logits, bf16_bits(hidden), bf16_bits(y))
@@ -124,48 +126,57 @@ def test_ep_decode_every_route_pattern(path):
 
 
 @pytest.mark.parametrize("path", ["fused", "staged"])
-def test_skewed_prefill_full_size_sampled(path):
+def test_skewed_prefill_full_size(path):
     dev = require_gpu()
     wl = I.WORKLOADS["zipf_prefill_T65536_E256_k8_H7168"]
+    T, k, H = wl.T, wl.k, wl.H
     logits = I.make_logits(wl)
-    hidden = I.make_hidden(wl)
+    hidden_d = I.make_hidden(wl, device=dev)
     y_dev = I.make_expert_out(wl.capacity, wl.H, device=dev)
     r = _router(wl, dev)
-    _run(r, path, logits.to(dev), hidden.to(dev), y_dev)
+    _run(r, path, logits.to(dev), hidden_d, y_dev)
     torch.cuda.synchronize()
+    assert r.device_status() == tdt.MOE_OK
     # gating and align in full
-    w_ref, ids_ref = oracle.topk_softmax(logits_for_oracle(logits), wl.k, wl.renormalize)
+    w_ref, ids_ref = oracle.topk_softmax(logits_for_oracle(logits), k, wl.renormalize)
     assert np.array_equal(np_i32(r.topk_ids), ids_ref)
     assert np.abs(r.topk_weights.cpu().numpy() - w_ref).max() <= TOPK_WEIGHT_ATOL
     al = oracle.align_permute(ids_ref, wl.E, wl.block_size)
     assert_align_equal(r.align, al, "skewed")
     counts = al["counts"]
     assert counts.max() > 8 * counts.mean()  # the Zipf bias makes a few experts hot
-    # gather: sampled rows, each recomputed by the oracle from its slot id
-    rng = np.random.default_rng(0)
+    # gather: every row below N_pad, chunk by chunk, against the oracle's gather of the chunk's slot ids
+    hidden_bits = bf16_bits(hidden_d)
     npad = int(al["num_tokens_post_pad"][0])
-    rows = np.unique(np.concatenate([rng.integers(0, npad, 512), [0, npad - 1]]))
-    sti = al["sorted_token_ids"][rows]
-    want = oracle.gather(bf16_bits(hidden), wl.k, sti, len(rows), len(rows))
-    got = bf16_bits(r.permuted[torch.from_numpy(rows).to(dev)])
-    real = sti != wl.T * wl.k
-    assert np.array_equal(got[real], want[real])
-    # combine: sampled tokens; the expert-output rows they read are copied back
-    toks = np.unique(np.concatenate([rng.integers(0, wl.T, 256), [0, wl.T - 1]]))
-    inv = al["inv_perm"].reshape(wl.T, wl.k)[toks]
-    used = np.unique(inv[inv >= 0])
-    y_rows = bf16_bits(y_dev[torch.from_numpy(used).long().to(dev)])
-    remap = np.full(wl.capacity, -1, np.int64)
-    remap[used] = np.arange(len(used))
-    inv_c = np.where(inv >= 0, remap[np.maximum(inv, 0)], -1).astype(np.int32).reshape(-1)
-    want = oracle.combine(y_rows, w_ref[toks], inv_c)
-    got = bf16_bits(r.out[torch.from_numpy(toks).long().to(dev)])
-    assert_combine_within_weight_tolerance(got, want, y_rows, inv_c, wl.k, "skewed sampled")
-    # the same tokens combined on the device from the oracle's weights: within 1 bf16 ulp
-    w_full = torch.from_numpy(w_ref).to(dev)
-    out2 = tdt.moe_combine(y_dev, w_full, r.align.inv_perm)
-    got2 = bf16_bits(out2[torch.from_numpy(toks).long().to(dev)])
-    assert ulp_distance_bf16(got2, want).max() <= COMBINE_MAX_ULP
+    rows_per_chunk = 1 << 15
+    for p0 in range(0, npad, rows_per_chunk):
+        p1 = min(npad, p0 + rows_per_chunk)
+        sti = al["sorted_token_ids"][p0:p1]
+        want = oracle.gather(hidden_bits, k, sti, p1 - p0, p1 - p0)
+        got = bf16_bits(r.permuted[p0:p1])
+        real = sti != T * k
+        assert np.array_equal(got[real], want[real]), f"gathered rows {p0}..{p1}"
+    del hidden_bits
+    # combine: every token, chunk by chunk; the expert-output rows a chunk reads are copied back
+    out2 = tdt.moe_combine(y_dev, torch.from_numpy(w_ref).to(dev), r.align.inv_perm)
+    torch.cuda.synchronize()
+    inv = al["inv_perm"].reshape(T, k)
+    toks_per_chunk = 2048
+    for t0 in range(0, T, toks_per_chunk):
+        t1 = min(T, t0 + toks_per_chunk)
+        inv_c = inv[t0:t1]
+        used = np.unique(inv_c[inv_c >= 0])
+        y_rows = bf16_bits(y_dev[torch.from_numpy(used).long().to(dev)])
+        remap = np.full(wl.capacity, -1, np.int64)
+        remap[used] = np.arange(len(used))
+        inv_r = np.where(inv_c >= 0, remap[np.maximum(inv_c, 0)], -1).astype(np.int32).reshape(-1)
+        want = oracle.combine(y_rows, w_ref[t0:t1], inv_r)
+        # the step's combine used the GPU gating weights: the propagated weight tolerance
+        assert_combine_within_weight_tolerance(bf16_bits(r.out[t0:t1]), want, y_rows, inv_r, k,
+                                               f"skewed tokens {t0}..{t1}")
+        # the combine on the oracle's weights: within 1 bf16 ulp
+        d = ulp_distance_bf16(bf16_bits(out2[t0:t1]), want)
+        assert d.max() <= COMBINE_MAX_ULP, (t0, d.max())
 
 
 @pytest.mark.parametrize("name", ["qwen3moe_prefill_T4096_E128_k8", "ep_decode_T2_E160_local40_k6"])
@@ -173,7 +184,7 @@ def test_repeat_steps_are_bit_identical(name):
     """Repeated steps, alternating the staged and the fused dispatch, give the same bits."""
     dev = require_gpu()
     wl = I.WORKLOADS[name]
-    logits, hidden = I.make_logits(wl).to(dev), I.make_hidden(wl).to(dev)
+    logits, hidden = I.make_logits(wl, device=dev), I.make_hidden(wl, device=dev)
     y = I.make_expert_out(wl.capacity, wl.H, device=dev)
     r = _router(wl, dev)
     first = None
@@ -212,3 +223,29 @@ def test_zero_tokens():
     torch.cuda.synchronize()
     ref = oracle.align_permute(np.zeros((0, 4), np.int32), 16, 8)
     assert_align_equal(r.align, ref, "T=0")
+
+
+@pytest.mark.parametrize("name", ["tiny_T64_E8_k2", "qwen3moe_prefill_T4096_E128_k8"])
+def test_host_step_pipeline_matches_serial_steps(name):
+    """The double-buffered end-to-end path: five steps with different inputs in flight together give, for
+    each step, the bits of the same step run alone, and step 0 matches the oracle."""
+    dev = require_gpu()
+    wl = I.WORKLOADS[name]
+    y = I.make_expert_out(wl.capacity, wl.H, device=dev)
+    ins = [(I.make_logits(wl, seed=s).pin_memory(), I.make_hidden(wl, seed=s).pin_memory()) for s in range(5)]
+    outs = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in range(5)]
+    r = _router(wl, dev)
+    pipe = tdt.HostStepPipeline(r, expert_out=y)
+    for (lg, hd), o in zip(ins, outs):
+        pipe.submit(lg, hd, o)
+    pipe.synchronize()
+    assert r.device_status() == tdt.MOE_OK
+    solo = _router(wl, dev)
+    for (lg, hd), o in zip(ins, outs):
+        want = solo.step(lg.to(dev), hd.to(dev), y)
+        torch.cuda.synchronize()
+        assert torch.equal(o, want.cpu())
+    lg, hd = ins[0]
+    ref = _oracle_pipeline(wl, lg, bf16_bits(hd), bf16_bits(y))
+    assert_combine_within_weight_tolerance(bf16_bits(outs[0]), ref[4], bf16_bits(y), ref[2]["inv_perm"], wl.k,
+                                           "pipelined step 0")
