@@ -5,8 +5,10 @@
 
 One step = MoeRouter.step over one batch: moe_route_dispatch (gating + align + permute-gather:
 three kernels, or one for decode-sized batches) -> moe_combine (the stand-in expert outputs replace
-the expert MLPs between gather and combine), replayed as one CUDA graph.  The decode workload also
-times every injected route pattern (routes given by the caller).  Inputs are resident in HBM.
+the expert MLPs between gather and combine), replayed as one CUDA graph.  Inputs are resident in HBM.
+The headline is the largest workload (65536 tokens, 256 experts, top-8, hidden 7168, Zipf-skewed
+routing); the same run also times the prefill, non-power-of-2 and decode workloads and reports them
+under ``workloads`` (the decode workload: every route pattern, the worst one reported).
 When one step moves more bytes than L2 holds (the prefill workloads), the K steps are replayed
 back to back between one pair of CUDA events on the launching stream; otherwise L2 is flushed (a
 256 MiB write, then a 256 MiB read, so no dirty flush lines are written back inside a timed step)
@@ -19,8 +21,9 @@ Also reported: per-stage device times and achieved HBM bandwidth from the algori
 the step's path and for the four stage entry points),
 the roofline of the dominant kernel against the measured copy peak, an end-to-end figure
 through MoeRouter.step_from_host (pinned host inputs copied in and the output copied back
-inside the timed region), SM clocks sampled during the timed region, and the CPU oracle
-timed on this host as a baseline.  ``--impl reference`` times the CPU oracle alone.
+inside the timed region, double-buffered over two streams), SM clocks sampled while the workload
+is measured, and the CPU oracle timed on this host as a baseline (per stage and in total).
+``--impl reference`` times the CPU oracle alone.
 """
 from __future__ import annotations
 
@@ -66,7 +69,9 @@ def parse_args():
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
     p.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    p.add_argument("--workload", default=None, help="workload name (default: the Qwen3-MoE-like prefill)")
+    p.add_argument("--workload", default=None,
+                   help="workload name (default: the skewed 65536-token prefill, with the other workloads as sub-records)")
+    p.add_argument("--no-sub-workloads", action="store_true", help="time the headline workload only")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-graph", action="store_true", help="launch the calls directly instead of a graph")
     p.add_argument("--flush-always", action="store_true",
@@ -173,27 +178,49 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle leg --
-def oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, t0: int, n: int):
-    """The oracle pipeline on tokens [t0, t0+n) of the workload (gate, align, gather, combine)."""
+ORACLE_STAGES = ("topk", "align", "gather", "combine")
+
+
+def oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, t0: int, n: int, times=None):
+    """The oracle pipeline on tokens [t0, t0+n) of the workload (gate, align, gather, combine);
+    appends each stage's wall time (s) to ``times[stage]`` when given."""
+    clk = time.perf_counter
+    a = clk()
     w, ids = oracle_mod.topk_softmax(logits_np[t0:t0 + n], wl.k, wl.renormalize)
+    b = clk()
     al = oracle_mod.align_permute(ids, wl.E, wl.block_size, emap_np, wl.experts_local)
+    c = clk()
     npad = int(al["num_tokens_post_pad"][0])
     oracle_mod.gather(hidden_bits[t0:t0 + n], wl.k, al["sorted_token_ids"], npad, al["capacity"])
+    d = clk()
     oracle_mod.combine(y_bits[:al["capacity"]], w, al["inv_perm"])
+    e = clk()
+    if times is not None:
+        for name, dt in zip(ORACLE_STAGES, (b - a, c - b, d - c, e - d)):
+            times[name].append(dt)
     return n
 
 
+def oracle_sample_tokens(wl) -> int:
+    """Tokens of the workload in one oracle pass of the CPU baseline (a few seconds of CPU work)."""
+    return min(wl.T, 2048 if wl.H > 4096 else 4096)
+
+
 def host_inputs_numpy(wl, seed: int, T_max: int):
+    """The first T_max tokens of the workload as numpy arrays for the oracle (bf16 as uint16 bits).
+    The counter-based generator gives the same bits on any device; the large buffers are generated on
+    the GPU when there is one (faster) and copied to the host."""
     import numpy as np
     import torch
     from token_dispatch_topk_b200 import inputs as I
+    gen = "cuda" if torch.cuda.is_available() else "cpu"
     T = min(wl.T, T_max)
     logits = I.make_logits(wl, seed=seed, T=T)
     logits_np = logits.view(torch.int16).numpy().view(np.uint16) if logits.dtype == torch.bfloat16 else logits.numpy()
-    hidden = I.make_hidden(wl, seed=seed, T=T)
+    hidden = I.make_hidden(wl, seed=seed, T=T, device=gen).cpu()
     hidden_bits = hidden.view(torch.int16).numpy().view(np.uint16)
     cap = T * wl.k + wl.experts_local * (wl.block_size - 1)
-    y = I.make_expert_out(cap, wl.H, seed=seed)
+    y = I.make_expert_out(cap, wl.H, seed=seed, device=gen).cpu()
     y_bits = y.view(torch.int16).numpy().view(np.uint16)
     emap = I.expert_map(wl)
     return logits_np, hidden_bits, y_bits, None if emap is None else emap.numpy()
@@ -213,22 +240,26 @@ def host_cpu() -> dict:
     return {"model": model, "logical_cores": os.cpu_count()}
 
 
-def cpu_oracle_rate(wl, seed: int, budget_s: float, T_max: int = 4096):
-    """Tokens/s of the oracle on this host over a bounded sample (single-threaded)."""
+def cpu_oracle_rate(wl, seed: int, budget_s: float, runs: int = 5):
+    """Tokens/s of the oracle on this host (single-threaded) over a bounded token sample: the median
+    over up to `runs` passes (fewer when the budget runs out), per stage and in total."""
     import oracle as oracle_mod
     oracle_mod.default()
-    logits_np, hidden_bits, y_bits, emap_np = host_inputs_numpy(wl, seed, T_max)
+    logits_np, hidden_bits, y_bits, emap_np = host_inputs_numpy(wl, seed, oracle_sample_tokens(wl))
     T = logits_np.shape[0]
-    done, reps = 0, 0
+    times = {s: [] for s in ORACLE_STAGES}
     t_start = time.perf_counter()
-    while True:
-        done += oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, T)
-        reps += 1
-        el = time.perf_counter() - t_start
-        if el >= budget_s or reps >= 1000:
+    passes = 0
+    while passes < runs:
+        oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, T, times)
+        passes += 1
+        if time.perf_counter() - t_start >= budget_s:
             break
-    return {"value": done / el, "unit": UNIT, "cores": 1, "kind": "oracle",
-            "sample": f"{reps} oracle passes over the first {T} tokens of the workload ({el:.1f} s, single thread)",
+    per_stage = {s: statistics.median(v) for s, v in times.items()}
+    total = statistics.median([sum(times[s][i] for s in ORACLE_STAGES) for i in range(passes)])
+    return {"value": T / total, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"the first {T} tokens of the workload, median of {passes} oracle passes, single thread",
+            "per_stage_ms": {s: 1e3 * v for s, v in per_stage.items()}, "total_ms": 1e3 * total,
             "host": host_cpu()}
 
 
@@ -242,7 +273,7 @@ def run_reference(args, wl):
     steps, warm = args.steps, args.warmup
     # calibrate the per-step sample so that warmup + steps fit the time budget
     T_cal = min(wl.T, 64)
-    logits_np, hidden_bits, y_bits, emap_np = host_inputs_numpy(wl, args.seed, min(wl.T, 4096))
+    logits_np, hidden_bits, y_bits, emap_np = host_inputs_numpy(wl, args.seed, oracle_sample_tokens(wl))
     t = time.perf_counter()
     oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, T_cal)
     per_token = max((time.perf_counter() - t) / T_cal, 1e-7)
@@ -250,10 +281,11 @@ def run_reference(args, wl):
     n = int(max(1, min(logits_np.shape[0], per_step_budget / per_token)))
     for i in range(warm):
         oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, 0, n)
+    times = {s: [] for s in ORACLE_STAGES}
     t = time.perf_counter()
     for i in range(steps):
         t0 = (i * n) % max(1, logits_np.shape[0] - n + 1)
-        oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, t0, n)
+        oracle_pass(oracle_mod, wl, logits_np, hidden_bits, y_bits, emap_np, t0, n, times)
     el = time.perf_counter() - t
     value = steps * n / el
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": steps,
@@ -262,6 +294,7 @@ def run_reference(args, wl):
             "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"}},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
                              "sample": f"{n} tokens of the workload per step, single-threaded C++ oracle",
+                             "per_stage_ms": {s: 1e3 * statistics.median(v) for s, v in times.items()},
                              "host": host_cpu()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -269,68 +302,95 @@ def run_reference(args, wl):
 
 
 # ------------------------------------------------------------------------ GPU leg --
-def main():
-    args = parse_args()
-    from token_dispatch_topk_b200 import inputs as I
-    wl = I.WORKLOADS[args.workload or I.DEFAULT_WORKLOAD]
-    if args.impl == "reference":
-        return run_reference(args, wl)
+class Ctx:
+    """What every workload measurement shares: the device, stream, L2 flush buffers, rank info."""
 
+    def __init__(self, args, dev, ws, rank):
+        import torch
+        self.args, self.dev, self.ws, self.rank = args, dev, ws, rank
+        self.stream = torch.cuda.Stream(device=dev)
+        self.flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+        self.flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
+        self.l2_bytes = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20))
+        self.sms = torch.cuda.get_device_properties(dev).multi_processor_count
+        self.uuid = None
+        try:
+            self.uuid = str(torch.cuda.get_device_properties(dev).uuid)
+        except Exception:
+            pass
+
+    def flush(self, i=0):
+        # write a buffer larger than L2, then read another one: L2 is left holding only clean
+        # lines of a buffer the step never touches, so no flush write-back lands in a timed step
+        self.flush_buf.fill_(i & 0xFF)
+        self.flush_read.max()
+
+
+def stage_kernels(wl, r, sms: int) -> dict:
+    """The kernels each entry point launches for this workload (the library's selection rules; the
+    lane-gating rule is moe_gate::lane_gating_fits in csrc/gate_lane.cuh)."""
+    sk = dict(STAGE_KERNEL)
+    elem = 2 if wl.logits_dtype == "bf16" else 4
+    lanes = wl.k <= 8 and (wl.E * elem) % 16 == 0 and (
+        (wl.E <= 64 and wl.T >= 1024) or (elem == 2 and wl.E <= 256 and wl.T >= 16384))
+    if r.small_batch:
+        sk["dispatch"] = "route_small_kernel"
+    elif lanes:
+        sk["dispatch"] = "gate_count_lanes_kernel+tile_scan_kernel+place_gather_kernel"
+    if lanes:
+        sk["topk"] = "topk_lane_kernel"
+    P = wl.T * wl.k
+    if 4096 < P <= 65536:  # the fused path's tile kernels, placement only
+        sk["align"] = "gate_count_kernel+tile_scan_kernel+place_gather_kernel<false>"
+    elif P > 65536 or wl.experts_local > 512:  # beyond one cluster: the two-kernel align
+        sk["align"] = "align_count_kernel+align_place_kernel"
+    if wl.T * (-(-wl.H * 2 // 4096)) < sms:  # fewer 4 KB row chunks than SMs: the small-batch combine
+        sk["combine"] = "combine_small_kernel"
+    return sk
+
+
+def measure_workload(wl, ctx: Ctx, headline: bool) -> dict:
+    """Time one workload's step on this rank's GPU; the headline also gets e2e, clocks and the CPU baseline."""
     import torch
-    import torch.distributed as dist
     import token_dispatch_topk_b200 as tdt
+    from token_dispatch_topk_b200 import inputs as I
     from token_dispatch_topk_b200.dist import max_over_ranks, rank_seed
 
-    ws, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if ws > 1:
-        from datetime import timedelta
-        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    args, dev, stream, ws, rank = ctx.args, ctx.dev, ctx.stream, ctx.ws, ctx.rank
     seed = rank_seed(args.seed, rank)  # an independent batch per rank
-    tdt.load_library()
-
-    # ---- inputs resident in HBM
-    logits_h = I.make_logits(wl, seed=seed)
-    hidden_h = I.make_hidden(wl, seed=seed)
-    logits = logits_h.to(dev)
-    hidden = hidden_h.to(dev)
+    # ---- inputs resident in HBM (counter-based generator: the same bits as on the host)
+    logits = I.make_logits(wl, seed=seed, device=dev)
+    hidden = I.make_hidden(wl, seed=seed, device=dev)
     y = I.make_expert_out(wl.capacity, wl.H, seed=seed, device=dev)
     r = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, E_local=wl.E_local,
                       expert_map=I.expert_map(wl), logits_dtype=logits.dtype, device=dev)
-    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
-    flush_read = torch.ones(L2_FLUSH_BYTES // 4, dtype=torch.int32, device=dev)
-
-    def flush(i=0):
-        # write a buffer larger than L2, then read another one: L2 is left holding only clean
-        # lines of a buffer the step never touches, so no flush write-back lands in a timed step
-        flush_buf.fill_(i & 0xFF)
-        flush_read.max()
-
-    stream = torch.cuda.Stream(device=dev)
+    flush = ctx.flush
+    sampler = ClockSampler(ctx.uuid) if (rank == 0 and headline) else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.4)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
         for _ in range(3):
             r.step(logits, hidden, y)
     stream.synchronize()
     if r.device_status() != tdt.MOE_OK:
-        raise RuntimeError("device status after warm-up steps is not MOE_OK")
+        raise RuntimeError(f"{wl.name}: device status after warm-up steps is not MOE_OK")
     R = int(r.align.counts.sum().item())
     npad = int(r.align.num_tokens_post_pad.item())
     NB = r.align.expert_ids.numel()
-    if r.small_batch:
-        launches_per_step = 2  # route_small_kernel, combine_small_kernel
-    else:
-        launches_per_step = 4  # gate_count_kernel, tile_scan_kernel, place_gather_kernel, combine kernel
+    launches_per_step = 2 if r.small_batch else 4  # route_small + combine_small, or gate_count, tile_scan, place_gather, combine
 
     use_graph = not args.no_graph
     graphs = {}
+
+    def capture(fn):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            fn()
+        return g
+
     if use_graph:
-        def capture(fn):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                fn()
-            return g
         graphs["step"] = capture(lambda: r.step(logits, hidden, y))
     stage_fns = {"step": lambda: r.step(logits, hidden, y)}
 
@@ -339,6 +399,8 @@ def main():
             graphs[name].replay()
         else:
             stage_fns[name]()
+
+    step_samples = {}
 
     def timed(name, iters, warm):
         """Sum of per-iteration event times (ms), L2 flushed before each iteration."""
@@ -357,8 +419,6 @@ def main():
         step_samples[name] = per_step
         return sum(per_step)
 
-    step_samples = {}
-
     def timed_back_to_back(name, iters, warm):
         """Time (ms) of `iters` steps replayed back to back between one pair of events (no flush:
         used when one step's bytes exceed L2, so no step finds its inputs left there by the last)."""
@@ -376,28 +436,20 @@ def main():
 
     abytes = algorithmic_bytes(wl, R, r.capacity, NB)
     step_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
-    l2_bytes = int(getattr(torch.cuda.get_device_properties(dev), "L2_cache_size", 0) or (126 << 20))
-    back_to_back = step_bytes > l2_bytes and not args.flush_always
+    back_to_back = step_bytes > ctx.l2_bytes and not args.flush_always
 
     # ---- the timed region: K steps
-    uuid = None
-    try:
-        uuid = str(torch.cuda.get_device_properties(dev).uuid)
-    except Exception:
-        pass
-    sampler = ClockSampler(uuid) if rank == 0 else None
     if ws > 1:
+        import torch.distributed as dist
         dist.barrier()
     torch.cuda.synchronize()
-    if sampler:
-        sampler.start()
-        time.sleep(0.4)
+    t_region = time.perf_counter()
     if back_to_back:
         total_ms = timed_back_to_back("step", args.steps, args.warmup)
     else:
         total_ms = timed("step", args.steps, args.warmup)
     torch.cuda.synchronize()
-    clocks = sampler.stop() if sampler else None
+    t_region = time.perf_counter() - t_region
     total_ms = max_over_ranks(total_ms, dev)
     if ws > 1:
         dist.barrier()
@@ -419,27 +471,7 @@ def main():
     peak, peak_src = measured_peaks()
     abytes["dispatch"] = abytes["topk"] + abytes["align"] + abytes["gather"]
     st_iters = args.stage_steps or min(args.steps, 500)
-
-    stage_kernel = dict(STAGE_KERNEL)
-    # the kernels each entry point launches for this workload (the library's selection rules; the
-    # lane-gating rule is moe_gate::lane_gating_fits in csrc/gate_lane.cuh)
-    elem = 2 if wl.logits_dtype == "bf16" else 4
-    lanes = wl.k <= 8 and (wl.E * elem) % 16 == 0 and (
-        (wl.E <= 64 and wl.T >= 1024) or (elem == 2 and wl.E <= 256 and wl.T >= 16384))
-    if r.small_batch:
-        stage_kernel["dispatch"] = "route_small_kernel"
-    elif lanes:
-        stage_kernel["dispatch"] = "gate_count_lanes_kernel+tile_scan_kernel+place_gather_kernel"
-    if lanes:
-        stage_kernel["topk"] = "topk_lane_kernel"
-    P = wl.T * wl.k
-    if 4096 < P <= 65536:  # the fused path's tile kernels, placement only
-        stage_kernel["align"] = "gate_count_kernel+tile_scan_kernel+place_gather_kernel<false>"
-    elif P > 65536 or wl.experts_local > 512:  # beyond one cluster: the two-kernel align
-        stage_kernel["align"] = "align_count_kernel+align_place_kernel"
-    sms = torch.cuda.get_device_properties(dev).multi_processor_count
-    if wl.T * (-(-wl.H * 2 // 4096)) < sms:  # fewer 4 KB row chunks than SMs: the small-batch combine
-        stage_kernel["combine"] = "combine_small_kernel"
+    stage_kernel = stage_kernels(wl, r, ctx.sms)
 
     def stage_times(names, calls):
         marks = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(len(names) + 1)]
@@ -451,9 +483,7 @@ def main():
                 marks[i + 1].record()
 
         if use_graph:
-            g_inst = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_inst, stream=stream):
-                instrumented()
+            g_inst = capture(instrumented)
         sums = [0.0] * len(names)
         warm = min(args.warmup, 10)
         with torch.cuda.stream(stream):
@@ -477,21 +507,15 @@ def main():
                          "timing": "CUDA events between the stages of the step graph"}
         return out
 
-    stages = stage_times(("topk", "align", "gather", "combine"),
-                         [lambda: r.gate(logits), lambda: r.align_permute(),
-                          lambda: r.gather(hidden, hidden_ready=True), lambda: r.combine(y)])
+    stages = stage_times(ORACLE_STAGES, [lambda: r.gate(logits), lambda: r.align_permute(),
+                                         lambda: r.gather(hidden, hidden_ready=True), lambda: r.combine(y)])
     stages_fused = stage_times(("dispatch", "combine"), [lambda: r.dispatch(logits, hidden), lambda: r.combine(y)])
+
     # the dominant single kernel of the step: the combine (about half of the bytes) above the
     # small-batch limits; for small batches the longer of the step's two kernels.  Its launch time
     # is measured without the per-step event floor: a graph of n x [L2 flush, launch] minus a graph
     # of n x [L2 flush], both replayed between one pair of events on the launching stream.
     def launch_us(fn, n=20, reps=5):
-        def cap(body):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                body()
-            return g
-
         def both():
             for i in range(n):
                 flush(i)
@@ -501,7 +525,7 @@ def main():
             for i in range(n):
                 flush(i)
 
-        ga, gb = cap(both), cap(flush_only)
+        ga, gb = capture(both), capture(flush_only)
         res = []
         with torch.cuda.stream(stream):
             for g in (ga, gb):
@@ -519,14 +543,10 @@ def main():
         return 1e3 * (res[0] - res[1]) / n
 
     in_step = stages_fused
-    if r.small_batch:
-        dom = max(in_step, key=lambda n: in_step[n]["us"])
-    else:
-        dom = "combine"
+    dom = max(in_step, key=lambda n: in_step[n]["us"]) if r.small_batch else "combine"
     dom_fn = (lambda: r.combine(y)) if dom == "combine" else (lambda: r.dispatch(logits, hidden))
     dom_us = launch_us(dom_fn)
     ach = abytes[dom] / (dom_us * 1e-6) / 1e9
-    total_bytes = abytes["topk"] + abytes["align"] + abytes["gather"] + abytes["combine"]
     roofline = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
                 "traffic": ncu_traffic(stage_kernel[dom], wl.name), "kernel": stage_kernel[dom],
                 "peak_source": peak_src, "launch_us": dom_us,
@@ -538,7 +558,7 @@ def main():
     patterns = None
     if wl.name.startswith("ep_decode"):
         w_inj = I.decode_pattern_weights(seed=seed).to(dev)
-        patterns, device = {}, {}
+        pat_us, device = {}, {}
         for pname in I.DECODE_PATTERNS:
             ids_p = I.decode_pattern_ids(pname).to(dev)
             fn = (lambda ids_p=ids_p: r.step_routes(ids_p, w_inj, hidden, y))
@@ -546,76 +566,146 @@ def main():
                 graphs["pattern"] = capture(fn)
             stage_fns["pattern"] = fn
             n_it = min(args.steps, 500)
-            patterns[pname] = 1e3 * timed("pattern", n_it, min(args.warmup, 10)) / n_it
+            pat_us[pname] = 1e3 * timed("pattern", n_it, min(args.warmup, 10)) / n_it
             device[pname] = launch_us(fn)
         device["logits"] = launch_us(lambda: r.step(logits, hidden, y))
-        patterns = {"us_per_step": patterns, "worst_us": max(patterns.values()),
-                    "worst": max(patterns, key=patterns.get),
+        patterns = {"us_per_step": pat_us, "worst_us": max(pat_us.values()),
+                    "worst": max(pat_us, key=pat_us.get),
                     "device_us_per_step": device, "device_worst_us": max(device.values()),
+                    "device_worst": max(device, key=device.get),
                     "device_timing": "graph of 20 x [L2 flush, step] minus graph of 20 x [L2 flush], per step "
                                      "(kernels and the gaps between them, without the per-step event latency)",
                     "path": "MoeRouter.step_routes: moe_route_dispatch (given routes) + moe_combine, one graph each"}
         if r.device_status() != tdt.MOE_OK:
             raise RuntimeError("device status after the route-pattern steps is not MOE_OK")
 
-    # ---- end to end through the public API, from pinned host buffers
-    e2e_steps = args.e2e_steps or min(args.steps, 200)
-    lp, hp = logits_h.pin_memory(), hidden_h.pin_memory()
-    out_h = torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory()
-    with torch.cuda.stream(stream):
-        for _ in range(3):
-            r.step_from_host(lp, hp, y, out_h, stream)
-        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(e2e_steps)]
-        for a, b in evs:
-            a.record(stream)
-            r.step_from_host(lp, hp, y, out_h, stream)
-            b.record(stream)
-    stream.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in evs)
-    e2e_ms = max_over_ranks(e2e_ms, dev)
-    h2d = lp.numel() * lp.element_size() + hp.numel() * hp.element_size()
-    d2h = out_h.numel() * out_h.element_size()
-    e2e = {"value": ws * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h, "steps": e2e_steps,
-           "api": "MoeRouter.step_from_host (pinned H2D of logits+hidden, moe_route_dispatch + moe_combine, "
-                  "D2H of out)"}
+    total_bytes = step_bytes
+    rec = {
+        "workload": wl.name, "T": wl.T, "E": wl.E, "E_local": wl.experts_local, "k": wl.k, "H": wl.H,
+        "value": value, "unit": UNIT, "ms_per_step": ms_per_step,
+        "achieved_hbm_gbs": total_bytes / (ms_per_step * 1e-3) / 1e9,
+        "algorithmic_bytes_per_step": total_bytes,
+        "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
+        "hbm_frac_of_measured_peak": total_bytes / (ms_per_step * 1e-3) / 1e9 / peak,
+        "routed_slots_local": R, "num_tokens_post_pad": npad,
+        "l2": (f"not flushed: steps replayed back to back, each moving {step_bytes / 2**20:.0f} MiB "
+               f"> L2 ({ctx.l2_bytes >> 20} MiB)") if back_to_back else
+              (f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write + "
+               f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)"),
+        "flushed_ms_per_step": flushed_ms_per_step, "flushed_step_us_percentiles": flushed_pct_us,
+        "step_path": "moe_route_dispatch (single kernel) + moe_combine" if r.small_batch else
+                     "moe_route_dispatch (three kernels) + moe_combine",
+        "roofline": roofline, "stages": stages_fused, "stages_four_call_path": stages,
+        "decode_route_patterns": patterns, "launches_per_step": launches_per_step,
+        "timed_region_s": t_region,
+    }
 
+    if headline:
+        # ---- end to end through the public API, from pinned host buffers (double-buffered: the next
+        # step's host->device copies and the previous step's device->host copy overlap the step)
+        e2e_steps = args.e2e_steps or min(args.steps, 200)
+        logits_h = logits.cpu().pin_memory()
+        hidden_h = hidden.cpu().pin_memory()
+        outs_h = [torch.empty((wl.T, wl.H), dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        pipe = tdt.HostStepPipeline(r, expert_out=y)
+        for i in range(3):
+            pipe.submit(logits_h, hidden_h, outs_h[i % 2])
+        pipe.synchronize()
+        e0, e1 = pipe.timed(lambda i: pipe.submit(logits_h, hidden_h, outs_h[i % 2]), e2e_steps)
+        e2e_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+        h2d = logits_h.numel() * logits_h.element_size() + hidden_h.numel() * hidden_h.element_size()
+        d2h = outs_h[0].numel() * outs_h[0].element_size()
+        rec["e2e"] = {"value": ws * wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h, "steps": e2e_steps, "ms_per_step": e2e_ms / e2e_steps,
+                      "api": "HostStepPipeline over MoeRouter (pinned H2D of logits+hidden on one copy stream, "
+                             "moe_route_dispatch + moe_combine, D2H of out on another; two buffer sets)"}
+        del pipe
+        if r.device_status() != tdt.MOE_OK:
+            raise RuntimeError("device status after the timed steps is not MOE_OK")
+        rec["clocks"] = sampler.stop() if sampler else None
+        if rec["clocks"] is not None:
+            rec["clocks"]["window"] = ("sampled every 200 ms from before the warm-up steps to the end of the "
+                                       "end-to-end steps (timed steps, per-stage and per-launch timing inside)")
+        rec["gpu_launches"] = launches_per_step * args.steps
+        if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+            rec["cpu_baseline"] = cpu_oracle_rate(wl, seed, args.cpu_seconds)
+    del graphs
     if r.device_status() != tdt.MOE_OK:
-        raise RuntimeError("device status after the timed steps is not MOE_OK")
+        raise RuntimeError(f"{wl.name}: device status at the end is not MOE_OK")
+    return rec
 
-    cpu = None
-    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
-        cpu = cpu_oracle_rate(wl, seed, args.cpu_seconds)
+
+TARGETS = {  # end-to-end targets: fraction of 8 TB/s, or device time of the worst decode route pattern
+    "qwen3moe_prefill_T4096_E128_k8": ("hbm_frac_of_8tbs", 0.70),
+    "nonpow2_T16384_E60_k4": ("hbm_frac_of_8tbs", 0.70),
+    "zipf_prefill_T65536_E256_k8_H7168": ("hbm_frac_of_8tbs", 0.70),
+    "ep_decode_T2_E160_local40_k6": ("device_worst_us", 10.0),
+}
+
+
+def target_status(rec: dict):
+    t = TARGETS.get(rec["workload"])
+    if t is None:
+        return None
+    key, bar = t
+    if key == "device_worst_us":
+        v = rec["decode_route_patterns"]["device_worst_us"]
+        return {"device_worst_us": v, "bar_us": bar, "met": v < bar}
+    return {key: rec[key], "bar": bar, "met": rec[key] >= bar}
+
+
+def main():
+    args = parse_args()
+    from token_dispatch_topk_b200 import inputs as I
+    wl = I.WORKLOADS[args.workload or I.DEFAULT_WORKLOAD]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+
+    import torch
+    import torch.distributed as dist
+    import token_dispatch_topk_b200 as tdt
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        from datetime import timedelta
+        dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
+    tdt.load_library()
+    ctx = Ctx(args, dev, ws, rank)
+
+    head = measure_workload(wl, ctx, headline=True)
+    head["target"] = target_status(head)
+    subs = []
+    if args.workload is None and not args.no_sub_workloads:
+        torch.cuda.empty_cache()
+        for name in I.BENCH_SUB_WORKLOADS:
+            rec = measure_workload(I.WORKLOADS[name], ctx, headline=False)
+            rec["target"] = target_status(rec)
+            subs.append(rec)
+            torch.cuda.empty_cache()
 
     if rank == 0:
         line = {
-            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": head["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "dtype_detail": "bf16 activations, fp32 gating math and combine accumulation, int32 indices",
-            "data": "synthetic (seeded; see token_dispatch_topk_b200/inputs.py)",
+            "data": "synthetic (seeded, counter-based; see token_dispatch_topk_b200/inputs.py)",
             "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
-                       "l2": (f"not flushed: steps replayed back to back, each moving {step_bytes / 2**20:.0f} MiB "
-                              f"> L2 ({l2_bytes >> 20} MiB)") if back_to_back else
-                             (f"flushed between timed steps ({L2_FLUSH_BYTES >> 20} MiB write + "
-                              f"{L2_FLUSH_BYTES >> 20} MiB read of another buffer)"),
-                       "cuda_graph": use_graph,
+                       "l2": head["l2"], "cuda_graph": not args.no_graph,
                        "parallelism": "one independent batch per GPU" if ws > 1 else "single GPU"},
-            "achieved_hbm_gbs": total_bytes / (ms_per_step * 1e-3) / 1e9,
-            "algorithmic_bytes_per_step": total_bytes,
-            "hbm_frac_of_8tbs": total_bytes / (ms_per_step * 1e-3) / 8e12,
-            "routed_slots_local": R, "num_tokens_post_pad": npad,
-            "flushed_ms_per_step": flushed_ms_per_step, "flushed_step_us_percentiles": flushed_pct_us,
-            "step_path": "moe_route_dispatch (single kernel) + moe_combine" if r.small_batch else
-                         "moe_route_dispatch (three kernels) + moe_combine",
-            "roofline": roofline, "stages": stages_fused, "stages_four_call_path": stages, "e2e": e2e,
-            "decode_route_patterns": patterns,
-            "cpu_baseline": cpu,
-            "gpu_launches": launches_per_step * args.steps, "launches_per_step": launches_per_step,
-            "clocks": clocks,
+            **{k: head[k] for k in ("achieved_hbm_gbs", "algorithmic_bytes_per_step", "hbm_frac_of_8tbs",
+                                    "hbm_frac_of_measured_peak", "routed_slots_local", "num_tokens_post_pad",
+                                    "flushed_ms_per_step", "flushed_step_us_percentiles", "step_path", "roofline",
+                                    "stages", "stages_four_call_path", "decode_route_patterns", "target",
+                                    "timed_region_s")},
+            "e2e": head["e2e"], "cpu_baseline": head.get("cpu_baseline"),
+            "gpu_launches": head["gpu_launches"], "launches_per_step": head["launches_per_step"],
+            "clocks": head["clocks"],
+            "workloads": subs,
         }
         print(json.dumps(line), flush=True)
-    del graphs
     if ws > 1:
         dist.barrier()
         dist.destroy_process_group()

@@ -16,6 +16,6 @@ from .binding import (  # noqa: F401
     moe_route_dispatch, moe_route_dispatch_workspace_bytes, moe_topk_softmax, moe_version, moe_workspace_init,
     status_string, alloc_dispatch_workspace,
 )
-from .router import MoeRouter  # noqa: F401
+from .router import HostStepPipeline, MoeRouter  # noqa: F401
 
-__all__ = [n for n in dir() if n.startswith("moe_") or n in ("MoeRouter", "MoeError", "AlignResult")]
+__all__ = [n for n in dir() if n.startswith("moe_") or n in ("MoeRouter", "HostStepPipeline", "MoeError", "AlignResult")]

@@ -122,3 +122,74 @@ class MoeRouter:
         a = B.moe_read_status(self.workspace, stream)
         b = B.moe_read_status(self.dispatch_workspace, stream)
         return a if a != B.MOE_OK else b
+
+
+class HostStepPipeline:
+    """End-to-end routing steps from pinned host buffers, with the copies overlapped.
+
+    Each ``submit`` enqueues one step: the host->device copies of its logits and hidden rows on a copy
+    stream, the step (moe_route_dispatch + moe_combine) on a compute stream, and the device->host copy
+    of its combined output on a third stream.  ``depth`` sets of device input and output buffers
+    rotate, so step i's inputs are copied in while step i-1 runs and step i-2's output is copied out
+    (the two copy directions share no engine).  Events order each buffer set's reuse: a set's inputs
+    are overwritten only after the step that read them, its output only after that output has been
+    copied out.  The router's other device buffers (routes, align outputs, gathered rows) are used by
+    the compute stream alone, in step order.  ``expert_out`` stands in for the expert MLPs' output.
+    Host output buffers must stay untouched until ``synchronize`` (or the step's own copy) is done."""
+
+    def __init__(self, router: MoeRouter, expert_out: torch.Tensor, depth: int = 2):
+        self.r = router
+        self.y = expert_out
+        self.depth = depth
+        dev = router.device
+        self.h2d = torch.cuda.Stream(device=dev)
+        self.comp = torch.cuda.Stream(device=dev)
+        self.d2h = torch.cuda.Stream(device=dev)
+        self.logits = [torch.empty_like(router.logits_dev) for _ in range(depth)]
+        self.hidden = [torch.empty_like(router.hidden_dev) for _ in range(depth)]
+        self.out = [torch.empty_like(router.out) for _ in range(depth)]
+        self.in_ready = [torch.cuda.Event() for _ in range(depth)]
+        self.in_free = [torch.cuda.Event() for _ in range(depth)]
+        self.done = [torch.cuda.Event() for _ in range(depth)]
+        self.out_free = [torch.cuda.Event() for _ in range(depth)]
+        self.i = 0
+
+    def submit(self, logits_host: torch.Tensor, hidden_host: torch.Tensor, out_host: torch.Tensor) -> None:
+        b = self.i % self.depth
+        r = self.r
+        self.h2d.wait_event(self.in_free[b])  # (no-op before the set's first use)
+        with torch.cuda.stream(self.h2d):
+            self.logits[b].copy_(logits_host, non_blocking=True)
+            self.hidden[b].copy_(hidden_host, non_blocking=True)
+            self.in_ready[b].record(self.h2d)
+        self.comp.wait_event(self.in_ready[b])
+        self.comp.wait_event(self.out_free[b])
+        with torch.cuda.stream(self.comp):
+            r.dispatch(self.logits[b], self.hidden[b], stream=self.comp)
+            B.moe_combine(self.y, r.topk_weights, r.align.inv_perm, self.out[b], device_status=r.workspace,
+                          stream=self.comp)
+            self.in_free[b].record(self.comp)
+            self.done[b].record(self.comp)
+        self.d2h.wait_event(self.done[b])
+        with torch.cuda.stream(self.d2h):
+            out_host.copy_(self.out[b], non_blocking=True)
+            self.out_free[b].record(self.d2h)
+        self.i += 1
+
+    def synchronize(self) -> None:
+        for s in (self.h2d, self.comp, self.d2h):
+            s.synchronize()
+
+    def timed(self, submit_one, n: int):
+        """Run ``submit_one(i)`` for i < n between two timing events: one on the copy-in stream before the
+        first copy, one on the copy-out stream after the last copy (which follows every earlier step).
+        Returns the two events, completed."""
+        torch.cuda.synchronize(self.r.device)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(self.h2d)
+        for i in range(n):
+            submit_one(i)
+        e1.record(self.d2h)
+        self.synchronize()
+        return e0, e1
