@@ -111,7 +111,7 @@ __device__ __forceinline__ uint64_t global_ns() {
 // Between polls the warp sleeps (__nanosleep, 32 ns doubling to 256 ns) so that waiting warps
 // take no issue slots from the warps doing the work.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64_t limit_ns = kWaitLimitNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_ns();
   unsigned sleep_ns = 32;
@@ -119,8 +119,26 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     __nanosleep(sleep_ns);
     if (mbar_try_wait(bar, parity)) return true;
     if (sleep_ns < 256) sleep_ns <<= 1;
-    if (global_ns() - t0 > kWaitLimitNs) return false;
+    if (global_ns() - t0 > limit_ns) return false;
   }
+}
+
+// Test hooks kept in words 2 and 3 of a dispatch workspace header (zero in normal use, which is what
+// moe_workspace_init leaves): word 2 holds bits that withhold one event a bounded wait depends on, so
+// that a test can make that wait run out and check the MOE_ERR_TIMEOUT it records; word 3 is the wait
+// limit in microseconds (0: the default of about two seconds).
+constexpr uint32_t kHookWithholdRowLoads = 1u;     // placement + gather: never issue the hidden-row loads
+constexpr uint32_t kHookWithholdTilePublish = 2u;  // gating: tile 0 never publishes its counts
+struct WaitHooks {
+  uint32_t withhold;
+  uint64_t limit_ns;
+};
+__device__ __forceinline__ WaitHooks read_hooks(const int32_t* ws_header) {
+  const uint2 v = __ldcg(reinterpret_cast<const uint2*>(ws_header + 2));  // written by the host, not cached in L1
+  WaitHooks h;
+  h.withhold = v.x;
+  h.limit_ns = v.y == 0u ? kWaitLimitNs : static_cast<uint64_t>(v.y) * 1000ull;
+  return h;
 }
 
 // Named barrier over `nthreads` threads (a multiple of 32) of this CTA.
