@@ -14,7 +14,11 @@ back to back between one pair of CUDA events on the launching stream; otherwise 
 256 MiB write, then a 256 MiB read, so no dirty flush lines are written back inside a timed step)
 before each step and every step is timed with its own pair of events (``--flush-always`` forces
 this mode; the flushed figure is reported beside the other).  The result is the max over ranks.
-N > 1 runs one independent batch per GPU (weak scaling: the path has no cross-token exchange).
+N > 1 runs the layer expert-parallel (strong scaling): every rank routes the same tokens with its own
+contiguous block of E/N experts, combines its local slots into the owners' receive buffers (CUDA IPC,
+the stores crossing NVLink) and reduces the rows it owns (dist.EpExchange); a step ends with the
+layer output spread over the ranks.  ``--dp`` runs one independent batch per GPU instead (weak
+scaling, no exchange); ``--ep`` takes the expert-parallel step on one GPU too.
 Rank 0 prints one JSON line.
 
 Also reported: per-stage device times and achieved HBM bandwidth from the algorithmic bytes (for
@@ -72,6 +76,8 @@ def parse_args():
     p.add_argument("--workload", default=None,
                    help="workload name (default: the skewed 65536-token prefill, with the other workloads as sub-records)")
     p.add_argument("--no-sub-workloads", action="store_true", help="time the headline workload only")
+    p.add_argument("--dp", action="store_true", help="N > 1: one independent batch per GPU (no exchange)")
+    p.add_argument("--ep", action="store_true", help="the expert-parallel step even on one GPU")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-graph", action="store_true", help="launch the calls directly instead of a graph")
     p.add_argument("--flush-always", action="store_true",
@@ -635,6 +641,106 @@ def measure_workload(wl, ctx: Ctx, headline: bool) -> dict:
     return rec
 
 
+def measure_ep(wl, ctx: Ctx) -> dict:
+    """The expert-parallel layer step over the ranks (strong scaling): every rank routes the same T tokens
+    with its own block of experts (moe_route_dispatch), combines its local slots into the owners'
+    receive buffers and reduces the rows it owns (dist.EpExchange: a stream synchronisation and a
+    process-group barrier inside every step, so no CUDA graph).  Timed with CUDA events on the
+    launching stream around K steps, max over ranks; value = T * K / that time."""
+    import torch
+    import torch.distributed as dist
+    import token_dispatch_topk_b200 as tdt
+    from token_dispatch_topk_b200 import inputs as I
+    from token_dispatch_topk_b200.dist import EpExchange, ep_expert_map, max_over_ranks
+
+    args, dev, stream, ws, rank = ctx.args, ctx.dev, ctx.stream, ctx.ws, ctx.rank
+    emap, El = ep_expert_map(wl.E, ws, rank)
+    logits = I.make_logits(wl, seed=args.seed, device=dev)  # the same tokens on every rank
+    hidden = I.make_hidden(wl, seed=args.seed, device=dev)
+    r = tdt.MoeRouter(wl.T, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, E_local=El, expert_map=emap,
+                      logits_dtype=logits.dtype, device=dev)
+    y = I.make_expert_out(r.capacity, wl.H, seed=args.seed * 16 + 5 + rank, device=dev)  # this rank's experts
+    ex = EpExchange(wl.T, wl.H, dev)
+
+    def step():
+        r.dispatch(logits, hidden, stream=stream)
+        ex.combine_reduce(y, r.topk_weights, r.align.inv_perm, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    stream.synchronize()
+    if r.device_status() != tdt.MOE_OK:
+        raise RuntimeError("expert-parallel warm-up: device status is not MOE_OK")
+    sampler = ClockSampler(ctx.uuid) if rank == 0 else None
+    if sampler:
+        sampler.start()
+        time.sleep(0.4)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    total_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    # end to end: the step's inputs copied in from pinned host memory, this owner's rows copied out
+    logits_h, hidden_h = logits.cpu().pin_memory(), hidden.cpu().pin_memory()
+    lo, hi = ex.ranges[rank]
+    out_h = torch.empty((hi - lo, wl.H), dtype=torch.bfloat16).pin_memory()
+    e2e_steps = args.e2e_steps or min(args.steps, 200)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        f0.record(stream)
+        for _ in range(e2e_steps):
+            r.logits_dev.copy_(logits_h, non_blocking=True)
+            r.hidden_dev.copy_(hidden_h, non_blocking=True)
+            r.dispatch(r.logits_dev, r.hidden_dev, stream=stream)
+            out = ex.combine_reduce(y, r.topk_weights, r.align.inv_perm, stream=stream)
+            out_h.copy_(out, non_blocking=True)
+        f1.record(stream)
+    stream.synchronize()
+    e2e_ms = max_over_ranks(f0.elapsed_time(f1), dev)
+    clocks = sampler.stop() if sampler else None
+    if r.device_status() != tdt.MOE_OK:
+        raise RuntimeError("expert-parallel steps: device status is not MOE_OK")
+    R = int(r.align.counts.sum().item())
+    nvlink_bytes = sum((b - a) * wl.H * 2 for o, (a, b) in enumerate(ex.ranges) if o != rank)
+    # kernels per step: the dispatch (one kernel for decode-sized batches; else gating + placement, and
+    # the tile-scan kernel when the tiles times the local experts exceed the lookback's limit), one
+    # combine per owner with tokens, one reduce on an owner with tokens
+    if r.small_batch:
+        n_dispatch = 1
+    else:
+        rt = 32 if (wl.T + 15) // 16 > ctx.sms * 4 else 16
+        elem = 2 if wl.logits_dtype == "bf16" else 4
+        if wl.k <= 8 and (wl.E * elem) % 16 == 0 and ((wl.E <= 64 and wl.T >= 1024) or
+                                                      (elem == 2 and wl.E <= 256 and wl.T >= 16384)):
+            rt = 32
+        n_dispatch = 2 if -(-wl.T // rt) * El <= 65536 else 3
+    per_step = n_dispatch + sum(1 for a, b in ex.ranges if b > a) + (1 if hi > lo else 0)
+    return {"workload": wl.name, "value": wl.T * args.steps / (total_ms / 1e3), "unit": UNIT,
+            "ms_per_step": total_ms / args.steps, "E_local": El, "routed_slots_local_rank0": R,
+            "owned_tokens_rank0": hi - lo, "peer_store_bytes_per_rank_per_step": nvlink_bytes,
+            "launches_per_step": per_step, "gpu_launches": per_step * args.steps, "clocks": clocks,
+            "e2e": {"value": wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": logits_h.numel() * logits_h.element_size() +
+                    hidden_h.numel() * hidden_h.element_size(),
+                    "d2h_bytes_per_step": out_h.numel() * out_h.element_size(), "steps": e2e_steps,
+                    "api": "MoeRouter.dispatch + EpExchange.combine_reduce, pinned H2D of logits and hidden, "
+                           "D2H of this owner's rows (rank 0's bytes)"},
+            "parallelism": f"expert parallel over {ws} ranks ({El} local experts each): moe_route_dispatch, "
+                           f"moe_combine into the owners' receive buffers (CUDA IPC), barrier, moe_reduce_partials",
+            "timing": "CUDA events around K steps on the launching stream (host barrier inside each step), "
+                      "max over ranks"}
+
+
 TARGETS = {  # end-to-end targets: fraction of 8 TB/s, or device time of the worst decode route pattern
     "qwen3moe_prefill_T4096_E128_k8": ("hbm_frac_of_8tbs", 0.70),
     "nonpow2_T16384_E60_k4": ("hbm_frac_of_8tbs", 0.70),
@@ -674,6 +780,23 @@ def main():
     tdt.load_library()
     ctx = Ctx(args, dev, ws, rank)
 
+    if (ws > 1 and not args.dp) or args.ep:
+        rec = measure_ep(wl, ctx)
+        if rank == 0:
+            print(json.dumps({
+                "metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded, counter-based; see token_dispatch_topk_b200/inputs.py)",
+                "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
+                           "parallelism": rec["parallelism"], "cuda_graph": False},
+                "expert_parallel": rec, "gpu_launches": rec["gpu_launches"], "clocks": rec["clocks"],
+                "e2e": rec["e2e"], "cpu_baseline": None}), flush=True)
+        if ws > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
+
     head = measure_workload(wl, ctx, headline=True)
     head["target"] = target_status(head)
     subs = []
@@ -694,7 +817,7 @@ def main():
             "data": "synthetic (seeded, counter-based; see token_dispatch_topk_b200/inputs.py)",
             "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
                        "l2": head["l2"], "cuda_graph": not args.no_graph,
-                       "parallelism": "one independent batch per GPU" if ws > 1 else "single GPU"},
+                       "parallelism": "one independent batch per GPU (--dp)" if ws > 1 else "single GPU"},
             **{k: head[k] for k in ("achieved_hbm_gbs", "algorithmic_bytes_per_step", "hbm_frac_of_8tbs",
                                     "hbm_frac_of_measured_peak", "routed_slots_local", "num_tokens_post_pad",
                                     "flushed_ms_per_step", "flushed_step_us_percentiles", "step_path", "roofline",

@@ -4,7 +4,8 @@
     over the ranks;
   * expert parallel: each rank owns a contiguous block of experts (``ep_expert_map``), routes the
     same tokens with its map (the oracle stands in for the rank's kernels here), combines its
-    local slots into a bf16 partial, and ``ep_reduce_partials`` sums the partials over the ranks.
+    local slots into a bf16 partial, and ``ep_reduce_partials`` all-gathers the partials and sums
+    them in rank order (the oracle's reduce stands in for moe_reduce_partials).
     The result must match the oracle's single-rank combine of all slots within the rounding of
     the two partials and the final sum; the expert outputs are a function of (global expert,
     token) so that every rank builds its own expert-grouped rows consistently.
@@ -65,7 +66,12 @@ def _worker(rank, world, port, q):
         logits = torch.cat([logits, logits.flip(1) * 0.5], dim=1).contiguous()
         bits = logits.view(torch.int16).numpy().view(np.uint16)
         _, _, partial = _rank_partial(bits, T, E, k, H, bs, world, rank)
-        summed = D.ep_reduce_partials(torch.from_numpy(partial.view(np.int16)).view(torch.bfloat16))
+        def oracle_reduce(parts):  # the oracle stands in for moe_reduce_partials on the CPU
+            bits = np.stack([p.view(torch.int16).numpy().view(np.uint16) for p in parts])
+            return torch.from_numpy(oracle.reduce_partials(bits).view(np.int16)).view(torch.bfloat16)
+
+        summed = D.ep_reduce_partials(torch.from_numpy(partial.view(np.int16)).view(torch.bfloat16),
+                                      reduce=oracle_reduce)
         out["partial"] = partial
         out["summed"] = summed.view(torch.int16).numpy().view(np.uint16)
         out["bits"] = bits
@@ -101,6 +107,9 @@ def test_expert_parallel_partials_sum_to_the_full_combine(two_ranks):
     assert np.array_equal(bits, two_ranks[1]["bits"])
     s0, s1 = two_ranks[0]["summed"], two_ranks[1]["summed"]
     assert np.array_equal(s0, s1), "every rank holds the same reduced output"
+    # the all-gather baseline sums in rank order: bit-identical to the oracle's reduce of the partials
+    both = np.stack([two_ranks[0]["partial"], two_ranks[1]["partial"]])
+    assert np.array_equal(s0, oracle.reduce_partials(both))
     # single rank owning every expert
     w, ids, full = _rank_partial(bits, T, E, k, H, bs, 1, 0)
     p0 = bf16_bits_to_f32(two_ranks[0]["partial"]).astype(np.float64)

@@ -6,13 +6,22 @@ Two uses:
   * expert parallel: every rank routes the same tokens with its own ``expert_map`` (a contiguous
     block of experts, ``ep_expert_map``); its combine is the partial sum over its local slots, and
     the one exchange of the layer is the sum of those partials over the ranks: fp32 sum of the bf16
-    partials, rounded once to bf16.  Two forms:
-      - ``ep_reduce_partials``: an NCCL all-reduce of the widened partials;
-      - reduce-scatter through the library: ``ep_combine_to_owners`` (each rank's combine writes each
-        owner's token range into the owner's receive buffer, ``ep_token_range``), then, after a
-        barrier, ``ep_reduce_received`` on every owner (moe_reduce_partials, rank order).  The
-        receive buffers of a multi-GPU run are peer memory (e.g. symmetric memory); the tests run
-        the ranks on one GPU with local buffers in their place.
+    partials in ascending rank order, rounded once to bf16.  Two forms:
+      - ``EpExchange`` (the library's form, a reduce-scatter): each rank's moe_combine writes each
+        owner's token range (``ep_token_range``) of its partial straight into its slot of that
+        owner's receive buffer, in the owner's memory, shared between the processes through CUDA IPC
+        (on several GPUs the combine's own stores cross NVLink; plain 16-byte stores, no TMA, no
+        multicast); each rank then synchronises its stream and joins a process-group barrier, so
+        that every store into every owner's buffer has completed before any owner reads; then each
+        owner runs moe_reduce_partials over its slots in rank order.  Two receive buffers alternate
+        between steps, so one barrier per step also keeps a step's stores away from the buffer the
+        owner is still reducing from the step before;
+      - ``ep_reduce_partials``: an all-gather of the whole partials through the process group, then
+        the same rank-ordered reduce on every rank (bit-identical to the reduce-scatter's rows; the
+        collective baseline).
+    ``ep_combine_to_owners`` and ``ep_reduce_received`` are the two halves of the reduce-scatter for
+    callers that manage their own buffers; a caller must order every rank's combine before the
+    owners' reduces (synchronise the combine's stream, or wait on its event, before a barrier).
 
 The exchange follows the expert-parallel decode of the "b70-optimization-lab: 2026-07-16 MTP1
 M=2 compact scheduler closure note" (scheduler paragraph: each rank derives its local expert row
@@ -98,11 +107,74 @@ def ep_reduce_received(received, out: Optional[torch.Tensor] = None, stream=None
     return moe_reduce_partials(received, out=out, stream=stream)
 
 
-def ep_reduce_partials(partial: torch.Tensor, group: Optional[dist.ProcessGroup] = None) -> torch.Tensor:
-    """Sum the ranks' bf16 partial combines [T, H]: widened to fp32, summed over the ranks, rounded
-    once to bf16 (round-to-nearest-even).  Returns a new tensor; with one rank, the partial."""
+def ep_reduce_partials(partial: torch.Tensor, group: Optional[dist.ProcessGroup] = None,
+                       reduce=None) -> torch.Tensor:
+    """Sum the ranks' bf16 partial combines [T, H] (the collective baseline of the exchange): an
+    all-gather of every rank's partial, then the fp32 sum in ascending rank order from +0, rounded
+    once to bf16, on every rank.  ``reduce`` maps the list of partials (rank order) to the sum;
+    default: moe_reduce_partials on the partials' device.  Returns a new tensor; with one rank, a
+    copy of the partial."""
     if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size(group) == 1:
         return partial.clone()
-    acc = partial.float()
-    dist.all_reduce(acc, op=dist.ReduceOp.SUM, group=group)
-    return acc.to(torch.bfloat16)
+    parts = [torch.empty_like(partial) for _ in range(dist.get_world_size(group))]
+    dist.all_gather(parts, partial.contiguous(), group=group)
+    if reduce is None:
+        from .binding import moe_reduce_partials
+        return moe_reduce_partials(parts)
+    return reduce(parts)
+
+
+class EpExchange:
+    """The expert-parallel exchange as a reduce-scatter through the owners' memory (see the module
+    docstring).  One object per rank, created by every rank of ``group`` together (it exchanges
+    CUDA IPC handles of the receive buffers through the process group).
+
+    ``combine_reduce(expert_out, topk_weights, inv_perm)`` runs one step: this rank's partial combine
+    into every owner's receive buffer, the barrier, and this owner's reduce; it returns this owner's
+    rows of the layer output ([hi - lo, H] bf16 for ``ep_token_range(T, world, rank)``), in a buffer the
+    next step overwrites.  Without a process group it is a single rank's exchange (its own buffer)."""
+
+    def __init__(self, T: int, H: int, device, group: Optional[dist.ProcessGroup] = None, buffers: int = 2):
+        from torch.multiprocessing.reductions import reduce_tensor
+        self.group = group
+        grouped = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size(group) if grouped else 1  # one rank: its own buffer, no barrier
+        self.rank = dist.get_rank(group) if grouped else 0
+        self.T, self.H = T, H
+        self.ranges = [ep_token_range(T, self.world, o) for o in range(self.world)]
+        lo, hi = self.ranges[self.rank]
+        rows = max(1, hi - lo)  # every owner shares a buffer, even one without tokens
+        self.recv = [torch.zeros((self.world, rows, H), dtype=torch.bfloat16, device=device) for _ in range(buffers)]
+        self.out = torch.empty((hi - lo, H), dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize(device)
+        if self.world > 1:
+            mine = [reduce_tensor(b) for b in self.recv]
+            handles = [None] * self.world
+            dist.all_gather_object(handles, mine, group=group)
+            # remote[b][o]: owner o's receive buffer b, as mapped in this process
+            self.remote = [[self.recv[b] if o == self.rank else handles[o][b][0](*handles[o][b][1])
+                            for o in range(self.world)] for b in range(buffers)]
+            dist.barrier(group=group)
+        else:
+            self.remote = [[b] for b in self.recv]
+        self.step_index = 0
+
+    def destinations(self, b: int):
+        """This rank's slot in every owner's receive buffer b (owner order)."""
+        return [self.remote[b][o][self.rank, :hi - lo] for o, (lo, hi) in enumerate(self.ranges)]
+
+    def combine_reduce(self, expert_out: torch.Tensor, topk_weights: torch.Tensor, inv_perm: torch.Tensor,
+                       device_status: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        from .binding import moe_reduce_partials
+        b = self.step_index % len(self.recv)
+        self.step_index += 1
+        s = torch.cuda.current_stream() if stream is None else stream
+        ep_combine_to_owners(expert_out, topk_weights, inv_perm, self.destinations(b), device_status=device_status,
+                             stream=s)
+        if self.world > 1:
+            s.synchronize()                 # this rank's stores into every owner's buffer have completed
+            dist.barrier(group=self.group)  # ... and every other rank's into this owner's
+        lo, hi = self.ranges[self.rank]
+        if hi > lo:
+            moe_reduce_partials([self.recv[b][r, :hi - lo] for r in range(self.world)], out=self.out, stream=s)
+        return self.out
