@@ -2,9 +2,7 @@
 the CPU oracle pipeline, through the C ABI.
 
 Two kernel paths sit behind the call: one kernel with one CTA per slot for small batches
-(T <= 32, T*k <= 256 and E <= 256) and the tiled path above that, whose prefix over the tiles is
-either a decoupled lookback inside the gating kernel (tiles x local experts <= 65536) or a separate
-per-expert scan kernel (above).  Shapes cover both sides of every
+(T <= 32, T*k <= 256 and E <= 256) and the tiled three-kernel path above that.  Shapes cover both sides of every
 one of those limits, one and many gating tiles with a ragged last tile, maps with remote and
 out-of-range values, every gating vector width, k up to 32, 1024 experts, T = 0 and the decode size,
 with logits-derived routes and with routes given by the caller.  Bars as for the stage entry points:
@@ -71,11 +69,10 @@ CASES = [
     ("lanes_bf16_E56_k7_strided_map", 1111, 56, 7, torch.bfloat16, False, "strided", 14, 16, 32),
     ("lanes_wide_bf16_E256_k8_strided_map", 16500, 256, 8, torch.bfloat16, True, "strided", 64, 128, 16),
     ("lanes_wide_bf16_E192_k5_ties", 16401, 192, 5, torch.bfloat16, False, None, 192, 32, 8),
-    # prefix over the tiles: per-expert scan kernel (tiles x local experts > 65536) with one warp per row;
-    # lookback windows that wrap more than once (lanes kernel: 128 predecessor flags per window)
-    ("tile_scan_kernel_E512", 5000, 512, 8, torch.bfloat16, True, None, 512, 16, 64),
-    ("lookback_many_windows_fp32_E60", 16400, 60, 4, torch.float32, False, None, 60, 64, 16),
-    ("lookback_row4_pad_E61", 4000, 61, 3, torch.bfloat16, True, None, 61, 5, 16),
+    # many tiles and many local experts (a long tile scan per expert); a ragged fp32 lanes batch
+    ("many_tiles_E512", 5000, 512, 8, torch.bfloat16, True, None, 512, 16, 64),
+    ("lanes_fp32_E60_ragged", 16400, 60, 4, torch.float32, False, None, 60, 64, 16),
+    ("lanes_bf16_E61_no_lanes_odd", 4000, 61, 3, torch.bfloat16, True, None, 61, 5, 16),
 ]
 
 
@@ -225,10 +222,9 @@ def test_dispatch_sigmoid_scoring(T, E, k, dtype, renorm, E_local, bs, H):
     assert np.array_equal(bf16_bits(perm[:npad])[real], perm_ref[:npad][real])
 
 
-def test_dispatch_workspace_shared_across_sizes_and_prefix_modes():
-    """One workspace, large enough for every call, used by calls of different sizes whose prefix over
-    the tiles takes the lookback or the scan kernel: each call is correct whatever the previous one
-    left in the workspace (lookback flags carry the call's epoch and a tag no count can carry)."""
+def test_dispatch_workspace_shared_across_sizes():
+    """One workspace, large enough for every call, used by calls of different sizes and tile layouts:
+    each call is correct whatever the previous one left in the workspace."""
     dev = require_gpu()
     shapes = [(3000, 60, 4, 60), (5000, 512, 8, 512), (3000, 60, 4, 60), (700, 128, 8, 128), (5000, 512, 8, 512),
               (700, 128, 8, 128)]

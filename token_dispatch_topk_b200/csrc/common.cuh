@@ -127,8 +127,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, uint64
 // moe_workspace_init leaves): word 2 holds bits that withhold one event a bounded wait depends on, so
 // that a test can make that wait run out and check the MOE_ERR_TIMEOUT it records; word 3 is the wait
 // limit in microseconds (0: the default of about two seconds).
-constexpr uint32_t kHookWithholdRowLoads = 1u;     // placement + gather: never issue the hidden-row loads
-constexpr uint32_t kHookWithholdTilePublish = 2u;  // gating: tile 0 never publishes its counts
+constexpr uint32_t kHookWithholdRowLoads = 1u;  // placement + gather: never issue the hidden-row loads
 struct WaitHooks {
   uint32_t withhold;
   uint64_t limit_ns;

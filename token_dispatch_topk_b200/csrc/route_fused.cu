@@ -8,27 +8,21 @@
 // scheduler closure note.  The outputs are exactly those of moe_topk_softmax +
 // moe_align_permute + moe_gather; only the kernel boundaries move.
 //
-// Batches above the small-batch limits take two kernels (three when the tile counts are too many
-// for the lookback), chained by programmatic dependent launch:
+// Batches above the small-batch limits take three kernels, chained by programmatic dependent
+// launch:
 // gate_count_kernel (one CTA per tile of 16 or 32 tokens; 16 when the tiles of a batch fit on
 // the SMs at once, so that each warp gates one row):
 //   A. each warp gates rows of the tile (gate_row: one warp per row) and writes topk_weights and
 //      topk_ids; the local expert of every slot of the tile goes to shared memory;
 //   B. stable ranks inside the tile: each warp owns a contiguous run of the tile's slots, counts
 //      it into its own shared-memory row, the rows are scanned across warps, and each slot's rank
-//      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm;
-//   C. the prefix of the tile counts over the tiles, in the same pass (decoupled lookback, the
-//      "single pass" form of the block alignment's prefix): CTAs take their tiles in ticket order,
-//      publish the tile's per-expert counts with a flag, and look back over the flags of the tiles
-//      before theirs (one flag per thread, a whole window at once) until the nearest tile that has
-//      published its inclusive prefix; the aggregates in between plus that prefix give the tile's
-//      base per expert, which the tile publishes in turn; the last tile's inclusive prefix is the
-//      expert totals.  Every flag wait is bounded in time (MOE_ERR_TIMEOUT in the status word).
-//      When the tiles times the local experts exceed kLookbackMaxCells (the lookback would read too
-//      much), the counts go to the workspace expert-major instead and tile_scan_kernel (one CTA per
-//      local expert) turns each expert's row of tile counts into its prefix after a kernel boundary.
+//      = earlier warps' count + earlier peers in its warp; the rank is parked in inv_perm and the
+//      tile's per-expert counts go to the workspace, expert-major ([E_local][tiles]).
 //   gate_count_lanes_kernel replaces it for many short rows (moe_gate::lane_gating_fits): one
 //   CTA per tile of 32 tokens, up to eight lanes per row (gate_lane.cuh), the same ranks and counts.
+// tile_scan_kernel (one CTA per local expert): the expert's row of tile counts becomes the
+//   exclusive prefix over the tiles (the tile bases) and its total goes to the workspace.
+//   Nothing waits on another CTA: the kernel boundary is the only grid-wide step.
 // place_gather_kernel (one warp per CTA, up to 8 tokens, TMA staging as in gather_tma_kernel):
 //   bulk-loads its hidden rows first (hidden is an input of the call, complete before the first
 //   kernel ran); scans the padded expert totals into the offsets itself (E_local values, in
@@ -48,11 +42,7 @@ namespace {
 
 constexpr int kGcWarps = 16;
 constexpr int kGcThreads = kGcWarps * 32;
-constexpr int kWsHeaderBytes = 256;  // status word, test hooks, lookback ticket / done count / epoch
-constexpr int kWsTicketWord = 4;     // header word: next tile ticket (wraps to 0 after the last tile)
-constexpr int kWsDoneWord = 5;       // header word: tiles finished in this call
-constexpr int kWsEpochByte = 24;     // header bytes 24..31: number of completed lookback calls (u64)
-constexpr int64_t kLookbackMaxCells = 65536;  // lookback when num_tiles * E_local is at most this
+constexpr int kWsHeaderBytes = 256;  // status word, test hooks (words 2 and 3), padding
 constexpr int kRowsPerTile = 32;       // tile height of the lane kernel and of the align entry point
 constexpr int kRowsPerTileSmall = 16;  // tile height of gate_count_kernel when all tiles fit at once
 constexpr int kGcCtasPerSm = 4;        // gate_count_kernel CTAs resident per SM (2048 threads)
@@ -89,14 +79,8 @@ struct DispatchArgs {
   int32_t* n_pad;
   int32_t* inv_perm;
   int32_t* status;
-  int32_t* tile_counts;  // tile bases: tile_counts[e * base_stride_e + tile * base_stride_t]
+  int32_t* tile_counts;  // [E_local][num_tiles]: tile counts, then tile bases
   int32_t* totals;       // [E_local]
-  int base_stride_e, base_stride_t;  // [E_local][num_tiles] (tile scan) or [num_tiles][E_local] (lookback)
-  // lookback only (gate kernels with kLookback)
-  unsigned long long* flags;  // [num_tiles]: tag | (epoch << 2) | state, state 1 = aggregate, 2 = inclusive prefix
-  int32_t* agg;               // [num_tiles][row4]: each tile's counts
-  int32_t* incl;              // [num_tiles][row4]: each tile's inclusive prefix
-  int row4;                   // E_local rounded up to a multiple of 4 (16-byte rows)
 };
 
 // Local expert of global expert g (or -1: remote); out-of-range values are flagged.
@@ -132,23 +116,20 @@ __device__ __forceinline__ int padded_rows(int c, int bs, int bs_shift) {
 }
 
 // Shared memory of gate_count_kernel (ints): s_le[rows_per_tile * k] | whist[kGcWarps][E_local] |
-// masks[kGcWarps][E_local] | (lookback) s_cnt[row4] | s_excl[row4]
-__host__ __device__ inline int row4_of(int E_local) { return (E_local + 3) & ~3; }
-__host__ __device__ inline size_t gc_smem_ints(int rows_per_tile, int k, int E_local, bool lookback) {
-  return static_cast<size_t>(rows_per_tile) * k + 2 * static_cast<size_t>(kGcWarps) * E_local +
-         (lookback ? 2 * static_cast<size_t>(row4_of(E_local)) : 0);
+// masks[kGcWarps][E_local]
+__host__ __device__ inline size_t gc_smem_ints(int rows_per_tile, int k, int E_local) {
+  return static_cast<size_t>(rows_per_tile) * k + 2 * static_cast<size_t>(kGcWarps) * E_local;
 }
 
 // Stable ranks inside a tile, by the CTA's `nwarps` warps (all threads call this, after s_le is
 // complete): warp w owns a contiguous run of the tile's 32-slot chunks and counts it into its row of
 // `whist` ([nwarps][E_local], zero on entry); the rows are scanned across warps per expert (the
-// tile's counts go to s_cnt for the lookback, or to the workspace expert-major for the tile scan
-// when s_cnt is null); each slot's rank = earlier warps' count of its
+// tile's counts go to the workspace, expert-major); each slot's rank = earlier warps' count of its
 // expert + the warp's running count + earlier peers in its chunk.  The rank is parked in inv_perm
 // as (rank << 10) | local expert for place_gather_kernel; remote slots get -1.  `masks`
 // ([nwarps][E_local]) is zero on entry and left zero.
 __device__ __forceinline__ void rank_tile_slots(const DispatchArgs& a, const int* s_le, int nslots, int64_t row0,
-                                                int tile, int* whist, unsigned* masks, int nwarps, int* s_cnt) {
+                                                int tile, int* whist, unsigned* masks, int nwarps) {
   const int El = a.E_local, k = a.k;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int nthreads = nwarps * 32;
@@ -171,11 +152,7 @@ __device__ __forceinline__ void rank_tile_slots(const DispatchArgs& a, const int
       whist[w * El + e] = run;
       run += c;
     }
-    if (s_cnt != nullptr) {
-      s_cnt[e] = run;  // the lookback publishes it
-    } else {
-      a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = run;
-    }
+    a.tile_counts[static_cast<int64_t>(e) * a.num_tiles + tile] = run;
   }
   __syncthreads();
   for (int c = c0; c < c1; ++c) {
@@ -193,201 +170,25 @@ __device__ __forceinline__ void rank_tile_slots(const DispatchArgs& a, const int
   }
 }
 
-// ------------------------------------------------------------------------------------------
-// Decoupled lookback over the tiles (single pass).  Tiles are taken in ticket order (a CTA's tile is
-// the ticket it draws after its predecessor kernel has finished), so every tile a CTA waits for
-// belongs to a CTA that has already started: the waits always end while the GPU is healthy, and
-// each one is bounded in time besides.  The workspace header holds the ticket (wrapping to 0 after
-// the last tile), the count of finished tiles and an epoch (completed calls): a flag is current
-// when it carries this call's epoch, so no flag is ever reset.
-constexpr unsigned long long kFlagAggregate = 1ull;
-constexpr unsigned long long kFlagPrefix = 2ull;
-// Top bit of every flag: no count, base or total the workspace holds (all non-negative int32) can
-// look like a flag, whatever earlier calls of other sizes or modes left where the flags now are.
-constexpr unsigned long long kFlagTag = 1ull << 63;
-
-__device__ __forceinline__ unsigned long long ld_acquire_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-__device__ __forceinline__ void st_release_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-
-// State of a tile's flag in this call (kFlagAggregate or kFlagPrefix), once published; 0 when the
-// bounded wait runs out.
-__device__ __forceinline__ int wait_tile_flag(const unsigned long long* f, unsigned long long epoch, uint64_t limit_ns) {
-  const unsigned long long want = kFlagTag | (epoch << 2);
-  unsigned long long v = ld_acquire_u64(f);
-  if ((v & ~3ull) == want && (v & 3ull) != 0ull) return static_cast<int>(v & 3ull);
-  const uint64_t t0 = moe::global_ns();
-  unsigned sleep_ns = 32;
-  for (;;) {
-    __nanosleep(sleep_ns);
-    v = ld_acquire_u64(f);
-    if ((v & ~3ull) == want && (v & 3ull) != 0ull) return static_cast<int>(v & 3ull);
-    if (sleep_ns < 256) sleep_ns <<= 1;
-    if (moe::global_ns() - t0 > limit_ns) return 0;
-  }
-}
-
-__device__ __forceinline__ unsigned long long* ws_epoch(const DispatchArgs& a) {
-  return reinterpret_cast<unsigned long long*>(reinterpret_cast<char*>(a.status) + kWsEpochByte);
-}
-
-// This CTA's tile (its ticket) and the call's epoch, drawn by thread 0 after the predecessor kernel
-// has finished (the previous call's last tile left the ticket at 0 and advanced the epoch).
-__device__ __forceinline__ void lookback_enter(const DispatchArgs& a, int* s_tile, unsigned long long* s_epoch) {
-  if (threadIdx.x == 0) {
-    unsigned* words = reinterpret_cast<unsigned*>(a.status);
-    *s_tile = static_cast<int>(atomicInc(words + kWsTicketWord, static_cast<unsigned>(a.num_tiles - 1)));
-    *s_epoch = __ldcg(ws_epoch(a));
-  }
-  __syncthreads();
-}
-
-// The tile's exclusive prefix over the tiles before it, per local expert (all NT threads call this
-// after the tile's counts are in s_cnt).  Publishes the aggregate, looks back over windows of NT
-// predecessor flags (thread i waits for tile hi - i) until the nearest tile with an inclusive prefix,
-// adds that prefix and the aggregates in between (16-byte loads from L2, many tiles in parallel),
-// then publishes the tile's own inclusive prefix and writes its base (and, for the last tile, the
-// expert totals).  Finally counts the tile as done; the call's last tile advances the epoch.
-// Shared memory: s_cnt [row4], s_excl [row4], s_ctl [1].
-template <int NT>
-__device__ void tile_lookback(const DispatchArgs& a, int tile, unsigned long long epoch, const moe::WaitHooks& hooks,
-                              const int* s_cnt, int* s_excl, int* s_ctl) {
-  const int tid = threadIdx.x;
-  const int El = a.E_local, R4 = a.row4, N = a.num_tiles;
-  const bool valid = tile < N;  // a ticket past the last tile: the workspace was not initialised
-  if (!valid && tid == 0) moe::record_status(a.status, MOE_ERR_WORKSPACE);
-  if (valid) {
-    int32_t* my_agg = a.agg + static_cast<int64_t>(tile) * R4;
-    for (int e = tid; e < R4; e += NT) {
-      const int c = e < El ? s_cnt[e] : 0;
-      my_agg[e] = c;
-      s_excl[e] = 0;
-      if (tile == 0) a.incl[e] = c;
-    }
-    if (tid == 0) s_ctl[0] = NT << 1;
-    __syncthreads();
-    const bool withhold = tile == 0 && (hooks.withhold & moe::kHookWithholdTilePublish) != 0u;
-    if (tid == 0 && !withhold) {
-      __threadfence();
-      st_release_u64(a.flags + tile, kFlagTag | (epoch << 2) | (tile == 0 ? kFlagPrefix : kFlagAggregate));
-    }
-    if (tile > 0) {
-      const int Q = R4 >> 2;                     // 16-byte quads per row
-      const int par = NT >= Q ? NT / Q : 1;      // predecessor rows summed side by side
-      int hi = tile - 1;                         // nearest predecessor not yet added
-      for (;;) {
-        // thread i: the tile i places back; the lowest such thread that ends the lookback wins:
-        // (i << 1) | 0 for an inclusive prefix to add, (i << 1) | 1 to stop with nothing to add
-        // (past tile 0, or a wait that ran out)
-        const int j = hi - tid;
-        int cand = NT << 1;
-        if (j < 0) {
-          cand = (tid << 1) | 1;
-        } else {
-          const int state = wait_tile_flag(a.flags + j, epoch, hooks.limit_ns);
-          if (state == 0) {
-            moe::record_status(a.status, MOE_ERR_TIMEOUT);
-            cand = (tid << 1) | 1;
-          } else if (state == static_cast<int>(kFlagPrefix)) {
-            cand = tid << 1;
-          }
-        }
-        if (cand < (NT << 1)) atomicMin(s_ctl, cand);
-        __syncthreads();
-        const int ctl = s_ctl[0];
-        const int stop = ctl >> 1;  // window positions [0, stop) add their aggregates
-        const bool add_prefix = stop < NT && (ctl & 1) == 0;
-        for (int qq = tid; qq < Q * par; qq += NT) {
-          const int q = qq % Q, r0 = qq / Q;
-          int4 acc = make_int4(0, 0, 0, 0);
-          for (int t = r0; t < stop; t += par) {
-            const int4 v = __ldcg(reinterpret_cast<const int4*>(a.agg + static_cast<int64_t>(hi - t) * R4) + q);
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-          }
-          if (r0 == 0 && add_prefix) {
-            const int4 v = __ldcg(reinterpret_cast<const int4*>(a.incl + static_cast<int64_t>(hi - stop) * R4) + q);
-            acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-          }
-          if (par > 1) {
-            atomicAdd(s_excl + 4 * q + 0, acc.x);
-            atomicAdd(s_excl + 4 * q + 1, acc.y);
-            atomicAdd(s_excl + 4 * q + 2, acc.z);
-            atomicAdd(s_excl + 4 * q + 3, acc.w);
-          } else {
-            s_excl[4 * q + 0] += acc.x;
-            s_excl[4 * q + 1] += acc.y;
-            s_excl[4 * q + 2] += acc.z;
-            s_excl[4 * q + 3] += acc.w;
-          }
-        }
-        __syncthreads();
-        if (stop < NT) break;
-        hi -= NT;
-        if (tid == 0) s_ctl[0] = NT << 1;
-        __syncthreads();
-      }
-      int32_t* my_incl = a.incl + static_cast<int64_t>(tile) * R4;
-      for (int e = tid; e < R4; e += NT) my_incl[e] = s_excl[e] + (e < El ? s_cnt[e] : 0);
-      __syncthreads();
-      if (tid == 0) {
-        __threadfence();
-        st_release_u64(a.flags + tile, kFlagTag | (epoch << 2) | kFlagPrefix);
-      }
-    }
-    int32_t* my_base = a.tile_counts + static_cast<int64_t>(tile) * a.base_stride_t;
-    for (int e = tid; e < El; e += NT) {
-      const int ex = tile > 0 ? s_excl[e] : 0;
-      my_base[e] = ex;
-      if (tile == N - 1) a.totals[e] = ex + s_cnt[e];
-    }
-  }
-  __syncthreads();
-  if (tid == 0) {
-    __threadfence();
-    unsigned* words = reinterpret_cast<unsigned*>(a.status);
-    if (atomicAdd(words + kWsDoneWord, 1u) == static_cast<unsigned>(N - 1)) {
-      words[kWsDoneWord] = 0u;  // every tile has read the epoch: the next call gets a new one
-      *ws_epoch(a) = (epoch + 1ull) & ((1ull << 61) - 1ull);
-    }
-  }
-}
-
-template <typename TIn, int VEC, int CPL, bool kLookback>
+template <typename TIn, int VEC, int CPL>
 __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) {
   extern __shared__ int smem[];
-  __shared__ int s_tile, s_ctl;
-  __shared__ unsigned long long s_epoch;
   const int k = a.k, El = a.E_local, RT = a.rows_per_tile;
   int* s_le = smem;
   int* whist = s_le + RT * k;
   unsigned* masks = reinterpret_cast<unsigned*>(whist + kGcWarps * El);
-  int* s_cnt = reinterpret_cast<int*>(masks + kGcWarps * El);
-  int* s_excl = s_cnt + a.row4;
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tile = blockIdx.x;
+  const int64_t row0 = static_cast<int64_t>(tile) * RT;
+  const int rows = static_cast<int>((a.T - row0) < RT ? (a.T - row0) : RT);
   for (int i = tid; i < kGcWarps * El; i += kGcThreads) {
     whist[i] = 0;
     masks[i] = 0u;
   }
+  __syncthreads();
   moe::pdl_wait();  // the logits may come from the previous kernel
   moe::pdl_launch_dependents();
-  moe::WaitHooks hooks{0u, moe::kWaitLimitNs};
-  int tile = blockIdx.x;
-  if constexpr (kLookback) {
-    hooks = moe::read_hooks(a.status);
-    lookback_enter(a, &s_tile, &s_epoch);
-    tile = s_tile < a.num_tiles ? s_tile : a.num_tiles;  // past the last tile: no rows (flagged below)
-  } else {
-    __syncthreads();
-  }
-  const int64_t row0 = static_cast<int64_t>(tile) * RT;
-  const int rows = static_cast<int>((a.T - row0) < RT ? ((a.T - row0) > 0 ? (a.T - row0) : 0) : RT);
 
   // A. gating, one warp per row (or the routes the caller gave)
   const TIn* logits = static_cast<const TIn*>(a.logits);
@@ -409,12 +210,7 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
   __syncthreads();
 
   // B. stable ranks inside the tile
-  rank_tile_slots(a, s_le, rows * k, row0, tile, whist, masks, kGcWarps, kLookback ? s_cnt : nullptr);
-  // C. the tile bases: the prefix over the tiles, in this pass
-  if constexpr (kLookback) {
-    __syncthreads();
-    tile_lookback<kGcThreads>(a, s_tile, s_epoch, hooks, s_cnt, s_excl, &s_ctl);
-  }
+  rank_tile_slots(a, s_le, rows * k, row0, tile, whist, masks, kGcWarps);
 }
 
 // One CTA of G warps per tile of kRowsPerTile tokens, G lanes per row: the tile's logits are staged
@@ -422,39 +218,28 @@ __global__ void __launch_bounds__(kGcThreads) gate_count_kernel(DispatchArgs a) 
 // warps rank the tile's slots and write its per-expert counts (rank_tile_slots, as gate_count_kernel).
 // Shared memory: staged rows [kRowsPerTile * stride chunks] | whist [G][E_local] | peer masks
 // [G][E_local] | s_le [kRowsPerTile * K].
-template <typename TIn, int K, int G, bool kLookback>
+template <typename TIn, int K, int G>
 __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a, int cpr) {
   constexpr int NT = 32 * G;
   extern __shared__ __align__(16) uint4 s_rows[];
-  __shared__ int s_tile, s_ctl;
-  __shared__ unsigned long long s_epoch;
   const int El = a.E_local;
   const int stride = moe_gate::lane_tile_stride(cpr);
   int* whist = reinterpret_cast<int*>(s_rows + kRowsPerTile * stride);
   unsigned* masks = reinterpret_cast<unsigned*>(whist + G * El);
   int* s_le = reinterpret_cast<int*>(masks + G * El);
-  int* s_cnt = s_le + kRowsPerTile * K;
-  int* s_excl = s_cnt + a.row4;
   const int tid = threadIdx.x;
+  const int tile = blockIdx.x;
+  const int64_t row0 = static_cast<int64_t>(tile) * kRowsPerTile;
+  const int rows = static_cast<int>((a.T - row0) < kRowsPerTile ? (a.T - row0) : kRowsPerTile);  // >= 1
   for (int e = tid; e < G * El; e += NT) {
     whist[e] = 0;
     masks[e] = 0u;
   }
   moe::pdl_wait();  // the logits may come from the previous kernel
   moe::pdl_launch_dependents();
-  moe::WaitHooks hooks{0u, moe::kWaitLimitNs};
-  int tile = blockIdx.x;
-  if constexpr (kLookback) {
-    hooks = moe::read_hooks(a.status);
-    lookback_enter(a, &s_tile, &s_epoch);
-    tile = s_tile < a.num_tiles ? s_tile : a.num_tiles;  // past the last tile: no rows (flagged below)
-  }
-  const int64_t row0 = static_cast<int64_t>(tile) * kRowsPerTile;
-  const int rows = static_cast<int>((a.T - row0) < kRowsPerTile ? ((a.T - row0) > 0 ? (a.T - row0) : 0)
-                                                                : kRowsPerTile);
-  if (rows > 0) moe_gate::lane_tile_load(static_cast<const uint4*>(a.logits) + row0 * cpr, rows, cpr, stride, s_rows, tid, NT);
+  moe_gate::lane_tile_load(static_cast<const uint4*>(a.logits) + row0 * cpr, rows, cpr, stride, s_rows, tid, NT);
   __syncthreads();
-  if (rows > 0) {  // uniform
+  {
     const int r = tid / G, g = tid % G;
     const int rr = r < rows ? r : rows - 1;  // every lane takes part in the group's shuffles
     float w[K];
@@ -471,44 +256,35 @@ __global__ void __launch_bounds__(32 * G) gate_count_lanes_kernel(DispatchArgs a
     }
   }
   __syncthreads();
-  rank_tile_slots(a, s_le, rows * K, row0, tile, whist, masks, G, kLookback ? s_cnt : nullptr);
-  if constexpr (kLookback) {
-    __syncthreads();
-    tile_lookback<NT>(a, s_tile, s_epoch, hooks, s_cnt, s_excl, &s_ctl);
-  }
+  rank_tile_slots(a, s_le, rows * K, row0, tile, whist, masks, G);
 }
 
 using LanesKernel = void (*)(DispatchArgs, int);
 
-template <typename TIn, int K, bool LB>
+template <typename TIn, int K>
 LanesKernel lanes_kernel_g(int G) {
   switch (G) {
-    case 1: return &gate_count_lanes_kernel<TIn, K, 1, LB>;
-    case 2: return &gate_count_lanes_kernel<TIn, K, 2, LB>;
-    case 4: return &gate_count_lanes_kernel<TIn, K, 4, LB>;
-    case 8: return &gate_count_lanes_kernel<TIn, K, 8, LB>;
-    default: return nullptr;
-  }
-}
-
-template <typename TIn, bool LB>
-LanesKernel lanes_kernel_for_lb(int k, int G) {
-  switch (k) {
-    case 1: return lanes_kernel_g<TIn, 1, LB>(G);
-    case 2: return lanes_kernel_g<TIn, 2, LB>(G);
-    case 3: return lanes_kernel_g<TIn, 3, LB>(G);
-    case 4: return lanes_kernel_g<TIn, 4, LB>(G);
-    case 5: return lanes_kernel_g<TIn, 5, LB>(G);
-    case 6: return lanes_kernel_g<TIn, 6, LB>(G);
-    case 7: return lanes_kernel_g<TIn, 7, LB>(G);
-    case 8: return lanes_kernel_g<TIn, 8, LB>(G);
+    case 1: return &gate_count_lanes_kernel<TIn, K, 1>;
+    case 2: return &gate_count_lanes_kernel<TIn, K, 2>;
+    case 4: return &gate_count_lanes_kernel<TIn, K, 4>;
+    case 8: return &gate_count_lanes_kernel<TIn, K, 8>;
     default: return nullptr;
   }
 }
 
 template <typename TIn>
-LanesKernel lanes_kernel_for(int k, int G, bool lookback) {
-  return lookback ? lanes_kernel_for_lb<TIn, true>(k, G) : lanes_kernel_for_lb<TIn, false>(k, G);
+LanesKernel lanes_kernel_for(int k, int G) {
+  switch (k) {
+    case 1: return lanes_kernel_g<TIn, 1>(G);
+    case 2: return lanes_kernel_g<TIn, 2>(G);
+    case 3: return lanes_kernel_g<TIn, 3>(G);
+    case 4: return lanes_kernel_g<TIn, 4>(G);
+    case 5: return lanes_kernel_g<TIn, 5>(G);
+    case 6: return lanes_kernel_g<TIn, 6>(G);
+    case 7: return lanes_kernel_g<TIn, 7>(G);
+    case 8: return lanes_kernel_g<TIn, 8>(G);
+    default: return nullptr;
+  }
 }
 
 // One CTA per local expert: its row of tile counts -> exclusive prefix over the tiles, in place;
@@ -615,7 +391,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     }
   }
   moe::pdl_launch_dependents();
-  moe::pdl_wait();  // ranks, tile bases and totals (gate_count_kernel, or tile_scan_kernel after it)
+  moe::pdl_wait();  // ranks (gate_count_kernel), tile bases and totals (tile_scan_kernel)
 
   // the slots' parked values (rank in the tile << 10 | local expert, or -1) and their tiles' bases
   // are loaded first, so that these loads are in flight during the offsets scan
@@ -633,7 +409,7 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
     base[m] = 0;
     if (pv[m] >= 0 && (pv[m] & 1023) < El) {
       const int64_t tile = (t0 + e / k) >> a.rt_shift;
-      base[m] = a.tile_counts[static_cast<int64_t>(pv[m] & 1023) * a.base_stride_e + tile * a.base_stride_t];
+      base[m] = a.tile_counts[static_cast<int64_t>(pv[m] & 1023) * a.num_tiles + tile];
     }
   }
 
@@ -970,12 +746,7 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
 template <typename TIn, int VEC, int CPL>
 struct GateCountFamily {
   using Fn = void (*)(DispatchArgs);
-  static Fn get() { return &gate_count_kernel<TIn, VEC, CPL, false>; }
-};
-template <typename TIn, int VEC, int CPL>
-struct GateCountLbFamily {
-  using Fn = void (*)(DispatchArgs);
-  static Fn get() { return &gate_count_kernel<TIn, VEC, CPL, true>; }
+  static Fn get() { return &gate_count_kernel<TIn, VEC, CPL>; }
 };
 template <typename TIn, int VEC, int CPL>
 struct SmallFamily {
@@ -1033,82 +804,26 @@ moe_status_t launch_tile_scan(const DispatchArgs& a, int E_local, cudaStream_t s
                                          dim3(kTsThreadsSmall), 0, st, a);
 }
 
-// Workspace layout after the 256-byte header.  Tile scan: tile counts (then bases) [E_local][tiles],
-// totals [E_local].  Lookback: flags [tiles] (u64), aggregates, inclusive prefixes and bases
-// [tiles][row4] each, totals [E_local].
 struct FusedLayout {
   int num_tiles;
-  bool lookback;
-  size_t tile_counts_off, totals_off, flags_off, agg_off, incl_off, bytes;
+  size_t tile_counts_off, totals_off, bytes;
 };
 
-bool use_lookback(int64_t num_tiles, int E_local) {
-  return num_tiles * static_cast<int64_t>(E_local) <= kLookbackMaxCells;
-}
-
-size_t align256(size_t x) { return (x + 255) & ~size_t{255}; }
-
-FusedLayout fused_layout(int64_t T, int E_local, int rows_per_tile, bool lookback) {
+FusedLayout fused_layout(int64_t T, int E_local, int rows_per_tile) {
   FusedLayout l{};
   const int64_t nt = (T + rows_per_tile - 1) / rows_per_tile;
   l.num_tiles = nt < 1 ? 1 : static_cast<int>(nt);
-  l.lookback = lookback;
-  const size_t N = static_cast<size_t>(l.num_tiles);
-  if (!lookback) {
-    l.tile_counts_off = kWsHeaderBytes;
-    l.totals_off = l.tile_counts_off + align256(N * E_local * 4);
-  } else {
-    const size_t row = static_cast<size_t>(row4_of(E_local)) * 4;
-    l.flags_off = kWsHeaderBytes;
-    l.agg_off = l.flags_off + align256(N * 8);
-    l.incl_off = l.agg_off + align256(N * row);
-    l.tile_counts_off = l.incl_off + align256(N * row);
-    l.totals_off = l.tile_counts_off + align256(N * row);
-  }
+  l.tile_counts_off = kWsHeaderBytes;
+  l.totals_off = l.tile_counts_off + ((static_cast<size_t>(l.num_tiles) * E_local * 4 + 255) & ~size_t{255});
   l.bytes = l.totals_off + static_cast<size_t>(E_local) * 4;
   return l;
-}
-
-// Layout for a call: the lookback when the tiles times the local experts are few enough.
-FusedLayout fused_layout_for(int64_t T, int E_local, int rows_per_tile) {
-  const int64_t nt = (T + rows_per_tile - 1) / rows_per_tile;
-  return fused_layout(T, E_local, rows_per_tile, use_lookback(nt < 1 ? 1 : nt, E_local));
-}
-
-// Workspace bytes that cover both modes at a tile height (the larger of the two).
-size_t fused_workspace_bytes(int64_t T, int E_local, int rows_per_tile) {
-  const size_t a = fused_layout(T, E_local, rows_per_tile, false).bytes;
-  const size_t b = fused_layout(T, E_local, rows_per_tile, true).bytes;
-  return a > b ? a : b;
-}
-
-// Fill the tile-count fields of the kernel arguments for a layout.
-void set_layout_args(DispatchArgs& a, const FusedLayout& lay, void* workspace) {
-  char* ws = static_cast<char*>(workspace);
-  a.num_tiles = lay.num_tiles;
-  a.row4 = row4_of(a.E_local);
-  a.tile_counts = reinterpret_cast<int32_t*>(ws + lay.tile_counts_off);
-  a.totals = reinterpret_cast<int32_t*>(ws + lay.totals_off);
-  if (lay.lookback) {
-    a.flags = reinterpret_cast<unsigned long long*>(ws + lay.flags_off);
-    a.agg = reinterpret_cast<int32_t*>(ws + lay.agg_off);
-    a.incl = reinterpret_cast<int32_t*>(ws + lay.incl_off);
-    a.base_stride_e = 1;
-    a.base_stride_t = a.row4;
-  } else {
-    a.flags = nullptr;
-    a.agg = nullptr;
-    a.incl = nullptr;
-    a.base_stride_e = lay.num_tiles;
-    a.base_stride_t = 1;
-  }
 }
 
 }  // namespace
 
 extern "C" size_t moe_route_dispatch_workspace_bytes(int64_t T, int32_t k, int32_t E_local) {
   if (T < 0 || k < 1 || E_local < 1) return 0;
-  return fused_workspace_bytes(T, E_local, kRowsPerTileSmall);  // the larger of the two tile heights' layouts
+  return fused_layout(T, E_local, kRowsPerTileSmall).bytes;  // the larger of the two tile heights' layouts
 }
 
 extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype, const void* hidden, int64_t T,
@@ -1169,9 +884,10 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   int rt = kRowsPerTile;
   if (!lanes && (T + kRowsPerTileSmall - 1) / kRowsPerTileSmall <= static_cast<int64_t>(sms) * kGcCtasPerSm)
     rt = kRowsPerTileSmall;
-  const FusedLayout lay = fused_layout_for(T, E_local, rt);
+  const FusedLayout lay = fused_layout(T, E_local, rt);
   a.rows_per_tile = rt;
   a.rt_shift = rt == kRowsPerTileSmall ? 4 : 5;
+  a.num_tiles = lay.num_tiles;
   a.topk_weights = topk_weights;
   a.topk_ids = topk_ids;
   a.counts = counts;
@@ -1181,7 +897,8 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   a.n_pad = num_tokens_post_pad;
   a.inv_perm = inv_perm;
   a.status = static_cast<int32_t*>(workspace);
-  set_layout_args(a, lay, workspace);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.tile_counts_off);
+  a.totals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.totals_off);
 
   // gating geometry of the warp-per-row kernels: widest aligned vector that spreads the row over the warp
   int vec_max = 16 / elem;
@@ -1214,12 +931,10 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
   if (lanes) {
     const int cpr = E * elem / 16;
     const int G = moe_gate::lane_gate_lanes(cpr);
-    LanesKernel lk = dtype == MOE_DTYPE_BF16 ? lanes_kernel_for<__nv_bfloat16>(k, G, lay.lookback)
-                                            : lanes_kernel_for<float>(k, G, lay.lookback);
+    LanesKernel lk = dtype == MOE_DTYPE_BF16 ? lanes_kernel_for<__nv_bfloat16>(k, G) : lanes_kernel_for<float>(k, G);
     if (lk == nullptr) return MOE_ERR_UNSUPPORTED;
     const size_t smem1 = static_cast<size_t>(kRowsPerTile) * moe_gate::lane_tile_stride(cpr) * sizeof(uint4) +
-                         (2 * static_cast<size_t>(G) * E_local + static_cast<size_t>(kRowsPerTile) * k +
-                          (lay.lookback ? 2 * static_cast<size_t>(a.row4) : 0)) * sizeof(int);
+                         (2 * static_cast<size_t>(G) * E_local + static_cast<size_t>(kRowsPerTile) * k) * sizeof(int);
     if (smem1 > 48 * 1024 &&
         cudaFuncSetAttribute(reinterpret_cast<const void*>(lk), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem1)) != cudaSuccess)
@@ -1229,15 +944,11 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
       return MOE_ERR_CUDA;
   } else {
     // the gating geometry does not matter when the routes are given (no row is gated)
-    GcKernel gk = lay.lookback
-                      ? (given_ids ? family_pick<GateCountLbFamily, float>(1, 1)
-                         : dtype == MOE_DTYPE_BF16 ? family_pick<GateCountLbFamily, __nv_bfloat16>(vec, cpl)
-                                                   : family_pick<GateCountLbFamily, float>(vec, cpl))
-                      : (given_ids ? family_pick<GateCountFamily, float>(1, 1)
-                         : dtype == MOE_DTYPE_BF16 ? family_pick<GateCountFamily, __nv_bfloat16>(vec, cpl)
-                                                   : family_pick<GateCountFamily, float>(vec, cpl));
+    GcKernel gk = given_ids ? family_pick<GateCountFamily, float>(1, 1)
+                  : dtype == MOE_DTYPE_BF16 ? family_pick<GateCountFamily, __nv_bfloat16>(vec, cpl)
+                                            : family_pick<GateCountFamily, float>(vec, cpl);
     if (gk == nullptr) return MOE_ERR_UNSUPPORTED;
-    const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local, lay.lookback) * sizeof(int);
+    const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
     if (smem1 > 48 * 1024 &&
         cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
                              static_cast<int>(smem1)) != cudaSuccess)
@@ -1245,7 +956,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
     if (moe_host::launch_pdl_max_shared(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
       return MOE_ERR_CUDA;
   }
-  if (!lay.lookback && launch_tile_scan(a, E_local, st) != MOE_OK) return MOE_ERR_CUDA;
+  if (launch_tile_scan(a, E_local, st) != MOE_OK) return MOE_ERR_CUDA;
 
   // tokens per CTA: at most kPgMaxTokens (and kPgCtaBytes of staged rows), chosen so that the CTAs
   // fill whole waves of kPgCtasPerSm per SM; shared memory sized so that no SM takes more
@@ -1270,7 +981,7 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
 // moe_align_permute through the tile kernels above (given routes, no gather).
 // ---------------------------------------------------------------------------------------------
 size_t moe_internal::align_tiles_workspace_bytes(int64_t T, int32_t E_local) {
-  return fused_workspace_bytes(T, E_local, kRowsPerTile);
+  return fused_layout(T, E_local, kRowsPerTile).bytes;
 }
 
 moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32_t k, int32_t E_global,
@@ -1290,9 +1001,10 @@ moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32
   a.P = T * k;
   a.C = moe_align_capacity(T, k, E_local, block_size);
   a.NB = static_cast<int>((a.C + block_size - 1) / block_size);
-  const FusedLayout lay = fused_layout_for(T, E_local, kRowsPerTile);
+  const FusedLayout lay = fused_layout(T, E_local, kRowsPerTile);
   a.rows_per_tile = kRowsPerTile;
   a.rt_shift = 5;
+  a.num_tiles = lay.num_tiles;
   a.topk_ids = const_cast<int32_t*>(topk_ids);  // read only: given_ids
   a.counts = counts;
   a.offsets = offsets;
@@ -1301,18 +1013,18 @@ moe_status_t moe_internal::align_tiles(const int32_t* topk_ids, int64_t T, int32
   a.n_pad = num_tokens_post_pad;
   a.inv_perm = inv_perm;
   a.status = static_cast<int32_t*>(workspace);
-  set_layout_args(a, lay, workspace);
+  a.tile_counts = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.tile_counts_off);
+  a.totals = reinterpret_cast<int32_t*>(static_cast<char*>(workspace) + lay.totals_off);
 
-  GcKernel gk = lay.lookback ? family_pick<GateCountLbFamily, float>(1, 1)  // no row is gated
-                             : family_pick<GateCountFamily, float>(1, 1);
-  const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local, lay.lookback) * sizeof(int);
+  GcKernel gk = family_pick<GateCountFamily, float>(1, 1);  // no row is gated
+  const size_t smem1 = gc_smem_ints(a.rows_per_tile, k, E_local) * sizeof(int);
   if (smem1 > 48 * 1024 &&
       cudaFuncSetAttribute(reinterpret_cast<const void*>(gk), cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem1)) != cudaSuccess)
     return MOE_ERR_CUDA;
   if (moe_host::launch_pdl_max_shared(gk, dim3(static_cast<unsigned>(a.num_tiles)), dim3(kGcThreads), smem1, st, a) != MOE_OK)
     return MOE_ERR_CUDA;
-  if (!lay.lookback && launch_tile_scan(a, E_local, st) != MOE_OK) return MOE_ERR_CUDA;
+  if (launch_tile_scan(a, E_local, st) != MOE_OK) return MOE_ERR_CUDA;
   // placement only: up to kPgMaxTokens tokens per one-warp CTA, the CTAs filling whole waves
   const int sms = moe_host::sm_count();
   if (sms <= 0) return MOE_ERR_CUDA;
