@@ -178,3 +178,94 @@ class EpExchange:
         if hi > lo:
             moe_reduce_partials([self.recv[b][r, :hi - lo] for r in range(self.world)], out=self.out, stream=s)
         return self.out
+
+
+class EpAllToAll:
+    """The expert-parallel layer with the tokens sharded over the ranks (the all-to-all form).
+
+    Rank r holds its own T_r tokens (``T_per_rank[r]``) and owns a contiguous block of experts.  One
+    ``step`` on every rank:
+      1. gating of this rank's tokens (moe_topk_softmax) into buffers the other ranks can read;
+      2. a barrier; each owner copies every rank's routes into one list (one peer copy per rank), aligns
+         them with its expert_map (moe_align_permute: the expert-grouped layout of every rank's slots
+         on its experts, rank by rank in slot order) and pulls the hidden rows it needs from each rank
+         (moe_gather with that rank's hidden rows as the source: bulk loads from the rank's memory);
+      3. the owner's experts run on the expert-grouped rows (``expert_out`` stands in for them here);
+      4. for every rank, the owner's moe_combine of that rank's slots on its experts is written straight
+         into the rank's receive buffer (stores into the rank's memory);
+      5. a barrier; each rank reduces its partials in ascending owner order (moe_reduce_partials): the
+         same sum as the replicated-token exchange (fp32 in rank order, rounded once to bf16).
+    The buffers other ranks read or write (routes, weights, hidden rows, receive buffers) are shared
+    through CUDA IPC.  The caller writes this step's hidden rows into ``hidden`` before ``step``.
+    Returns this rank's layer output [T_r, H] (overwritten by the next step)."""
+
+    def __init__(self, T_per_rank, E: int, k: int, H: int, block_size: int, renormalize: bool, device,
+                 group: Optional[dist.ProcessGroup] = None, logits_dtype=torch.bfloat16):
+        from torch.multiprocessing.reductions import reduce_tensor
+        from . import binding as B
+        self.group = group
+        self.world = dist.get_world_size(group)
+        self.rank = dist.get_rank(group)
+        assert len(T_per_rank) == self.world
+        self.T = list(int(t) for t in T_per_rank)
+        self.off = [sum(self.T[:r]) for r in range(self.world)]
+        self.T_total = sum(self.T)
+        self.E, self.k, self.H, self.block_size, self.renormalize = E, k, H, block_size, renormalize
+        emap, self.E_local = ep_expert_map(E, self.world, self.rank)
+        self.expert_map = emap.to(device)
+        Tr = self.T[self.rank]
+        # shared with the other ranks
+        self.topk_ids = torch.zeros((max(1, Tr), k), dtype=torch.int32, device=device)
+        self.topk_weights = torch.zeros((max(1, Tr), k), dtype=torch.float32, device=device)
+        self.hidden = torch.zeros((max(1, Tr), H), dtype=torch.bfloat16, device=device)
+        self.recv = torch.zeros((self.world, max(1, Tr), H), dtype=torch.bfloat16, device=device)
+        # this owner's own
+        self.ids_all = torch.zeros((max(1, self.T_total), k), dtype=torch.int32, device=device)
+        self.align = B.alloc_align_outputs(self.T_total, k, self.E_local, block_size, device)
+        self.capacity = self.align.capacity
+        self.workspace = B.alloc_workspace(self.T_total, k, self.E_local, device)
+        self.permuted = torch.empty((self.capacity, H), dtype=torch.bfloat16, device=device)
+        self.out = torch.empty((Tr, H), dtype=torch.bfloat16, device=device)
+        torch.cuda.synchronize(device)
+        mine = [reduce_tensor(t) for t in (self.topk_ids, self.topk_weights, self.hidden, self.recv)]
+        handles = [None] * self.world
+        dist.all_gather_object(handles, mine, group=group)
+        own = (self.topk_ids, self.topk_weights, self.hidden, self.recv)
+        peers = [own if o == self.rank else tuple(h[0](*h[1]) for h in handles[o]) for o in range(self.world)]
+        self.peer_ids, self.peer_w, self.peer_hidden, self.peer_recv = (list(x) for x in zip(*peers))
+        dist.barrier(group=group)
+
+    def slots(self, r: int) -> slice:
+        """Rank r's slots in this owner's list of every rank's routes."""
+        return slice(self.off[r] * self.k, (self.off[r] + self.T[r]) * self.k)
+
+    def step(self, logits: torch.Tensor, expert_out: torch.Tensor, stream=None) -> torch.Tensor:
+        from . import binding as B
+        s = torch.cuda.current_stream() if stream is None else stream
+        Tr, k = self.T[self.rank], self.k
+        with torch.cuda.stream(s):
+            if Tr:
+                B.moe_topk_softmax(logits, k, self.renormalize, self.topk_weights[:Tr], self.topk_ids[:Tr], s)
+            s.synchronize()
+            dist.barrier(group=self.group)  # every rank's routes and hidden rows are ready
+            for r in range(self.world):
+                if self.T[r]:
+                    self.ids_all[self.off[r]:self.off[r] + self.T[r]].copy_(self.peer_ids[r][:self.T[r]],
+                                                                            non_blocking=True)
+            B.moe_align_permute(self.ids_all[:self.T_total], self.E, self.block_size, self.expert_map, self.E_local,
+                                self.align, self.workspace, s)
+            inv = self.align.inv_perm
+            for r in range(self.world):
+                if self.T[r]:
+                    B.moe_gather(self.peer_hidden[r][:self.T[r]], k, inv[self.slots(r)], self.capacity,
+                                 permuted=self.permuted, device_status=self.workspace, stream=s)
+            # (the owner's experts run here on self.permuted; expert_out stands in for their output)
+            for r in range(self.world):
+                if self.T[r]:
+                    B.moe_combine(expert_out, self.peer_w[r][:self.T[r]], inv[self.slots(r)],
+                                  self.peer_recv[r][self.rank, :self.T[r]], device_status=self.workspace, stream=s)
+            s.synchronize()
+            dist.barrier(group=self.group)  # every owner's partial for every rank has landed
+            if Tr:
+                B.moe_reduce_partials([self.recv[o, :Tr] for o in range(self.world)], out=self.out, stream=s)
+        return self.out
