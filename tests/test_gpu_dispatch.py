@@ -69,7 +69,9 @@ CASES = [
     ("lanes_bf16_E56_k7_strided_map", 1111, 56, 7, torch.bfloat16, False, "strided", 14, 16, 32),
     ("lanes_wide_bf16_E256_k8_strided_map", 16500, 256, 8, torch.bfloat16, True, "strided", 64, 128, 16),
     ("lanes_wide_bf16_E192_k5_ties", 16401, 192, 5, torch.bfloat16, False, None, 192, 32, 8),
-    # many tiles and many local experts (a long tile scan per expert); a ragged fp32 lanes batch
+    # more tiles than the gating kernel's CTAs resident at once (625 tiles of 512 threads); many local
+    # experts (a long tile scan per expert); ragged lanes batches
+    ("many_tiles_fp32_E128", 20000, 128, 8, torch.float32, True, None, 128, 16, 16),
     ("many_tiles_E512", 5000, 512, 8, torch.bfloat16, True, None, 512, 16, 64),
     ("lanes_fp32_E60_ragged", 16400, 60, 4, torch.float32, False, None, 60, 64, 16),
     ("lanes_bf16_E61_no_lanes_odd", 4000, 61, 3, torch.bfloat16, True, None, 61, 5, 16),
