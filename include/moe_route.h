@@ -251,17 +251,17 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
                          int32_t k, int32_t H, int64_t capacity, void* out, int32_t* device_status, void* stream);
 
 /*
- * moe_route_dispatch -- gating, align and permute-gather in one call, as two kernels (one for
- * small batches) instead of four ("Upstream Reference", "File Index": the gate -> topk -> expand part of the FusedMoE
- * pipeline).  Every output is the same as from moe_topk_softmax (flags: MOE_RENORMALIZE) then
+ * moe_route_dispatch -- gating, align and permute-gather in one call, as three kernels (one for
+ * small batches) instead of the stage calls' four or more ("Upstream Reference", "File Index": the
+ * gate -> topk -> expand part of the FusedMoE pipeline).  Every output is the same as from moe_topk_softmax (flags: MOE_RENORMALIZE) then
  * moe_align_permute then moe_gather (without MOE_GATHER_ZERO_PAD), bit for bit:
  *   topk_weights [T,k], topk_ids [T,k], counts [E_local], offsets [E_local+1],
  *   sorted_token_ids [C], expert_ids [NB], num_tokens_post_pad [1], inv_perm [T*k],
  *   permuted [C, H] (rows of local slots; pad rows untouched).
  * For T > 32, T*k > 256 or E > 256: the first kernel gates tiles of tokens and counts each tile's slots
- * per local expert with their ranks inside the tile; the last of its CTAs to finish turns the
- * tile counts into the padded layout; the second kernel gives every slot its row and copies the
- * hidden rows there.  Smaller batches (decode) take one kernel with one CTA per slot: each CTA
+ * per local expert with their ranks inside the tile; the second turns each expert's tile counts into
+ * its prefix over the tiles and its total; the third scans the padded totals into the offsets, gives
+ * every slot its row and copies the hidden rows there.  Smaller batches (decode) take one kernel with one CTA per slot: each CTA
  * routes the whole batch by itself, CTA 0 writes the routing outputs and every CTA copies the
  * hidden row of its own slot.
  *   logits [T, E] bf16/fp32 (dtype); hidden [T, H] bf16, 16-byte aligned, H % 8 == 0 and
@@ -271,7 +271,10 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
  *   input (the align input of moe_align_permute), logits and topk_weights may be NULL and are
  *   not read or written; every other output is as from moe_align_permute + moe_gather.
  *   workspace: >= moe_route_dispatch_workspace_bytes(T, k, E_local) bytes, zeroed before its
- *   first use and left ready by every call; its first 4 bytes are the device status word.
+ *   first use and left ready by every call; its first 4 bytes are the device status word.  Words
+ *   2 and 3 are test hooks and must stay zero in normal use (moe_workspace_init zeroes them): a
+ *   nonzero word 2 makes the placement kernel withhold its hidden-row loads so that its bounded wait
+ *   runs out (MOE_ERR_TIMEOUT), word 3 sets that wait's limit in microseconds.
  *   Errors: as the three calls it replaces; UNSUPPORTED also for H > 65536.
  */
 MOE_API size_t moe_route_dispatch_workspace_bytes(int64_t T, int32_t k, int32_t E_local);
