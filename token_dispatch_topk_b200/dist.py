@@ -10,8 +10,8 @@ Two uses:
       - ``EpExchange`` (the library's form, a reduce-scatter): each rank's moe_combine writes each
         owner's token range (``ep_token_range``) of its partial straight into its slot of that
         owner's receive buffer, in the owner's memory, shared between the processes through CUDA IPC
-        (on several GPUs the combine's own stores cross NVLink; plain 16-byte stores, no TMA, no
-        multicast); each rank then synchronises its stream and joins a process-group barrier, so
+        and mapped in each rank's own device context (on several GPUs the combine's own stores cross
+        NVLink; plain 16-byte stores, no TMA, no multicast); each rank then synchronises its stream and joins a process-group barrier, so
         that every store into every owner's buffer has completed before any owner reads; then each
         owner runs moe_reduce_partials over its slots in rank order.  Two receive buffers alternate
         between steps, so one barrier per step also keeps a step's stores away from the buffer the
@@ -107,6 +107,26 @@ def ep_reduce_received(received, out: Optional[torch.Tensor] = None, stream=None
     return moe_reduce_partials(received, out=out, stream=stream)
 
 
+def _share(t: torch.Tensor):
+    """A picklable CUDA IPC handle of a device tensor (torch's own sharing of CUDA storage)."""
+    from torch.multiprocessing.reductions import reduce_tensor
+    return reduce_tensor(t)
+
+
+def _open_shared(handle, device) -> torch.Tensor:
+    """Map another process's tensor (a handle from ``_share``) into this process, opened in the context
+    of this rank's own device: the mapping is then this device's, with peer access enabled as needed,
+    so this device's kernels may read and write it (over NVLink when it lives on another GPU).  The
+    tensor reports this device; its memory is the other process's."""
+    from torch.multiprocessing.reductions import rebuild_cuda_tensor
+    fn, args = handle
+    if fn is not rebuild_cuda_tensor or len(args) != 15:
+        raise RuntimeError("unexpected CUDA IPC handle layout")
+    args = list(args)
+    args[6] = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    return fn(*args)
+
+
 def ep_reduce_partials(partial: torch.Tensor, group: Optional[dist.ProcessGroup] = None,
                        reduce=None) -> torch.Tensor:
     """Sum the ranks' bf16 partial combines [T, H] (the collective baseline of the exchange): an
@@ -135,7 +155,6 @@ class EpExchange:
     next step overwrites.  Without a process group it is a single rank's exchange (its own buffer)."""
 
     def __init__(self, T: int, H: int, device, group: Optional[dist.ProcessGroup] = None, buffers: int = 2):
-        from torch.multiprocessing.reductions import reduce_tensor
         self.group = group
         grouped = dist.is_available() and dist.is_initialized()
         self.world = dist.get_world_size(group) if grouped else 1  # one rank: its own buffer, no barrier
@@ -148,11 +167,11 @@ class EpExchange:
         self.out = torch.empty((hi - lo, H), dtype=torch.bfloat16, device=device)
         torch.cuda.synchronize(device)
         if self.world > 1:
-            mine = [reduce_tensor(b) for b in self.recv]
+            mine = [_share(b) for b in self.recv]
             handles = [None] * self.world
             dist.all_gather_object(handles, mine, group=group)
             # remote[b][o]: owner o's receive buffer b, as mapped in this process
-            self.remote = [[self.recv[b] if o == self.rank else handles[o][b][0](*handles[o][b][1])
+            self.remote = [[self.recv[b] if o == self.rank else _open_shared(handles[o][b], device)
                             for o in range(self.world)] for b in range(buffers)]
             dist.barrier(group=group)
         else:
@@ -201,7 +220,6 @@ class EpAllToAll:
 
     def __init__(self, T_per_rank, E: int, k: int, H: int, block_size: int, renormalize: bool, device,
                  group: Optional[dist.ProcessGroup] = None, logits_dtype=torch.bfloat16):
-        from torch.multiprocessing.reductions import reduce_tensor
         from . import binding as B
         self.group = group
         self.world = dist.get_world_size(group)
@@ -227,11 +245,12 @@ class EpAllToAll:
         self.permuted = torch.empty((self.capacity, H), dtype=torch.bfloat16, device=device)
         self.out = torch.empty((Tr, H), dtype=torch.bfloat16, device=device)
         torch.cuda.synchronize(device)
-        mine = [reduce_tensor(t) for t in (self.topk_ids, self.topk_weights, self.hidden, self.recv)]
+        mine = [_share(t) for t in (self.topk_ids, self.topk_weights, self.hidden, self.recv)]
         handles = [None] * self.world
         dist.all_gather_object(handles, mine, group=group)
         own = (self.topk_ids, self.topk_weights, self.hidden, self.recv)
-        peers = [own if o == self.rank else tuple(h[0](*h[1]) for h in handles[o]) for o in range(self.world)]
+        peers = [own if o == self.rank else tuple(_open_shared(h, device) for h in handles[o])
+                 for o in range(self.world)]
         self.peer_ids, self.peer_w, self.peer_hidden, self.peer_recv = (list(x) for x in zip(*peers))
         dist.barrier(group=group)
 
