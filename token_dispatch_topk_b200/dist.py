@@ -113,6 +113,19 @@ def _share(t: torch.Tensor):
     return reduce_tensor(t)
 
 
+def _check_peer_access(device, group: Optional[dist.ProcessGroup] = None) -> None:
+    """Every rank's device must reach every other rank's device directly (NVLink or PCIe peer access)
+    before buffers are shared: the kernels read and write the peers' memory with plain loads and stores.
+    Raises on this rank when one cannot; gathers the ranks' device indices through the process group."""
+    me = torch.device(device).index
+    me = torch.cuda.current_device() if me is None else me
+    devs = [None] * dist.get_world_size(group)
+    dist.all_gather_object(devs, me, group=group)
+    for d in devs:
+        if d != me and not torch.cuda.can_device_access_peer(me, d):
+            raise RuntimeError(f"device {me} cannot access device {d} directly: no shared receive buffers")
+
+
 def _open_shared(handle, device) -> torch.Tensor:
     """Map another process's tensor (a handle from ``_share``) into this process, opened in the context
     of this rank's own device: the mapping is then this device's, with peer access enabled as needed,
@@ -167,6 +180,7 @@ class EpExchange:
         self.out = torch.empty((hi - lo, H), dtype=torch.bfloat16, device=device)
         torch.cuda.synchronize(device)
         if self.world > 1:
+            _check_peer_access(device, group)
             mine = [_share(b) for b in self.recv]
             handles = [None] * self.world
             dist.all_gather_object(handles, mine, group=group)
@@ -216,14 +230,16 @@ class EpAllToAll:
          same sum as the replicated-token exchange (fp32 in rank order, rounded once to bf16).
     The buffers other ranks read or write (routes, weights, hidden rows, receive buffers) are shared
     through CUDA IPC.  The caller writes this step's hidden rows into ``hidden`` before ``step``.
-    Returns this rank's layer output [T_r, H] (overwritten by the next step)."""
+    Returns this rank's layer output [T_r, H] (overwritten by the next step).  Without a process
+    group it is a single rank's layer (its own buffers, no barrier)."""
 
     def __init__(self, T_per_rank, E: int, k: int, H: int, block_size: int, renormalize: bool, device,
                  group: Optional[dist.ProcessGroup] = None, logits_dtype=torch.bfloat16):
         from . import binding as B
         self.group = group
-        self.world = dist.get_world_size(group)
-        self.rank = dist.get_rank(group)
+        grouped = dist.is_available() and dist.is_initialized()
+        self.world = dist.get_world_size(group) if grouped else 1  # one rank: its own buffers, no barrier
+        self.rank = dist.get_rank(group) if grouped else 0
         assert len(T_per_rank) == self.world
         self.T = list(int(t) for t in T_per_rank)
         self.off = [sum(self.T[:r]) for r in range(self.world)]
@@ -245,14 +261,18 @@ class EpAllToAll:
         self.permuted = torch.empty((self.capacity, H), dtype=torch.bfloat16, device=device)
         self.out = torch.empty((Tr, H), dtype=torch.bfloat16, device=device)
         torch.cuda.synchronize(device)
-        mine = [_share(t) for t in (self.topk_ids, self.topk_weights, self.hidden, self.recv)]
-        handles = [None] * self.world
-        dist.all_gather_object(handles, mine, group=group)
         own = (self.topk_ids, self.topk_weights, self.hidden, self.recv)
-        peers = [own if o == self.rank else tuple(_open_shared(h, device) for h in handles[o])
-                 for o in range(self.world)]
+        if self.world > 1:
+            _check_peer_access(device, group)
+            mine = [_share(t) for t in own]
+            handles = [None] * self.world
+            dist.all_gather_object(handles, mine, group=group)
+            peers = [own if o == self.rank else tuple(_open_shared(h, device) for h in handles[o])
+                     for o in range(self.world)]
+            dist.barrier(group=group)
+        else:
+            peers = [own]
         self.peer_ids, self.peer_w, self.peer_hidden, self.peer_recv = (list(x) for x in zip(*peers))
-        dist.barrier(group=group)
 
     def slots(self, r: int) -> slice:
         """Rank r's slots in this owner's list of every rank's routes."""
@@ -265,8 +285,9 @@ class EpAllToAll:
         with torch.cuda.stream(s):
             if Tr:
                 B.moe_topk_softmax(logits, k, self.renormalize, self.topk_weights[:Tr], self.topk_ids[:Tr], s)
-            s.synchronize()
-            dist.barrier(group=self.group)  # every rank's routes and hidden rows are ready
+            if self.world > 1:
+                s.synchronize()
+                dist.barrier(group=self.group)  # every rank's routes and hidden rows are ready
             for r in range(self.world):
                 if self.T[r]:
                     self.ids_all[self.off[r]:self.off[r] + self.T[r]].copy_(self.peer_ids[r][:self.T[r]],
@@ -283,8 +304,9 @@ class EpAllToAll:
                 if self.T[r]:
                     B.moe_combine(expert_out, self.peer_w[r][:self.T[r]], inv[self.slots(r)],
                                   self.peer_recv[r][self.rank, :self.T[r]], device_status=self.workspace, stream=s)
-            s.synchronize()
-            dist.barrier(group=self.group)  # every owner's partial for every rank has landed
+            if self.world > 1:
+                s.synchronize()
+                dist.barrier(group=self.group)  # every owner's partial for every rank has landed
             if Tr:
                 B.moe_reduce_partials([self.recv[o, :Tr] for o in range(self.world)], out=self.out, stream=s)
         return self.out
