@@ -193,9 +193,11 @@ MOE_API moe_status_t moe_align_permute(const int32_t* topk_ids, int64_t T, int32
  *   - no workspace: the completion ticket and the per-tile expert counters live in a fixed
  *     1 MiB array inside the library, one per GPU that loads it, held until the process exits;
  *   - it always runs the count + place tile kernels; sizes whose scratch would exceed that
- *     array (a 256-byte header plus 4 bytes per local expert per tile of up to 8192 slots,
- *     > 1 MiB, e.g. E_local = 1024 with more than about 1M slots) return MOE_ERR_UNSUPPORTED
- *     before anything is enqueued;
+ *     array return MOE_ERR_UNSUPPORTED before anything is enqueued.  The scratch is a 256-byte
+ *     header plus 4 bytes per local expert per tile; a tile holds 2048 slots, doubled (up to
+ *     8192) while there would be more than 256 tiles, and above 4096 slots at least 16 tiles'
+ *     counters are kept.  With E_local = 1024, for example, up to 2 088 960 slots fit, except
+ *     522 241 to 524 288 and 1 044 481 to 1 048 576 (256 tiles);
  *   - device_status: a caller device int32 that collects device-side errors, or NULL.
  *   It calls no cudaMalloc, cudaFree or other allocating routine.  The first call in each
  *   CUDA context (the device's primary context; again after a device reset, which makes a new

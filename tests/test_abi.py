@@ -173,5 +173,8 @@ def test_noalloc_rejects_sizes_beyond_its_scratch_on_the_host():
     f = lib.moe_align_permute_noalloc
     assert f(p, 522241, 4, 1024, N, 1024, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED
     assert f(p, 1 << 18, 4, 1024, N, 1024, 64, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED
+    # every size whose tiles number 256 (of 2048, 4096 or 8192 slots) is beyond the array
+    for slots in (522241, 524288, 1044481, 1048576, 2088961):
+        assert f(p, slots, 1, 1024, N, 1024, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED, slots
     assert f(p, 4, 4, 2048, N, 2048, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_UNSUPPORTED  # E_local > 1024
     assert f(p, 4, 4, 8, N, 4, 16, p, p, p, p, p, p, N, N) == B.MOE_ERR_INVALID_ARG  # identity map, E_local != E
