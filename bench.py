@@ -18,7 +18,9 @@ N > 1 runs the layer expert-parallel (strong scaling): every rank routes the sam
 contiguous block of E/N experts, combines its local slots into the owners' receive buffers (CUDA IPC,
 the stores crossing NVLink) and reduces the rows it owns (dist.EpExchange); a step ends with the
 layer output spread over the ranks.  ``--dp`` runs one independent batch per GPU instead (weak
-scaling, no exchange); ``--ep`` takes the expert-parallel step on one GPU too.
+scaling, no exchange); ``--ep`` takes the expert-parallel step on one GPU too; ``--a2a`` shards the
+workload's tokens over the ranks instead (dist.EpAllToAll: each owner pulls the hidden rows its
+experts need from every rank and pushes each rank's partial combine back).
 Rank 0 prints one JSON line.
 
 Also reported: per-stage device times and achieved HBM bandwidth from the algorithmic bytes (for
@@ -50,6 +52,7 @@ METRIC = "routed tokens/s (gate+align+permute+combine) and achieved HBM GB/s vs 
 UNIT = "tokens/s"
 L2_FLUSH_BYTES = 256 << 20
 FALLBACK_HBM_GBS = 6650.0
+NVLINK_PEER_GBS = 770.0  # measured peer copy on this machine's B200s, per direction per GPU
 KERNEL_SOURCES = {
     "topk_row_warp_kernel": "token_dispatch_topk_b200/csrc/topk_softmax.cu",
     "align_cluster_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
@@ -78,6 +81,8 @@ def parse_args():
     p.add_argument("--no-sub-workloads", action="store_true", help="time the headline workload only")
     p.add_argument("--dp", action="store_true", help="N > 1: one independent batch per GPU (no exchange)")
     p.add_argument("--ep", action="store_true", help="the expert-parallel step even on one GPU")
+    p.add_argument("--a2a", action="store_true",
+                   help="the expert-parallel layer with the tokens sharded over the ranks (EpAllToAll)")
     p.add_argument("--seed", type=int, default=0)
     p.add_argument("--no-graph", action="store_true", help="launch the calls directly instead of a graph")
     p.add_argument("--flush-always", action="store_true",
@@ -725,9 +730,19 @@ def measure_ep(wl, ctx: Ctx) -> dict:
             rt = 32
         n_dispatch = 2 if -(-wl.T // rt) * El <= 65536 else 3
     per_step = n_dispatch + sum(1 for a, b in ex.ranges if b > a) + (1 if hi > lo else 0)
+    step_s = total_ms / args.steps / 1e3
+    # roofline of the exchange: the bytes this rank's combine stores into other ranks' memory, against the
+    # measured peer-copy bandwidth of this machine (770 GB/s per direction per GPU; 900 GB/s nominal)
+    nvlink = None if nvlink_bytes == 0 else {
+        "bound": "nvlink", "bytes_per_step": nvlink_bytes, "peak": NVLINK_PEER_GBS, "unit": "GB/s",
+        "achieved": nvlink_bytes / step_s / 1e9, "frac": nvlink_bytes / step_s / 1e9 / NVLINK_PEER_GBS,
+        "target_ms_per_step": 1e3 * nvlink_bytes / (NVLINK_PEER_GBS * 1e9),
+        "note": "achieved = this rank's peer-store bytes over the whole step time (the step also gates, "
+                "gathers and reduces)"}
     return {"workload": wl.name, "value": wl.T * args.steps / (total_ms / 1e3), "unit": UNIT,
             "ms_per_step": total_ms / args.steps, "E_local": El, "routed_slots_local_rank0": R,
             "owned_tokens_rank0": hi - lo, "peer_store_bytes_per_rank_per_step": nvlink_bytes,
+            "nvlink_roofline": nvlink,
             "launches_per_step": per_step, "gpu_launches": per_step * args.steps, "clocks": clocks,
             "e2e": {"value": wl.T * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
                     "h2d_bytes_per_step": logits_h.numel() * logits_h.element_size() +
@@ -738,6 +753,60 @@ def measure_ep(wl, ctx: Ctx) -> dict:
             "parallelism": f"expert parallel over {ws} ranks ({El} local experts each): moe_route_dispatch, "
                            f"moe_combine into the owners' receive buffers (CUDA IPC), barrier, moe_reduce_partials",
             "timing": "CUDA events around K steps on the launching stream (host barrier inside each step), "
+                      "max over ranks"}
+
+
+def measure_a2a(wl, ctx: Ctx) -> dict:
+    """The expert-parallel layer with the workload's T tokens sharded over the ranks (dist.EpAllToAll,
+    strong scaling): rank r gates its own token range; every owner aligns every rank's routes on its
+    experts, pulls the hidden rows it needs and pushes each rank's partial combine back; each rank
+    reduces its partials.  Two barriers per step (no CUDA graph).  CUDA events around K steps on the
+    launching stream, max over ranks; value = T * K / that time."""
+    import torch
+    import torch.distributed as dist
+    import token_dispatch_topk_b200 as tdt
+    from token_dispatch_topk_b200 import inputs as I
+    from token_dispatch_topk_b200.dist import EpAllToAll, ep_token_range, max_over_ranks
+
+    args, dev, stream, ws, rank = ctx.args, ctx.dev, ctx.stream, ctx.ws, ctx.rank
+    ranges = [ep_token_range(wl.T, ws, r) for r in range(ws)]
+    lo, hi = ranges[rank]
+    T_per_rank = [b - a for a, b in ranges]
+    logits = I.make_logits(wl, seed=args.seed, device=dev)[lo:hi].contiguous()  # this rank's tokens
+    ex = EpAllToAll(T_per_rank, wl.E, wl.k, wl.H, wl.block_size, wl.renormalize, dev, logits_dtype=logits.dtype)
+    ex.hidden[:hi - lo].copy_(I.hidden_rows(torch.arange(lo, hi), wl.H, seed=args.seed, device=dev))
+    y = I.make_expert_out(ex.capacity, wl.H, seed=args.seed * 16 + 5 + rank, device=dev)  # this owner's experts
+
+    def step():
+        ex.step(logits, y, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            step()
+    stream.synchronize()
+    if tdt.moe_read_status(ex.workspace) != tdt.MOE_OK:
+        raise RuntimeError("all-to-all warm-up: device status is not MOE_OK")
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+    stream.synchronize()
+    total_ms = max_over_ranks(e0.elapsed_time(e1), dev)
+    if tdt.moe_read_status(ex.workspace) != tdt.MOE_OK:
+        raise RuntimeError("all-to-all steps: device status is not MOE_OK")
+    per_step = 1 + ws + sum(1 for t in T_per_rank if t) * 2 + (1 if hi > lo else 0) + 2  # gate, align (2), gathers, combines, reduce
+    return {"workload": wl.name, "value": wl.T * args.steps / (total_ms / 1e3), "unit": UNIT,
+            "ms_per_step": total_ms / args.steps, "E_local": ex.E_local, "tokens_rank0": T_per_rank[0],
+            "launches_per_step_approx": per_step,
+            "parallelism": f"expert parallel over {ws} ranks, tokens sharded ({T_per_rank[0]} on rank 0): gating, "
+                           f"align of every rank's routes, moe_gather pulling rows from each rank, moe_combine "
+                           f"pushing partials, barrier, moe_reduce_partials",
+            "timing": "CUDA events around K steps on the launching stream (host barriers inside each step), "
                       "max over ranks"}
 
 
@@ -779,6 +848,22 @@ def main():
         dist.init_process_group("nccl", device_id=dev, timeout=timedelta(seconds=120))
     tdt.load_library()
     ctx = Ctx(args, dev, ws, rank)
+
+    if args.a2a:
+        rec = measure_a2a(wl, ctx)
+        if rank == 0:
+            print(json.dumps({
+                "metric": METRIC, "value": rec["value"], "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+                "warmup": args.warmup, "ms_per_step": rec["ms_per_step"], "higher_is_better": True,
+                "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+                "data": "synthetic (seeded, counter-based; see token_dispatch_topk_b200/inputs.py)",
+                "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
+                           "parallelism": rec["parallelism"], "cuda_graph": False},
+                "expert_parallel_all_to_all": rec, "e2e": None, "cpu_baseline": None}), flush=True)
+        if ws > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return 0
 
     if (ws > 1 and not args.dp) or args.ep:
         rec = measure_ep(wl, ctx)
