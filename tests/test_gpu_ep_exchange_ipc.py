@@ -20,7 +20,7 @@ import oracle
 
 pytestmark = pytest.mark.gpu
 
-T, E, K, H, BS, STEPS = 301, 48, 6, 136, 8, 3
+E, K, H, BS, STEPS = 48, 6, 136, 8, 3
 
 
 def _free_port() -> int:
@@ -33,7 +33,7 @@ def _bits(t):
     return t.detach().contiguous().cpu().view(torch.int16).numpy().view(np.uint16)
 
 
-def _worker(rank, world, port, q):
+def _worker(rank, world, T, port, q):
     import torch.distributed as dist
     import token_dispatch_topk_b200 as tdt
     from token_dispatch_topk_b200 import dist as D
@@ -65,14 +65,15 @@ def _worker(rank, world, port, q):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("world", [2, 3])
-def test_ep_exchange_through_ipc_on_one_gpu(world):
+@pytest.mark.parametrize("T,world", [(301, 2), (301, 3), (2, 3)], ids=["T301_two_ranks", "T301_three_ranks",
+                                                                      "decode_T2_owner_without_tokens"])
+def test_ep_exchange_through_ipc_on_one_gpu(T, world):
     assert torch.cuda.is_available()
     oracle.default()
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
+    procs = [ctx.Process(target=_worker, args=(r, world, T, port, q)) for r in range(world)]
     for p in procs:
         p.start()
     res = dict(q.get(timeout=300) for _ in procs)
