@@ -640,6 +640,8 @@ def measure_workload(wl, ctx: Ctx, headline: bool) -> dict:
         rec["gpu_launches"] = launches_per_step * args.steps
         if rank == 0 and ws == 1 and not args.no_cpu_baseline:
             rec["cpu_baseline"] = cpu_oracle_rate(wl, seed, args.cpu_seconds)
+    elif rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        rec["cpu_baseline"] = cpu_oracle_rate(wl, seed, min(3.0, args.cpu_seconds))  # per stage, a shorter budget
     del graphs
     if r.device_status() != tdt.MOE_OK:
         raise RuntimeError(f"{wl.name}: device status at the end is not MOE_OK")
