@@ -130,13 +130,16 @@ def _open_shared(handle, device) -> torch.Tensor:
     """Map another process's tensor (a handle from ``_share``) into this process, opened in the context
     of this rank's own device: the mapping is then this device's, with peer access enabled as needed,
     so this device's kernels may read and write it (over NVLink when it lives on another GPU).  The
-    tensor reports this device; its memory is the other process's."""
+    tensor reports this device; its memory is the other process's.  The owner synchronised its device
+    before sharing and the handles travel through the process group afterwards, so no IPC event is
+    opened to order the first use."""
     from torch.multiprocessing.reductions import rebuild_cuda_tensor
     fn, args = handle
     if fn is not rebuild_cuda_tensor or len(args) != 15:
         raise RuntimeError("unexpected CUDA IPC handle layout")
     args = list(args)
     args[6] = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    args[14] = False  # event_sync_required
     return fn(*args)
 
 
