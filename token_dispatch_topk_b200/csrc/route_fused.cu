@@ -521,20 +521,22 @@ place_gather_kernel(DispatchArgs a, const uint8_t* __restrict__ hidden, uint32_t
 // A decode batch is a handful of tokens: its routing is a short chain of dependent steps, and one
 // SM writing every hidden row to its slots would be bound by that SM's store bandwidth.  So the
 // grid has one CTA per slot s = t*k + j; every CTA gates all T rows, ranks the slots and scans the
-// local experts (no CTA waits for another); CTA 0 writes the routing outputs; CTA s copies the
-// hidden row of token t to the row of slot s when the slot is local.  The row is loaded into
+// local experts (no CTA waits for another); the routing outputs are shared out over the CTAs, so
+// that no CTA's stores lengthen the chain; CTA s copies the hidden row of token t to the row of
+// slot s when the slot is local.  The row is loaded into
 // registers at kernel entry, so its memory latency overlaps the gating loads.  The phases are
 // laid out for latency (few barriers, no serial searches):
 //   A. hidden row -> registers; expert map -> shared memory; warp w gates rows w, w + 8, ...
 //      (or reads the caller's routes);
 //   B. per warp of 32 slots: local expert, rank among the warp's earlier slots of the same expert
-//      and the warp's count of it (a 32-step shuffle loop); the first slot of each expert in the
+//      and the warp's count of it (one match.any); the first slot of each expert in the
 //      warp records the count in the warp's row of a histogram;
 //   C. per expert (one per thread): count = sum of the warp rows, blocks = ceil(count/bs),
-//      exclusive scan of the blocks over the experts; CTA 0 writes counts, offsets, the expert's
-//      expert_ids and its pad rows;
+//      exclusive scan of the blocks over the experts; each CTA writes counts, offsets, expert_ids
+//      and the pad rows of a contiguous share of the experts;
 //   D. row of slot s = offset of its expert + its expert's slots in earlier warps + its rank;
-//      CTA 0 writes sorted_token_ids, inv_perm and the tail past N_pad; CTA s copies its row.
+//      CTA s writes sorted_token_ids[row] and inv_perm[s] and copies its row; the tail past
+//      N_pad is shared out over the CTAs.
 constexpr int kSmallThreads = 256;
 constexpr int kSmallWarps = kSmallThreads / 32;
 constexpr int kSmallMaxTokens = 32;
@@ -578,6 +580,8 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
   // grid (k, T): this CTA copies the row of slot tok * k + j (no CTA has a slot when P == 0)
   const int tok = blockIdx.y, slot = tok * k + static_cast<int>(blockIdx.x);
   const bool lead = blockIdx.x == 0 && blockIdx.y == 0;
+  // the expert-owned outputs and the tail are shared out over the grid's CTAs (cta = slot)
+  const int ncta = static_cast<int>(gridDim.x * gridDim.y), cta = slot;
   for (int i = tid; i < nw * El; i += kSmallThreads) whist[i] = 0;
 
   moe::pdl_wait();  // logits, routes and hidden may come from the previous kernel
@@ -634,15 +638,9 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
         }
       }
     }
-    int cnt = 0;
-#pragma unroll
-    for (int j = 0; j < 32; ++j) {
-      const int lj = __shfl_sync(0xffffffffu, le, j);
-      const int same = (lj == le) ? 1 : 0;
-      cnt += same;
-      rank += (j < lane) ? same : 0;
-    }
-    if (le >= 0 && rank == 0) whist[warp * El + le] = cnt;
+    const unsigned same = __match_any_sync(0xffffffffu, le);  // lanes of this warp with the same local expert
+    rank = __popc(same & moe::lanemask_lt());
+    if (le >= 0 && rank == 0) whist[warp * El + le] = __popc(same);
     if (tid < P) {
       s_le[tid] = le;
       s_rk[tid] = rank;
@@ -650,9 +648,12 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
   }
   __syncthreads();
 
-  // C. per expert: count, blocks, exclusive scan of the blocks; expert-owned outputs (CTA 0)
+  // C. per expert: count, blocks, exclusive scan of the blocks; each CTA writes the expert-owned
+  //    outputs of its share of the experts
   const int ept = (El + kSmallThreads - 1) / kSmallThreads;  // experts per thread, consecutive
   const int e0 = tid * ept;
+  const int epc = (El + ncta - 1) / ncta;  // experts per CTA, consecutive
+  const int my_e0 = cta * epc, my_e1 = my_e0 + epc;
   int cnt_e[kSmallExpertsPerThread], nb_e[kSmallExpertsPerThread];
   int sum = 0;
 #pragma unroll
@@ -690,7 +691,7 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
     if (i < ept && e < El) {
       const int off = before * bs;
       s_off[e] = off;
-      if (lead) {
+      if (e >= my_e0 && e < my_e1) {
         counts[e] = cnt_e[i];
         offsets[e] = off;
         for (int b = 0; b < nb_e[i]; ++b) expert_ids[before + b] = e;
@@ -705,41 +706,38 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
   }
   __syncthreads();
 
-  // D. slot rows; the tail past N_pad (CTA 0); this CTA's hidden row to its slot row
-  if (lead) {
-    if (tid < P) {
-      int r = -1;
-      if (le >= 0) {
-        r = s_off[le] + rank;
-        for (int w = 0; w < warp; ++w) r += whist[w * El + le];
-        if (static_cast<int64_t>(r) >= C) {  // < N_pad <= C for consistent inputs
-          moe::record_status(status, MOE_ERR_BAD_ROW);
-          r = -1;
-        } else {
-          sorted_ids[r] = tid;
-        }
-      }
-      inv_perm[tid] = r;
-    }
-    for (int64_t i = static_cast<int64_t>(total) + tid; i < C; i += kSmallThreads) sorted_ids[i] = pad_value;
-    for (int b = total_blocks + tid; b < NB; b += kSmallThreads) expert_ids[b] = -1;
-  }
+  // D. this CTA's slot: its row (sorted_token_ids, inv_perm) and the copy of its hidden row; a share
+  //    of the tail past N_pad
   if (slot < P) {
     const int le_s = s_le[slot];
+    int row = -1;
     if (le_s >= 0) {
-      int row = s_off[le_s] + s_rk[slot];
+      row = s_off[le_s] + s_rk[slot];
       for (int w = 0; w < (slot >> 5); ++w) row += whist[w * El + le_s];
-      if (static_cast<int64_t>(row) < C) {
-        uint4* dst = permuted + static_cast<int64_t>(row) * nvec;
-#pragma unroll
-        for (int i = 0; i < kSmallPrefetch; ++i) {
-          const int v = tid + i * kSmallThreads;
-          if (v < nvec) dst[v] = pre[i];
-        }
-        for (int v = tid + kSmallPrefetch * kSmallThreads; v < nvec; v += kSmallThreads) dst[v] = __ldg(src + v);
+      if (static_cast<int64_t>(row) >= C) {  // < N_pad <= C for consistent inputs
+        if (tid == 0) moe::record_status(status, MOE_ERR_BAD_ROW);
+        row = -1;
       }
     }
+    if (tid == 0) {
+      inv_perm[slot] = row;
+      if (row >= 0) sorted_ids[row] = slot;
+    }
+    if (row >= 0) {
+      uint4* dst = permuted + static_cast<int64_t>(row) * nvec;
+#pragma unroll
+      for (int i = 0; i < kSmallPrefetch; ++i) {
+        const int v = tid + i * kSmallThreads;
+        if (v < nvec) dst[v] = pre[i];
+      }
+      for (int v = tid + kSmallPrefetch * kSmallThreads; v < nvec; v += kSmallThreads) dst[v] = __ldg(src + v);
+    }
   }
+  const int64_t stride = static_cast<int64_t>(ncta) * kSmallThreads;
+  for (int64_t i = static_cast<int64_t>(total) + static_cast<int64_t>(cta) * kSmallThreads + tid; i < C; i += stride)
+    sorted_ids[i] = pad_value;
+  for (int64_t b = static_cast<int64_t>(total_blocks) + static_cast<int64_t>(cta) * kSmallThreads + tid; b < NB; b += stride)
+    expert_ids[b] = -1;
 }
 
 // Kernel families instantiated per gating geometry (logits type, vector width, chunks per lane).
