@@ -64,7 +64,7 @@ class MoeRouter:
     def dispatch(self, logits: Optional[torch.Tensor], hidden: torch.Tensor, stream=None,
                  topk_ids: Optional[torch.Tensor] = None):
         """gate + align + permute-gather through the fused entry point (one kernel for small batches,
-        two above).  With ``topk_ids`` given, those routes are aligned instead of gating ``logits``."""
+        three above).  With ``topk_ids`` given, those routes are aligned instead of gating ``logits``."""
         given = topk_ids is not None
         return B.moe_route_dispatch(None if given else logits, hidden, self.k, self.renormalize, self.block_size,
                                     self.expert_map, self.E_local, None if given else self.topk_weights,
