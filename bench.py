@@ -719,18 +719,9 @@ def measure_ep(wl, ctx: Ctx) -> dict:
         raise RuntimeError("expert-parallel steps: device status is not MOE_OK")
     R = int(r.align.counts.sum().item())
     nvlink_bytes = sum((b - a) * wl.H * 2 for o, (a, b) in enumerate(ex.ranges) if o != rank)
-    # kernels per step: the dispatch (one kernel for decode-sized batches; else gating + placement, and
-    # the tile-scan kernel when the tiles times the local experts exceed the lookback's limit), one
-    # combine per owner with tokens, one reduce on an owner with tokens
-    if r.small_batch:
-        n_dispatch = 1
-    else:
-        rt = 32 if (wl.T + 15) // 16 > ctx.sms * 4 else 16
-        elem = 2 if wl.logits_dtype == "bf16" else 4
-        if wl.k <= 8 and (wl.E * elem) % 16 == 0 and ((wl.E <= 64 and wl.T >= 1024) or
-                                                      (elem == 2 and wl.E <= 256 and wl.T >= 16384)):
-            rt = 32
-        n_dispatch = 2 if -(-wl.T // rt) * El <= 65536 else 3
+    # kernels per step: the dispatch (one kernel for decode-sized batches; else gating, tile scan and
+    # placement), one combine per owner with tokens, one reduce on an owner with tokens
+    n_dispatch = 1 if r.small_batch else 3
     per_step = n_dispatch + sum(1 for a, b in ex.ranges if b > a) + (1 if hi > lo else 0)
     step_s = total_ms / args.steps / 1e3
     # roofline of the exchange: the bytes this rank's combine stores into other ranks' memory, against the
@@ -801,10 +792,16 @@ def measure_a2a(wl, ctx: Ctx) -> dict:
     total_ms = max_over_ranks(e0.elapsed_time(e1), dev)
     if tdt.moe_read_status(ex.workspace) != tdt.MOE_OK:
         raise RuntimeError("all-to-all steps: device status is not MOE_OK")
-    per_step = 1 + ws + sum(1 for t in T_per_rank if t) * 2 + (1 if hi > lo else 0) + 2  # gate, align (2), gathers, combines, reduce
+    # kernels per step: gating of this rank's tokens; the align of every rank's routes (one cluster kernel
+    # up to 4096 slots, the three tile kernels up to 65536, count + place above or past 512 local experts);
+    # a gather and a combine per rank with tokens; the reduce of this rank's rows
+    P = wl.T * wl.k
+    n_align = 3 if 4096 < P <= 65536 else (1 if P <= 4096 and ex.E_local <= 512 else 2)
+    own = 1 if hi > lo else 0
+    per_step = own + n_align + 2 * sum(1 for t in T_per_rank if t) + own
     return {"workload": wl.name, "value": wl.T * args.steps / (total_ms / 1e3), "unit": UNIT,
             "ms_per_step": total_ms / args.steps, "E_local": ex.E_local, "tokens_rank0": T_per_rank[0],
-            "launches_per_step_approx": per_step,
+            "launches_per_step": per_step, "gpu_launches": per_step * args.steps,
             "parallelism": f"expert parallel over {ws} ranks, tokens sharded ({T_per_rank[0]} on rank 0): gating, "
                            f"align of every rank's routes, moe_gather pulling rows from each rank, moe_combine "
                            f"pushing partials, barrier, moe_reduce_partials",
@@ -861,7 +858,8 @@ def main():
                 "data": "synthetic (seeded, counter-based; see token_dispatch_topk_b200/inputs.py)",
                 "config": {"workload": wl.name, **{k: v for k, v in wl.as_config().items() if k != "name"},
                            "parallelism": rec["parallelism"], "cuda_graph": False},
-                "expert_parallel_all_to_all": rec, "e2e": None, "cpu_baseline": None}), flush=True)
+                "expert_parallel_all_to_all": rec, "gpu_launches": rec["gpu_launches"], "e2e": None,
+                "cpu_baseline": None}), flush=True)
         if ws > 1:
             dist.barrier()
             dist.destroy_process_group()

@@ -27,6 +27,7 @@ def test_expert_parallel_bench_modes(mode):
         assert key in d, key
     assert d["value"] > 0 and d["scaling"] == "strong" and d["n_gpus"] == 1
     assert d["config"]["workload"] == "tiny_T64_E8_k2"
+    assert d["gpu_launches"] > 0
 
 
 def test_default_bench_line_carries_the_contract_keys():
