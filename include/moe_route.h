@@ -227,6 +227,9 @@ MOE_API moe_status_t moe_align_permute_noalloc(const int32_t* topk_ids, int64_t 
  *              (this needs sorted_token_ids and num_tokens_post_pad; otherwise
  *              they may be NULL).  Rows >= N_pad are never written.
  *   Each hidden row is read once and written to all its local destinations.
+ *   Without MOE_GATHER_HIDDEN_READY the rows are read after inv_perm, and the
+ *   row of a token with no local slot is not read at all (in an expert-parallel
+ *   layer, hidden may be another GPU's memory).
  *   device_status: a device int32 (e.g. the align workspace) or NULL; a row
  *   outside [-1, capacity) is skipped and MOE_ERR_BAD_ROW recorded.
  *   Errors: INVALID_ARG (sizes, null pointers, H % 8 != 0, misaligned pointers).

@@ -9,7 +9,8 @@
 // Both stages are token-major and bandwidth-bound.  The main kernels move rows with TMA
 // bulk copies (cp.async.bulk, no multicast) through shared memory:
 //   gather_tma_kernel:  each hidden row is bulk-loaded once and bulk-stored to every
-//                       local destination row of its token.
+//                       local destination row of its token; rows loaded after the wait for
+//                       inv_perm are only those of tokens with a local slot.
 //   combine_tma_kernel: a producer warp bulk-loads the local slot rows of each (token,
 //                       column chunk) into a ring of stages; consumer warps run the fp32
 //                       fused multiply-adds in ascending slot order from +0 and store one
@@ -115,19 +116,20 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
   }
   __syncwarp();
   const bool evict_first = row_bytes <= moe::kEvictFirstMaxRowBytes;
-  auto load_rows = [&]() {
+  auto load_rows = [&](unsigned mask) {  // bit i: load the row of token t0 + i
     if (lane == 0) {
-      moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(n) * row_bytes);
+      moe::mbar_arrive_expect_tx(&bar, static_cast<uint32_t>(__popc(mask)) * row_bytes);
       for (int i = 0; i < n; ++i) {
-        moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes,
-                       hidden + (t0 + i) * static_cast<int64_t>(row_bytes), row_bytes, &bar, evict_first);
+        if ((mask >> i) & 1u)
+          moe::bulk_load(rows + static_cast<size_t>(i) * row_bytes,
+                         hidden + (t0 + i) * static_cast<int64_t>(row_bytes), row_bytes, &bar, evict_first);
       }
     }
   };
-  if (hidden_ready) load_rows();  // hidden predates the previous kernel: load it while that kernel finishes
+  const unsigned all_rows = n >= 32 ? 0xffffffffu : (1u << n) - 1u;
+  if (hidden_ready) load_rows(all_rows);  // hidden predates the previous kernel: load it while that kernel finishes
   moe::pdl_launch_dependents();
   moe::pdl_wait();                 // inv_perm comes from the previous kernel
-  if (!hidden_ready) load_rows();
   const int nslots = n * k;  // <= 8 * 32
   int32_t dst[8];
 #pragma unroll
@@ -142,6 +144,16 @@ gather_tma_kernel(const uint8_t* __restrict__ hidden, int64_t T, uint32_t row_by
       }
     }
     dst[m] = r;
+  }
+  if (!hidden_ready) {
+    // loaded after the wait: only the rows of tokens with a local slot (a token whose slots are all
+    // remote is never stored, and its row may sit in another GPU's memory)
+    unsigned need = 0u;
+#pragma unroll
+    for (int m = 0; m < 8; ++m) {
+      if (dst[m] >= 0) need |= 1u << ((lane + 32 * m) / k);
+    }
+    load_rows(__reduce_or_sync(0xffffffffu, need));
   }
   if (!moe::mbar_wait(&bar, 0)) {
     moe::record_status(status, MOE_ERR_TIMEOUT);
