@@ -65,6 +65,7 @@ KERNEL_SOURCES = {
     "topk_lane_kernel": "token_dispatch_topk_b200/csrc/topk_softmax.cu",
     "align_count_kernel+align_place_kernel": "token_dispatch_topk_b200/csrc/align_permute.cu",
     "route_small_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
+    "route_decode_kernel": "token_dispatch_topk_b200/csrc/route_fused.cu",
 }
 STAGE_KERNEL = {"topk": "topk_row_warp_kernel", "align": "align_cluster_kernel", "gather": "gather_tma_kernel",
                 "combine": "combine_tma_kernel", "dispatch": "gate_count_kernel+tile_scan_kernel+place_gather_kernel"}
@@ -345,7 +346,7 @@ def stage_kernels(wl, r, sms: int) -> dict:
     lanes = wl.k <= 8 and (wl.E * elem) % 16 == 0 and (
         (wl.E <= 64 and wl.T >= 1024) or (elem == 2 and wl.E <= 256 and wl.T >= 16384))
     if r.small_batch:
-        sk["dispatch"] = "route_small_kernel"
+        sk["dispatch"] = "route_decode_kernel" if wl.T * wl.k <= 32 else "route_small_kernel"
     elif lanes:
         sk["dispatch"] = "gate_count_lanes_kernel+tile_scan_kernel+place_gather_kernel"
     if lanes:
@@ -390,7 +391,7 @@ def measure_workload(wl, ctx: Ctx, headline: bool) -> dict:
     R = int(r.align.counts.sum().item())
     npad = int(r.align.num_tokens_post_pad.item())
     NB = r.align.expert_ids.numel()
-    launches_per_step = 2 if r.small_batch else 4  # route_small + combine_small, or gate_count, tile_scan, place_gather, combine
+    launches_per_step = 2 if r.small_batch else 4  # the decode kernel + combine, or gate_count, tile_scan, place_gather, combine
 
     use_graph = not args.no_graph
     graphs = {}

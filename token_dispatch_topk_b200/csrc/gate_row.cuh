@@ -177,19 +177,46 @@ __device__ __forceinline__ void pop_front_if(K (&k)[NV], bool hit) {
   k[NV - 1] = hit ? K(0) : k[NV - 1];
 }
 
-// Top-k of one row (all 32 lanes of the warp call it).  Lanes 0..k-1 return the expert of rank
-// `lane` in my_e and its weight in my_w; other lanes' outputs are unspecified.  `mode`: bits
-// kGateRenorm and kGateSigmoid.  Softmax weights are exp(x - m) over the full-row sum (or over the
-// k selected); sigmoid weights are 1 / (1 + exp(-x)) each (or over their sum, 1/k if it is 0).
+// The selection key of an expert: bf16 logits give a 32-bit key, fp32 logits a 64-bit one (see the
+// file comment); 0 is below every real key.
+template <typename TIn>
+struct GateKey {
+  using type = uint64_t;
+};
+template <>
+struct GateKey<__nv_bfloat16> {
+  using type = uint32_t;
+};
+
+template <typename TIn>
+__device__ __forceinline__ int key_expert(typename GateKey<TIn>::type key) {
+  if constexpr (sizeof(TIn) == 2) {
+    return static_cast<int>(0xffffu - (key & 0xffffu));
+  } else {
+    return static_cast<int>(0xffffffffu - static_cast<uint32_t>(key));
+  }
+}
+
+template <typename TIn>
+__device__ __forceinline__ float key_value(typename GateKey<TIn>::type key) {
+  if constexpr (sizeof(TIn) == 2) {
+    return ordered16_to_float(key >> 16);
+  } else {
+    return ordered_to_float(static_cast<uint32_t>(key >> 32));
+  }
+}
+
+// The selection half of gate_row (all 32 lanes of the warp call it): lanes 0..k-1 return the key of
+// rank `lane` in my_key; every lane returns the row's largest key in best0 and, for the softmax
+// without renormalisation, the full-row denominator Z (else 0).
 template <typename TIn, int VEC, int CPL>
-__device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int k, int mode, int lane,
-                                         int& my_e, float& my_w) {
+__device__ __forceinline__ void gate_row_select(const TIn* __restrict__ rp, int E, int k, int mode, int lane,
+                                                typename GateKey<TIn>::type& my_key,
+                                                typename GateKey<TIn>::type& best0, float& Z) {
   constexpr int NV = CPL * VEC;
   const int n_chunks = E / VEC;
-  const bool renormalize = (mode & kGateRenorm) != 0;
-  const bool sigmoid = (mode & kGateSigmoid) != 0;
-  float m = 0.f, Z = 0.f, S = 0.f, my_p = 0.f;
-  my_e = 0;
+  const bool full_row_z = (mode & (kGateRenorm | kGateSigmoid)) == 0;
+  Z = 0.f;
 
   if constexpr (sizeof(TIn) == 2) {
     uint32_t key[NV];
@@ -206,7 +233,8 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
         for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0u;
       }
     }
-    uint32_t my_key = 0u, best0 = 0u;
+    my_key = 0u;
+    best0 = 0u;
     constexpr bool kSorted = NV <= 8;  // few keys per lane: keep them sorted, the lane's top is key[0]
     if constexpr (kSorted) sort_desc<NV>(key);
     for (int j = 0; j < k; ++j) {
@@ -220,8 +248,8 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
       best = __reduce_max_sync(0xffffffffu, best);
       if (j == 0) {
         best0 = best;
-        if (!renormalize && !sigmoid) {  // full-row denominator, from the keys before any is retired
-          m = ordered16_to_float(best >> 16);
+        if (full_row_z) {  // full-row denominator, from the keys before any is retired
+          const float m = ordered16_to_float(best >> 16);
           float z = 0.f;
 #pragma unroll
           for (int i = 0; i < NV; ++i) {
@@ -238,13 +266,6 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
       }
       if (lane == j) my_key = best;
     }
-    m = ordered16_to_float(best0 >> 16);
-    if (lane < k) {
-      const float xj = ordered16_to_float(my_key >> 16);
-      my_p = sigmoid ? 1.f / (1.f + expf(-xj)) : expf(xj - m);
-      my_e = static_cast<int>(0xffffu - (my_key & 0xffffu));
-    }
-    if (renormalize) S = warp_sum(my_p);
   } else {
     uint64_t key[NV];
 #pragma unroll
@@ -260,8 +281,8 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
         for (int i = 0; i < VEC; ++i) key[c * VEC + i] = 0ull;
       }
     }
-    uint64_t my_key = 0ull;
-    uint32_t hi0 = 0u;
+    my_key = 0ull;
+    best0 = 0ull;
     constexpr bool kSorted = NV <= 8;
     if constexpr (kSorted) sort_desc<NV>(key);
     for (int j = 0; j < k; ++j) {
@@ -277,9 +298,9 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
                                                              ? static_cast<uint32_t>(mine) : 0u);
       const uint64_t best = (static_cast<uint64_t>(hi) << 32) | lo;
       if (j == 0) {
-        hi0 = hi;
-        if (!renormalize && !sigmoid) {
-          m = ordered_to_float(hi);
+        best0 = best;
+        if (full_row_z) {
+          const float m = ordered_to_float(hi);
           float z = 0.f;
 #pragma unroll
           for (int i = 0; i < NV; ++i) {
@@ -296,19 +317,44 @@ __device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int 
       }
       if (lane == j) my_key = best;
     }
-    m = ordered_to_float(hi0);
-    if (lane < k) {
-      const float xj = ordered_to_float(static_cast<uint32_t>(my_key >> 32));
-      my_p = sigmoid ? 1.f / (1.f + expf(-xj)) : expf(xj - m);
-      my_e = static_cast<int>(0xffffffffu - static_cast<uint32_t>(my_key));
-    }
-    if (renormalize) S = warp_sum(my_p);
   }
+}
+
+// The weights half of gate_row (all 32 lanes call it, with gate_row_select's outputs): lanes 0..k-1
+// return the expert of rank `lane` in my_e and its weight in my_w; other lanes' outputs are
+// unspecified.  Softmax weights are exp(x - m) over Z (or over the k selected when renormalising);
+// sigmoid weights are 1 / (1 + exp(-x)) each (or over their sum, 1/k if it is 0).
+template <typename TIn>
+__device__ __forceinline__ void gate_row_weights(typename GateKey<TIn>::type my_key, typename GateKey<TIn>::type best0,
+                                                 float Z, int k, int mode, int lane, int& my_e, float& my_w) {
+  const bool renormalize = (mode & kGateRenorm) != 0;
+  const bool sigmoid = (mode & kGateSigmoid) != 0;
+  const float m = key_value<TIn>(best0);
+  float my_p = 0.f, S = 0.f;
+  my_e = 0;
+  if (lane < k) {
+    const float xj = key_value<TIn>(my_key);
+    my_p = sigmoid ? 1.f / (1.f + expf(-xj)) : expf(xj - m);
+    my_e = key_expert<TIn>(my_key);
+  }
+  if (renormalize) S = warp_sum(my_p);
   if (sigmoid) {
     my_w = renormalize ? (S > 0.f ? my_p / S : 1.f / static_cast<float>(k)) : my_p;
   } else {
     my_w = my_p / (renormalize ? S : Z);
   }
+}
+
+// Top-k of one row (all 32 lanes of the warp call it).  Lanes 0..k-1 return the expert of rank
+// `lane` in my_e and its weight in my_w; other lanes' outputs are unspecified.  `mode`: bits
+// kGateRenorm and kGateSigmoid (see gate_row_weights).
+template <typename TIn, int VEC, int CPL>
+__device__ __forceinline__ void gate_row(const TIn* __restrict__ rp, int E, int k, int mode, int lane,
+                                         int& my_e, float& my_w) {
+  typename GateKey<TIn>::type key, best0;
+  float Z;
+  gate_row_select<TIn, VEC, CPL>(rp, E, k, mode, lane, key, best0, Z);
+  gate_row_weights<TIn>(key, best0, Z, k, mode, lane, my_e, my_w);
 }
 
 }  // namespace moe_gate

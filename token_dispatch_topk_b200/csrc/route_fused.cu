@@ -740,6 +740,212 @@ route_small_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, u
     expert_ids[b] = -1;
 }
 
+// Decode batches of at most one warp of slots (P <= 32): the outputs of route_small_kernel with two
+// CTA barriers instead of three, and the softmax weights off the routing chain.  Grid and row copy as
+// in route_small_kernel (one CTA per slot).
+//   A. hidden row -> registers; expert map -> shared memory; warp w selects the top-k of rows w, w + 8,
+//      ... (moe_gate::gate_row_select; the selected keys go to shared memory), or reads the caller's
+//      routes;
+//   B. the last warp: local expert of each slot, its rank among earlier slots of the same expert and
+//      the expert's count (one match.any), blocks per expert, exclusive scan of the blocks over the
+//      local experts (one warp over shared memory).  Meanwhile the other warps of CTA 0 turn the
+//      selected keys into the weights (moe_gate::gate_row_weights) and write topk_weights and topk_ids;
+//   C. each CTA: its slot's row (offset of its expert + rank), sorted_token_ids and inv_perm, and the
+//      copy of its hidden row; the expert-owned outputs of a contiguous share of the experts and a
+//      share of the tail past N_pad.
+constexpr int kDecodeMaxSlots = 32;
+template <typename TIn, int VEC, int CPL, bool kGivenIds>
+__global__ void __launch_bounds__(kSmallThreads)
+route_decode_kernel(DispatchArgs a, const uint4* __restrict__ hidden, int nvec, uint4* __restrict__ permuted) {
+  using KeyT = typename moe_gate::GateKey<TIn>::type;
+  __shared__ int s_map[kSmallMaxExperts];
+  __shared__ int s_cnt[kSmallMaxExperts];  // slots per local expert
+  __shared__ int s_blk[kSmallMaxExperts];  // blocks per local expert, then their exclusive scan
+  __shared__ int s_ge[kDecodeMaxSlots];
+  __shared__ int s_le[kDecodeMaxSlots];
+  __shared__ int s_rk[kDecodeMaxSlots];
+  __shared__ KeyT s_key[kDecodeMaxSlots];    // selected keys, slot order
+  __shared__ KeyT s_best[kDecodeMaxSlots];   // per row: its largest key
+  __shared__ float s_z[kDecodeMaxSlots];     // per row: the full-row denominator (softmax without renormalising)
+  __shared__ int s_total_blocks;
+  // every parameter, read into registers at entry (moe::pin), before the kernel waits for anything
+  const int T = moe::pin(static_cast<int>(a.T)), k = moe::pin(a.k), E = moe::pin(a.E), El = moe::pin(a.E_local);
+  const int bs = moe::pin(a.bs), bs_shift = moe::pin(a.bs_shift), NB = moe::pin(a.NB);
+  const int renormalize = moe::pin(a.renormalize);
+  const int64_t C = moe::pin(a.C);
+  const TIn* logits = moe::pin(static_cast<const TIn*>(a.logits));
+  const int32_t* expert_map = moe::pin(a.expert_map);
+  int32_t* topk_ids = moe::pin(a.topk_ids);
+  float* topk_weights = moe::pin(a.topk_weights);
+  int32_t* counts = moe::pin(a.counts);
+  int32_t* offsets = moe::pin(a.offsets);
+  int32_t* sorted_ids = moe::pin(a.sorted_ids);
+  int32_t* expert_ids = moe::pin(a.expert_ids);
+  int32_t* n_pad = moe::pin(a.n_pad);
+  int32_t* inv_perm = moe::pin(a.inv_perm);
+  int32_t* status = moe::pin(a.status);
+  hidden = moe::pin(hidden);
+  permuted = moe::pin(permuted);
+  nvec = moe::pin(nvec);
+  const int P = T * k;  // <= kDecodeMaxSlots
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int tok = blockIdx.y, slot = tok * k + static_cast<int>(blockIdx.x);
+  const bool lead = blockIdx.x == 0 && blockIdx.y == 0;
+  const int ncta = static_cast<int>(gridDim.x * gridDim.y), cta = slot;
+  for (int e = tid; e < El; e += kSmallThreads) {
+    s_cnt[e] = 0;
+    s_blk[e] = 0;
+  }
+
+  moe::pdl_wait();  // logits, routes and hidden may come from the previous kernel
+  moe::pdl_launch_dependents();
+  // A. this CTA's hidden row, the expert map and the gating loads, in flight together
+  const uint4* src = hidden + static_cast<int64_t>(slot < P ? tok : 0) * nvec;
+  uint4 pre[kSmallPrefetch];
+#pragma unroll
+  for (int i = 0; i < kSmallPrefetch; ++i) {
+    const int v = tid + i * kSmallThreads;
+    if (slot < P && v < nvec) pre[i] = __ldg(src + v);
+  }
+  int mv[kSmallExpertsPerThread];
+#pragma unroll
+  for (int i = 0; i < kSmallExpertsPerThread; ++i) {
+    const int g = tid + i * kSmallThreads;
+    mv[i] = g < E ? (expert_map != nullptr ? __ldg(expert_map + g) : g) : 0;
+  }
+  if constexpr (kGivenIds) {
+    if (tid < P) s_ge[tid] = topk_ids[tid];
+  } else {
+    for (int row = warp; row < T; row += kSmallWarps) {
+      KeyT key, best0;
+      float z;
+      moe_gate::gate_row_select<TIn, VEC, CPL>(logits + static_cast<int64_t>(row) * E, E, k, renormalize, lane, key,
+                                               best0, z);
+      if (lane < k) {
+        s_ge[row * k + lane] = moe_gate::key_expert<TIn>(key);
+        s_key[row * k + lane] = key;
+      }
+      if (lane == 0) {
+        s_best[row] = best0;
+        s_z[row] = z;
+      }
+    }
+  }
+#pragma unroll
+  for (int i = 0; i < kSmallExpertsPerThread; ++i) {
+    const int g = tid + i * kSmallThreads;
+    if (g < E) s_map[g] = mv[i];
+  }
+  __syncthreads();
+
+  // B. ranks, counts and the block scan (last warp); the weights (the other warps of CTA 0)
+  if (warp == kSmallWarps - 1) {
+    int le = -1;
+    if (lane < P) {
+      const int g = s_ge[lane];
+      if (static_cast<unsigned>(g) >= static_cast<unsigned>(E)) {
+        if (lead) moe::record_status(status, MOE_ERR_BAD_EXPERT_ID);
+      } else {
+        le = s_map[g];
+        if (le < -1 || le >= El) {
+          if (lead) moe::record_status(status, MOE_ERR_BAD_EXPERT_ID);
+          le = -1;
+        }
+      }
+    }
+    const unsigned same = __match_any_sync(0xffffffffu, le);  // lanes with the same local expert
+    const int rank = __popc(same & moe::lanemask_lt());
+    if (le >= 0 && rank == 0) {
+      const int c = __popc(same);
+      s_cnt[le] = c;
+      s_blk[le] = bs_shift >= 0 ? (c + bs - 1) >> bs_shift : (c + bs - 1) / bs;
+    }
+    if (lane < P) {
+      s_le[lane] = le;
+      s_rk[lane] = rank;
+    }
+    __syncwarp();
+    const int per = (El + 31) >> 5;  // lane l scans a contiguous run of the local experts
+    const int e0 = lane * per < El ? lane * per : El;
+    const int e1 = e0 + per < El ? e0 + per : El;
+    int sum = 0;
+    for (int e = e0; e < e1; ++e) sum += s_blk[e];
+    int incl = sum;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += v;
+    }
+    int run = incl - sum;
+    for (int e = e0; e < e1; ++e) {
+      const int b = s_blk[e];
+      s_blk[e] = run;
+      run += b;
+    }
+    if (lane == 31) s_total_blocks = incl;
+  } else if (!kGivenIds && lead) {
+    for (int row = warp; row < T; row += kSmallWarps - 1) {
+      int e;
+      float w;
+      moe_gate::gate_row_weights<TIn>(lane < k ? s_key[row * k + lane] : KeyT(0), s_best[row], s_z[row], k, renormalize,
+                                      lane, e, w);
+      if (lane < k) {
+        topk_weights[row * k + lane] = w;
+        topk_ids[row * k + lane] = e;
+      }
+    }
+  }
+  __syncthreads();
+
+  // C. this CTA's slot and its row; a share of the expert-owned outputs and of the tail
+  const int total_blocks = s_total_blocks;
+  const int total = total_blocks * bs;  // N_pad
+  const int32_t pad_value = P;
+  if (slot < P) {
+    const int le_s = s_le[slot];
+    int row = -1;
+    if (le_s >= 0) {
+      row = s_blk[le_s] * bs + s_rk[slot];
+      if (static_cast<int64_t>(row) >= C) {  // < N_pad <= C for consistent inputs
+        if (tid == 0) moe::record_status(status, MOE_ERR_BAD_ROW);
+        row = -1;
+      }
+    }
+    if (tid == 0) {
+      inv_perm[slot] = row;
+      if (row >= 0) sorted_ids[row] = slot;
+    }
+    if (row >= 0) {
+      uint4* dst = permuted + static_cast<int64_t>(row) * nvec;
+#pragma unroll
+      for (int i = 0; i < kSmallPrefetch; ++i) {
+        const int v = tid + i * kSmallThreads;
+        if (v < nvec) dst[v] = pre[i];
+      }
+      for (int v = tid + kSmallPrefetch * kSmallThreads; v < nvec; v += kSmallThreads) dst[v] = __ldg(src + v);
+    }
+  }
+  const int epc = (El + ncta - 1) / ncta;  // experts per CTA, consecutive
+  const int my_e1 = (cta + 1) * epc < El ? (cta + 1) * epc : El;
+  for (int e = cta * epc + tid; e < my_e1; e += kSmallThreads) {
+    const int c = s_cnt[e], b0 = s_blk[e];
+    const int nb = c == 0 ? 0 : bs_shift >= 0 ? (c + bs - 1) >> bs_shift : (c + bs - 1) / bs;
+    counts[e] = c;
+    offsets[e] = b0 * bs;
+    for (int b = 0; b < nb; ++b) expert_ids[b0 + b] = e;
+    for (int p = b0 * bs + c; p < (b0 + nb) * bs; ++p) sorted_ids[p] = pad_value;
+  }
+  if (lead && tid == 0) {
+    offsets[El] = total;
+    n_pad[0] = total;
+  }
+  const int64_t stride = static_cast<int64_t>(ncta) * kSmallThreads;
+  for (int64_t i = static_cast<int64_t>(total) + static_cast<int64_t>(cta) * kSmallThreads + tid; i < C; i += stride)
+    sorted_ids[i] = pad_value;
+  for (int64_t b = static_cast<int64_t>(total_blocks) + static_cast<int64_t>(cta) * kSmallThreads + tid; b < NB; b += stride)
+    expert_ids[b] = -1;
+}
+
 // Kernel families instantiated per gating geometry (logits type, vector width, chunks per lane).
 template <typename TIn, int VEC, int CPL>
 struct GateCountFamily {
@@ -750,6 +956,11 @@ template <typename TIn, int VEC, int CPL>
 struct SmallFamily {
   using Fn = void (*)(DispatchArgs, const uint4*, int, uint4*);
   static Fn get() { return &route_small_kernel<TIn, VEC, CPL, false>; }
+};
+template <typename TIn, int VEC, int CPL>
+struct DecodeFamily {
+  using Fn = void (*)(DispatchArgs, const uint4*, int, uint4*);
+  static Fn get() { return &route_decode_kernel<TIn, VEC, CPL, false>; }
 };
 using GcKernel = GateCountFamily<float, 1, 1>::Fn;
 using SmallKernel = SmallFamily<float, 1, 1>::Fn;
@@ -917,7 +1128,11 @@ extern "C" moe_status_t moe_route_dispatch(const void* logits, moe_dtype_t dtype
 
   // small batches: one kernel, one CTA per slot
   if (small_batch) {
-    SmallKernel sk = given_ids ? &route_small_kernel<float, 1, 1, true>
+    // at most one warp of slots: route_decode_kernel (two CTA barriers); above: route_small_kernel
+    const bool one_warp = P <= kDecodeMaxSlots;
+    SmallKernel sk = given_ids ? (one_warp ? &route_decode_kernel<float, 1, 1, true> : &route_small_kernel<float, 1, 1, true>)
+                     : one_warp ? (dtype == MOE_DTYPE_BF16 ? family_pick<DecodeFamily, __nv_bfloat16>(vec, cpl)
+                                                          : family_pick<DecodeFamily, float>(vec, cpl))
                      : dtype == MOE_DTYPE_BF16 ? family_pick<SmallFamily, __nv_bfloat16>(vec, cpl)
                                                : family_pick<SmallFamily, float>(vec, cpl);
     if (sk == nullptr) return MOE_ERR_UNSUPPORTED;
