@@ -266,9 +266,9 @@ MOE_API moe_status_t moe_combine(const void* expert_out, const float* topk_weigh
  * For T > 32, T*k > 256 or E > 256: the first kernel gates tiles of tokens and counts each tile's slots
  * per local expert with their ranks inside the tile; the second turns each expert's tile counts into
  * its prefix over the tiles and its total; the third scans the padded totals into the offsets, gives
- * every slot its row and copies the hidden rows there.  Smaller batches (decode) take one kernel with one CTA per slot: each CTA
- * routes the whole batch by itself, CTA 0 writes the routing outputs and every CTA copies the
- * hidden row of its own slot.
+ * every slot its row and copies the hidden rows there.  Smaller batches (decode) take one kernel with one
+ * CTA per slot: each CTA routes the whole batch by itself, writes its own slot's row and a share of the
+ * other routing outputs, and copies the hidden row of its slot.
  *   logits [T, E] bf16/fp32 (dtype); hidden [T, H] bf16, 16-byte aligned, H % 8 == 0 and
  *   H <= 65536; expert_map and E_local as for moe_align_permute.
  *   flags: MOE_RENORMALIZE, MOE_SCORING_SIGMOID (as for moe_topk_softmax);
