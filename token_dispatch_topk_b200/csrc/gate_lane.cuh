@@ -9,13 +9,15 @@
 // gate_row.cuh spends a warp on each row: k rounds of warp-wide reductions, a few hundred
 // instructions per row, which makes gating of many short rows (say E = 60 experts, T = 16K tokens)
 // bound by instruction issue.  Here a CTA stages 32 rows in shared memory and G lanes (up to 8)
-// scan each row once, inserting every logit into a register-resident list of the K largest (2 * K
-// instructions per bf16 logit, as unique 32-bit keys; about 5 * K per fp32 logit, as value and
-// index); the G lists are merged with log2(G) shuffle rounds.  Several times fewer instructions per
-// row than the warp-per-row kernel.
+// scan each row once.  bf16 logits become unique 32-bit keys, and their K largest come from sorting
+// networks (a sort of each 16-byte chunk, then bitonic merges of the lists: about 5 instructions per
+// logit for K = 8).  fp32 logits are inserted into a register-resident list of the K largest, as value
+// and index (about 5 * K instructions per logit).  The G lists are merged with log2(G) shuffle rounds.
+// That is several times fewer instructions per row than the warp-per-row kernel.
 //
-// Order: logits arrive in ascending expert order and a logit moves ahead only of kept logits it
-// strictly exceeds, so among equal logits the lower index stays ahead (+0 and -0 compare equal).
+// Order: fp32 logits arrive in ascending expert order and a logit moves ahead only of kept logits it
+// strictly exceeds, so among equal logits the lower index stays ahead (+0 and -0 compare equal); bf16
+// keys hold the inverted index below the value, so the same order is the keys' order.
 #pragma once
 
 #include <cuda_runtime.h>
@@ -110,43 +112,59 @@ struct LaneTopK {
 };
 
 // bf16 logits: the ordered 16-bit value above, 0xFFFF - expert below, so the keys of a row are
-// unique and their order is the selection order (0 is below every key of a finite logit).  The K
-// largest keys are kept sorted descending: a key bubbles down the list with one max and one min
-// per entry.  Keys being unique, the list holds the K largest keys whatever order they arrive in.
-template <int K>
-struct LaneTopKey {
-  uint32_t v[K];
-
-  __device__ __forceinline__ void init() {
-#pragma unroll
-    for (int p = 0; p < K; ++p) v[p] = 0u;
-  }
-
-  __device__ __forceinline__ void insert(uint32_t x) {
-#pragma unroll
-    for (int p = 0; p < K; ++p) {
-      const uint32_t hi = v[p] > x ? v[p] : x;
-      x = v[p] > x ? x : v[p];
-      v[p] = hi;
-    }
-  }
-};
-
+// unique and their order is the selection order (0 is below every key of a finite logit).  Keys being
+// unique, the K largest of a set do not depend on the order in which its parts are combined, so they
+// are found with sorting networks: each 16-byte chunk's 8 keys are sorted (Batcher's 19
+// compare-exchanges), and two descending lists of KP keys (KP = K rounded up to a power of two,
+// padded with 0) give the KP largest of both as max(a[i], b[KP-1-i]), a bitonic sequence that
+// log2(KP) rounds of half-cleaners sort.  No chain runs through all the keys of a row, so most
+// compare-exchanges are independent.
 __device__ __forceinline__ uint32_t bf16_key(uint32_t bits16, int e) {
   return (ordered16(bits16) << 16) | (0xffffu - static_cast<uint32_t>(e));
 }
 
 template <int K>
-__device__ __forceinline__ void lane_insert_chunk_keys(LaneTopKey<K>& t, const uint4 q, int j) {
+struct KeyListSize {
+  static constexpr int value = K <= 1 ? 1 : (K <= 2 ? 2 : (K <= 4 ? 4 : 8));
+};
+
+// v bitonic -> v sorted descending (half-cleaners at distance KP/2, ..., 1).
+template <int KP>
+__device__ __forceinline__ void bitonic_sort_desc(uint32_t (&v)[KP]) {
+#pragma unroll
+  for (int d = KP / 2; d >= 1; d >>= 1) {
+#pragma unroll
+    for (int i = 0; i < KP; ++i) {
+      if ((i & d) == 0) {
+        const uint32_t a = v[i], b = v[i + d];
+        v[i] = a > b ? a : b;
+        v[i + d] = a > b ? b : a;
+      }
+    }
+  }
+}
+
+// l, o descending -> l = the KP largest of both, descending.
+template <int KP>
+__device__ __forceinline__ void merge_top_keys(uint32_t (&l)[KP], const uint32_t (&o)[KP]) {
+#pragma unroll
+  for (int i = 0; i < KP; ++i) {
+    const uint32_t b = o[KP - 1 - i];
+    l[i] = l[i] > b ? l[i] : b;
+  }
+  bitonic_sort_desc<KP>(l);
+}
+
+// The KP largest keys of one 16-byte chunk of bf16 logits (chunk j of the row), descending.
+template <int KP>
+__device__ __forceinline__ void chunk_top_keys(const uint4 q, int j, uint32_t (&out)[KP]) {
   const int i = 8 * j;
-  t.insert(bf16_key(q.x & 0xffffu, i));
-  t.insert(bf16_key(q.x >> 16, i + 1));
-  t.insert(bf16_key(q.y & 0xffffu, i + 2));
-  t.insert(bf16_key(q.y >> 16, i + 3));
-  t.insert(bf16_key(q.z & 0xffffu, i + 4));
-  t.insert(bf16_key(q.z >> 16, i + 5));
-  t.insert(bf16_key(q.w & 0xffffu, i + 6));
-  t.insert(bf16_key(q.w >> 16, i + 7));
+  uint32_t c[8] = {bf16_key(q.x & 0xffffu, i),     bf16_key(q.x >> 16, i + 1), bf16_key(q.y & 0xffffu, i + 2),
+                   bf16_key(q.y >> 16, i + 3),     bf16_key(q.z & 0xffffu, i + 4), bf16_key(q.z >> 16, i + 5),
+                   bf16_key(q.w & 0xffffu, i + 6), bf16_key(q.w >> 16, i + 7)};
+  sort_desc<8>(c);
+#pragma unroll
+  for (int r = 0; r < KP; ++r) out[r] = c[r];
 }
 
 // Insert the logits of one 16-byte chunk (chunk j of the row) in ascending expert order.
@@ -185,7 +203,7 @@ constexpr int kLaneMaxChunks = 4;  // chunks one lane holds: cpr / G rounded up,
 // `mode`: kGateRenorm, kGateSigmoid.  Every lane of the group returns the K experts in selection
 // order and their weights.
 // Merge, after each lane's scan, pairwise over shuffle distance 1, 2, then 4:
-//   bf16: the keys are unique, so inserting the partner's K keys gives the K largest of both.
+//   bf16: the keys are unique, so the bitonic merge of the partner's list gives the K largest of both.
 //   fp32: the list of the lower chunks is the base and the other is inserted into it in its own
 //   order.  Every expert of the inserted list has a higher index than every expert of the base,
 //   and among equal logits the inserted list keeps the lower index ahead, so the merged list is
@@ -201,24 +219,29 @@ __device__ __forceinline__ void lane_gate_row(const uint4* __restrict__ srow, in
   }
   LaneTopK<K> t;
   if constexpr (sizeof(TIn) == 2) {
-    LaneTopKey<K> kt;
-    kt.init();
+    constexpr int KP = KeyListSize<K>::value;
+    uint32_t kt[KP];
+#pragma unroll
+    for (int r = 0; r < KP; ++r) kt[r] = 0u;
 #pragma unroll
     for (int u = 0; u < kLaneMaxChunks; ++u) {
-      if (j0 + u < j1) lane_insert_chunk_keys<K>(kt, q[u], j0 + u);
+      if (j0 + u < j1) {
+        uint32_t c[KP];
+        chunk_top_keys<KP>(q[u], j0 + u, c);
+        merge_top_keys<KP>(kt, c);
+      }
     }
 #pragma unroll
     for (int d = 1; d < G; d <<= 1) {
-      uint32_t o[K];
+      uint32_t o[KP];
 #pragma unroll
-      for (int r = 0; r < K; ++r) o[r] = __shfl_xor_sync(0xffffffffu, kt.v[r], d);
-#pragma unroll
-      for (int r = 0; r < K; ++r) kt.insert(o[r]);
+      for (int r = 0; r < KP; ++r) o[r] = __shfl_xor_sync(0xffffffffu, kt[r], d);
+      merge_top_keys<KP>(kt, o);
     }
 #pragma unroll
     for (int r = 0; r < K; ++r) {
-      t.v[r] = ordered16_to_float(kt.v[r] >> 16);
-      t.e[r] = static_cast<int>(0xffffu - (kt.v[r] & 0xffffu));
+      t.v[r] = ordered16_to_float(kt[r] >> 16);
+      t.e[r] = static_cast<int>(0xffffu - (kt[r] & 0xffffu));
     }
   } else {
     t.init();
